@@ -1,0 +1,134 @@
+/*
+ * attn_jvp.h -- C ABI of the fused attention + Jacobian-vector-product
+ * forward pass for NVIDIA B200 (sm_100a).
+ *
+ * The operation (rCM, "Large-scale diffusion distillation via
+ * score-regularized continuous-time consistency", §3.2 / App. C, as the
+ * anthology record LIT-783 summarises it: FlashAttention-2 and its JVP in one
+ * tiled pass, for self- and cross-attention; the model card "rCM Consistency
+ * Distillation Diffusion Model", Research Highlights, names the open-source
+ * FlashAttention-2 JVP kernel).  For every batch b, head h and query row i:
+ *
+ *   S   = s * Q K^T                   P  = row-softmax(S)
+ *   dS  = s * (tQ K^T + Q tK^T)       mu = rowsum(P .* dS)
+ *   O   = P V
+ *   tO  = (P .* (dS - mu)) V + P tV   (the derivative of O along (tQ, tK, tV))
+ *   lse = ln sum_j exp(S_ij)          (natural log, fp32)
+ *
+ * computed in one pass over the keys with an online softmax: P and dS are
+ * never written to memory.  Non-causal, no mask, no dropout; Lq may differ
+ * from Lk (cross-attention).  s is a constant (no derivative with respect to
+ * it).
+ *
+ * Layout: every tensor is a contiguous row-major [B][H][L][d] array (the
+ * layout of a PyTorch [B, H, L, d] tensor); the tangents tQ, tK, tV share the
+ * layout of Q, K, V (the anthology record notes that context parallelism
+ * distributes the QKV tangents like QKV).  lse is [B][H][Lq] fp32.
+ *
+ * Ownership and execution: all pointers are DEVICE pointers owned by the
+ * caller.  The library allocates no device memory per call and keeps no
+ * per-call state.  Calls are stream-ordered and asynchronous: they return
+ * after enqueueing work on `stream` (a cudaStream_t; NULL = legacy default
+ * stream) and do not synchronise.  Calls are thread-safe.  Inputs must not
+ * alias outputs.  Non-finite inputs give unspecified (but memory-safe)
+ * results.
+ *
+ * Errors: argument checks run on the host before any launch and return a
+ * negative ajvp_status; nothing is enqueued then.  A failed launch returns
+ * AJVP_ERR_CUDA and the cudaError_t is kept per thread
+ * (attn_jvp_last_cuda_error).  Every wait inside the kernels is bounded: if a
+ * pipeline wait ever exceeds the wait bound, the kernel records
+ * AJVP_ERR_TIMEOUT in a device status word, releases what it holds and
+ * returns; attn_jvp_check_device_status reads (and clears) that word.
+ */
+#ifndef ATTN_JVP_H
+#define ATTN_JVP_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    AJVP_OK = 0,
+    AJVP_ERR_INVALID_ARG = -1,        /* null pointer, negative size, Lk == 0, non-finite scale */
+    AJVP_ERR_UNSUPPORTED_DIM = -2,    /* head dimension d not supported by this entry point */
+    AJVP_ERR_MISALIGNED = -3,         /* a pointer breaks the alignment rule of the entry point */
+    AJVP_ERR_UNSUPPORTED_DEVICE = -4, /* current device is not compute capability 10.0 */
+    AJVP_ERR_TIMEOUT = -5,            /* a kernel wait ran past its bound (device status word) */
+    AJVP_ERR_CUDA = -6,               /* a CUDA runtime/driver call failed */
+    AJVP_ERR_TOO_LARGE = -7           /* a size exceeds the documented maximum */
+} ajvp_status;
+
+/*
+ * attn_jvp_fwd -- bf16 I/O, fp32 accumulation, tcgen05 tensor-core kernel.
+ *
+ *   q, tq      : const __nv_bfloat16 [B][H][Lq][d]
+ *   k, v, tk, tv: const __nv_bfloat16 [B][H][Lk][d]
+ *   o, to      : __nv_bfloat16 [B][H][Lq][d]   (outputs, round-to-nearest-even)
+ *   lse        : float [B][H][Lq], or NULL to skip it
+ *   scale      : the softmax scale s (finite)
+ *   stream     : cudaStream_t, or NULL
+ *
+ * Supported: d == 128; B, H, Lq >= 0; Lk >= 1; Lq, Lk < 2^31;
+ * B*H*ceil(Lq/128) < 2^31.  B*H == 0 or Lq == 0 is a no-op returning AJVP_OK.
+ * Every pointer must be 16-byte aligned (tensor-memory-accelerator rule).
+ * The current device must be compute capability 10.0 (B200).
+ * Returns AJVP_OK once the kernel is enqueued.
+ */
+int attn_jvp_fwd(const void *q, const void *k, const void *v,
+                 const void *tq, const void *tk, const void *tv,
+                 void *o, void *to, float *lse,
+                 int64_t B, int64_t H, int64_t Lq, int64_t Lk, int64_t d,
+                 float scale, void *stream);
+
+/*
+ * attn_jvp_fwd_f32 -- fp32 I/O, fp32 arithmetic (CUDA-core kernel), for the
+ * accuracy-critical configuration.  Same math, layout and error rules as
+ * attn_jvp_fwd, with float tensors.  Supported: 1 <= d <= 256; pointers
+ * 4-byte aligned.  Any compute capability 10.0 device.
+ */
+int attn_jvp_fwd_f32(const float *q, const float *k, const float *v,
+                     const float *tq, const float *tk, const float *tv,
+                     float *o, float *to, float *lse,
+                     int64_t B, int64_t H, int64_t Lq, int64_t Lk, int64_t d,
+                     float scale, void *stream);
+
+/* Static, human-readable description of an ajvp_status value. */
+const char *attn_jvp_strerror(int status);
+
+/* cudaError_t behind the calling thread's last AJVP_ERR_CUDA (0 if none). */
+int attn_jvp_last_cuda_error(void);
+
+/*
+ * Synchronise `stream`, then read and clear the device status word of the
+ * current device.  Returns AJVP_OK, AJVP_ERR_TIMEOUT (some kernel wait ran
+ * past its bound since the last check) or AJVP_ERR_CUDA.
+ */
+int attn_jvp_check_device_status(void *stream);
+
+/*
+ * Bound, in nanoseconds, on any single pipeline wait inside the kernels
+ * (default 2e9, i.e. 2 s; 0 restores the default).  Applies to launches made
+ * after the call, process-wide.
+ */
+int attn_jvp_set_wait_bound_ns(uint64_t ns);
+
+/*
+ * Failure-detection self test: enqueue a one-warp kernel that waits, through
+ * the same bounded-wait routine the attention kernel uses, on a barrier that
+ * nothing ever completes, with a bound of `bound_ns`.  The kernel gives up,
+ * records AJVP_ERR_TIMEOUT in the device status word and returns; the GPU
+ * context stays usable.  Returns AJVP_OK once enqueued.
+ */
+int attn_jvp_selftest_wait_timeout(uint64_t bound_ns, void *stream);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int attn_jvp_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_JVP_H */
