@@ -1,0 +1,35 @@
+"""Fused attention + Jacobian-vector product (forward-mode tangent) for
+NVIDIA B200 (sm_100a): O = softmax(s Q K^T) V and tO, its derivative along
+(tQ, tK, tV), in one tiled pass -- the attention hot path of rCM's
+continuous-time consistency distillation.
+
+The computation lives in the CUDA library ``libattnjvp.so`` (C ABI in
+``include/attn_jvp.h``); this package is its ctypes binding plus the seeded
+synthetic-input generator.  The library is loaded on first use and a missing
+build raises.
+"""
+from ._binding import (  # noqa: F401
+    AJVP_ERR_CUDA,
+    AJVP_ERR_INVALID_ARG,
+    AJVP_ERR_MISALIGNED,
+    AJVP_ERR_TIMEOUT,
+    AJVP_ERR_TOO_LARGE,
+    AJVP_ERR_UNSUPPORTED_DEVICE,
+    AJVP_ERR_UNSUPPORTED_DIM,
+    AJVP_OK,
+    AttnJvpError,
+    attn_jvp,
+    attn_jvp_fwd,
+    attn_jvp_fwd_f32,
+    check_device_status,
+    load_library,
+    selftest_wait_timeout,
+    set_wait_bound_ns,
+    strerror,
+    version,
+)
+
+__all__ = [
+    "attn_jvp", "attn_jvp_fwd", "attn_jvp_fwd_f32", "check_device_status", "load_library",
+    "selftest_wait_timeout", "set_wait_bound_ns", "strerror", "version", "AttnJvpError",
+]

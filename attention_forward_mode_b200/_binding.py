@@ -1,0 +1,180 @@
+"""ctypes binding of the C ABI in ``include/attn_jvp.h``.
+
+Argument marshalling only: shape/dtype/device checks of torch tensors, raw
+pointers handed to the library, status codes turned into exceptions.  Every
+step of the computation runs in the library's CUDA kernels; there is no other
+implementation to fall back to, so a missing library raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libattnjvp.so")
+
+AJVP_OK = 0
+AJVP_ERR_INVALID_ARG = -1
+AJVP_ERR_UNSUPPORTED_DIM = -2
+AJVP_ERR_MISALIGNED = -3
+AJVP_ERR_UNSUPPORTED_DEVICE = -4
+AJVP_ERR_TIMEOUT = -5
+AJVP_ERR_CUDA = -6
+AJVP_ERR_TOO_LARGE = -7
+
+# every symbol the header declares
+EXPORTED = ("attn_jvp_fwd", "attn_jvp_fwd_f32", "attn_jvp_strerror", "attn_jvp_last_cuda_error",
+            "attn_jvp_check_device_status", "attn_jvp_set_wait_bound_ns",
+            "attn_jvp_selftest_wait_timeout", "attn_jvp_version")
+
+_lock = threading.Lock()
+_lib = None
+
+
+class AttnJvpError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(what)
+
+
+def load_library(path: str = LIB_PATH):
+    """Load (once) and type the shared library.  Raises if it is missing."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(path):
+            raise RuntimeError(f"CUDA library not built: {path} is missing "
+                               "(run `python -m attention_forward_mode_b200.build`)")
+        lib = ctypes.CDLL(path)
+        vp, i64, f32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_float
+        fwd_args = [vp] * 9 + [i64] * 5 + [f32, vp]
+        lib.attn_jvp_fwd.argtypes = fwd_args
+        lib.attn_jvp_fwd.restype = ctypes.c_int
+        lib.attn_jvp_fwd_f32.argtypes = fwd_args
+        lib.attn_jvp_fwd_f32.restype = ctypes.c_int
+        lib.attn_jvp_strerror.argtypes = [ctypes.c_int]
+        lib.attn_jvp_strerror.restype = ctypes.c_char_p
+        lib.attn_jvp_last_cuda_error.argtypes = []
+        lib.attn_jvp_last_cuda_error.restype = ctypes.c_int
+        lib.attn_jvp_check_device_status.argtypes = [vp]
+        lib.attn_jvp_check_device_status.restype = ctypes.c_int
+        lib.attn_jvp_set_wait_bound_ns.argtypes = [ctypes.c_uint64]
+        lib.attn_jvp_set_wait_bound_ns.restype = ctypes.c_int
+        lib.attn_jvp_selftest_wait_timeout.argtypes = [ctypes.c_uint64, vp]
+        lib.attn_jvp_selftest_wait_timeout.restype = ctypes.c_int
+        lib.attn_jvp_version.argtypes = []
+        lib.attn_jvp_version.restype = ctypes.c_int
+        _lib = lib
+        return lib
+
+
+def strerror(status: int) -> str:
+    return load_library().attn_jvp_strerror(int(status)).decode()
+
+
+def _check(status: int, where: str):
+    if status != AJVP_OK:
+        lib = load_library()
+        msg = f"{where}: {strerror(status)} (status {status})"
+        if status == AJVP_ERR_CUDA:
+            msg += f", cudaError {lib.attn_jvp_last_cuda_error()}"
+        raise AttnJvpError(status, msg)
+
+
+def _stream_handle(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _prepare(q, k, v, tq, tk, tv, o, to, lse, dtype, want_lse):
+    for name, x in (("q", q), ("k", k), ("v", v), ("tq", tq), ("tk", tk), ("tv", tv)):
+        if not isinstance(x, torch.Tensor) or not x.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+        if x.dtype != dtype:
+            raise ValueError(f"{name} must be {dtype}, got {x.dtype}")
+        if x.dim() != 4 or not x.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous [B, H, L, d] tensor")
+    B, H, Lq, d = q.shape
+    Lk = k.shape[2]
+    if tq.shape != q.shape:
+        raise ValueError("tq must have the shape of q")
+    for name, x in (("k", k), ("v", v), ("tk", tk), ("tv", tv)):
+        if x.shape != (B, H, Lk, d):
+            raise ValueError(f"{name} must be [B, H, Lk, d] = {(B, H, Lk, d)}, got {tuple(x.shape)}")
+    if o is None:
+        o = torch.empty_like(q)
+    if to is None:
+        to = torch.empty_like(q)
+    if want_lse and lse is None:
+        lse = torch.empty((B, H, Lq), device=q.device, dtype=torch.float32)
+    for name, x, shp, dt in (("o", o, q.shape, dtype), ("to", to, q.shape, dtype)):
+        if x.shape != shp or x.dtype != dt or not x.is_contiguous() or not x.is_cuda:
+            raise ValueError(f"{name} must be a contiguous CUDA {dt} tensor of shape {tuple(shp)}")
+    if lse is not None and (lse.shape != (B, H, Lq) or lse.dtype != torch.float32 or not lse.is_contiguous()):
+        raise ValueError("lse must be a contiguous float32 [B, H, Lq] tensor")
+    return o, to, lse, (B, H, Lq, Lk, d)
+
+
+def attn_jvp_fwd(q, k, v, tq, tk, tv, scale=None, o=None, to=None, lse=None, stream=None, want_lse=True):
+    """O, tO, lse for bf16 [B, H, L, d] CUDA tensors (d = 128), through the
+    C ABI's ``attn_jvp_fwd`` (tcgen05 kernel).  Output tensors may be passed
+    in; otherwise they are allocated.  Asynchronous on ``stream`` (default:
+    torch's current stream)."""
+    o, to, lse, (B, H, Lq, Lk, d) = _prepare(q, k, v, tq, tk, tv, o, to, lse, torch.bfloat16, want_lse)
+    if scale is None:
+        scale = d ** -0.5
+    lib = load_library()
+    rc = lib.attn_jvp_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(tq), _ptr(tk), _ptr(tv), _ptr(o), _ptr(to), _ptr(lse),
+                          B, H, Lq, Lk, d, float(scale), _stream_handle(stream))
+    _check(rc, "attn_jvp_fwd")
+    return o, to, lse
+
+
+def attn_jvp_fwd_f32(q, k, v, tq, tk, tv, scale=None, o=None, to=None, lse=None, stream=None, want_lse=True):
+    """fp32-I/O variant through ``attn_jvp_fwd_f32`` (CUDA-core kernel, d <= 256)."""
+    o, to, lse, (B, H, Lq, Lk, d) = _prepare(q, k, v, tq, tk, tv, o, to, lse, torch.float32, want_lse)
+    if scale is None:
+        scale = d ** -0.5
+    lib = load_library()
+    rc = lib.attn_jvp_fwd_f32(_ptr(q), _ptr(k), _ptr(v), _ptr(tq), _ptr(tk), _ptr(tv), _ptr(o), _ptr(to),
+                              _ptr(lse), B, H, Lq, Lk, d, float(scale), _stream_handle(stream))
+    _check(rc, "attn_jvp_fwd_f32")
+    return o, to, lse
+
+
+def attn_jvp(q, k, v, tq, tk, tv, scale=None, **kw):
+    """Dispatch on the input dtype: bf16 -> attn_jvp_fwd, fp32 -> attn_jvp_fwd_f32."""
+    if q.dtype == torch.bfloat16:
+        return attn_jvp_fwd(q, k, v, tq, tk, tv, scale, **kw)
+    if q.dtype == torch.float32:
+        return attn_jvp_fwd_f32(q, k, v, tq, tk, tv, scale, **kw)
+    raise ValueError(f"unsupported dtype {q.dtype}")
+
+
+def check_device_status(stream=None) -> int:
+    """Synchronise ``stream`` and read-and-clear the device status word."""
+    return load_library().attn_jvp_check_device_status(_stream_handle(stream))
+
+
+def set_wait_bound_ns(ns: int) -> None:
+    _check(load_library().attn_jvp_set_wait_bound_ns(int(ns)), "attn_jvp_set_wait_bound_ns")
+
+
+def selftest_wait_timeout(bound_ns: int, stream=None) -> None:
+    _check(load_library().attn_jvp_selftest_wait_timeout(int(bound_ns), _stream_handle(stream)),
+           "attn_jvp_selftest_wait_timeout")
+
+
+def version() -> int:
+    return load_library().attn_jvp_version()

@@ -1,0 +1,270 @@
+// api.cu -- C ABI of the attention + JVP forward library (see
+// include/attn_jvp.h for the contract of every entry point).
+//
+// Host side only: argument checks, tensor-map encoding, launch on the
+// caller's stream, error mapping.  No device memory is allocated here.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "attn_jvp.h"
+#include "jvp_f32.cuh"
+#include "jvp_sm100.cuh"
+
+namespace {
+
+constexpr int kVersion = 100;  // 0.1.0
+constexpr uint64_t kDefaultBoundNs = 2000000000ull;
+constexpr int kMaxDevices = 64;
+
+thread_local int t_last_cuda_error = 0;
+std::atomic<uint64_t> g_bound_ns{kDefaultBoundNs};
+
+// per-device one-time set-up: capability check and kernel attributes
+struct DeviceState {
+    std::once_flag once;
+    int status = AJVP_OK;
+    int cuda_error = 0;
+};
+DeviceState g_dev[kMaxDevices];
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+std::once_flag g_encode_once;
+EncodeTiledFn g_encode = nullptr;
+
+int fail_cuda(cudaError_t e) {
+    t_last_cuda_error = (int)e;
+    return AJVP_ERR_CUDA;
+}
+
+int device_setup(int *dev_out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail_cuda(e);
+    if (dev < 0 || dev >= kMaxDevices) return AJVP_ERR_UNSUPPORTED_DEVICE;
+    DeviceState &st = g_dev[dev];
+    std::call_once(st.once, [&]() {
+        int major = 0, minor = 0;
+        cudaError_t e1 = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+        cudaError_t e2 = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+        if (e1 != cudaSuccess || e2 != cudaSuccess) {
+            st.status = AJVP_ERR_CUDA;
+            st.cuda_error = (int)(e1 != cudaSuccess ? e1 : e2);
+            return;
+        }
+        if (major != 10 || minor != 0) {
+            st.status = AJVP_ERR_UNSUPPORTED_DEVICE;
+            return;
+        }
+        cudaError_t e3 = cudaFuncSetAttribute(ajvp::sm100::attn_jvp_fwd_kernel,
+                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                              (int)ajvp::sm100::SMEM_BYTES);
+        cudaError_t e4 = cudaFuncSetAttribute(ajvp::f32::attn_jvp_fwd_f32_kernel,
+                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                              (int)ajvp::f32::smem_bytes(ajvp::f32::DMAX));
+        if (e3 != cudaSuccess || e4 != cudaSuccess) {
+            st.status = AJVP_ERR_CUDA;
+            st.cuda_error = (int)(e3 != cudaSuccess ? e3 : e4);
+        }
+    });
+    if (st.status == AJVP_ERR_CUDA) t_last_cuda_error = st.cuda_error;
+    *dev_out = dev;
+    return st.status;
+}
+
+int get_encoder() {
+    std::call_once(g_encode_once, []() {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    });
+    return g_encode ? AJVP_OK : AJVP_ERR_CUDA;
+}
+
+// [BH][L][d] bf16 tensor, boxes of 64 columns x box_rows rows, 128-byte swizzle
+int encode_3d(CUtensorMap *m, const void *ptr, int64_t d, int64_t L, int64_t BH, uint32_t box_rows) {
+    cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)L, (cuuint64_t)BH};
+    cuuint64_t strides[2] = {(cuuint64_t)(d * 2), (cuuint64_t)(L * d * 2)};
+    cuuint32_t box[3] = {64u, box_rows, 1u};
+    cuuint32_t estr[3] = {1u, 1u, 1u};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        t_last_cuda_error = (int)r;
+        return AJVP_ERR_CUDA;
+    }
+    return AJVP_OK;
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+// Checks shared by both entry points; sets *noop when there is nothing to do.
+int check_common(const void *q, const void *k, const void *v, const void *tq, const void *tk, const void *tv,
+                 const void *o, const void *to, int64_t B, int64_t H, int64_t Lq, int64_t Lk, int64_t d,
+                 float scale, bool *noop) {
+    *noop = false;
+    if (B < 0 || H < 0 || Lq < 0 || Lk < 1 || d < 1) return AJVP_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return AJVP_ERR_INVALID_ARG;
+    if (B == 0 || H == 0 || Lq == 0) {
+        *noop = true;
+        return AJVP_OK;
+    }
+    if (!q || !k || !v || !tq || !tk || !tv || !o || !to) return AJVP_ERR_INVALID_ARG;
+    if (Lq >= (int64_t(1) << 31) || Lk >= (int64_t(1) << 31) || B * H >= (int64_t(1) << 31))
+        return AJVP_ERR_TOO_LARGE;
+    return AJVP_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int attn_jvp_fwd(const void *q, const void *k, const void *v, const void *tq, const void *tk, const void *tv,
+                 void *o, void *to, float *lse, int64_t B, int64_t H, int64_t Lq, int64_t Lk, int64_t d,
+                 float scale, void *stream) {
+    bool noop = false;
+    int rc = check_common(q, k, v, tq, tk, tv, o, to, B, H, Lq, Lk, d, scale, &noop);
+    if (rc != AJVP_OK || noop) return rc;
+    if (d != ajvp::sm100::HD) return AJVP_ERR_UNSUPPORTED_DIM;
+    const void *ptrs[9] = {q, k, v, tq, tk, tv, o, to, lse};
+    for (int i = 0; i < 9; ++i)
+        if (ptrs[i] && !aligned(ptrs[i], 16)) return AJVP_ERR_MISALIGNED;
+    const int64_t BH = B * H;
+    const int64_t n_qtiles = (Lq + ajvp::sm100::BR - 1) / ajvp::sm100::BR;
+    if (n_qtiles * BH >= (int64_t(1) << 31)) return AJVP_ERR_TOO_LARGE;
+
+    int dev = 0;
+    rc = device_setup(&dev);
+    if (rc != AJVP_OK) return rc;
+    rc = get_encoder();
+    if (rc != AJVP_OK) return rc;
+
+    ajvp::sm100::Params p;
+    std::memset(&p, 0, sizeof(p));
+    if ((rc = encode_3d(&p.tm_q, q, d, Lq, BH, 128)) != AJVP_OK) return rc;
+    if ((rc = encode_3d(&p.tm_tq, tq, d, Lq, BH, 128)) != AJVP_OK) return rc;
+    if ((rc = encode_3d(&p.tm_k, k, d, Lk, BH, 64)) != AJVP_OK) return rc;
+    if ((rc = encode_3d(&p.tm_tk, tk, d, Lk, BH, 64)) != AJVP_OK) return rc;
+    if ((rc = encode_3d(&p.tm_v, v, d, Lk, BH, 64)) != AJVP_OK) return rc;
+    if ((rc = encode_3d(&p.tm_tv, tv, d, Lk, BH, 64)) != AJVP_OK) return rc;
+    if ((rc = encode_3d(&p.tm_o, o, d, Lq, BH, 128)) != AJVP_OK) return rc;
+    if ((rc = encode_3d(&p.tm_to, to, d, Lq, BH, 128)) != AJVP_OK) return rc;
+    p.lse = lse;
+    p.Lq = (int)Lq;
+    p.Lk = (int)Lk;
+    p.n_qtiles = (int)n_qtiles;
+    p.scale = scale;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.bound_ns = g_bound_ns.load();
+
+    ajvp::sm100::attn_jvp_fwd_kernel<<<(unsigned)(n_qtiles * BH), ajvp::sm100::NTHREADS, ajvp::sm100::SMEM_BYTES,
+                                       (cudaStream_t)stream>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail_cuda(e);
+    return AJVP_OK;
+}
+
+int attn_jvp_fwd_f32(const float *q, const float *k, const float *v, const float *tq, const float *tk,
+                     const float *tv, float *o, float *to, float *lse, int64_t B, int64_t H, int64_t Lq, int64_t Lk,
+                     int64_t d, float scale, void *stream) {
+    bool noop = false;
+    int rc = check_common(q, k, v, tq, tk, tv, o, to, B, H, Lq, Lk, d, scale, &noop);
+    if (rc != AJVP_OK || noop) return rc;
+    if (d > ajvp::f32::DMAX) return AJVP_ERR_UNSUPPORTED_DIM;
+    const void *ptrs[9] = {q, k, v, tq, tk, tv, o, to, lse};
+    for (int i = 0; i < 9; ++i)
+        if (ptrs[i] && !aligned(ptrs[i], 4)) return AJVP_ERR_MISALIGNED;
+    const int64_t BH = B * H;
+    const int64_t n_qtiles = (Lq + ajvp::f32::BR - 1) / ajvp::f32::BR;
+    if (n_qtiles * BH >= (int64_t(1) << 31)) return AJVP_ERR_TOO_LARGE;
+
+    int dev = 0;
+    rc = device_setup(&dev);
+    if (rc != AJVP_OK) return rc;
+    ajvp::f32::attn_jvp_fwd_f32_kernel<<<(unsigned)(n_qtiles * BH), ajvp::f32::WARPS * 32,
+                                         ajvp::f32::smem_bytes((int)d), (cudaStream_t)stream>>>(
+        q, k, v, tq, tk, tv, o, to, lse, (int)Lq, (int)Lk, (int)d, (int)n_qtiles, scale);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail_cuda(e);
+    return AJVP_OK;
+}
+
+const char *attn_jvp_strerror(int status) {
+    switch (status) {
+        case AJVP_OK: return "success";
+        case AJVP_ERR_INVALID_ARG: return "invalid argument (null pointer, negative size, Lk < 1 or non-finite scale)";
+        case AJVP_ERR_UNSUPPORTED_DIM: return "unsupported head dimension for this entry point";
+        case AJVP_ERR_MISALIGNED: return "pointer not aligned as the entry point requires";
+        case AJVP_ERR_UNSUPPORTED_DEVICE: return "current device is not compute capability 10.0 (B200)";
+        case AJVP_ERR_TIMEOUT: return "a kernel wait ran past its bound";
+        case AJVP_ERR_CUDA: return "CUDA runtime or driver error";
+        case AJVP_ERR_TOO_LARGE: return "a size exceeds the supported maximum";
+        default: return "unknown status";
+    }
+}
+
+int attn_jvp_last_cuda_error(void) { return t_last_cuda_error; }
+
+int attn_jvp_check_device_status(void *stream) {
+    cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return fail_cuda(e);
+    int word = 0;
+    e = cudaMemcpyFromSymbol(&word, ajvp::g_status_word, sizeof(int));
+    if (e != cudaSuccess) return fail_cuda(e);
+    if (word != 0) {
+        const int zero = 0;
+        e = cudaMemcpyToSymbol(ajvp::g_status_word, &zero, sizeof(int));
+        if (e != cudaSuccess) return fail_cuda(e);
+        return AJVP_ERR_TIMEOUT;
+    }
+    return AJVP_OK;
+}
+
+int attn_jvp_set_wait_bound_ns(uint64_t ns) {
+    g_bound_ns.store(ns == 0 ? kDefaultBoundNs : ns);
+    return AJVP_OK;
+}
+
+int attn_jvp_version(void) { return kVersion; }
+
+}  // extern "C"
+
+// ------------------------------------------------------- failure self test
+namespace {
+__global__ void selftest_wait_kernel(unsigned long long bound_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    const uint32_t b = ajvp::smem_u32(&bar);
+    if (threadIdx.x == 0) {
+        ajvp::mbar_init(b, 1);
+        abort_flag = 0;
+        ajvp::fence_barrier_init();
+    }
+    __syncwarp();
+    // nothing ever arrives on `bar`: the bounded wait must give up
+    bool ok = ajvp::mbar_wait(b, 0, reinterpret_cast<volatile int *>(&abort_flag), bound_ns);
+    ok = __all_sync(0xffffffffu, ok);
+    (void)ok;
+}
+}  // namespace
+
+extern "C" int attn_jvp_selftest_wait_timeout(uint64_t bound_ns, void *stream) {
+    int dev = 0;
+    int rc = device_setup(&dev);
+    if (rc != AJVP_OK) return rc;
+    if (bound_ns == 0 || bound_ns > 10000000000ull) return AJVP_ERR_INVALID_ARG;
+    selftest_wait_kernel<<<1, 32, 0, (cudaStream_t)stream>>>((unsigned long long)bound_ns);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail_cuda(e);
+    return AJVP_OK;
+}

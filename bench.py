@@ -1,0 +1,424 @@
+"""Benchmark of the fused attention + JVP forward pass on B200.
+
+One step = one call of the C ABI's ``attn_jvp_fwd`` on the whole workload
+(the 32760-token video self-attention JVP by default: B=1, H=12,
+Lq=Lk=32760, d=128, bf16 I/O).  Metric: attention+JVP TFLOP/s, counting
+12 * Lq * Lk * d FLOPs per head, and its fraction of the measured B200 dense
+bf16 tensor peak.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+For N > 1 launch one process per GPU with torch.distributed.run; every rank
+runs its own replica of the workload (independent problems, no data-path
+collective: weak scaling) and rank 0 prints one JSON line with the job-wide
+aggregate over the max-over-ranks device time.
+
+``--impl reference`` times the fp64 CPU oracle (plain loops, OpenMP) on a
+bounded sample of the same workload on this machine's host cores: the only
+other implementation there is of this computation.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from attention_forward_mode_b200.workloads import BENCH_WORKLOAD, WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "attention+JVP TFLOP/s (12·Lq·Lk·d/head) and % of B200 BF16 tensor peak"
+FALLBACK_BF16_TFLOPS = 1590.0
+KERNEL_SOURCES = ["attention_forward_mode_b200/csrc/jvp_sm100.cuh", "attention_forward_mode_b200/csrc/ptx_sm100.cuh"]
+TRAFFIC_FILE = "profiles/attn_jvp_fwd_kernel.video_selfattn_b1h12_l32760.md"
+L2_BYTES = 126 * 1024 * 1024
+
+
+# ------------------------------------------------------------------ helpers
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def init_dist(world: int, local: int, backend: str = "nccl", timeout_s: int = 300):
+    import datetime
+
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        kw = {"device_id": torch.device("cuda", local)} if backend == "nccl" else {}
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s), **kw)
+    return dist
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Max of a per-rank float over all ranks (identity for one rank)."""
+    if world <= 1:
+        return value
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_value(flops_per_rank_step: float, steps: int, world: int, max_seconds: float) -> float:
+    """Whole-job TFLOP/s: every rank's work over the slowest rank's time."""
+    return flops_per_rank_step * steps * world / max_seconds / 1e12
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            j = json.load(f)
+        return float(j["bf16_tflops"]), float(j.get("bf16_tflops_sustained", j["bf16_tflops"])), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic():
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the kernel source as it stands (else None)."""
+    path = os.path.join(ROOT, TRAFFIC_FILE)
+    if not os.path.exists(path):
+        return None
+    fields = {}
+    for line in open(path):
+        if ":" in line and line.strip().startswith(("traffic_bytes_per_launch", "kernel_source_sha")):
+            k, v = line.split(":", 1)
+            fields[k.strip()] = v.strip().strip("`")
+    if fields.get("kernel_source_sha") != kernel_source_sha():
+        return None
+    try:
+        return float(fields["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling while the timed region runs."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.gpu), "-lms", "100"], stdout=self.out,
+                                         stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        if getattr(self, "out", None):
+            self.out.close()
+
+    def summary(self):
+        rows = []
+        try:
+            for line in open(self.path):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9 and parts[1].replace(".", "").isdigit():
+                    rows.append(parts)
+        except Exception:
+            pass
+        finally:
+            try:
+                os.unlink(self.path)
+            except Exception:
+                pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["clock sampling unavailable"], "samples": 0}
+        sm = [float(r[1]) for r in rows]
+        mx = max(float(r[2]) for r in rows)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower().startswith("active")})
+        loaded = [s for s in sm if s > 0.5 * mx] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": reasons, "samples": len(rows),
+                "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit()) if rows else None}
+
+
+# ------------------------------------------------------------- CPU oracle
+def oracle_sample(w, inputs_cpu_head, seconds: float, seed: int = 0):
+    """Time the fp64 oracle on query rows of one head (all Lk keys) for about
+    ``seconds``; returns (TFLOP/s-equivalent, rows, elapsed, threads)."""
+    import oracle
+    q, k, v, tq, tk, tv = inputs_cpu_head
+    g = torch.Generator().manual_seed(seed)
+    # calibrate on two rows per oracle thread (rows are spread over threads)
+    probe = max(4, 2 * oracle.num_threads())
+    idx = torch.randperm(q.shape[0], generator=g)[:probe]
+    t0 = time.perf_counter()
+    oracle.attn_jvp(q[idx][None], k[None], v[None], tq[idx][None], tk[None], tv[None], w.scale)
+    per_row = max((time.perf_counter() - t0) / probe, 1e-6)
+    rows = int(max(1, min(q.shape[0], seconds / per_row)))
+    idx = torch.randperm(q.shape[0], generator=g)[:rows]
+    qs, tqs = q[idx][None], tq[idx][None]
+    t0 = time.perf_counter()
+    oracle.attn_jvp(qs, k[None], v[None], tqs, tk[None], tv[None], w.scale)
+    el = time.perf_counter() - t0
+    flops = 12.0 * rows * w.Lk * w.d
+    return flops / el / 1e12, rows, el, oracle.num_threads()
+
+
+def head0_cpu(inp):
+    return tuple(inp[n][0, 0].detach().cpu() for n in ("q", "k", "v", "tq", "tk", "tv"))
+
+
+# ------------------------------------------------------------------ arms
+def run_reference(args, w):
+    rank, world, local = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+    oracle.build()
+    inp = make_inputs(w, seed=0, device="cpu")
+    head = head0_cpu(inp)
+    del inp
+    total_steps = args.steps + args.warmup
+    per_step = max(0.5, args.reference_seconds / max(1, total_steps))
+    # bounded sample per step: rows of head 0 sized to ~per_step seconds
+    for _ in range(args.warmup):
+        oracle_sample(w, head, per_step)
+    vals, rows_total, el_total = [], 0, 0.0
+    threads = oracle.num_threads()
+    for s in range(args.steps):
+        v, rows, el, threads = oracle_sample(w, head, per_step, seed=s + 1)
+        vals.append(v)
+        rows_total += rows
+        el_total += el
+    value = 12.0 * rows_total * w.Lk * w.d / el_total / 1e12
+    sample = (f"{rows_total} query rows of head 0 over {args.steps} steps (each all {w.Lk} keys), "
+              f"{el_total:.1f} s of fp64 oracle time")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * el_total / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(w, world),
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w, world):
+    in_bytes = w.B * w.H * (2 * w.Lq + 4 * w.Lk) * w.d * w.elem_size
+    return {"workload": w.name, "B": w.B, "H": w.H, "Lq": w.Lq, "Lk": w.Lk, "d": w.d, "scale": w.scale,
+            "io": w.dtype, "parallelism": "single GPU" if world == 1 else f"{world} independent replicas",
+            "l2": (f"inputs larger than L2 ({in_bytes / 1e6:.0f} MB vs {L2_BYTES / 1e6:.0f} MB), no flush"
+                   if in_bytes > L2_BYTES else "L2 flushed between steps")}
+
+
+def run_ours(args, w):
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = init_dist(world, local)
+    import attention_forward_mode_b200 as ajvp
+    ajvp.load_library()
+
+    inp = make_inputs(w, seed=rank, device=dev)
+    o = torch.empty_like(inp["q"])
+    to = torch.empty_like(inp["q"])
+    lse = torch.empty((w.B, w.H, w.Lq), device=dev, dtype=torch.float32)
+    stream = torch.cuda.current_stream(dev)
+    in_bytes = sum(t.numel() * t.element_size() for t in inp.values())
+    flush = None
+    if in_bytes <= L2_BYTES:
+        flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def step():
+        if flush is not None:
+            flush.zero_()
+        ajvp.attn_jvp_fwd(inp["q"], inp["k"], inp["v"], inp["tq"], inp["tk"], inp["tv"], w.scale,
+                          o=o, to=to, lse=lse, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if ajvp.check_device_status(stream) != ajvp.AJVP_OK:
+        raise RuntimeError("kernel wait bound exceeded during warm-up")
+
+    # ---- device-timed region: K launches, events on the launching stream
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clocks:
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    ms = ev0.elapsed_time(ev1)
+    ms_max = max_over_ranks(ms, world, dev)
+    status = ajvp.check_device_status(stream)
+    if status != ajvp.AJVP_OK:
+        raise RuntimeError(f"kernel reported {ajvp.strerror(status)}")
+    value = aggregate_value(w.flops, args.steps, world, ms_max / 1e3)
+    per_launch_s = ms / 1e3 / args.steps
+    achieved = w.flops / per_launch_s / 1e12
+
+    # ---- end to end: pinned host inputs -> device -> C ABI -> host, every step
+    host_in = {n: t.detach().to("cpu").pin_memory() for n, t in inp.items()}
+    host_o = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    host_to = torch.empty(to.shape, dtype=to.dtype).pin_memory()
+    host_lse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = host_o.numel() * 2 + host_to.numel() * 2 + host_lse.numel() * 4
+
+    def e2e_step():
+        for n in inp:
+            inp[n].copy_(host_in[n], non_blocking=True)
+        ajvp.attn_jvp_fwd(inp["q"], inp["k"], inp["v"], inp["tq"], inp["tk"], inp["tv"], w.scale,
+                          o=o, to=to, lse=lse, stream=stream)
+        host_o.copy_(o, non_blocking=True)
+        host_to.copy_(to, non_blocking=True)
+        host_lse.copy_(lse, non_blocking=True)
+
+    e2e_steps = max(1, min(args.steps, args.e2e_steps))
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    ev2, ev3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev2.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    ev3.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(ev2.elapsed_time(ev3), world, dev)
+    e2e_value = aggregate_value(w.flops, e2e_steps, world, e2e_ms / 1e3)
+
+    line = None
+    if rank == 0:
+        burst, sustained, src = measured_peaks()
+        clk = clocks.summary()
+        line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": workload_config(w, world),
+                "pct_of_bf16_peak": 100.0 * value / world / burst,
+                "roofline": {"bound": "tensor", "achieved": achieved, "peak": burst, "unit": "TFLOP/s",
+                             "frac": achieved / burst, "traffic": committed_traffic(),
+                             "peak_source": f"{src} bf16 dense (burst) from MEASURED_PEAKS.json"
+                             if src == "measured" else "fallback 1.59 PFLOP/s",
+                             "kernel": "attn_jvp_fwd_kernel", "algorithmic_flops_per_launch": w.flops,
+                             "algorithmic_bytes_per_launch": w.io_bytes},
+                "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                        "d2h_bytes_per_step": d2h, "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps},
+                "gpu_launches": args.steps,
+                "clocks": clk}
+        # CPU oracle next to the kernel: rank 0 at N = 1 only
+        if world == 1 and not args.no_cpu_baseline:
+            v, rows, el, threads = oracle_sample(w, head0_cpu(inp), args.cpu_seconds)
+            line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                                    "sample": f"{rows} random query rows of head 0 against all {w.Lk} keys "
+                                              f"({el:.1f} s, fp64, OpenMP)"}
+        if world == 1 and not args.no_eager:
+            line["eager_torch_jvp"] = eager_reference(w, inp)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def eager_reference(w, inp, chunk: int = 8192):
+    """torch.func.jvp of softmax(s q k^T) v in the I/O dtype on the GPU,
+    looped over heads and 8192-row query chunks (what fits in memory);
+    one untimed pass, then one timed pass."""
+    def attn(q, k, v):
+        return torch.softmax((q @ k.transpose(-1, -2)) * w.scale, dim=-1) @ v
+
+    def one_pass():
+        for b in range(w.B):
+            for h in range(w.H):
+                k, v, tk, tv = (inp[n][b, h] for n in ("k", "v", "tk", "tv"))
+                for r0 in range(0, w.Lq, chunk):
+                    q = inp["q"][b, h, r0:r0 + chunk]
+                    tq = inp["tq"][b, h, r0:r0 + chunk]
+                    torch.func.jvp(attn, (q, k, v), (tq, tk, tv))
+    try:
+        one_pass()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        one_pass()
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1)
+        return {"value": w.flops / (ms / 1e3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms,
+                "how": f"torch.func.jvp, {w.dtype}, per head, {chunk}-row query chunks, summed"}
+    except Exception as exc:  # e.g. out of memory on a shared GPU
+        torch.cuda.empty_cache()
+        return {"value": None, "unit": "TFLOP/s", "error": f"{type(exc).__name__}: {exc}"[:200]}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=BENCH_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--reference-seconds", type=float, default=90.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-eager", action="store_true")
+    ap.add_argument("--heads", type=int, default=None,
+                    help="override H (small profiling captures); the JSON config shows the H used")
+    args = ap.parse_args(argv)
+    args.warmup = max(3, args.warmup)  # timing rule: at least 3 untimed warm-up steps
+    w = WORKLOADS[args.workload]
+    if args.heads is not None:
+        import dataclasses
+        w = dataclasses.replace(w, H=args.heads, name=f"{w.name}_h{args.heads}")
+    if w.dtype != "bf16" and args.impl == "ours":
+        ap.error("the benchmark times the bf16 tensor-core path")
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ours(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -46,6 +46,12 @@
 
 #include <stdint.h>
 
+#if defined(__GNUC__)
+#define AJVP_API __attribute__((visibility("default")))
+#else
+#define AJVP_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -77,7 +83,7 @@ typedef enum {
  * The current device must be compute capability 10.0 (B200).
  * Returns AJVP_OK once the kernel is enqueued.
  */
-int attn_jvp_fwd(const void *q, const void *k, const void *v,
+AJVP_API int attn_jvp_fwd(const void *q, const void *k, const void *v,
                  const void *tq, const void *tk, const void *tv,
                  void *o, void *to, float *lse,
                  int64_t B, int64_t H, int64_t Lq, int64_t Lk, int64_t d,
@@ -89,31 +95,31 @@ int attn_jvp_fwd(const void *q, const void *k, const void *v,
  * attn_jvp_fwd, with float tensors.  Supported: 1 <= d <= 256; pointers
  * 4-byte aligned.  Any compute capability 10.0 device.
  */
-int attn_jvp_fwd_f32(const float *q, const float *k, const float *v,
+AJVP_API int attn_jvp_fwd_f32(const float *q, const float *k, const float *v,
                      const float *tq, const float *tk, const float *tv,
                      float *o, float *to, float *lse,
                      int64_t B, int64_t H, int64_t Lq, int64_t Lk, int64_t d,
                      float scale, void *stream);
 
 /* Static, human-readable description of an ajvp_status value. */
-const char *attn_jvp_strerror(int status);
+AJVP_API const char *attn_jvp_strerror(int status);
 
 /* cudaError_t behind the calling thread's last AJVP_ERR_CUDA (0 if none). */
-int attn_jvp_last_cuda_error(void);
+AJVP_API int attn_jvp_last_cuda_error(void);
 
 /*
  * Synchronise `stream`, then read and clear the device status word of the
  * current device.  Returns AJVP_OK, AJVP_ERR_TIMEOUT (some kernel wait ran
  * past its bound since the last check) or AJVP_ERR_CUDA.
  */
-int attn_jvp_check_device_status(void *stream);
+AJVP_API int attn_jvp_check_device_status(void *stream);
 
 /*
  * Bound, in nanoseconds, on any single pipeline wait inside the kernels
  * (default 2e9, i.e. 2 s; 0 restores the default).  Applies to launches made
  * after the call, process-wide.
  */
-int attn_jvp_set_wait_bound_ns(uint64_t ns);
+AJVP_API int attn_jvp_set_wait_bound_ns(uint64_t ns);
 
 /*
  * Failure-detection self test: enqueue a one-warp kernel that waits, through
@@ -122,10 +128,10 @@ int attn_jvp_set_wait_bound_ns(uint64_t ns);
  * records AJVP_ERR_TIMEOUT in the device status word and returns; the GPU
  * context stays usable.  Returns AJVP_OK once enqueued.
  */
-int attn_jvp_selftest_wait_timeout(uint64_t bound_ns, void *stream);
+AJVP_API int attn_jvp_selftest_wait_timeout(uint64_t bound_ns, void *stream);
 
 /* Library version, major * 10000 + minor * 100 + patch. */
-int attn_jvp_version(void);
+AJVP_API int attn_jvp_version(void);
 
 #ifdef __cplusplus
 }

@@ -1,0 +1,93 @@
+"""C ABI checks that need no GPU: the library loads, exports every symbol
+the header declares, and rejects bad arguments on the host before touching
+CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from attention_forward_mode_b200 import _binding as B
+from attention_forward_mode_b200 import build as build_mod
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_mod.build()
+    return B.load_library()
+
+
+def header_functions():
+    text = open(os.path.join(ROOT, "include", "attn_jvp.h")).read()
+    return sorted(set(re.findall(r"AJVP_API\s+[\w\s\*]*?\b(attn_jvp_\w+)\s*\(", text)))
+
+
+def test_header_matches_binding_list():
+    assert header_functions() == sorted(B.EXPORTED)
+
+
+def test_every_header_symbol_exported(lib):
+    raw = ctypes.CDLL(B.LIB_PATH)
+    for name in header_functions():
+        assert hasattr(raw, name), name
+
+
+def test_version_and_strerror(lib):
+    assert lib.attn_jvp_version() == 100
+    for code in range(-7, 1):
+        assert len(lib.attn_jvp_strerror(code)) > 5
+    assert b"unknown" in lib.attn_jvp_strerror(-99)
+
+
+def _call(lib, fn="attn_jvp_fwd", ptr=16, B_=1, H=1, Lq=8, Lk=8, d=128, scale=0.1, lse=None):
+    f = getattr(lib, fn)
+    p = ctypes.c_void_p(ptr) if ptr is not None else None
+    return f(p, p, p, p, p, p, p, p, lse, B_, H, Lq, Lk, d, scale, None)
+
+
+@pytest.mark.parametrize("fn", ["attn_jvp_fwd", "attn_jvp_fwd_f32"])
+def test_host_side_rejections(lib, fn):
+    # none of these reach a CUDA call: checked on the host first
+    assert _call(lib, fn, Lk=0) == B.AJVP_ERR_INVALID_ARG
+    assert _call(lib, fn, Lq=-1) == B.AJVP_ERR_INVALID_ARG
+    assert _call(lib, fn, B_=-2) == B.AJVP_ERR_INVALID_ARG
+    assert _call(lib, fn, d=0) == B.AJVP_ERR_INVALID_ARG
+    assert _call(lib, fn, scale=float("nan")) == B.AJVP_ERR_INVALID_ARG
+    assert _call(lib, fn, scale=float("inf")) == B.AJVP_ERR_INVALID_ARG
+    assert _call(lib, fn, ptr=None) == B.AJVP_ERR_INVALID_ARG
+    assert _call(lib, fn, Lq=1 << 31) == B.AJVP_ERR_TOO_LARGE
+    assert _call(lib, fn, Lk=1 << 31) == B.AJVP_ERR_TOO_LARGE
+    # empty work is a successful no-op (null pointers allowed then)
+    assert _call(lib, fn, ptr=None, Lq=0) == B.AJVP_OK
+    assert _call(lib, fn, ptr=None, B_=0) == B.AJVP_OK
+    assert _call(lib, fn, ptr=None, H=0) == B.AJVP_OK
+
+
+def test_bf16_dim_and_alignment_rules(lib):
+    assert _call(lib, d=64) == B.AJVP_ERR_UNSUPPORTED_DIM
+    assert _call(lib, d=256) == B.AJVP_ERR_UNSUPPORTED_DIM
+    assert _call(lib, ptr=24) == B.AJVP_ERR_MISALIGNED
+    assert _call(lib, lse=ctypes.c_void_p(20)) == B.AJVP_ERR_MISALIGNED
+
+
+def test_f32_dim_and_alignment_rules(lib):
+    assert _call(lib, "attn_jvp_fwd_f32", d=257) == B.AJVP_ERR_UNSUPPORTED_DIM
+    assert _call(lib, "attn_jvp_fwd_f32", ptr=18) == B.AJVP_ERR_MISALIGNED
+
+
+def test_no_gpu_reports_cuda_or_device_error(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    # valid arguments: the first CUDA call fails on a machine without a GPU
+    rc = _call(lib, ptr=1 << 20)
+    assert rc in (B.AJVP_ERR_CUDA, B.AJVP_ERR_UNSUPPORTED_DEVICE)
+
+
+def test_binding_raises_without_cuda_tensors(lib):
+    import torch
+    x = torch.zeros(1, 1, 4, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        B.attn_jvp_fwd(x, x, x, x, x, x)
