@@ -65,9 +65,10 @@ enum : int {
     B_VT_EMPTY = 7,  // +stage
     B_SD_FULL = 9,   // +buffer
     B_P_FULL = 11,   // +buffer
-    B_PV_DONE = 13,
-    B_MMA_DRAIN = 14,
-    N_BARS = 15
+    B_PV_DONE = 13,   // one phase per P.V pair (rescale waits on the previous tile's)
+    B_O_FULL = 14,    // single use: every MMA of the CTA has completed
+    B_MMA_DRAIN = 15,
+    N_BARS = 16
 };
 constexpr uint32_t OFF_TMEM_SLOT = 8 * N_BARS;   // u32
 constexpr uint32_t OFF_ABORT = OFF_TMEM_SLOT + 4;  // int
@@ -114,6 +115,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
             mbar_init(BAR(B_P_FULL + s), 128);
         }
         mbar_init(BAR(B_PV_DONE), 1);
+        mbar_init(BAR(B_O_FULL), 1);
         mbar_init(BAR(B_MMA_DRAIN), 1);
         *abort_flag = 0;
         fence_barrier_init();
@@ -250,6 +252,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                 if (ok) ok = issue_pv(j - 1);
             }
             if (ok) ok = issue_pv(nk - 1);
+            // O and T are final once everything issued so far completes.  (A parity wait
+            // on B_PV_DONE for the last tile would be ambiguous: that barrier may still be
+            // two phases behind when the softmax warps finish their last tile.)
+            if (ok) mma_commit(BAR(B_O_FULL));
             // every MMA issued must finish before tensor memory is released
             mma_commit(BAR(B_MMA_DRAIN));
             mbar_wait_drain(BAR(B_MMA_DRAIN), 0, bound);
@@ -291,14 +297,24 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                 for (int i = 1; i < BC; ++i)
                     if (i >= valid) x[i] = x[0];  // neutral for the max; p forced to 0 below
             }
-            float mx = x[0];
+            // row max (min for a negative scale) over 8 independent chains
+            float m8[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) m8[k] = x[k];
             if (c >= 0.f) {
 #pragma unroll
-                for (int i = 1; i < BC; ++i) mx = fmaxf(mx, x[i]);
+                for (int i = 8; i < BC; ++i) m8[i & 7] = fmaxf(m8[i & 7], x[i]);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) m8[k] = fmaxf(m8[k], m8[k + 4]);
+                m8[0] = fmaxf(fmaxf(m8[0], m8[2]), fmaxf(m8[1], m8[3]));
             } else {
 #pragma unroll
-                for (int i = 1; i < BC; ++i) mx = fminf(mx, x[i]);
+                for (int i = 8; i < BC; ++i) m8[i & 7] = fminf(m8[i & 7], x[i]);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) m8[k] = fminf(m8[k], m8[k + 4]);
+                m8[0] = fminf(fminf(m8[0], m8[2]), fminf(m8[1], m8[3]));
             }
+            const float mx = m8[0];
             const float m_tile = mx * c;
             if (j == 0) {
                 m_ref = m_tile;
@@ -330,47 +346,50 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                 }
             }
             const float neg_m = -m_ref;
-            float lsum = 0.f;
 #pragma unroll
-            for (int i = 0; i < BC; ++i) {
-                x[i] = ex2_approx(fmaf(x[i], c, neg_m));
-            }
+            for (int i = 0; i < BC; ++i) x[i] = ex2_approx(fmaf(x[i], c, neg_m));
             if (valid < BC) {
 #pragma unroll
                 for (int i = 1; i < BC; ++i)
                     if (i >= valid) x[i] = 0.f;
             }
+            // dS' is loaded while P is packed and stored (different columns)
+            uint32_t d0[32], d1[32];
+            tmem_ld32(t_s + 64, d0);
+            tmem_ld32(t_s + 96, d1);
+            float lsum;
             {
+                float ls[4] = {0.f, 0.f, 0.f, 0.f};
                 uint32_t pk[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    lsum += x[2 * i] + x[2 * i + 1];
+                    ls[i & 3] += x[2 * i] + x[2 * i + 1];
                     pk[i] = pack_bf16x2(x[2 * i], x[2 * i + 1]);
                 }
                 tmem_st32(t_s, pk);  // P over S's first 32 columns
+                lsum = (ls[0] + ls[1]) + (ls[2] + ls[3]);
             }
-            float gsum = 0.f;
+            float gsum;
             {
-                uint32_t d0[32], d1[32];
-                tmem_ld32(t_s + 64, d0);
-                tmem_ld32(t_s + 96, d1);
                 tmem_wait_ld();
+                float gs[4] = {0.f, 0.f, 0.f, 0.f};
                 uint32_t pd[32];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const float t0 = x[2 * i] * __uint_as_float(d0[2 * i]) * s_lin;
                     const float t1 = x[2 * i + 1] * __uint_as_float(d0[2 * i + 1]) * s_lin;
-                    gsum += t0 + t1;
+                    gs[i & 3] += t0 + t1;
                     pd[i] = pack_bf16x2(t0, t1);
                 }
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const float t0 = x[32 + 2 * i] * __uint_as_float(d1[2 * i]) * s_lin;
                     const float t1 = x[32 + 2 * i + 1] * __uint_as_float(d1[2 * i + 1]) * s_lin;
-                    gsum += t0 + t1;
+                    gs[i & 3] += t0 + t1;
                     pd[16 + i] = pack_bf16x2(t0, t1);
                 }
                 tmem_st32(t_s + 64, pd);  // P.*s dS' over dS''s first 32 columns
+                gsum = (gs[0] + gs[1]) + (gs[2] + gs[3]);
             }
             l += lsum;
             g += gsum;
@@ -380,7 +399,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
         }
 
         if (ok) {
-            ok = mbar_wait(BAR(B_PV_DONE), (nk - 1) & 1, abort_flag, bound);
+            ok = mbar_wait(BAR(B_O_FULL), 0, abort_flag, bound);
             ok = __all_sync(0xffffffffu, ok);
         }
         if (ok) {
