@@ -1,6 +1,6 @@
 // jvp_sm100.cuh -- fused attention + Jacobian-vector product, bf16 I/O,
-// fp32 accumulation, for sm_100a (B200): TMA tile loads through an mbarrier
-// pipeline, tcgen05 MMAs accumulating in tensor memory, warp-specialised
+// fp32 accumulation, for sm_100a (B200): TMA tile loads through mbarrier
+// pipelines, tcgen05 MMAs accumulating in tensor memory, warp-specialised
 // roles.
 //
 // The method (rCM, anthology record LIT-783, §3.2 / App. C): one tiled pass
@@ -16,23 +16,31 @@
 // (the centred JVP expression, rearranged with rowsum(P) = 1).  P and dS are
 // never written to global memory.
 //
-// CTA = 128 query rows of one (batch, head); 256 threads:
-//   warp 0      TMA producer (one lane): Q, tQ once; K|tK and V|tV tiles
-//               through two 2-stage rings.
-//   warp 1      MMA issuer (one lane), per 64-key tile j:
-//                 [S_j | dS'_j]  = Q  [K_j | tK_j]^T      (N = 128)
-//                        dS'_j  += tQ K_j^T               (N = 64)
-//                 [O | T]       += P_j  [V_j | tV_j]      (N = 256, A in TMEM)
-//                        T      += PdS_j V_j              (N = 128, A in TMEM)
-//   warp 2      tensor-memory allocation / release.
-//   warps 4-7   softmax + JVP statistics (one thread per query row, rows are
-//               TMEM lanes), lazy rescale of O and T, epilogue.
+// One CTA owns 128 query rows of one (batch, head); 384 threads:
+//   warp 0       TMA producer (one lane): Q, tQ once; K|tK and V|tV tiles
+//                through two 2-stage rings.
+//   warp 1       MMA issuer (one lane), per 64-key tile j:
+//                  [S_j | dS'_j]  = Q  [K_j | tK_j]^T      (N = 128)
+//                         dS'_j  += tQ K_j^T               (N = 64)
+//                  [O | T]       += P_j  [V_j | tV_j]      (N = 256, A in TMEM)
+//                         T      += PdS_j V_j              (N = 128, A in TMEM)
+//   warp 2       tensor-memory allocation / release.
+//   warps 4-7    softmax group 0: keys 0-31 of every tile,
+//   warps 8-11   softmax group 1: keys 32-63 of every tile.
+//                One thread per (query row, group); rows are TMEM lanes.  The
+//                two groups exchange their partial row maxima through shared
+//                memory once per tile, so both keep the same reference max
+//                and partial sums l, g that add up at the end.  Each group
+//                rescales half of the accumulators (group 0 O, group 1 T) and
+//                writes half of the outputs.
 //
 // Tensor memory (512 columns x 128 lanes of fp32):
 //   [0,128) O_acc   [128,256) T_acc   [256,384) S/dS' buffer 0
 //   [384,512) S/dS' buffer 1    (S at +0, dS' at +64 inside a buffer)
-// bf16 P_j is written over S_j's first 32 columns and bf16 (P.*s dS')_j over
-// dS'_j's first 32 columns; they are the A operands of the second MMA pair.
+// bf16 P is written over S and bf16 P.*s dS' over dS', each group inside its
+// own 32 columns (group 0 at +0, group 1 at +32), so neither group overwrites
+// values the other still has to read.  They are the A operands of the
+// second MMA pair: 16 keys = 8 TMEM columns per K-step.
 #pragma once
 
 #include "ptx_sm100.cuh"
@@ -40,48 +48,60 @@
 namespace ajvp {
 namespace sm100 {
 
-constexpr int BR = 128;       // query rows per CTA
-constexpr int BC = 64;        // keys per tile
-constexpr int HD = 128;       // head dimension
-constexpr int NTHREADS = 256;
+constexpr int BR = 128;  // query rows per CTA
+constexpr int BC = 64;   // keys per tile
+constexpr int HD = 128;  // head dimension
+constexpr int NTHREADS = 384;
+constexpr int SOFTMAX_THREADS = 256;
+constexpr int STAGES = 2;
 
-// shared memory map (offsets from a 1024-byte aligned base)
-constexpr uint32_t CHUNK_Q = 128 * 128;            // one 64-column chunk of a 128-row tile (bytes)
-constexpr uint32_t CHUNK_K = 64 * 128;             // one 64-column chunk of a 64-row tile
-constexpr uint32_t SM_Q = 0;                       // Q  [2 chunks][128 rows][128 B]
-constexpr uint32_t SM_TQ = SM_Q + 2 * CHUNK_Q;     // tQ
-constexpr uint32_t STAGE_BYTES = 4 * CHUNK_K;      // 32 KB
-constexpr uint32_t SM_KT = SM_TQ + 2 * CHUNK_Q;    // K|tK ring, 2 stages
-constexpr uint32_t SM_VT = SM_KT + 2 * STAGE_BYTES;  // V|tV ring, 2 stages
-constexpr uint32_t SM_BAR = SM_VT + 2 * STAGE_BYTES;
-constexpr uint32_t SMEM_BYTES = SM_BAR + 256 + 1024;  // + alignment slack
+constexpr uint32_t CHUNK_Q = 128 * 128;  // one 64-column chunk of a 128-row tile (bytes)
+constexpr uint32_t CHUNK_K = 64 * 128;   // one 64-column chunk of a 64-row tile
+constexpr uint32_t SM_Q = 0;             // Q  [2 chunks][128 rows][128 B]
+constexpr uint32_t SM_TQ = SM_Q + 2 * CHUNK_Q;
+constexpr uint32_t KT_STAGE = 4 * CHUNK_K;  // [K c0 | tK c0 | K c1 | tK c1]
+constexpr uint32_t VT_STAGE = 4 * CHUNK_K;  // [V c0 | V c1 | tV c0 | tV c1]
+constexpr uint32_t KT_CHUNK = 2 * CHUNK_K;  // stride between 64-column chunks of the K side
+constexpr uint32_t SM_KT = SM_TQ + 2 * CHUNK_Q;
+constexpr uint32_t SM_VT = SM_KT + STAGES * KT_STAGE;
+constexpr uint32_t SM_BAR = SM_VT + STAGES * VT_STAGE;
+constexpr uint32_t SM_XCH = SM_BAR + 256;  // fp32 [2 buffers][2 groups][128 rows] partial maxima,
+                                           // then [l, g][2 groups][128 rows] final sums
+constexpr uint32_t XCH_FLOATS = 2 * 2 * 128 + 2 * 2 * 128;
+constexpr uint32_t SMEM_BYTES = SM_XCH + 4 * XCH_FLOATS + 1024;  // + alignment slack
 
-// barrier slots (8 bytes each) inside SM_BAR
+// barrier slots (8 bytes each).  Two MMA commits per key tile:
+//   B_SD_FULL[j % 2]  S_j / dS'_j complete: the softmax may read them, and
+//                     K-side stage j % 2 (same index) may be refilled
+//   B_VT_EMPTY[j % 2] P_j.V_j etc. complete: V-side stage j % 2 may be
+//                     refilled, and O / T may be rescaled before P_{j+1}.V
 enum : int {
     B_Q_FULL = 0,
-    B_KT_FULL = 1,   // +stage
-    B_KT_EMPTY = 3,  // +stage
-    B_VT_FULL = 5,   // +stage
-    B_VT_EMPTY = 7,  // +stage
-    B_SD_FULL = 9,   // +buffer
-    B_P_FULL = 11,   // +buffer
-    B_PV_DONE = 13,   // one phase per P.V pair (rescale waits on the previous tile's)
-    B_O_FULL = 14,    // single use: every MMA of the CTA has completed
-    B_MMA_DRAIN = 15,
-    N_BARS = 16
+    B_KT_FULL = 1,   // + stage
+    B_VT_FULL = 3,   // + stage
+    B_VT_EMPTY = 5,  // + stage
+    B_SD_FULL = 7,   // + buffer (= K-side stage)
+    B_P_FULL = 9,    // + buffer
+    B_O_FULL = 11,   // single use: every MMA of the tile has completed
+    B_MMA_DRAIN = 12,
+    N_BARS = 13
 };
-constexpr uint32_t OFF_TMEM_SLOT = 8 * N_BARS;   // u32
+static_assert(STAGES == 2, "the K-side ring reuses the two S/dS' buffer barriers");
+constexpr uint32_t OFF_TMEM_SLOT = 8 * N_BARS;     // u32
 constexpr uint32_t OFF_ABORT = OFF_TMEM_SLOT + 4;  // int
 
 constexpr uint32_t TM_O = 0, TM_T = 128, TM_BUF = 256;
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units: P entries stay <= 256
 
+// named barriers of the 256 softmax threads
+constexpr uint32_t NB_TILE = 2, NB_EPI = 1;
+
 struct Params {
     CUtensorMap tm_q, tm_tq, tm_k, tm_tk, tm_v, tm_tv, tm_o, tm_to;
     float *lse;
-    int Lq, Lk, n_qtiles;
-    float scale;       // s
-    float scale_log2;  // s * log2(e)
+    int Lq, Lk, n_qtiles;  // n_qtiles: 128-row query tiles per (batch, head)
+    float scale;           // s
+    float scale_log2;      // s * log2(e)
     unsigned long long bound_ns;
 };
 
@@ -106,15 +126,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
 
     if (threadIdx.x == 0) {
         mbar_init(BAR(B_Q_FULL), 1);
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < STAGES; ++s) {
             mbar_init(BAR(B_KT_FULL + s), 1);
-            mbar_init(BAR(B_KT_EMPTY + s), 1);
             mbar_init(BAR(B_VT_FULL + s), 1);
             mbar_init(BAR(B_VT_EMPTY + s), 1);
-            mbar_init(BAR(B_SD_FULL + s), 1);
-            mbar_init(BAR(B_P_FULL + s), 128);
         }
-        mbar_init(BAR(B_PV_DONE), 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(BAR(B_SD_FULL + b), 1);
+            mbar_init(BAR(B_P_FULL + b), SOFTMAX_THREADS);
+        }
         mbar_init(BAR(B_O_FULL), 1);
         mbar_init(BAR(B_MMA_DRAIN), 1);
         *abort_flag = 0;
@@ -141,7 +161,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
         // ------------------------------------------------------ TMA producer
         if (lane == 0) {
             bool ok = true;
-            int kt_last[2] = {-1, -1}, vt_last[2] = {-1, -1};
+            int kt_last[STAGES], vt_last[STAGES];
+            for (int s = 0; s < STAGES; ++s) kt_last[s] = vt_last[s] = -1;
             mbar_arrive_expect_tx(BAR(B_Q_FULL), 4 * CHUNK_Q);
             tma_load_3d(base + SM_Q, &p.tm_q, BAR(B_Q_FULL), 0, q0, bh);
             tma_load_3d(base + SM_Q + CHUNK_Q, &p.tm_q, BAR(B_Q_FULL), 64, q0, bh);
@@ -150,15 +171,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
             // order of use by the MMA warp: KT_0, KT_1, VT_0, KT_2, VT_1, ...
             for (int t = 0; t <= nk && ok; ++t) {
                 if (t < nk) {
-                    const int s = t & 1;
-                    if (!mbar_wait(BAR(B_KT_EMPTY + s), ((t >> 1) & 1) ^ 1, abort_flag, bound)) {
+                    const int s = t % STAGES;
+                    // stage s is free once S/dS' of tile t - 2 are complete
+                    if (!mbar_wait(BAR(B_SD_FULL + s), ((t / STAGES) & 1) ^ 1, abort_flag, bound)) {
                         ok = false;
                         break;
                     }
-                    const uint32_t st = base + SM_KT + s * STAGE_BYTES;
+                    const uint32_t st = base + SM_KT + s * KT_STAGE;
                     const uint32_t fb = BAR(B_KT_FULL + s);
                     const int y = t * BC;
-                    mbar_arrive_expect_tx(fb, STAGE_BYTES);
+                    mbar_arrive_expect_tx(fb, KT_STAGE);
                     // chunk c: K rows then tK rows, so [K | tK] is one N = 128 operand
                     tma_load_3d(st, &p.tm_k, fb, 0, y, bh);
                     tma_load_3d(st + CHUNK_K, &p.tm_tk, fb, 0, y, bh);
@@ -168,15 +190,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                 }
                 if (t >= 1) {
                     const int i = t - 1;
-                    const int s = i & 1;
-                    if (!mbar_wait(BAR(B_VT_EMPTY + s), ((i >> 1) & 1) ^ 1, abort_flag, bound)) {
+                    const int s = i % STAGES;
+                    if (!mbar_wait(BAR(B_VT_EMPTY + s), ((i / STAGES) & 1) ^ 1, abort_flag, bound)) {
                         ok = false;
                         break;
                     }
-                    const uint32_t st = base + SM_VT + s * STAGE_BYTES;
+                    const uint32_t st = base + SM_VT + s * VT_STAGE;
                     const uint32_t fb = BAR(B_VT_FULL + s);
                     const int y = i * BC;
-                    mbar_arrive_expect_tx(fb, STAGE_BYTES);
+                    mbar_arrive_expect_tx(fb, VT_STAGE);
                     // [V c0 | V c1 | tV c0 | tV c1]: N-chunks 64 columns apart (LBO)
                     tma_load_3d(st, &p.tm_v, fb, 0, y, bh);
                     tma_load_3d(st + CHUNK_K, &p.tm_v, fb, 64, y, bh);
@@ -187,9 +209,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
             }
             // let every copy already issued land before shared memory is released
             mbar_wait_drain(BAR(B_Q_FULL), 0, bound);
-            for (int s = 0; s < 2; ++s) {
-                if (kt_last[s] >= 0) mbar_wait_drain(BAR(B_KT_FULL + s), (kt_last[s] >> 1) & 1, bound);
-                if (vt_last[s] >= 0) mbar_wait_drain(BAR(B_VT_FULL + s), (vt_last[s] >> 1) & 1, bound);
+            for (int s = 0; s < STAGES; ++s) {
+                if (kt_last[s] >= 0) mbar_wait_drain(BAR(B_KT_FULL + s), (kt_last[s] / STAGES) & 1, bound);
+                if (vt_last[s] >= 0) mbar_wait_drain(BAR(B_VT_FULL + s), (vt_last[s] / STAGES) & 1, bound);
             }
         }
         __syncwarp();
@@ -200,50 +222,55 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
             constexpr uint32_t ID_D = idesc_bf16_f32(128, 64, 0);    // tQ K^T
             constexpr uint32_t ID_OT = idesc_bf16_f32(128, 256, 1);  // P [V|tV]
             constexpr uint32_t ID_T = idesc_bf16_f32(128, 128, 1);   // PdS V
+            // K-major operands: 128-byte rows, 8-row groups 1024 B apart; V: 64-column
+            // chunks CHUNK_K apart (LBO), 8-key groups 1024 B apart (SBO)
+            const uint64_t dq = smem_desc_sw128(base + SM_Q, 16, 1024);
+            const uint64_t dtq = smem_desc_sw128(base + SM_TQ, 16, 1024);
+            const uint64_t dk0 = smem_desc_sw128(base + SM_KT, 16, 1024);
+            const uint64_t dv0 = smem_desc_sw128(base + SM_VT, CHUNK_K, 1024);
             bool ok = mbar_wait(BAR(B_Q_FULL), 0, abort_flag, bound);
             auto issue_sd = [&](int j) -> bool {
-                const int s = j & 1;
-                if (!mbar_wait(BAR(B_KT_FULL + s), (j >> 1) & 1, abort_flag, bound)) return false;
+                const int s = j % STAGES;
+                const int b = j & 1;
+                if (!mbar_wait(BAR(B_KT_FULL + s), (j / STAGES) & 1, abort_flag, bound)) return false;
                 tc_fence_after();
-                const uint32_t kst = base + SM_KT + s * STAGE_BYTES;
-                const uint32_t t_s = tbase + TM_BUF + 128u * s;
+                const uint64_t dk = desc_add(dk0, s * KT_STAGE);
+                const uint32_t t_s = tbase + TM_BUF + 128u * b;
 #pragma unroll
                 for (int kk = 0; kk < HD / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * 2 * CHUNK_K + (kk & 3) * 32;
+                    const uint32_t off = (kk >> 2) * KT_CHUNK + (kk & 3) * 32;
                     const uint32_t offq = (kk >> 2) * CHUNK_Q + (kk & 3) * 32;
-                    mma_ss(t_s, smem_desc_sw128(base + SM_Q + offq, 16, 1024),
-                           smem_desc_sw128(kst + off, 16, 1024), ID_SD, kk > 0 ? 1u : 0u);
+                    mma_ss(t_s, desc_add(dq, offq), desc_add(dk, off), ID_SD, kk > 0 ? 1u : 0u);
                 }
 #pragma unroll
                 for (int kk = 0; kk < HD / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * 2 * CHUNK_K + (kk & 3) * 32;
+                    const uint32_t off = (kk >> 2) * KT_CHUNK + (kk & 3) * 32;
                     const uint32_t offq = (kk >> 2) * CHUNK_Q + (kk & 3) * 32;
-                    mma_ss(t_s + 64, smem_desc_sw128(base + SM_TQ + offq, 16, 1024),
-                           smem_desc_sw128(kst + off, 16, 1024), ID_D, 1u);
+                    mma_ss(t_s + 64, desc_add(dtq, offq), desc_add(dk, off), ID_D, 1u);
                 }
-                mma_commit(BAR(B_SD_FULL + s));
-                mma_commit(BAR(B_KT_EMPTY + s));
+                mma_commit(BAR(B_SD_FULL + b));
                 return true;
             };
             auto issue_pv = [&](int i) -> bool {
-                const int s = i & 1;
-                if (!mbar_wait(BAR(B_P_FULL + s), (i >> 1) & 1, abort_flag, bound)) return false;
-                if (!mbar_wait(BAR(B_VT_FULL + s), (i >> 1) & 1, abort_flag, bound)) return false;
+                const int s = i % STAGES;
+                const int b = i & 1;
+                if (!mbar_wait(BAR(B_P_FULL + b), (i >> 1) & 1, abort_flag, bound)) return false;
+                if (!mbar_wait(BAR(B_VT_FULL + s), (i / STAGES) & 1, abort_flag, bound)) return false;
                 tc_fence_after();
-                const uint32_t vst = base + SM_VT + s * STAGE_BYTES;
-                const uint32_t t_s = tbase + TM_BUF + 128u * s;
+                const uint64_t dv = desc_add(dv0, s * VT_STAGE);
+                const uint32_t t_s = tbase + TM_BUF + 128u * b;
 #pragma unroll
                 for (int kk = 0; kk < BC / 16; ++kk) {
-                    mma_ts(tbase + TM_O, t_s + 8u * kk, smem_desc_sw128(vst + kk * 2048, CHUNK_K, 1024), ID_OT,
-                           (i > 0 || kk > 0) ? 1u : 0u);
+                    // keys 16kk..16kk+15: group kk/2's columns, 8 columns per K-step
+                    const uint32_t a_col = (kk >> 1) * 32 + (kk & 1) * 8;
+                    mma_ts(tbase + TM_O, t_s + a_col, desc_add(dv, kk * 2048), ID_OT, (i > 0 || kk > 0) ? 1u : 0u);
                 }
 #pragma unroll
                 for (int kk = 0; kk < BC / 16; ++kk) {
-                    mma_ts(tbase + TM_T, t_s + 64 + 8u * kk, smem_desc_sw128(vst + kk * 2048, CHUNK_K, 1024),
-                           ID_T, 1u);
+                    const uint32_t a_col = 64 + (kk >> 1) * 32 + (kk & 1) * 8;
+                    mma_ts(tbase + TM_T, t_s + a_col, desc_add(dv, kk * 2048), ID_T, 1u);
                 }
                 mma_commit(BAR(B_VT_EMPTY + s));
-                mma_commit(BAR(B_PV_DONE));
                 return true;
             };
             if (ok) ok = issue_sd(0);
@@ -252,9 +279,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                 if (ok) ok = issue_pv(j - 1);
             }
             if (ok) ok = issue_pv(nk - 1);
-            // O and T are final once everything issued so far completes.  (A parity wait
-            // on B_PV_DONE for the last tile would be ambiguous: that barrier may still be
-            // two phases behind when the softmax warps finish their last tile.)
+            // O and T are final once everything issued so far completes (a dedicated
+            // barrier: a parity wait on a per-tile barrier could be ambiguous here)
             if (ok) mma_commit(BAR(B_O_FULL));
             // every MMA issued must finish before tensor memory is released
             mma_commit(BAR(B_MMA_DRAIN));
@@ -263,59 +289,70 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
         __syncwarp();
     } else if (warp >= 4) {
         // ---------------------------------------- softmax, JVP statistics, epilogue
-        const int wl = warp - 4;
+        const int grp = (warp - 4) >> 2;  // key columns 32*grp .. 32*grp+31 of each tile
+        const int wl = warp & 3;          // TMEM lane quadrant
         const int row = wl * 32 + lane;
         const uint32_t lane_off = (uint32_t)(wl * 32) << 16;
+        const uint32_t col0 = 32u * (uint32_t)grp;
         const float c = p.scale_log2;
-        const float s_lin = p.scale;
+        const float2 c2 = make_float2(c, c);
+        const float2 s2 = make_float2(p.scale, p.scale);
+        const bool up = c >= 0.f;  // row max of c*S is c * max(S) (min(S) for c < 0)
+        const float sentinel = up ? -INFINITY : INFINITY;
+        float *xch = reinterpret_cast<float *>(gbase + SM_XCH);
         float m_ref = -INFINITY, l = 0.f, g = 0.f;
-        bool ok = true;
+        bool failed = false;
 
         for (int j = 0; j < nk; ++j) {
             const int b = j & 1;
             const uint32_t t_s = tbase + lane_off + TM_BUF + 128u * b;
-            ok = mbar_wait(BAR(B_SD_FULL + b), (j >> 1) & 1, abort_flag, bound);
-            ok = __all_sync(0xffffffffu, ok);
-            if (!ok) break;
-            tc_fence_after();
-
-            float x[BC];
-            {
-                uint32_t r0[32], r1[32];
-                tmem_ld32(t_s, r0);
-                tmem_ld32(t_s + 32, r1);
+            if (!failed) failed = !mbar_wait_warp(BAR(B_SD_FULL + b), (j >> 1) & 1, abort_flag, bound);
+            uint32_t xs[32], xd[32];
+            const int valid = p.Lk - j * BC - (int)col0;  // keys of this group inside Lk (may be <= 0)
+            float part = sentinel;
+            if (!failed) {
+                tc_fence_after();
+                tmem_ld32(t_s + col0, xs);
+                tmem_ld32(t_s + 64 + col0, xd);
                 tmem_wait_ld();
+                if (valid < 32) {
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    x[i] = __uint_as_float(r0[i]);
-                    x[i + 32] = __uint_as_float(r1[i]);
+                    for (int i = 0; i < 32; ++i)
+                        if (i >= valid) xs[i] = __float_as_uint(sentinel);
                 }
+                float m4[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) m4[k] = __uint_as_float(xs[k]);
+                if (up) {
+#pragma unroll
+                    for (int i = 4; i < 28; i += 8)
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+                            m4[k] = fmax3(m4[k], __uint_as_float(xs[i + k]), __uint_as_float(xs[i + 4 + k]));
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) m4[k] = fmaxf(m4[k], __uint_as_float(xs[28 + k]));
+                    part = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]);
+                } else {
+#pragma unroll
+                    for (int i = 4; i < 28; i += 8)
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+                            m4[k] = fmin3(m4[k], __uint_as_float(xs[i + k]), __uint_as_float(xs[i + 4 + k]));
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) m4[k] = fminf(m4[k], __uint_as_float(xs[28 + k]));
+                    part = fminf(fmin3(m4[0], m4[1], m4[2]), m4[3]);
+                }
+                xch[(b * 2 + grp) * 128 + row] = part;
             }
-            const int valid = p.Lk - j * BC;  // >= 1
-            if (valid < BC) {
-#pragma unroll
-                for (int i = 1; i < BC; ++i)
-                    if (i >= valid) x[i] = x[0];  // neutral for the max; p forced to 0 below
+            // both groups' partial maxima are in shared memory; every softmax
+            // thread reaches this barrier each tile, and a failure anywhere
+            // ends the loop for all of them together
+            if (named_bar_or(NB_TILE, SOFTMAX_THREADS, failed)) {
+                failed = true;
+                break;
             }
-            // row max (min for a negative scale) over 8 independent chains
-            float m8[8];
-#pragma unroll
-            for (int k = 0; k < 8; ++k) m8[k] = x[k];
-            if (c >= 0.f) {
-#pragma unroll
-                for (int i = 8; i < BC; ++i) m8[i & 7] = fmaxf(m8[i & 7], x[i]);
-#pragma unroll
-                for (int k = 0; k < 4; ++k) m8[k] = fmaxf(m8[k], m8[k + 4]);
-                m8[0] = fmaxf(fmaxf(m8[0], m8[2]), fmaxf(m8[1], m8[3]));
-            } else {
-#pragma unroll
-                for (int i = 8; i < BC; ++i) m8[i & 7] = fminf(m8[i & 7], x[i]);
-#pragma unroll
-                for (int k = 0; k < 4; ++k) m8[k] = fminf(m8[k], m8[k + 4]);
-                m8[0] = fminf(fminf(m8[0], m8[2]), fminf(m8[1], m8[3]));
-            }
-            const float mx = m8[0];
-            const float m_tile = mx * c;
+            const float other = xch[(b * 2 + (grp ^ 1)) * 128 + row];
+            const float m_tile = (up ? fmaxf(part, other) : fminf(part, other)) * c;
             if (j == 0) {
                 m_ref = m_tile;
             } else {
@@ -328,88 +365,85 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                     }
                     l *= alpha;
                     g *= alpha;
-                    // O and T may only be touched once PV_{j-1} is complete
-                    ok = mbar_wait(BAR(B_PV_DONE), (j - 1) & 1, abort_flag, bound);
-                    ok = __all_sync(0xffffffffu, ok);
-                    if (!ok) break;
-                    tc_fence_after();
+                    // O and T may only be touched once the P.V products of tile j-1
+                    // are complete (the V-side barrier of its stage); group 0
+                    // rescales O, group 1 rescales T
+                    failed = !mbar_wait_warp(BAR(B_VT_EMPTY + ((j - 1) & 1)), ((j - 1) >> 1) & 1, abort_flag, bound);
+                    if (!failed) {
+                        tc_fence_after();
 #pragma unroll 1
-                    for (int cc = 0; cc < 8; ++cc) {
-                        uint32_t r[32];
-                        const uint32_t ta = tbase + lane_off + TM_O + 32u * cc;
-                        tmem_ld32(ta, r);
-                        tmem_wait_ld();
+                        for (int cc = 0; cc < 4; ++cc) {
+                            uint32_t r[32];
+                            const uint32_t ta = tbase + lane_off + 128u * (uint32_t)grp + 32u * cc;
+                            tmem_ld32(ta, r);
+                            tmem_wait_ld();
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-                        tmem_st32(ta, r);
+                            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+                            tmem_st32(ta, r);
+                        }
                     }
                 }
             }
-            const float neg_m = -m_ref;
+            if (failed) continue;  // the next tile's barrier carries the failure to everyone
+            const float2 nm2 = make_float2(-m_ref, -m_ref);
+            float pv[32];
 #pragma unroll
-            for (int i = 0; i < BC; ++i) x[i] = ex2_approx(fmaf(x[i], c, neg_m));
-            if (valid < BC) {
-#pragma unroll
-                for (int i = 1; i < BC; ++i)
-                    if (i >= valid) x[i] = 0.f;
+            for (int i = 0; i < 16; ++i) {
+                const float2 y =
+                    __ffma2_rn(make_float2(__uint_as_float(xs[2 * i]), __uint_as_float(xs[2 * i + 1])), c2, nm2);
+                pv[2 * i] = ex2_approx(y.x);
+                pv[2 * i + 1] = ex2_approx(y.y);
             }
-            // dS' is loaded while P is packed and stored (different columns)
-            uint32_t d0[32], d1[32];
-            tmem_ld32(t_s + 64, d0);
-            tmem_ld32(t_s + 96, d1);
-            float lsum;
-            {
-                float ls[4] = {0.f, 0.f, 0.f, 0.f};
-                uint32_t pk[32];
+            if (valid < 32) {
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    ls[i & 3] += x[2 * i] + x[2 * i + 1];
-                    pk[i] = pack_bf16x2(x[2 * i], x[2 * i + 1]);
-                }
-                tmem_st32(t_s, pk);  // P over S's first 32 columns
-                lsum = (ls[0] + ls[1]) + (ls[2] + ls[3]);
+                for (int i = 0; i < 32; ++i)
+                    if (i >= valid) pv[i] = 0.f;
             }
-            float gsum;
-            {
-                tmem_wait_ld();
-                float gs[4] = {0.f, 0.f, 0.f, 0.f};
-                uint32_t pd[32];
+            float2 ls2a = make_float2(0.f, 0.f), ls2b = ls2a, gs2a = ls2a, gs2b = ls2a;
+            uint32_t pk[16], pd[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const float t0 = x[2 * i] * __uint_as_float(d0[2 * i]) * s_lin;
-                    const float t1 = x[2 * i + 1] * __uint_as_float(d0[2 * i + 1]) * s_lin;
-                    gs[i & 3] += t0 + t1;
-                    pd[i] = pack_bf16x2(t0, t1);
+            for (int i = 0; i < 16; ++i) {
+                const float2 pp = make_float2(pv[2 * i], pv[2 * i + 1]);
+                const float2 dd = make_float2(__uint_as_float(xd[2 * i]), __uint_as_float(xd[2 * i + 1]));
+                const float2 t = __fmul2_rn(__fmul2_rn(pp, dd), s2);  // p * s dS'
+                if (i & 1) {
+                    ls2b = __fadd2_rn(ls2b, pp);
+                    gs2b = __fadd2_rn(gs2b, t);
+                } else {
+                    ls2a = __fadd2_rn(ls2a, pp);
+                    gs2a = __fadd2_rn(gs2a, t);
                 }
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const float t0 = x[32 + 2 * i] * __uint_as_float(d1[2 * i]) * s_lin;
-                    const float t1 = x[32 + 2 * i + 1] * __uint_as_float(d1[2 * i + 1]) * s_lin;
-                    gs[i & 3] += t0 + t1;
-                    pd[16 + i] = pack_bf16x2(t0, t1);
-                }
-                tmem_st32(t_s + 64, pd);  // P.*s dS' over dS''s first 32 columns
-                gsum = (gs[0] + gs[1]) + (gs[2] + gs[3]);
+                pk[i] = pack_bf16x2(pp.x, pp.y);
+                pd[i] = pack_bf16x2(t.x, t.y);
             }
-            l += lsum;
-            g += gsum;
+            tmem_st16(t_s + col0, pk);       // P over this group's S columns
+            tmem_st16(t_s + 64 + col0, pd);  // P.*s dS' over this group's dS' columns
+            l += (ls2a.x + ls2b.x) + (ls2a.y + ls2b.y);
+            g += (gs2a.x + gs2b.x) + (gs2a.y + gs2b.y);
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(BAR(B_P_FULL + b));
         }
 
-        if (ok) {
-            ok = mbar_wait(BAR(B_O_FULL), 0, abort_flag, bound);
-            ok = __all_sync(0xffffffffu, ok);
+        if (!failed) failed = !mbar_wait_warp(BAR(B_O_FULL), 0, abort_flag, bound);
+        float *lg = xch + 2 * 2 * 128;  // [l, g][group][row]
+        if (!failed) {
+            lg[(0 * 2 + grp) * 128 + row] = l;
+            lg[(1 * 2 + grp) * 128 + row] = g;
         }
-        if (ok) {
+        const bool any_failed = named_bar_or(NB_EPI, SOFTMAX_THREADS, failed);
+        if (!any_failed) {
             tc_fence_after();
-            const float inv_l = 1.f / l;
-            const float mu = g * inv_l;
-            // stage O into the Q tile's shared memory and tO into tQ's, in the
-            // 128-byte-swizzled layout of the store tensor maps
+            const float lt = l + lg[(0 * 2 + (grp ^ 1)) * 128 + row];
+            const float gt = g + lg[(1 * 2 + (grp ^ 1)) * 128 + row];
+            const float inv_l = 1.f / lt;
+            const float mu = gt * inv_l;
+            // group grp writes output columns 64*grp .. 64*grp+63: O into the Q
+            // tile's shared memory, tO into tQ's, in the 128-byte-swizzled
+            // layout of the store tensor maps
 #pragma unroll 1
-            for (int pc = 0; pc < 4; ++pc) {
+            for (int h = 0; h < 2; ++h) {
+                const int pc = 2 * grp + h;
                 uint32_t ro[32], rt[32];
                 tmem_ld32(tbase + lane_off + TM_O + 32u * pc, ro);
                 tmem_ld32(tbase + lane_off + TM_T + 32u * pc, rt);
@@ -424,8 +458,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                     wo[i] = pack_bf16x2(o0, o1);
                     wt[i] = pack_bf16x2(t0, t1);
                 }
-                const uint32_t chunk_off = (uint32_t)(pc >> 1) * CHUNK_Q + (uint32_t)row * 128u;
-                const uint32_t unit0 = (uint32_t)(pc & 1) * 4u;
+                const uint32_t chunk_off = (uint32_t)grp * CHUNK_Q + (uint32_t)row * 128u;
+                const uint32_t unit0 = (uint32_t)h * 4u;
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     const uint32_t phys = (((unit0 + u) ^ (uint32_t)(row & 7)) * 16u);
@@ -435,16 +469,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                                  wt[4 * u + 3]);
                 }
             }
-            if (p.lse != nullptr && q0 + row < p.Lq) {
+            if (grp == 0 && p.lse != nullptr && q0 + row < p.Lq) {
                 p.lse[(size_t)bh * (size_t)p.Lq + (size_t)(q0 + row)] =
-                    (m_ref + __log2f(l)) * 0.69314718055994531f;
+                    (m_ref + __log2f(lt)) * 0.69314718055994531f;
             }
         }
         fence_proxy_async_smem();
-        // all four softmax warps reach this barrier on every path (a warp that
-        // gave up skips only the work), so it cannot hang
-        named_bar_sync(1, 128);
-        if (wl == 0 && lane == 0 && ok && *abort_flag == 0) {
+        named_bar_sync(NB_EPI, SOFTMAX_THREADS);  // staging complete (every softmax thread gets here)
+        if (warp == 4 && lane == 0 && !any_failed && *abort_flag == 0) {
             tma_store_3d(&p.tm_o, base + SM_Q, 0, q0, bh);
             tma_store_3d(&p.tm_o, base + SM_Q + CHUNK_Q, 64, q0, bh);
             tma_store_3d(&p.tm_to, base + SM_TQ, 0, q0, bh);
