@@ -21,6 +21,7 @@ from ._binding import (  # noqa: F401
     attn_jvp,
     attn_jvp_fwd,
     attn_jvp_fwd_f32,
+    attn_jvp_fwd_f32out,
     check_device_status,
     load_library,
     selftest_wait_timeout,
@@ -30,6 +31,6 @@ from ._binding import (  # noqa: F401
 )
 
 __all__ = [
-    "attn_jvp", "attn_jvp_fwd", "attn_jvp_fwd_f32", "check_device_status", "load_library",
+    "attn_jvp", "attn_jvp_fwd", "attn_jvp_fwd_f32", "attn_jvp_fwd_f32out", "check_device_status", "load_library",
     "selftest_wait_timeout", "set_wait_bound_ns", "strerror", "version", "AttnJvpError",
 ]

@@ -26,7 +26,7 @@ AJVP_ERR_CUDA = -6
 AJVP_ERR_TOO_LARGE = -7
 
 # every symbol the header declares
-EXPORTED = ("attn_jvp_fwd", "attn_jvp_fwd_f32", "attn_jvp_strerror", "attn_jvp_last_cuda_error",
+EXPORTED = ("attn_jvp_fwd", "attn_jvp_fwd_f32out", "attn_jvp_fwd_f32", "attn_jvp_strerror", "attn_jvp_last_cuda_error",
             "attn_jvp_check_device_status", "attn_jvp_set_wait_bound_ns",
             "attn_jvp_selftest_wait_timeout", "attn_jvp_version")
 
@@ -56,6 +56,8 @@ def load_library(path: str = LIB_PATH):
         lib.attn_jvp_fwd.restype = ctypes.c_int
         lib.attn_jvp_fwd_f32.argtypes = fwd_args
         lib.attn_jvp_fwd_f32.restype = ctypes.c_int
+        lib.attn_jvp_fwd_f32out.argtypes = fwd_args
+        lib.attn_jvp_fwd_f32out.restype = ctypes.c_int
         lib.attn_jvp_strerror.argtypes = [ctypes.c_int]
         lib.attn_jvp_strerror.restype = ctypes.c_char_p
         lib.attn_jvp_last_cuda_error.argtypes = []
@@ -97,7 +99,7 @@ def _ptr(t) -> int | None:
     return None if t is None else t.data_ptr()
 
 
-def _prepare(q, k, v, tq, tk, tv, o, to, lse, dtype, want_lse):
+def _prepare(q, k, v, tq, tk, tv, o, to, lse, dtype, want_lse, out_dtype=None):
     for name, x in (("q", q), ("k", k), ("v", v), ("tq", tq), ("tk", tk), ("tv", tv)):
         if not isinstance(x, torch.Tensor) or not x.is_cuda:
             raise ValueError(f"{name} must be a CUDA tensor")
@@ -112,13 +114,14 @@ def _prepare(q, k, v, tq, tk, tv, o, to, lse, dtype, want_lse):
     for name, x in (("k", k), ("v", v), ("tk", tk), ("tv", tv)):
         if x.shape != (B, H, Lk, d):
             raise ValueError(f"{name} must be [B, H, Lk, d] = {(B, H, Lk, d)}, got {tuple(x.shape)}")
+    out_dtype = dtype if out_dtype is None else out_dtype
     if o is None:
-        o = torch.empty_like(q)
+        o = torch.empty(q.shape, device=q.device, dtype=out_dtype)
     if to is None:
-        to = torch.empty_like(q)
+        to = torch.empty(q.shape, device=q.device, dtype=out_dtype)
     if want_lse and lse is None:
         lse = torch.empty((B, H, Lq), device=q.device, dtype=torch.float32)
-    for name, x, shp, dt in (("o", o, q.shape, dtype), ("to", to, q.shape, dtype)):
+    for name, x, shp, dt in (("o", o, q.shape, out_dtype), ("to", to, q.shape, out_dtype)):
         if x.shape != shp or x.dtype != dt or not x.is_contiguous() or not x.is_cuda:
             raise ValueError(f"{name} must be a contiguous CUDA {dt} tensor of shape {tuple(shp)}")
     if lse is not None and (lse.shape != (B, H, Lq) or lse.dtype != torch.float32 or not lse.is_contiguous()):
@@ -138,6 +141,20 @@ def attn_jvp_fwd(q, k, v, tq, tk, tv, scale=None, o=None, to=None, lse=None, str
     rc = lib.attn_jvp_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(tq), _ptr(tk), _ptr(tv), _ptr(o), _ptr(to), _ptr(lse),
                           B, H, Lq, Lk, d, float(scale), _stream_handle(stream))
     _check(rc, "attn_jvp_fwd")
+    return o, to, lse
+
+
+def attn_jvp_fwd_f32out(q, k, v, tq, tk, tv, scale=None, o=None, to=None, lse=None, stream=None, want_lse=True):
+    """bf16 inputs, fp32 O and tO, through ``attn_jvp_fwd_f32out`` (tcgen05
+    kernel with split-bf16 probability operands; d = 128)."""
+    o, to, lse, (B, H, Lq, Lk, d) = _prepare(q, k, v, tq, tk, tv, o, to, lse, torch.bfloat16, want_lse,
+                                            out_dtype=torch.float32)
+    if scale is None:
+        scale = d ** -0.5
+    lib = load_library()
+    rc = lib.attn_jvp_fwd_f32out(_ptr(q), _ptr(k), _ptr(v), _ptr(tq), _ptr(tk), _ptr(tv), _ptr(o), _ptr(to),
+                                 _ptr(lse), B, H, Lq, Lk, d, float(scale), _stream_handle(stream))
+    _check(rc, "attn_jvp_fwd_f32out")
     return o, to, lse
 
 

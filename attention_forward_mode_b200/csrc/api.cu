@@ -63,9 +63,12 @@ int device_setup(int *dev_out) {
             st.status = AJVP_ERR_UNSUPPORTED_DEVICE;
             return;
         }
-        cudaError_t e3 = cudaFuncSetAttribute(ajvp::sm100::attn_jvp_fwd_kernel,
+        cudaError_t e3 = cudaFuncSetAttribute(ajvp::sm100::attn_jvp_fwd_kernel<false>,
                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
                                               (int)ajvp::sm100::SMEM_BYTES);
+        if (e3 == cudaSuccess)
+            e3 = cudaFuncSetAttribute(ajvp::sm100::attn_jvp_fwd_kernel<true>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ajvp::sm100::SMEM_BYTES);
         cudaError_t e4 = cudaFuncSetAttribute(ajvp::f32::attn_jvp_fwd_f32_kernel,
                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
                                               (int)ajvp::f32::smem_bytes(ajvp::f32::DMAX));
@@ -125,11 +128,10 @@ int check_common(const void *q, const void *k, const void *v, const void *tq, co
     return AJVP_OK;
 }
 
-}  // namespace
-
-extern "C" {
-
-int attn_jvp_fwd(const void *q, const void *k, const void *v, const void *tq, const void *tk, const void *tv,
+// Shared host path of the two tensor-core entry points (kSplit: fp32 outputs,
+// split-bf16 probability operands).
+template <bool kSplit>
+int launch_sm100(const void *q, const void *k, const void *v, const void *tq, const void *tk, const void *tv,
                  void *o, void *to, float *lse, int64_t B, int64_t H, int64_t Lq, int64_t Lk, int64_t d,
                  float scale, void *stream) {
     bool noop = false;
@@ -157,8 +159,13 @@ int attn_jvp_fwd(const void *q, const void *k, const void *v, const void *tq, co
     if ((rc = encode_3d(&p.tm_tk, tk, d, Lk, BH, 64)) != AJVP_OK) return rc;
     if ((rc = encode_3d(&p.tm_v, v, d, Lk, BH, 64)) != AJVP_OK) return rc;
     if ((rc = encode_3d(&p.tm_tv, tv, d, Lk, BH, 64)) != AJVP_OK) return rc;
-    if ((rc = encode_3d(&p.tm_o, o, d, Lq, BH, 128)) != AJVP_OK) return rc;
-    if ((rc = encode_3d(&p.tm_to, to, d, Lq, BH, 128)) != AJVP_OK) return rc;
+    if (kSplit) {
+        p.o_f32 = static_cast<float *>(o);
+        p.to_f32 = static_cast<float *>(to);
+    } else {
+        if ((rc = encode_3d(&p.tm_o, o, d, Lq, BH, 128)) != AJVP_OK) return rc;
+        if ((rc = encode_3d(&p.tm_to, to, d, Lq, BH, 128)) != AJVP_OK) return rc;
+    }
     p.lse = lse;
     p.Lq = (int)Lq;
     p.Lk = (int)Lk;
@@ -167,11 +174,27 @@ int attn_jvp_fwd(const void *q, const void *k, const void *v, const void *tq, co
     p.scale_log2 = scale * 1.4426950408889634f;
     p.bound_ns = g_bound_ns.load();
 
-    ajvp::sm100::attn_jvp_fwd_kernel<<<(unsigned)(n_qtiles * BH), ajvp::sm100::NTHREADS, ajvp::sm100::SMEM_BYTES,
-                                       (cudaStream_t)stream>>>(p);
+    ajvp::sm100::attn_jvp_fwd_kernel<kSplit><<<(unsigned)(n_qtiles * BH), ajvp::sm100::NTHREADS,
+                                               ajvp::sm100::SMEM_BYTES, (cudaStream_t)stream>>>(p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail_cuda(e);
     return AJVP_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int attn_jvp_fwd(const void *q, const void *k, const void *v, const void *tq, const void *tk, const void *tv,
+                 void *o, void *to, float *lse, int64_t B, int64_t H, int64_t Lq, int64_t Lk, int64_t d,
+                 float scale, void *stream) {
+    return launch_sm100<false>(q, k, v, tq, tk, tv, o, to, lse, B, H, Lq, Lk, d, scale, stream);
+}
+
+int attn_jvp_fwd_f32out(const void *q, const void *k, const void *v, const void *tq, const void *tk,
+                        const void *tv, float *o, float *to, float *lse, int64_t B, int64_t H, int64_t Lq,
+                        int64_t Lk, int64_t d, float scale, void *stream) {
+    return launch_sm100<true>(q, k, v, tq, tk, tv, o, to, lse, B, H, Lq, Lk, d, scale, stream);
 }
 
 int attn_jvp_fwd_f32(const float *q, const float *k, const float *v, const float *tq, const float *tk,

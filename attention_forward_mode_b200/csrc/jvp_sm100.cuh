@@ -98,6 +98,7 @@ constexpr uint32_t NB_TILE = 2, NB_EPI = 1;
 
 struct Params {
     CUtensorMap tm_q, tm_tq, tm_k, tm_tk, tm_v, tm_tv, tm_o, tm_to;
+    float *o_f32, *to_f32;  // kSplit: fp32 outputs [B*H][Lq][128] (tm_o / tm_to unused)
     float *lse;
     int Lq, Lk, n_qtiles;  // n_qtiles: 128-row query tiles per (batch, head)
     float scale;           // s
@@ -105,6 +106,11 @@ struct Params {
     unsigned long long bound_ns;
 };
 
+// kSplit = false: bf16 P and P.*s dS' operands, bf16 outputs.
+// kSplit = true : P and P.*s dS' are each split into bf16 hi + lo parts
+//                 (x = hi + lo to ~16 significant bits), both multiplied into
+//                 O and T, and O, tO are written in fp32; 1.5x the MMA work.
+template <bool kSplit>
 __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_constant__ Params p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -270,6 +276,18 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                     const uint32_t a_col = 64 + (kk >> 1) * 32 + (kk & 1) * 8;
                     mma_ts(tbase + TM_T, t_s + a_col, desc_add(dv, kk * 2048), ID_T, 1u);
                 }
+                if (kSplit) {  // the lo parts sit 16 columns after the hi parts
+#pragma unroll
+                    for (int kk = 0; kk < BC / 16; ++kk) {
+                        const uint32_t a_col = 16 + (kk >> 1) * 32 + (kk & 1) * 8;
+                        mma_ts(tbase + TM_O, t_s + a_col, desc_add(dv, kk * 2048), ID_OT, 1u);
+                    }
+#pragma unroll
+                    for (int kk = 0; kk < BC / 16; ++kk) {
+                        const uint32_t a_col = 64 + 16 + (kk >> 1) * 32 + (kk & 1) * 8;
+                        mma_ts(tbase + TM_T, t_s + a_col, desc_add(dv, kk * 2048), ID_T, 1u);
+                    }
+                }
                 mma_commit(BAR(B_VT_EMPTY + s));
                 return true;
             };
@@ -418,6 +436,20 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
             }
             tmem_st16(t_s + col0, pk);       // P over this group's S columns
             tmem_st16(t_s + 64 + col0, pd);  // P.*s dS' over this group's dS' columns
+            if (kSplit) {
+                // lo = x - hi, rounded to bf16: hi + lo carries ~16 significant bits
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float2 pp = make_float2(pv[2 * i], pv[2 * i + 1]);
+                    const float2 dd = make_float2(__uint_as_float(xd[2 * i]), __uint_as_float(xd[2 * i + 1]));
+                    const float2 t = __fmul2_rn(__fmul2_rn(pp, dd), s2);
+                    const uint32_t ph = pack_bf16x2(pp.x, pp.y), th = pack_bf16x2(t.x, t.y);
+                    pk[i] = pack_bf16x2(pp.x - __uint_as_float(ph << 16), pp.y - __uint_as_float(ph & 0xffff0000u));
+                    pd[i] = pack_bf16x2(t.x - __uint_as_float(th << 16), t.y - __uint_as_float(th & 0xffff0000u));
+                }
+                tmem_st16(t_s + col0 + 16, pk);
+                tmem_st16(t_s + 64 + col0 + 16, pd);
+            }
             l += (ls2a.x + ls2b.x) + (ls2a.y + ls2b.y);
             g += (gs2a.x + gs2b.x) + (gs2a.y + gs2b.y);
             tmem_wait_st();
@@ -438,11 +470,39 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
             const float gt = g + lg[(1 * 2 + (grp ^ 1)) * 128 + row];
             const float inv_l = 1.f / lt;
             const float mu = gt * inv_l;
-            // group grp writes output columns 64*grp .. 64*grp+63: O into the Q
-            // tile's shared memory, tO into tQ's, in the 128-byte-swizzled
-            // layout of the store tensor maps
+            // group grp writes output columns 64*grp .. 64*grp+63
+            if (kSplit) {
+                // fp32 outputs straight from registers, 16 bytes per store
+                const bool row_ok = q0 + row < p.Lq;
+                const size_t off = ((size_t)bh * (size_t)p.Lq + (size_t)(q0 + row)) * HD + 64u * (uint32_t)grp;
 #pragma unroll 1
-            for (int h = 0; h < 2; ++h) {
+                for (int h = 0; h < 2; ++h) {
+                    const int pc = 2 * grp + h;
+                    uint32_t ro[32], rt[32];
+                    tmem_ld32(tbase + lane_off + TM_O + 32u * pc, ro);
+                    tmem_ld32(tbase + lane_off + TM_T + 32u * pc, rt);
+                    tmem_wait_ld();
+                    if (row_ok) {
+                        float4 *po = reinterpret_cast<float4 *>(p.o_f32 + off + 32 * h);
+                        float4 *pt = reinterpret_cast<float4 *>(p.to_f32 + off + 32 * h);
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            float o4[4], t4[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                o4[e] = __uint_as_float(ro[4 * u + e]) * inv_l;
+                                t4[e] = fmaf(-mu, o4[e], __uint_as_float(rt[4 * u + e]) * inv_l);
+                            }
+                            po[u] = make_float4(o4[0], o4[1], o4[2], o4[3]);
+                            pt[u] = make_float4(t4[0], t4[1], t4[2], t4[3]);
+                        }
+                    }
+                }
+            }
+            // bf16 outputs: O into the Q tile's shared memory, tO into tQ's, in
+            // the 128-byte-swizzled layout of the store tensor maps
+#pragma unroll 1
+            for (int h = 0; h < (kSplit ? 0 : 2); ++h) {
                 const int pc = 2 * grp + h;
                 uint32_t ro[32], rt[32];
                 tmem_ld32(tbase + lane_off + TM_O + 32u * pc, ro);
@@ -476,7 +536,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
         }
         fence_proxy_async_smem();
         named_bar_sync(NB_EPI, SOFTMAX_THREADS);  // staging complete (every softmax thread gets here)
-        if (warp == 4 && lane == 0 && !any_failed && *abort_flag == 0) {
+        if (!kSplit && warp == 4 && lane == 0 && !any_failed && *abort_flag == 0) {
             tma_store_3d(&p.tm_o, base + SM_Q, 0, q0, bh);
             tma_store_3d(&p.tm_o, base + SM_Q + CHUNK_Q, 64, q0, bh);
             tma_store_3d(&p.tm_to, base + SM_TQ, 0, q0, bh);

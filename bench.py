@@ -253,8 +253,11 @@ def run_ours(args, w):
     ajvp.load_library()
 
     inp = make_inputs(w, seed=rank, device=dev)
-    o = torch.empty_like(inp["q"])
-    to = torch.empty_like(inp["q"])
+    # entry point: attn_jvp_fwd (bf16 outputs) or attn_jvp_fwd_f32out (fp32 outputs)
+    fwd = ajvp.attn_jvp_fwd if args.entry == "bf16" else ajvp.attn_jvp_fwd_f32out
+    out_dtype = torch.bfloat16 if args.entry == "bf16" else torch.float32
+    o = torch.empty(inp["q"].shape, device=dev, dtype=out_dtype)
+    to = torch.empty(inp["q"].shape, device=dev, dtype=out_dtype)
     lse = torch.empty((w.B, w.H, w.Lq), device=dev, dtype=torch.float32)
     stream = torch.cuda.current_stream(dev)
     in_bytes = sum(t.numel() * t.element_size() for t in inp.values())
@@ -265,7 +268,7 @@ def run_ours(args, w):
     def step():
         if flush is not None:
             flush.zero_()
-        ajvp.attn_jvp_fwd(inp["q"], inp["k"], inp["v"], inp["tq"], inp["tk"], inp["tv"], w.scale,
+        fwd(inp["q"], inp["k"], inp["v"], inp["tq"], inp["tk"], inp["tv"], w.scale,
                           o=o, to=to, lse=lse, stream=stream)
 
     for _ in range(args.warmup):
@@ -302,12 +305,12 @@ def run_ours(args, w):
     host_to = torch.empty(to.shape, dtype=to.dtype).pin_memory()
     host_lse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in host_in.values())
-    d2h = host_o.numel() * 2 + host_to.numel() * 2 + host_lse.numel() * 4
+    d2h = sum(t.numel() * t.element_size() for t in (host_o, host_to, host_lse))
 
     def e2e_step():
         for n in inp:
             inp[n].copy_(host_in[n], non_blocking=True)
-        ajvp.attn_jvp_fwd(inp["q"], inp["k"], inp["v"], inp["tq"], inp["tk"], inp["tv"], w.scale,
+        fwd(inp["q"], inp["k"], inp["v"], inp["tq"], inp["tk"], inp["tv"], w.scale,
                           o=o, to=to, lse=lse, stream=stream)
         host_o.copy_(o, non_blocking=True)
         host_to.copy_(to, non_blocking=True)
@@ -334,7 +337,8 @@ def run_ours(args, w):
         line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-                "config": workload_config(w, world),
+                "config": dict(workload_config(w, world), entry=("attn_jvp_fwd" if args.entry == "bf16"
+                                                                 else "attn_jvp_fwd_f32out")),
                 "pct_of_bf16_peak": 100.0 * value / world / burst,
                 "roofline": {"bound": "tensor", "achieved": achieved, "peak": burst, "unit": "TFLOP/s",
                              "frac": achieved / burst, "traffic": committed_traffic(),
@@ -405,6 +409,8 @@ def main(argv=None):
     ap.add_argument("--reference-seconds", type=float, default=90.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-eager", action="store_true")
+    ap.add_argument("--entry", choices=["bf16", "f32out"], default="bf16",
+                    help="f32out: time attn_jvp_fwd_f32out (fp32 outputs, split-bf16 probabilities)")
     ap.add_argument("--heads", type=int, default=None,
                     help="override H (small profiling captures); the JSON config shows the H used")
     args = ap.parse_args(argv)

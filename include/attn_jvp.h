@@ -90,6 +90,27 @@ AJVP_API int attn_jvp_fwd(const void *q, const void *k, const void *v,
                  float scale, void *stream);
 
 /*
+ * attn_jvp_fwd_f32out -- bf16 inputs, fp32 outputs, for when the tangent must
+ * be accurate beyond bf16 (the anthology record LIT-783, takeaway on §3.3 and
+ * Fig. 11: BF16 JVP error is much larger than BF16 output error).  Same
+ * tcgen05 kernel as attn_jvp_fwd, but the probabilities P and the tangent
+ * weights P.*s dS' are each carried as two bf16 parts (hi + lo, ~16
+ * significant bits) into the P.V products, and O, tO are written in fp32
+ * (1.5x the tensor-core work of attn_jvp_fwd).
+ *
+ *   q, k, v, tq, tk, tv : const __nv_bfloat16, layouts as attn_jvp_fwd
+ *   o, to               : float [B][H][Lq][d]
+ *   lse                 : float [B][H][Lq], or NULL
+ *
+ * Same sizes, alignment (16 bytes), device and error rules as attn_jvp_fwd.
+ */
+AJVP_API int attn_jvp_fwd_f32out(const void *q, const void *k, const void *v,
+                        const void *tq, const void *tk, const void *tv,
+                        float *o, float *to, float *lse,
+                        int64_t B, int64_t H, int64_t Lq, int64_t Lk, int64_t d,
+                        float scale, void *stream);
+
+/*
  * attn_jvp_fwd_f32 -- fp32 I/O, fp32 arithmetic (CUDA-core kernel), for the
  * accuracy-critical configuration.  Same math, layout and error rules as
  * attn_jvp_fwd, with float tensors.  Supported: 1 <= d <= 256; pointers

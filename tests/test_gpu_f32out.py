@@ -1,0 +1,99 @@
+"""attn_jvp_fwd_f32out (bf16 inputs, fp32 outputs, split-bf16 probability
+operands) against the fp64 oracle.
+
+Bound on max|err| / max|ref| for O and tO: 1e-4 * max(1, Lk / 8192).  The
+1e-4 is the fp32 bound; the factor models the error of fp32 accumulation in
+tensor memory, which grows with the number of accumulation steps into one
+accumulator (Lk / 16 MMA K-steps).  lse: 1e-5.  Also: the variant's errors
+must sit at least 10x below those of the bf16-output entry point on the same
+inputs (the point of the variant: BF16 JVP error is much larger than BF16
+output error)."""
+import numpy as np
+import pytest
+import torch
+
+import attention_forward_mode_b200 as ajvp
+import oracle
+from attention_forward_mode_b200.workloads import WORKLOADS, custom, sample_rows
+from gpu_common import compare_full, gpu_inputs, max_rel
+
+pytestmark = pytest.mark.gpu
+
+
+def tol(Lk):
+    t = 1e-4 * max(1.0, Lk / 8192.0)
+    return {"o": t, "to": t, "lse": 1e-5}
+
+
+def run_f32out(inp, scale):
+    out = ajvp.attn_jvp_fwd_f32out(inp["q"], inp["k"], inp["v"], inp["tq"], inp["tk"], inp["tv"], scale)
+    torch.cuda.synchronize()
+    assert out[0].dtype == torch.float32 and out[1].dtype == torch.float32
+    return out
+
+
+def check(err, what, Lk):
+    bound = tol(Lk)
+    for key in ("o", "to", "lse"):
+        assert err[key] <= bound[key], f"{what}: {key} max-rel error {err[key]:.3e} > {bound[key]:.1e} ({err})"
+
+
+@pytest.mark.parametrize("B,H,Lq,Lk", [(1, 1, 1, 1), (1, 2, 129, 127), (2, 3, 300, 700), (1, 1, 257, 4097)])
+def test_shapes_full(B, H, Lq, Lk):
+    w = custom(B, H, Lq, Lk, 128)
+    inp = gpu_inputs(w, seed=Lq + Lk)
+    err = compare_full(w, inp, run_f32out(inp, w.scale))
+    print(w.name, err)
+    check(err, w.name, Lk)
+
+
+@pytest.mark.parametrize("name", ["image_selfattn_b2h12_l4096_d128", "video_selfattn_b1h12_l32760_d128",
+                                  "video_crossattn_b1h40_lq32760_lk512_d128",
+                                  "video_selfattn_large_b1h40_l75600_d128"])
+def test_workloads_sampled(name):
+    w = WORKLOADS[name]
+    inp = gpu_inputs(w)
+    out = run_f32out(inp, w.scale)
+    bh = w.B * w.H
+    heads = sorted({0, bh // 2, bh - 1})
+    rows = sample_rows(w.Lq, 24)
+    idx = torch.tensor(rows, device="cuda")
+    fl = {n: t.reshape(-1, t.shape[-2], t.shape[-1]) for n, t in inp.items()}
+    got = [[], [], []]
+    ref = [[], [], []]
+    for h in heads:
+        q = fl["q"][h].index_select(0, idx).cpu()
+        tq = fl["tq"][h].index_select(0, idx).cpu()
+        k, v, tk, tv = (fl[n][h].cpu() for n in ("k", "v", "tk", "tv"))
+        r = oracle.attn_jvp(q[None], k[None], v[None], tq[None], tk[None], tv[None], w.scale)
+        for i in range(3):
+            ref[i].append(r[i][0])
+        got[0].append(out[0].reshape(-1, w.Lq, w.d)[h].index_select(0, idx).cpu().numpy())
+        got[1].append(out[1].reshape(-1, w.Lq, w.d)[h].index_select(0, idx).cpu().numpy())
+        got[2].append(out[2].reshape(-1, w.Lq)[h].index_select(0, idx).cpu().numpy())
+    err = {k: max_rel(np.stack(got[i]), np.stack(ref[i])) for i, k in enumerate(("o", "to", "lse"))}
+    print(name, err)
+    check(err, name, w.Lk)
+    del inp, out
+    torch.cuda.empty_cache()
+
+
+def test_tangent_error_far_below_bf16_path():
+    w = custom(1, 4, 640, 2048, 128)
+    inp = gpu_inputs(w, seed=21)
+    e32 = compare_full(w, inp, run_f32out(inp, w.scale))
+    o, to, lse = ajvp.attn_jvp_fwd(inp["q"], inp["k"], inp["v"], inp["tq"], inp["tk"], inp["tv"], w.scale)
+    torch.cuda.synchronize()
+    e16 = compare_full(w, inp, (o, to, lse))
+    print("f32out", e32, "bf16", e16)
+    assert e32["to"] * 10 <= e16["to"]
+    assert e32["o"] * 10 <= e16["o"]
+
+
+def test_zero_tangent_exact_zero():
+    w = custom(1, 2, 200, 300, 128)
+    inp = gpu_inputs(w, seed=2)
+    for n in ("tq", "tk", "tv"):
+        inp[n].zero_()
+    _, to, _ = run_f32out(inp, w.scale)
+    assert torch.count_nonzero(to).item() == 0
