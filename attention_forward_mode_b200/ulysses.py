@@ -1,0 +1,81 @@
+"""Ulysses context parallelism for the attention + JVP forward pass.
+
+rCM (anthology record LIT-783, §3.2 / App. C) runs its FlashAttention-2 JVP
+kernel under Ulysses context parallelism, with the tangents distributed like
+Q, K and V.  Each rank holds a sequence shard of every head:
+
+    q, tq        [B, H, Lq / P, d]      k, v, tk, tv  [B, H, Lk / P, d]
+
+An all-to-all turns that into full sequences for H / P heads per rank, the
+local fused kernel runs on them, and a second all-to-all returns O, tO and
+lse to sequence shards:
+
+    o, to        [B, H, Lq / P, d]      lse           [B, H, Lq / P]
+
+Rank r's sequence shard is rows r*L/P .. (r+1)*L/P - 1; rank r computes
+heads r*H/P .. (r+1)*H/P - 1.  H, Lq and Lk must divide by P.  The Q-side
+tensors (q, tq) and the K-side tensors (k, v, tk, tv) each travel in one
+packed all-to-all, the outputs in one more (plus one for lse).  The exchange
+uses torch.distributed (NCCL on GPUs); the attention itself is the library's
+kernel (``local_fn``, by default the C ABI entry point for the inputs'
+dtype).
+"""
+from __future__ import annotations
+
+import torch
+import torch.distributed as dist
+
+from ._binding import attn_jvp
+
+
+def _to_heads(x: torch.Tensor, world: int, group) -> torch.Tensor:
+    """[n, B, H, Ls, d] sequence shard -> [n, B, H/P, P*Ls, d] head shard."""
+    n, B, H, Ls, d = x.shape
+    hp = H // world
+    # [n, B, P, H/P, Ls, d] -> [P, n, B, H/P, Ls, d]: chunk p goes to rank p
+    send = x.reshape(n, B, world, hp, Ls, d).permute(2, 0, 1, 3, 4, 5).contiguous()
+    recv = torch.empty_like(send)
+    dist.all_to_all_single(recv, send, group=group)
+    # recv[p] = rank p's sequence rows for my heads -> [n, B, H/P, P, Ls, d]
+    return recv.permute(1, 2, 3, 0, 4, 5).reshape(n, B, hp, world * Ls, d)
+
+
+def _to_sequence(y: torch.Tensor, world: int, group) -> torch.Tensor:
+    """[n, B, H/P, P*Ls, e] head shard -> [n, B, H, Ls, e] sequence shard."""
+    n, B, hp, L, e = y.shape
+    Ls = L // world
+    # [n, B, H/P, P, Ls, e] -> [P, n, B, H/P, Ls, e]: sequence chunk p goes to rank p
+    send = y.reshape(n, B, hp, world, Ls, e).permute(3, 0, 1, 2, 4, 5).contiguous()
+    recv = torch.empty_like(send)
+    dist.all_to_all_single(recv, send, group=group)
+    # recv[p] = my sequence rows of rank p's heads -> [n, B, P, H/P, Ls, e]
+    return recv.permute(1, 2, 0, 3, 4, 5).reshape(n, B, world * hp, Ls, e)
+
+
+def ulysses_attn_jvp(q, k, v, tq, tk, tv, scale=None, group=None, local_fn=None):
+    """O, tO, lse for sequence-sharded inputs (see the module docstring).
+
+    ``local_fn(q, k, v, tq, tk, tv, scale) -> (o, to, lse)`` computes the
+    attention JVP of the gathered head shard; it defaults to the CUDA kernel
+    (``attn_jvp``).  Collective calls are made in the same order on every rank.
+    """
+    grouped = dist.is_initialized()
+    world = dist.get_world_size(group) if grouped else 1
+    B, H, Lqs, d = q.shape
+    Lks = k.shape[2]
+    if H % world != 0:
+        raise ValueError(f"heads ({H}) must divide by the group size ({world})")
+    if scale is None:
+        scale = d ** -0.5
+    fn = local_fn if local_fn is not None else attn_jvp
+    if not grouped:  # no process group: the plain local call
+        return fn(q, k, v, tq, tk, tv, scale)
+
+    qs = _to_heads(torch.stack((q, tq)), world, group)        # [2, B, H/P, Lq, d]
+    ks = _to_heads(torch.stack((k, v, tk, tv)), world, group)  # [4, B, H/P, Lk, d]
+    o, to, lse = fn(qs[0].contiguous(), ks[0].contiguous(), ks[1].contiguous(), qs[1].contiguous(),
+                    ks[2].contiguous(), ks[3].contiguous(), scale)
+    out = _to_sequence(torch.stack((o, to)), world, group)      # [2, B, H, Lq/P, d]
+    lse_s = _to_sequence(lse.unsqueeze(0).unsqueeze(-1).contiguous(), world, group)[0, ..., 0]
+    assert out.shape[3] == Lqs and ks.shape[3] == Lks * world
+    return out[0], out[1], lse_s

@@ -1,0 +1,37 @@
+"""The Ulysses wrapper on the GPU through NCCL: with a one-rank NCCL group the
+two all-to-all exchanges run for real (as identity exchanges) around the CUDA
+kernel, and the result must equal a direct attn_jvp_fwd call bit for bit.
+(Exchanges across several ranks are checked on CPU over gloo.)"""
+import datetime
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+
+import attention_forward_mode_b200 as ajvp
+from attention_forward_mode_b200.ulysses import ulysses_attn_jvp
+from attention_forward_mode_b200.workloads import custom, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+def test_one_rank_nccl_equals_direct_call():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    store = dist.TCPStore("127.0.0.1", port, 1, True, timeout=datetime.timedelta(seconds=60))
+    dist.init_process_group("nccl", store=store, rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=60), device_id=torch.device("cuda", 0))
+    try:
+        w = custom(1, 4, 384, 640, 128)
+        inp = make_inputs(w, seed=3, device="cuda")
+        a = ulysses_attn_jvp(inp["q"], inp["k"], inp["v"], inp["tq"], inp["tk"], inp["tv"], scale=w.scale)
+        b = ajvp.attn_jvp_fwd(inp["q"], inp["k"], inp["v"], inp["tq"], inp["tk"], inp["tv"], w.scale)
+        torch.cuda.synchronize()
+        for x, y in zip(a, b):
+            assert torch.equal(x, y)
+    finally:
+        dist.destroy_process_group()

@@ -1,0 +1,97 @@
+"""Ulysses context parallelism (sequence-sharded Q, K, V and tangents, all-to-all
+to head shards and back) on CPU ranks over gloo.  The local attention is the
+fp64 oracle, so the sharded result must equal the oracle on the unsharded
+tensors exactly: this checks the layout logic of the two exchanges."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _inputs(B, H, Lq, Lk, d, seed):
+    g = torch.Generator().manual_seed(seed)
+    shp_q, shp_k = (B, H, Lq, d), (B, H, Lk, d)
+    return {n: torch.randn(shp_q if n in ("q", "tq") else shp_k, generator=g, dtype=torch.float64)
+            for n in ("q", "k", "v", "tq", "tk", "tv")}
+
+
+def _oracle_fn(q, k, v, tq, tk, tv, scale):
+    import oracle
+    return tuple(torch.from_numpy(x) for x in oracle.attn_jvp(q, k, v, tq, tk, tv, scale))
+
+
+def _worker(rank, world, port, shape, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from attention_forward_mode_b200.ulysses import ulysses_attn_jvp
+        B, H, Lq, Lk, d = shape
+        full = _inputs(B, H, Lq, Lk, d, seed=7)
+        sq, sk = Lq // world, Lk // world
+        shard = {n: (t[:, :, rank * sq:(rank + 1) * sq] if n in ("q", "tq") else t[:, :, rank * sk:(rank + 1) * sk])
+                 .contiguous() for n, t in full.items()}
+        o, to, lse = ulysses_attn_jvp(shard["q"], shard["k"], shard["v"], shard["tq"], shard["tk"], shard["tv"],
+                                      scale=0.3, local_fn=_oracle_fn)
+        ro, rto, rlse = _oracle_fn(*(full[n] for n in ("q", "k", "v", "tq", "tk", "tv")), 0.3)
+        sl = slice(rank * sq, (rank + 1) * sq)
+        out[rank] = (bool(torch.equal(o, ro[:, :, sl])), bool(torch.equal(to, rto[:, :, sl])),
+                     bool(torch.equal(lse, rlse[:, :, sl])), tuple(o.shape), tuple(lse.shape))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.timeout(240)
+@pytest.mark.parametrize("world,shape", [(2, (1, 4, 24, 24, 8)),     # self-attention
+                                         (2, (2, 2, 16, 40, 4)),     # cross-attention, Lq != Lk
+                                         (4, (1, 8, 32, 20, 8))])    # four ranks
+def test_ulysses_matches_unsharded(world, shape):
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as m:
+        out = m.dict()
+        procs = [ctx.Process(target=_worker, args=(r, world, port, shape, out)) for r in range(world)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(200)
+        assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
+        res = dict(out)
+    B, H, Lq, Lk, d = shape
+    for r in range(world):
+        eq_o, eq_to, eq_lse, oshape, lshape = res[r]
+        assert oshape == (B, H, Lq // world, d) and lshape == (B, H, Lq // world)
+        assert eq_o and eq_to and eq_lse, res[r]
+
+
+def test_single_rank_is_the_local_call():
+    from attention_forward_mode_b200.ulysses import ulysses_attn_jvp
+    t = _inputs(1, 2, 8, 8, 4, seed=1)
+    a = ulysses_attn_jvp(t["q"], t["k"], t["v"], t["tq"], t["tk"], t["tv"], scale=0.5, local_fn=_oracle_fn)
+    b = _oracle_fn(t["q"], t["k"], t["v"], t["tq"], t["tk"], t["tv"], 0.5)
+    for x, y in zip(a, b):
+        assert np.array_equal(x.numpy(), y.numpy())
+
+
+def test_heads_must_divide():
+    from attention_forward_mode_b200 import ulysses
+    t = _inputs(1, 3, 8, 8, 4, seed=1)
+    orig = ulysses.dist.is_initialized, ulysses.dist.get_world_size
+    ulysses.dist.is_initialized = lambda: True
+    ulysses.dist.get_world_size = lambda group=None: 2
+    try:
+        with pytest.raises(ValueError):
+            ulysses.ulysses_attn_jvp(t["q"], t["k"], t["v"], t["tq"], t["tk"], t["tv"], local_fn=_oracle_fn)
+    finally:
+        ulysses.dist.is_initialized, ulysses.dist.get_world_size = orig
