@@ -16,13 +16,17 @@ from ._binding import (  # noqa: F401
     AJVP_ERR_TOO_LARGE,
     AJVP_ERR_UNSUPPORTED_DEVICE,
     AJVP_ERR_UNSUPPORTED_DIM,
+    AJVP_ERR_WORKSPACE,
     AJVP_OK,
     AttnJvpError,
     attn_jvp,
     attn_jvp_fwd,
     attn_jvp_fwd_f32,
     attn_jvp_fwd_f32out,
+    attn_jvp_fwd_host,
     check_device_status,
+    default_heads_per_chunk,
+    host_workspace_bytes,
     load_library,
     selftest_wait_timeout,
     set_wait_bound_ns,
@@ -31,6 +35,7 @@ from ._binding import (  # noqa: F401
 )
 
 __all__ = [
-    "attn_jvp", "attn_jvp_fwd", "attn_jvp_fwd_f32", "attn_jvp_fwd_f32out", "check_device_status", "load_library",
+    "attn_jvp", "attn_jvp_fwd", "attn_jvp_fwd_f32", "attn_jvp_fwd_f32out", "attn_jvp_fwd_host", "check_device_status",
+    "default_heads_per_chunk", "host_workspace_bytes", "load_library",
     "selftest_wait_timeout", "set_wait_bound_ns", "strerror", "version", "AttnJvpError",
 ]

@@ -6,6 +6,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdint>
@@ -181,6 +182,61 @@ int launch_sm100(const void *q, const void *k, const void *v, const void *tq, co
     return AJVP_OK;
 }
 
+// ---------------------------------------------------------- host pipeline
+// One staging buffer holds, for `nh` (batch, head) slabs, the six bf16 inputs,
+// the two bf16 outputs and lse, each array 256-byte aligned.
+constexpr uint64_t kStageAlign = 256;
+uint64_t round_up(uint64_t x) { return (x + kStageAlign - 1) / kStageAlign * kStageAlign; }
+
+struct StageLayout {
+    uint64_t q, tq, k, v, tk, tv, o, to, lse, bytes;  // offsets inside one buffer
+};
+
+StageLayout stage_layout(int64_t Lq, int64_t Lk, int64_t d, int64_t nh) {
+    StageLayout s;
+    const uint64_t qb = round_up((uint64_t)(nh * Lq * d * 2)), kb = round_up((uint64_t)(nh * Lk * d * 2));
+    const uint64_t lb = round_up((uint64_t)(nh * Lq * 4));
+    s.q = 0;
+    s.tq = s.q + qb;
+    s.k = s.tq + qb;
+    s.v = s.k + kb;
+    s.tk = s.v + kb;
+    s.tv = s.tk + kb;
+    s.o = s.tv + kb;
+    s.to = s.o + qb;
+    s.lse = s.to + qb;
+    s.bytes = s.lse + lb;
+    return s;
+}
+
+// Streams and events of one attn_jvp_fwd_host call, released on scope exit
+// (the driver defers the release of objects with work still pending).
+// Chunk c uses staging buffer c % kBuffers and compute stream 1 + c % 2, so
+// consecutive chunk kernels may overlap (the next one fills the SMs the
+// previous one's last wave leaves idle).
+constexpr int kBuffers = 3;
+struct HostPipe {
+    cudaStream_t st[4] = {nullptr, nullptr, nullptr, nullptr};  // copy in, compute x2, copy out
+    cudaEvent_t ev[1 + 3 * kBuffers] = {};                      // start, then in / comp / out per buffer
+    cudaEvent_t &start() { return ev[0]; }
+    cudaEvent_t &in(int b) { return ev[1 + b]; }
+    cudaEvent_t &comp(int b) { return ev[1 + kBuffers + b]; }
+    cudaEvent_t &out(int b) { return ev[1 + 2 * kBuffers + b]; }
+    cudaError_t create() {
+        cudaError_t e = cudaSuccess;
+        for (int i = 0; i < 4 && e == cudaSuccess; ++i) e = cudaStreamCreateWithFlags(&st[i], cudaStreamNonBlocking);
+        for (int i = 0; i < 1 + 3 * kBuffers && e == cudaSuccess; ++i)
+            e = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming);
+        return e;
+    }
+    ~HostPipe() {
+        for (cudaStream_t s : st)
+            if (s) cudaStreamDestroy(s);
+        for (cudaEvent_t x : ev)
+            if (x) cudaEventDestroy(x);
+    }
+};
+
 }  // namespace
 
 extern "C" {
@@ -195,6 +251,82 @@ int attn_jvp_fwd_f32out(const void *q, const void *k, const void *v, const void 
                         const void *tv, float *o, float *to, float *lse, int64_t B, int64_t H, int64_t Lq,
                         int64_t Lk, int64_t d, float scale, void *stream) {
     return launch_sm100<true>(q, k, v, tq, tk, tv, o, to, lse, B, H, Lq, Lk, d, scale, stream);
+}
+
+uint64_t attn_jvp_host_workspace_bytes(int64_t Lq, int64_t Lk, int64_t d, int64_t heads_per_chunk) {
+    if (Lq < 1 || Lk < 1 || d < 1 || heads_per_chunk < 1) return 0;
+    return kBuffers * stage_layout(Lq, Lk, d, heads_per_chunk).bytes;
+}
+
+int attn_jvp_fwd_host(const void *q, const void *k, const void *v, const void *tq, const void *tk, const void *tv,
+                      void *o, void *to, float *lse, int64_t B, int64_t H, int64_t Lq, int64_t Lk, int64_t d,
+                      float scale, void *workspace, uint64_t workspace_bytes, void *stream) {
+    bool noop = false;
+    int rc = check_common(q, k, v, tq, tk, tv, o, to, B, H, Lq, Lk, d, scale, &noop);
+    if (rc != AJVP_OK || noop) return rc;
+    if (d != ajvp::sm100::HD) return AJVP_ERR_UNSUPPORTED_DIM;
+    const int64_t BH = B * H;
+    const uint64_t one = stage_layout(Lq, Lk, d, 1).bytes;
+    if (!workspace || !aligned(workspace, kStageAlign) || workspace_bytes < kBuffers * one) return AJVP_ERR_WORKSPACE;
+    // heads per chunk: as many as the workspace holds, at most a quarter of B*H
+    int64_t nh = std::min<int64_t>((int64_t)(workspace_bytes / (kBuffers * one)), (BH + 3) / 4);
+    while (nh > 1 && kBuffers * stage_layout(Lq, Lk, d, nh).bytes > workspace_bytes) --nh;
+    nh = std::max<int64_t>(nh, 1);
+    const StageLayout L = stage_layout(Lq, Lk, d, nh);
+    int dev = 0;
+    if ((rc = device_setup(&dev)) != AJVP_OK) return rc;
+
+    HostPipe pipe;
+    cudaError_t e = pipe.create();
+    if (e != cudaSuccess) return fail_cuda(e);
+    const cudaStream_t caller = (cudaStream_t)stream;
+    if ((e = cudaEventRecord(pipe.start(), caller)) != cudaSuccess) return fail_cuda(e);
+    for (cudaStream_t s : pipe.st)
+        if ((e = cudaStreamWaitEvent(s, pipe.start(), 0)) != cudaSuccess) return fail_cuda(e);
+
+    const uint64_t qrow = (uint64_t)(Lq * d * 2), krow = (uint64_t)(Lk * d * 2);  // bytes per (b, h) slab
+    const int64_t nchunks = (BH + nh - 1) / nh;
+    const void *src[6] = {q, tq, k, v, tk, tv};
+    const uint64_t dst_off[6] = {L.q, L.tq, L.k, L.v, L.tk, L.tv};
+    for (int64_t c = 0; c < nchunks; ++c) {
+        const int b = (int)(c % kBuffers);
+        const int64_t h0 = c * nh, n = std::min<int64_t>(nh, BH - h0);
+        uint8_t *buf = static_cast<uint8_t *>(workspace) + (uint64_t)b * L.bytes;
+        // copy in, once the chunk that last used this buffer has been copied out
+        if (c >= kBuffers && (e = cudaStreamWaitEvent(pipe.st[0], pipe.out(b), 0)) != cudaSuccess)
+            return fail_cuda(e);
+        for (int t = 0; t < 6; ++t) {
+            const uint64_t row = t < 2 ? qrow : krow;
+            e = cudaMemcpyAsync(buf + dst_off[t], static_cast<const uint8_t *>(src[t]) + (uint64_t)h0 * row,
+                                (uint64_t)n * row, cudaMemcpyHostToDevice, pipe.st[0]);
+            if (e != cudaSuccess) return fail_cuda(e);
+        }
+        if ((e = cudaEventRecord(pipe.in(b), pipe.st[0])) != cudaSuccess) return fail_cuda(e);
+        // compute
+        const cudaStream_t cs = pipe.st[1 + (c & 1)];
+        if ((e = cudaStreamWaitEvent(cs, pipe.in(b), 0)) != cudaSuccess) return fail_cuda(e);
+        rc = launch_sm100<false>(buf + L.q, buf + L.k, buf + L.v, buf + L.tq, buf + L.tk, buf + L.tv, buf + L.o,
+                                 buf + L.to, lse ? reinterpret_cast<float *>(buf + L.lse) : nullptr, 1, n, Lq, Lk,
+                                 d, scale, cs);
+        if (rc != AJVP_OK) return rc;
+        if ((e = cudaEventRecord(pipe.comp(b), cs)) != cudaSuccess) return fail_cuda(e);
+        // copy out (in chunk order on one stream)
+        if ((e = cudaStreamWaitEvent(pipe.st[3], pipe.comp(b), 0)) != cudaSuccess) return fail_cuda(e);
+        e = cudaMemcpyAsync(static_cast<uint8_t *>(o) + (uint64_t)h0 * qrow, buf + L.o, (uint64_t)n * qrow,
+                            cudaMemcpyDeviceToHost, pipe.st[3]);
+        if (e == cudaSuccess)
+            e = cudaMemcpyAsync(static_cast<uint8_t *>(to) + (uint64_t)h0 * qrow, buf + L.to, (uint64_t)n * qrow,
+                                cudaMemcpyDeviceToHost, pipe.st[3]);
+        if (e == cudaSuccess && lse)
+            e = cudaMemcpyAsync(lse + h0 * Lq, buf + L.lse, (uint64_t)(n * Lq * 4), cudaMemcpyDeviceToHost,
+                                pipe.st[3]);
+        if (e != cudaSuccess) return fail_cuda(e);
+        if ((e = cudaEventRecord(pipe.out(b), pipe.st[3])) != cudaSuccess) return fail_cuda(e);
+    }
+    // the caller's stream continues once the last chunk (and so every chunk) is copied out
+    if ((e = cudaStreamWaitEvent(caller, pipe.out((int)((nchunks - 1) % kBuffers)), 0)) != cudaSuccess)
+        return fail_cuda(e);
+    return AJVP_OK;
 }
 
 int attn_jvp_fwd_f32(const float *q, const float *k, const float *v, const float *tq, const float *tk,
@@ -232,6 +364,7 @@ const char *attn_jvp_strerror(int status) {
         case AJVP_ERR_TIMEOUT: return "a kernel wait ran past its bound";
         case AJVP_ERR_CUDA: return "CUDA runtime or driver error";
         case AJVP_ERR_TOO_LARGE: return "a size exceeds the supported maximum";
+        case AJVP_ERR_WORKSPACE: return "device workspace missing, not 256-byte aligned or too small";
         default: return "unknown status";
     }
 }

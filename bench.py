@@ -307,14 +307,28 @@ def run_ours(args, w):
     h2d = sum(t.numel() * t.element_size() for t in host_in.values())
     d2h = sum(t.numel() * t.element_size() for t in (host_o, host_to, host_lse))
 
-    def e2e_step():
-        for n in inp:
-            inp[n].copy_(host_in[n], non_blocking=True)
-        fwd(inp["q"], inp["k"], inp["v"], inp["tq"], inp["tk"], inp["tv"], w.scale,
-                          o=o, to=to, lse=lse, stream=stream)
-        host_o.copy_(o, non_blocking=True)
-        host_to.copy_(to, non_blocking=True)
-        host_lse.copy_(lse, non_blocking=True)
+    if args.entry == "bf16":
+        # the library's host-buffer entry point: head chunks staged through a
+        # device workspace, copies in and out overlapped with the kernel
+        nh = ajvp.default_heads_per_chunk(w.B * w.H, w.Lq, w.Lk, w.d)
+        ws = torch.empty(ajvp.host_workspace_bytes(w.Lq, w.Lk, w.d, nh), dtype=torch.uint8, device=dev)
+        e2e_path = f"attn_jvp_fwd_host (pipelined, chunks of {nh} head(s))"
+
+        def e2e_step():
+            ajvp.attn_jvp_fwd_host(host_in["q"], host_in["k"], host_in["v"], host_in["tq"], host_in["tk"],
+                                   host_in["tv"], w.scale, o=host_o, to=host_to, lse=host_lse, workspace=ws,
+                                   stream=stream)
+    else:
+        e2e_path = "copy in, attn_jvp_fwd_f32out, copy out (serial on one stream)"
+
+        def e2e_step():
+            for n in inp:
+                inp[n].copy_(host_in[n], non_blocking=True)
+            fwd(inp["q"], inp["k"], inp["v"], inp["tq"], inp["tk"], inp["tv"], w.scale,
+                o=o, to=to, lse=lse, stream=stream)
+            host_o.copy_(o, non_blocking=True)
+            host_to.copy_(to, non_blocking=True)
+            host_lse.copy_(lse, non_blocking=True)
 
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
     e2e_step()
@@ -347,7 +361,8 @@ def run_ours(args, w):
                              "kernel": "attn_jvp_fwd_kernel", "algorithmic_flops_per_launch": w.flops,
                              "algorithmic_bytes_per_launch": w.io_bytes},
                 "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-                        "d2h_bytes_per_step": d2h, "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps},
+                        "d2h_bytes_per_step": d2h, "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps,
+                        "path": e2e_path},
                 "gpu_launches": args.steps,
                 "clocks": clk}
         # CPU oracle next to the kernel: rank 0 at N = 1 only

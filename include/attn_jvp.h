@@ -26,7 +26,8 @@
  * distributes the QKV tangents like QKV).  lse is [B][H][Lq] fp32.
  *
  * Ownership and execution: all pointers are DEVICE pointers owned by the
- * caller.  The library allocates no device memory per call and keeps no
+ * caller (except the data pointers of attn_jvp_fwd_host, which are host
+ * pointers).  The library allocates no device memory per call and keeps no
  * per-call state.  Calls are stream-ordered and asynchronous: they return
  * after enqueueing work on `stream` (a cudaStream_t; NULL = legacy default
  * stream) and do not synchronise.  Calls are thread-safe.  Inputs must not
@@ -64,7 +65,8 @@ typedef enum {
     AJVP_ERR_UNSUPPORTED_DEVICE = -4, /* current device is not compute capability 10.0 */
     AJVP_ERR_TIMEOUT = -5,            /* a kernel wait ran past its bound (device status word) */
     AJVP_ERR_CUDA = -6,               /* a CUDA runtime/driver call failed */
-    AJVP_ERR_TOO_LARGE = -7           /* a size exceeds the documented maximum */
+    AJVP_ERR_TOO_LARGE = -7,          /* a size exceeds the documented maximum */
+    AJVP_ERR_WORKSPACE = -8           /* workspace missing, misaligned or too small */
 } ajvp_status;
 
 /*
@@ -121,6 +123,46 @@ AJVP_API int attn_jvp_fwd_f32(const float *q, const float *k, const float *v,
                      float *o, float *to, float *lse,
                      int64_t B, int64_t H, int64_t Lq, int64_t Lk, int64_t d,
                      float scale, void *stream);
+
+/*
+ * attn_jvp_fwd_host -- the attn_jvp_fwd computation on HOST buffers.
+ *
+ *   q, k, v, tq, tk, tv : host __nv_bfloat16 arrays, layouts as attn_jvp_fwd
+ *   o, to               : host __nv_bfloat16 [B][H][Lq][d] (written)
+ *   lse                 : host float [B][H][Lq], or NULL
+ *   workspace           : DEVICE memory owned by the caller, 256-byte aligned,
+ *                         at least attn_jvp_host_workspace_bytes(Lq, Lk, d, 1)
+ *   workspace_bytes     : its size
+ *
+ * The (batch, head) slabs are processed in chunks of consecutive heads: while
+ * the kernel runs on one chunk, the next chunk's inputs are copied in and the
+ * previous chunk's outputs copied out (three staging buffers in the
+ * workspace used in turn; four internal streams: copy in, two compute
+ * streams taken in turn so that consecutive chunk kernels may overlap, copy
+ * out).  Chunk size: as many heads as three buffers in the workspace hold, at
+ * most a quarter of B*H (rounded up).
+ * Host buffers should be page-locked; pageable memory works but copies then
+ * do not overlap.  Stream-ordered on `stream` like attn_jvp_fwd: the work
+ * starts after what is already queued on `stream`, and work queued on
+ * `stream` afterwards (e.g. a synchronisation) sees the host outputs written.
+ * The internal streams and events are created and released per call, so the
+ * call must not be made while `stream` is being captured into a CUDA graph.
+ * Same size, device and error rules as attn_jvp_fwd, plus AJVP_ERR_WORKSPACE.
+ */
+AJVP_API int attn_jvp_fwd_host(const void *q, const void *k, const void *v,
+                      const void *tq, const void *tk, const void *tv,
+                      void *o, void *to, float *lse,
+                      int64_t B, int64_t H, int64_t Lq, int64_t Lk, int64_t d,
+                      float scale, void *workspace, uint64_t workspace_bytes,
+                      void *stream);
+
+/*
+ * Device workspace, in bytes, that attn_jvp_fwd_host needs to stage chunks
+ * of `heads_per_chunk` (batch, head) slabs (three staging buffers, every
+ * array 256-byte aligned).  Returns 0 for invalid sizes.
+ */
+AJVP_API uint64_t attn_jvp_host_workspace_bytes(int64_t Lq, int64_t Lk, int64_t d,
+                                       int64_t heads_per_chunk);
 
 /* Static, human-readable description of an ajvp_status value. */
 AJVP_API const char *attn_jvp_strerror(int status);

@@ -36,7 +36,7 @@ def test_every_header_symbol_exported(lib):
 
 def test_version_and_strerror(lib):
     assert lib.attn_jvp_version() == 100
-    for code in range(-7, 1):
+    for code in range(-8, 1):
         assert len(lib.attn_jvp_strerror(code)) > 5
     assert b"unknown" in lib.attn_jvp_strerror(-99)
 
@@ -70,6 +70,35 @@ def test_bf16_dim_and_alignment_rules(lib):
     assert _call(lib, d=256) == B.AJVP_ERR_UNSUPPORTED_DIM
     assert _call(lib, ptr=24) == B.AJVP_ERR_MISALIGNED
     assert _call(lib, lse=ctypes.c_void_p(20)) == B.AJVP_ERR_MISALIGNED
+
+
+def _call_host(lib, ptr=16, Lq=8, Lk=8, d=128, ws=256, ws_bytes=None):
+    p = ctypes.c_void_p(ptr) if ptr is not None else None
+    w = ctypes.c_void_p(ws) if ws is not None else None
+    if ws_bytes is None:
+        ws_bytes = lib.attn_jvp_host_workspace_bytes(Lq, Lk, d, 1)
+    return lib.attn_jvp_fwd_host(p, p, p, p, p, p, p, p, None, 1, 1, Lq, Lk, d, 0.1, w, ws_bytes, None)
+
+
+def test_host_workspace_bytes(lib):
+    f = lib.attn_jvp_host_workspace_bytes
+    assert f(0, 8, 128, 1) == 0 and f(8, 8, 128, 0) == 0
+    # three buffers; per buffer 2 q-side + 4 k-side inputs, 2 outputs, lse, each rounded to 256 bytes
+    per = 4 * 8 * 128 * 2 + 4 * 16 * 128 * 2 + 256
+    assert f(8, 16, 128, 1) == 3 * per
+    assert f(8, 16, 128, 3) == 3 * (4 * 3 * 8 * 128 * 2 + 4 * 3 * 16 * 128 * 2 + 256)
+    assert f(1, 1, 128, 1) == 3 * 9 * 256  # every array padded to its own 256-byte boundary
+
+
+def test_host_entry_rejections(lib):
+    # host-side checks, before any CUDA call
+    assert _call_host(lib, Lk=0) == B.AJVP_ERR_INVALID_ARG
+    assert _call_host(lib, d=64) == B.AJVP_ERR_UNSUPPORTED_DIM
+    assert _call_host(lib, ws=None) == B.AJVP_ERR_WORKSPACE
+    assert _call_host(lib, ws=128) == B.AJVP_ERR_WORKSPACE  # not 256-byte aligned
+    need = lib.attn_jvp_host_workspace_bytes(8, 8, 128, 1)
+    assert _call_host(lib, ws_bytes=need - 1) == B.AJVP_ERR_WORKSPACE
+    assert _call_host(lib, ptr=None, Lq=0, ws=None) == B.AJVP_OK  # empty: no-op
 
 
 def test_f32_dim_and_alignment_rules(lib):
