@@ -28,7 +28,8 @@ AJVP_ERR_WORKSPACE = -8
 
 # every symbol the header declares
 EXPORTED = ("attn_jvp_fwd", "attn_jvp_fwd_f32out", "attn_jvp_fwd_f32", "attn_jvp_fwd_host",
-            "attn_jvp_host_workspace_bytes", "attn_jvp_strerror", "attn_jvp_last_cuda_error",
+            "attn_jvp_fwd_host_noalloc", "attn_jvp_host_workspace_bytes", "attn_jvp_strerror",
+            "attn_jvp_last_cuda_error",
             "attn_jvp_check_device_status", "attn_jvp_set_wait_bound_ns",
             "attn_jvp_selftest_wait_timeout", "attn_jvp_version")
 
@@ -62,6 +63,8 @@ def load_library(path: str = LIB_PATH):
         lib.attn_jvp_fwd_f32out.restype = ctypes.c_int
         lib.attn_jvp_fwd_host.argtypes = [vp] * 9 + [i64] * 5 + [f32, vp, ctypes.c_uint64, vp]
         lib.attn_jvp_fwd_host.restype = ctypes.c_int
+        lib.attn_jvp_fwd_host_noalloc.argtypes = fwd_args
+        lib.attn_jvp_fwd_host_noalloc.restype = ctypes.c_int
         lib.attn_jvp_host_workspace_bytes.argtypes = [i64] * 4
         lib.attn_jvp_host_workspace_bytes.restype = ctypes.c_uint64
         lib.attn_jvp_strerror.argtypes = [ctypes.c_int]
@@ -181,6 +184,31 @@ def host_workspace_bytes(Lq: int, Lk: int, d: int, heads_per_chunk: int = 1) -> 
     return int(load_library().attn_jvp_host_workspace_bytes(int(Lq), int(Lk), int(d), int(heads_per_chunk)))
 
 
+def _prepare_host(q, k, v, tq, tk, tv, o, to, lse, want_lse):
+    for name, x in (("q", q), ("k", k), ("v", v), ("tq", tq), ("tk", tk), ("tv", tv)):
+        if not isinstance(x, torch.Tensor) or x.is_cuda or x.dtype != torch.bfloat16 or x.dim() != 4 \
+                or not x.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous bf16 [B, H, L, d] host tensor")
+    B, H, Lq, d = q.shape
+    Lk = k.shape[2]
+    if tq.shape != q.shape or any(x.shape != (B, H, Lk, d) for x in (k, v, tk, tv)):
+        raise ValueError("q, tq must be [B, H, Lq, d] and k, v, tk, tv [B, H, Lk, d]")
+    pin = q.is_pinned()
+    if o is None:
+        o = torch.empty(q.shape, dtype=torch.bfloat16, pin_memory=pin)
+    if to is None:
+        to = torch.empty(q.shape, dtype=torch.bfloat16, pin_memory=pin)
+    if want_lse and lse is None:
+        lse = torch.empty((B, H, Lq), dtype=torch.float32, pin_memory=pin)
+    for name, x in (("o", o), ("to", to)):
+        if x.is_cuda or x.shape != q.shape or x.dtype != torch.bfloat16 or not x.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous bf16 host tensor of shape {tuple(q.shape)}")
+    if lse is not None and (lse.is_cuda or lse.shape != (B, H, Lq) or lse.dtype != torch.float32
+                            or not lse.is_contiguous()):
+        raise ValueError("lse must be a contiguous float32 [B, H, Lq] host tensor")
+    return o, to, lse, (B, H, Lq, Lk, d)
+
+
 def default_heads_per_chunk(bh: int, Lq: int, Lk: int, d: int, target_bytes: int = 64 << 20) -> int:
     """Heads per staged chunk: about ``target_bytes`` of inputs and outputs
     (enough to keep each copy long against its launch cost), at least one
@@ -230,6 +258,21 @@ def attn_jvp_fwd_host(q, k, v, tq, tk, tv, scale=None, o=None, to=None, lse=None
                                _ptr(lse), B, H, Lq, Lk, d, float(scale), _ptr(workspace), workspace.numel(),
                                _stream_handle(stream))
     _check(rc, "attn_jvp_fwd_host")
+    return o, to, lse
+
+
+def attn_jvp_fwd_host_noalloc(q, k, v, tq, tk, tv, scale=None, o=None, to=None, lse=None, stream=None,
+                              want_lse=True):
+    """``attn_jvp_fwd_host`` staged through the library's static 64 MiB device
+    scratch instead of a workspace (the C call allocates no device memory).
+    Calls on different streams must not overlap.  Asynchronous on ``stream``."""
+    o, to, lse, (B, H, Lq, Lk, d) = _prepare_host(q, k, v, tq, tk, tv, o, to, lse, want_lse)
+    if scale is None:
+        scale = d ** -0.5
+    lib = load_library()
+    rc = lib.attn_jvp_fwd_host_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(tq), _ptr(tk), _ptr(tv), _ptr(o), _ptr(to),
+                                       _ptr(lse), B, H, Lq, Lk, d, float(scale), _stream_handle(stream))
+    _check(rc, "attn_jvp_fwd_host_noalloc")
     return o, to, lse
 
 

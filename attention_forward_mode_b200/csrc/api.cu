@@ -424,3 +424,49 @@ extern "C" int attn_jvp_selftest_wait_timeout(uint64_t bound_ns, void *stream) {
     if (e != cudaSuccess) return fail_cuda(e);
     return AJVP_OK;
 }
+
+// ------------------------------------------- host entry on static scratch
+// attn_jvp_fwd_host_noalloc stages its chunks in this file-scope device
+// array instead of a caller-supplied workspace.  Its device address is looked
+// up once per device (that device current) on the entry point's first call
+// there.  Nothing in it needs to start at zero: every byte a kernel reads is
+// first written by the same call's copies.
+namespace {
+constexpr uint64_t kNoallocScratchBytes = 64ull << 20;  // 64 MiB per device
+struct NoallocState {
+    std::once_flag once;
+    void *ptr = nullptr;
+    int cuda_error = 0;
+};
+NoallocState g_noalloc[kMaxDevices];
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
+
+extern "C" int attn_jvp_fwd_host_noalloc(const void *q, const void *k, const void *v, const void *tq,
+                                         const void *tk, const void *tv, void *o, void *to, float *lse, int64_t B,
+                                         int64_t H, int64_t Lq, int64_t Lk, int64_t d, float scale, void *stream) {
+    bool noop = false;
+    int rc = check_common(q, k, v, tq, tk, tv, o, to, B, H, Lq, Lk, d, scale, &noop);
+    if (rc != AJVP_OK || noop) return rc;
+    if (d != ajvp::sm100::HD) return AJVP_ERR_UNSUPPORTED_DIM;
+    // one (batch, head) slab, three staging buffers, must fit the scratch
+    if (attn_jvp_host_workspace_bytes(Lq, Lk, d, 1) > kNoallocScratchBytes) return AJVP_ERR_TOO_LARGE;
+    int dev = 0;
+    if ((rc = device_setup(&dev)) != AJVP_OK) return rc;
+    NoallocState &st = g_noalloc[dev];
+    std::call_once(st.once, [&]() {
+        void *p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e == cudaSuccess)
+            st.ptr = p;
+        else
+            st.cuda_error = (int)e;
+    });
+    if (!st.ptr) {
+        t_last_cuda_error = st.cuda_error;
+        return AJVP_ERR_CUDA;
+    }
+    return attn_jvp_fwd_host(q, k, v, tq, tk, tv, o, to, lse, B, H, Lq, Lk, d, scale, st.ptr,
+                             kNoallocScratchBytes, stream);
+}

@@ -26,8 +26,8 @@
  * distributes the QKV tangents like QKV).  lse is [B][H][Lq] fp32.
  *
  * Ownership and execution: all pointers are DEVICE pointers owned by the
- * caller (except the data pointers of attn_jvp_fwd_host, which are host
- * pointers).  The library allocates no device memory per call and keeps no
+ * caller (except the data pointers of attn_jvp_fwd_host and
+ * attn_jvp_fwd_host_noalloc, which are host pointers).  The library allocates no device memory per call and keeps no
  * per-call state.  Calls are stream-ordered and asynchronous: they return
  * after enqueueing work on `stream` (a cudaStream_t; NULL = legacy default
  * stream) and do not synchronise.  Calls are thread-safe.  Inputs must not
@@ -163,6 +163,38 @@ AJVP_API int attn_jvp_fwd_host(const void *q, const void *k, const void *v,
  */
 AJVP_API uint64_t attn_jvp_host_workspace_bytes(int64_t Lq, int64_t Lk, int64_t d,
                                        int64_t heads_per_chunk);
+
+/*
+ * attn_jvp_fwd_host_noalloc -- attn_jvp_fwd_host without a caller-supplied
+ * workspace: the chunks are staged in a static device array of the library
+ * (64 MiB per device, reserved when the library's device code is loaded on
+ * that device).  The pages have no counterpart: it exists for callers that
+ * cannot hand the library device memory (see attn_jvp_fwd_host for the
+ * computation, layouts and the host-buffer contract).
+ *
+ *   q, k, v, tq, tk, tv : host __nv_bfloat16 arrays, layouts as attn_jvp_fwd
+ *   o, to               : host __nv_bfloat16 [B][H][Lq][d] (written)
+ *   lse                 : host float [B][H][Lq], or NULL
+ *
+ * Maximum size: one (batch, head) slab in three staging buffers must fit the
+ * 64 MiB, i.e. attn_jvp_host_workspace_bytes(Lq, Lk, d, 1) <= 67108864
+ * (for d = 128 about Lq + Lk <= 21800); larger sizes return
+ * AJVP_ERR_TOO_LARGE before anything is enqueued.  Chunks hold as many heads
+ * as fit, at most a quarter of B*H.
+ * Allocates nothing (no cudaMalloc, cudaFree or allocating library call).
+ * The first call on a device looks up the array's device address there
+ * (cudaGetSymbolAddress, with that device current); make that first call
+ * before any stream capture begins.  Nothing in the array needs to start at
+ * zero.  The array is shared by every call on the device: calls on one
+ * stream are ordered and safe, but calls on different streams (or from
+ * different threads) whose executions overlap race on it and give undefined
+ * results; serialise them.  Other rules as attn_jvp_fwd_host.
+ */
+AJVP_API int attn_jvp_fwd_host_noalloc(const void *q, const void *k, const void *v,
+                              const void *tq, const void *tk, const void *tv,
+                              void *o, void *to, float *lse,
+                              int64_t B, int64_t H, int64_t Lq, int64_t Lk, int64_t d,
+                              float scale, void *stream);
 
 /* Static, human-readable description of an ajvp_status value. */
 AJVP_API const char *attn_jvp_strerror(int status);
