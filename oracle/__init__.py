@@ -12,6 +12,11 @@ FlashAttention-2 forward with its JVP; the oracle is the plain definition --
 O = softmax(s Q K^T) V and tO = d/dt O(Q + t tQ, K + t tK, V + t tV) at t = 0,
 written as sum_j P_ij (dS_ij - mu_i) V_j + sum_j P_ij tV_j with
 dS = s (tQ K^T + Q tK^T) and mu_i = sum_j P_ij dS_ij, plus lse = ln sum_j exp(S_ij).
+
+``attn_jvp_bwd_oracle.c`` is the backward counterpart: the gradients of
+L = <dO, O> + <dtO, tO> with respect to Q, K, V, tQ, tK, tV, written as the
+chain rule through the forward definition's steps in reverse order (the pages
+describe the forward only; this is the plain definition of its gradient).
 """
 from __future__ import annotations
 
@@ -25,21 +30,30 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "attn_jvp_oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
+_BWD_SRC = os.path.join(_HERE, "attn_jvp_bwd_oracle.c")
+_BWD_LIB = os.path.join(_HERE, "liboracle_bwd.so")
 _lock = threading.Lock()
 _lib = None
+_bwd_lib = None
+
+
+def _compile(src: str, lib: str, force: bool) -> str:
+    if force or not os.path.exists(lib) or os.path.getmtime(lib) < os.path.getmtime(src):
+        tmp = lib + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+                               "-o", tmp, src, "-lm"])
+        os.replace(tmp, lib)
+    return lib
 
 
 def build(force: bool = False) -> str:
-    """Compile the oracle to ``oracle/liboracle.so`` (gcc, -O2, OpenMP).
+    """Compile the oracles to ``oracle/liboracle.so`` (forward) and
+    ``oracle/liboracle_bwd.so`` (backward) with gcc -O2 and OpenMP.
 
     No -ffast-math: the oracle keeps IEEE fp64 semantics.
     """
-    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
-        tmp = _LIB + f".tmp{os.getpid()}"
-        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
-                               "-o", tmp, _SRC, "-lm"])
-        os.replace(tmp, _LIB)
-    return _LIB
+    _compile(_BWD_SRC, _BWD_LIB, force)
+    return _compile(_SRC, _LIB, force)
 
 
 def compile_variant(src_text: str, out_path: str) -> str:
@@ -55,6 +69,11 @@ def compile_variant(src_text: str, out_path: str) -> str:
 
 def source_text() -> str:
     with open(_SRC) as f:
+        return f.read()
+
+
+def bwd_source_text() -> str:
+    with open(_BWD_SRC) as f:
         return f.read()
 
 
@@ -79,6 +98,30 @@ def _get():
 def load_variant(path: str):
     """ctypes handle of a separately compiled oracle build."""
     return _bind(path)
+
+
+def _bind_bwd(path: str):
+    lib = ctypes.CDLL(path)
+    dp = ctypes.POINTER(ctypes.c_double)
+    ip = ctypes.POINTER(ctypes.c_int64)
+    lib.oracle_attn_jvp_bwd_f64.argtypes = ([dp] * 14 + [ctypes.c_int64] * 4 + [ctypes.c_double]
+                                            + [ip, ctypes.c_int64, ip, ctypes.c_int64])
+    lib.oracle_attn_jvp_bwd_f64.restype = ctypes.c_int
+    return lib
+
+
+def _get_bwd():
+    global _bwd_lib
+    with _lock:
+        if _bwd_lib is None:
+            build()
+            _bwd_lib = _bind_bwd(_BWD_LIB)
+        return _bwd_lib
+
+
+def load_bwd_variant(path: str):
+    """ctypes handle of a separately compiled backward-oracle build."""
+    return _bind_bwd(path)
 
 
 def num_threads() -> int:
@@ -138,3 +181,41 @@ def attn_jvp_rows(q, k, v, tq, tk, tv, scale: float, heads, rows):
     to = np.concatenate([x[1] for x in outs])
     lse = np.concatenate([x[2] for x in outs])
     return o, to, lse
+
+
+def attn_jvp_bwd(q, k, v, tq, tk, tv, dout, dtout, scale: float, qrows=None, krows=None, lib=None):
+    """Gradients of L = <dout, O> + <dtout, tO> with respect to q, k, v, tq,
+    tk, tv (O, tO as ``attn_jvp`` defines them), in fp64.
+
+    Inputs [..., L, d] (leading dims = batch*heads; any float dtype, widened
+    exactly).  ``qrows`` / ``krows``: optional lists of query rows / keys whose
+    gradients are wanted (default: all); key-side sums always run over every
+    query row.  Returns a dict of fp64 numpy arrays: dq, dtq [..., nq, d] and
+    dk, dv, dtk, dtv [..., nk, d].
+    """
+    q, k, v, tq, tk, tv, dout, dtout = (_f64(x) for x in (q, k, v, tq, tk, tv, dout, dtout))
+    lead = q.shape[:-2]
+    Lq, d = q.shape[-2], q.shape[-1]
+    Lk = k.shape[-2]
+    for x, L in ((tq, Lq), (dout, Lq), (dtout, Lq), (k, Lk), (v, Lk), (tk, Lk), (tv, Lk)):
+        if x.shape != tuple(lead) + (L, d):
+            raise ValueError(f"shape mismatch: {x.shape} vs {tuple(lead) + (L, d)}")
+    BH = int(np.prod(lead)) if lead else 1
+    qr = None if qrows is None else np.ascontiguousarray(np.asarray(qrows, dtype=np.int64))
+    kr = None if krows is None else np.ascontiguousarray(np.asarray(krows, dtype=np.int64))
+    nq = Lq if qr is None else len(qr)
+    nk = Lk if kr is None else len(kr)
+    out = {n: np.zeros(tuple(lead) + (nq, d)) for n in ("dq", "dtq")}
+    out.update({n: np.zeros(tuple(lead) + (nk, d)) for n in ("dk", "dv", "dtk", "dtv")})
+    dp = ctypes.POINTER(ctypes.c_double)
+    ip = ctypes.POINTER(ctypes.c_int64)
+    ptr = lambda a: a.ctypes.data_as(dp)  # noqa: E731
+    iptr = lambda a: None if a is None else a.ctypes.data_as(ip)  # noqa: E731
+    handle = lib if lib is not None else _get_bwd()
+    rc = handle.oracle_attn_jvp_bwd_f64(ptr(q), ptr(k), ptr(v), ptr(tq), ptr(tk), ptr(tv), ptr(dout), ptr(dtout),
+                                        ptr(out["dq"]), ptr(out["dk"]), ptr(out["dv"]), ptr(out["dtq"]),
+                                        ptr(out["dtk"]), ptr(out["dtv"]), BH, Lq, Lk, d, float(scale),
+                                        iptr(qr), nq, iptr(kr), nk)
+    if rc != 0:
+        raise RuntimeError(f"oracle_attn_jvp_bwd_f64 failed with {rc}")
+    return out
