@@ -20,11 +20,14 @@ from ._binding import (  # noqa: F401
     AJVP_OK,
     AttnJvpError,
     attn_jvp,
+    attn_jvp_bwd,
     attn_jvp_fwd,
     attn_jvp_fwd_f32,
     attn_jvp_fwd_f32out,
     attn_jvp_fwd_host,
     attn_jvp_fwd_host_noalloc,
+    attn_jvp_fwd_stats,
+    bwd_workspace_bytes,
     check_device_status,
     default_heads_per_chunk,
     host_workspace_bytes,
@@ -36,7 +39,7 @@ from ._binding import (  # noqa: F401
 )
 
 __all__ = [
-    "attn_jvp", "attn_jvp_fwd", "attn_jvp_fwd_f32", "attn_jvp_fwd_f32out", "attn_jvp_fwd_host", "attn_jvp_fwd_host_noalloc", "check_device_status",
+    "attn_jvp", "attn_jvp_bwd", "attn_jvp_fwd_stats", "bwd_workspace_bytes", "attn_jvp_fwd", "attn_jvp_fwd_f32", "attn_jvp_fwd_f32out", "attn_jvp_fwd_host", "attn_jvp_fwd_host_noalloc", "check_device_status",
     "default_heads_per_chunk", "host_workspace_bytes", "load_library",
     "selftest_wait_timeout", "set_wait_bound_ns", "strerror", "version", "AttnJvpError",
 ]

@@ -25,9 +25,11 @@ AJVP_ERR_TIMEOUT = -5
 AJVP_ERR_CUDA = -6
 AJVP_ERR_TOO_LARGE = -7
 AJVP_ERR_WORKSPACE = -8
+AJVP_ERR_DEVICE_LAYOUT = -9
 
 # every symbol the header declares
-EXPORTED = ("attn_jvp_fwd", "attn_jvp_fwd_f32out", "attn_jvp_fwd_f32", "attn_jvp_fwd_host",
+EXPORTED = ("attn_jvp_fwd", "attn_jvp_fwd_f32out", "attn_jvp_fwd_stats", "attn_jvp_bwd",
+            "attn_jvp_bwd_workspace_bytes", "attn_jvp_fwd_f32", "attn_jvp_fwd_host",
             "attn_jvp_fwd_host_noalloc", "attn_jvp_host_workspace_bytes", "attn_jvp_strerror",
             "attn_jvp_last_cuda_error",
             "attn_jvp_check_device_status", "attn_jvp_set_wait_bound_ns",
@@ -61,6 +63,12 @@ def load_library(path: str = LIB_PATH):
         lib.attn_jvp_fwd_f32.restype = ctypes.c_int
         lib.attn_jvp_fwd_f32out.argtypes = fwd_args
         lib.attn_jvp_fwd_f32out.restype = ctypes.c_int
+        lib.attn_jvp_fwd_stats.argtypes = [vp] * 10 + [i64] * 5 + [f32, vp]
+        lib.attn_jvp_fwd_stats.restype = ctypes.c_int
+        lib.attn_jvp_bwd.argtypes = [vp] * 18 + [i64] * 5 + [f32, vp, ctypes.c_uint64, vp]
+        lib.attn_jvp_bwd.restype = ctypes.c_int
+        lib.attn_jvp_bwd_workspace_bytes.argtypes = [i64] * 3
+        lib.attn_jvp_bwd_workspace_bytes.restype = ctypes.c_uint64
         lib.attn_jvp_fwd_host.argtypes = [vp] * 9 + [i64] * 5 + [f32, vp, ctypes.c_uint64, vp]
         lib.attn_jvp_fwd_host.restype = ctypes.c_int
         lib.attn_jvp_fwd_host_noalloc.argtypes = fwd_args
@@ -165,6 +173,66 @@ def attn_jvp_fwd_f32out(q, k, v, tq, tk, tv, scale=None, o=None, to=None, lse=No
                                  _ptr(lse), B, H, Lq, Lk, d, float(scale), _stream_handle(stream))
     _check(rc, "attn_jvp_fwd_f32out")
     return o, to, lse
+
+
+def attn_jvp_fwd_stats(q, k, v, tq, tk, tv, scale=None, o=None, to=None, lse=None, mu=None, stream=None):
+    """``attn_jvp_fwd`` that also returns mu (fp32 [B, H, Lq]), the row
+    statistic the backward needs beside lse.  Returns (o, to, lse, mu)."""
+    o, to, lse, (B, H, Lq, Lk, d) = _prepare(q, k, v, tq, tk, tv, o, to, lse, torch.bfloat16, True)
+    if mu is None:
+        mu = torch.empty((B, H, Lq), device=q.device, dtype=torch.float32)
+    if mu.shape != (B, H, Lq) or mu.dtype != torch.float32 or not mu.is_contiguous() or not mu.is_cuda:
+        raise ValueError("mu must be a contiguous float32 CUDA [B, H, Lq] tensor")
+    if scale is None:
+        scale = d ** -0.5
+    lib = load_library()
+    rc = lib.attn_jvp_fwd_stats(_ptr(q), _ptr(k), _ptr(v), _ptr(tq), _ptr(tk), _ptr(tv), _ptr(o), _ptr(to),
+                                _ptr(lse), _ptr(mu), B, H, Lq, Lk, d, float(scale), _stream_handle(stream))
+    _check(rc, "attn_jvp_fwd_stats")
+    return o, to, lse, mu
+
+
+def bwd_workspace_bytes(B: int, H: int, Lq: int) -> int:
+    """Device workspace ``attn_jvp_bwd`` needs (row statistics)."""
+    return int(load_library().attn_jvp_bwd_workspace_bytes(int(B), int(H), int(Lq)))
+
+
+GRAD_NAMES = ("dq", "dk", "dv", "dtq", "dtk", "dtv")
+
+
+def attn_jvp_bwd(q, k, v, tq, tk, tv, o, to, lse, mu, dout, dtout, scale=None, grads=None, workspace=None,
+                 stream=None):
+    """Gradients of <dout, O> + <dtout, tO> with respect to q, k, v, tq, tk,
+    tv, through the C ABI's ``attn_jvp_bwd`` (bf16, d = 128).  o, to, lse,
+    mu are the outputs of ``attn_jvp_fwd_stats`` on the same inputs.
+    ``grads``: optional dict of preallocated outputs.  Returns a dict
+    dq, dk, dv, dtq, dtk, dtv.  Asynchronous on ``stream``."""
+    _, _, _, (B, H, Lq, Lk, d) = _prepare(q, k, v, tq, tk, tv, o, to, lse, torch.bfloat16, True)
+    for name, x, shp, dt in (("mu", mu, (B, H, Lq), torch.float32), ("dout", dout, q.shape, torch.bfloat16),
+                             ("dtout", dtout, q.shape, torch.bfloat16)):
+        if not isinstance(x, torch.Tensor) or x.shape != shp or x.dtype != dt or not x.is_contiguous() \
+                or not x.is_cuda:
+            raise ValueError(f"{name} must be a contiguous CUDA {dt} tensor of shape {tuple(shp)}")
+    grads = dict(grads or {})
+    for name in GRAD_NAMES:
+        like = q if name in ("dq", "dtq") else k
+        if grads.get(name) is None:
+            grads[name] = torch.empty_like(like)
+        g = grads[name]
+        if g.shape != like.shape or g.dtype != torch.bfloat16 or not g.is_contiguous() or not g.is_cuda:
+            raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor of shape {tuple(like.shape)}")
+    if scale is None:
+        scale = d ** -0.5
+    if workspace is None:
+        workspace = torch.empty(max(1, bwd_workspace_bytes(B, H, Lq)), dtype=torch.uint8, device=q.device)
+    if not workspace.is_cuda or workspace.dtype != torch.uint8 or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA uint8 tensor")
+    lib = load_library()
+    rc = lib.attn_jvp_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(tq), _ptr(tk), _ptr(tv), _ptr(o), _ptr(to), _ptr(lse),
+                          _ptr(mu), _ptr(dout), _ptr(dtout), *(_ptr(grads[n]) for n in GRAD_NAMES), B, H, Lq, Lk, d,
+                          float(scale), _ptr(workspace), workspace.numel(), _stream_handle(stream))
+    _check(rc, "attn_jvp_bwd")
+    return grads
 
 
 def attn_jvp_fwd_f32(q, k, v, tq, tk, tv, scale=None, o=None, to=None, lse=None, stream=None, want_lse=True):

@@ -14,6 +14,7 @@
 #include <mutex>
 
 #include "attn_jvp.h"
+#include "jvp_bwd_sm100.cuh"
 #include "jvp_f32.cuh"
 #include "jvp_sm100.cuh"
 
@@ -70,6 +71,15 @@ int device_setup(int *dev_out) {
         if (e3 == cudaSuccess)
             e3 = cudaFuncSetAttribute(ajvp::sm100::attn_jvp_fwd_kernel<true>,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ajvp::sm100::SMEM_BYTES);
+        if (e3 == cudaSuccess)
+            e3 = cudaFuncSetAttribute(ajvp::bwd::attn_jvp_bwd_kernel<ajvp::bwd::ROLE_Q>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ajvp::bwd::SMEM_BYTES);
+        if (e3 == cudaSuccess)
+            e3 = cudaFuncSetAttribute(ajvp::bwd::attn_jvp_bwd_kernel<ajvp::bwd::ROLE_K>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ajvp::bwd::SMEM_BYTES);
+        if (e3 == cudaSuccess)
+            e3 = cudaFuncSetAttribute(ajvp::bwd::attn_jvp_bwd_kernel<ajvp::bwd::ROLE_V>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ajvp::bwd::SMEM_BYTES);
         cudaError_t e4 = cudaFuncSetAttribute(ajvp::f32::attn_jvp_fwd_f32_kernel,
                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
                                               (int)ajvp::f32::smem_bytes(ajvp::f32::DMAX));
@@ -134,13 +144,13 @@ int check_common(const void *q, const void *k, const void *v, const void *tq, co
 template <bool kSplit>
 int launch_sm100(const void *q, const void *k, const void *v, const void *tq, const void *tk, const void *tv,
                  void *o, void *to, float *lse, int64_t B, int64_t H, int64_t Lq, int64_t Lk, int64_t d,
-                 float scale, void *stream) {
+                 float scale, void *stream, float *mu = nullptr) {
     bool noop = false;
     int rc = check_common(q, k, v, tq, tk, tv, o, to, B, H, Lq, Lk, d, scale, &noop);
     if (rc != AJVP_OK || noop) return rc;
     if (d != ajvp::sm100::HD) return AJVP_ERR_UNSUPPORTED_DIM;
-    const void *ptrs[9] = {q, k, v, tq, tk, tv, o, to, lse};
-    for (int i = 0; i < 9; ++i)
+    const void *ptrs[10] = {q, k, v, tq, tk, tv, o, to, lse, mu};
+    for (int i = 0; i < 10; ++i)
         if (ptrs[i] && !aligned(ptrs[i], 16)) return AJVP_ERR_MISALIGNED;
     const int64_t BH = B * H;
     const int64_t n_qtiles = (Lq + ajvp::sm100::BR - 1) / ajvp::sm100::BR;
@@ -168,6 +178,7 @@ int launch_sm100(const void *q, const void *k, const void *v, const void *tq, co
         if ((rc = encode_3d(&p.tm_to, to, d, Lq, BH, 128)) != AJVP_OK) return rc;
     }
     p.lse = lse;
+    p.mu = mu;
     p.Lq = (int)Lq;
     p.Lk = (int)Lk;
     p.n_qtiles = (int)n_qtiles;
@@ -177,6 +188,45 @@ int launch_sm100(const void *q, const void *k, const void *v, const void *tq, co
 
     ajvp::sm100::attn_jvp_fwd_kernel<kSplit><<<(unsigned)(n_qtiles * BH), ajvp::sm100::NTHREADS,
                                                ajvp::sm100::SMEM_BYTES, (cudaStream_t)stream>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail_cuda(e);
+    return AJVP_OK;
+}
+
+// ---------------------------------------------------------------- backward
+// Row statistics {lse log2(e), mu, a, D} per query row, plus BN rows of
+// padding that the streamed statistics copies of the last tile may read.
+uint64_t bwd_stats_bytes(int64_t BH, int64_t Lq) {
+    return ((uint64_t)(BH * Lq + ajvp::bwd::BN) * 16u + 255u) / 256u * 256u;
+}
+
+template <int ROLE>
+int launch_bwd_role(const void *const r[4], const void *const c[4], void *out0, void *out1, const void *stats,
+                    int64_t BH, int64_t Lrow, int64_t Lcol, int64_t Lq, int64_t d, float scale, float out_scale,
+                    cudaStream_t stream) {
+    using namespace ajvp::bwd;
+    int rc;
+    Params p;
+    std::memset(&p, 0, sizeof(p));
+    const int nr = ROLE == ROLE_V ? 2 : 4;
+    for (int i = 0; i < 4; ++i) {
+        const void *rp = i < nr ? r[i] : r[0];  // ROLE_V leaves R2, R3 unused
+        if ((rc = encode_3d(&p.tm_r[i], rp, d, Lrow, BH, 128)) != AJVP_OK) return rc;
+        if ((rc = encode_3d(&p.tm_c[i], c[i], d, Lcol, BH, 64)) != AJVP_OK) return rc;
+    }
+    if ((rc = encode_3d(&p.tm_out[0], out0, d, Lrow, BH, 128)) != AJVP_OK) return rc;
+    if ((rc = encode_3d(&p.tm_out[1], out1, d, Lrow, BH, 128)) != AJVP_OK) return rc;
+    const int64_t n_rtiles = (Lrow + BM - 1) / BM;
+    p.stats = static_cast<const float4 *>(stats);
+    p.Lrow = (int)Lrow;
+    p.Lcol = (int)Lcol;
+    p.Lq = (int)Lq;
+    p.n_rtiles = (int)n_rtiles;
+    p.scale = scale;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.out_scale = out_scale;
+    p.bound_ns = g_bound_ns.load();
+    attn_jvp_bwd_kernel<ROLE><<<(unsigned)(n_rtiles * BH), NTHREADS, SMEM_BYTES, stream>>>(p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail_cuda(e);
     return AJVP_OK;
@@ -251,6 +301,82 @@ int attn_jvp_fwd_f32out(const void *q, const void *k, const void *v, const void 
                         const void *tv, float *o, float *to, float *lse, int64_t B, int64_t H, int64_t Lq,
                         int64_t Lk, int64_t d, float scale, void *stream) {
     return launch_sm100<true>(q, k, v, tq, tk, tv, o, to, lse, B, H, Lq, Lk, d, scale, stream);
+}
+
+int attn_jvp_fwd_stats(const void *q, const void *k, const void *v, const void *tq, const void *tk, const void *tv,
+                       void *o, void *to, float *lse, float *mu, int64_t B, int64_t H, int64_t Lq, int64_t Lk,
+                       int64_t d, float scale, void *stream) {
+    if (B > 0 && H > 0 && Lq > 0 && (!lse || !mu)) return AJVP_ERR_INVALID_ARG;
+    return launch_sm100<false>(q, k, v, tq, tk, tv, o, to, lse, B, H, Lq, Lk, d, scale, stream, mu);
+}
+
+uint64_t attn_jvp_bwd_workspace_bytes(int64_t B, int64_t H, int64_t Lq) {
+    if (B < 0 || H < 0 || Lq < 0) return 0;
+    return bwd_stats_bytes(B * H, Lq);
+}
+
+int attn_jvp_bwd(const void *q, const void *k, const void *v, const void *tq, const void *tk, const void *tv,
+                 const void *o, const void *to, const float *lse, const float *mu, const void *dout,
+                 const void *dtout, void *dq, void *dk, void *dv, void *dtq, void *dtk, void *dtv, int64_t B,
+                 int64_t H, int64_t Lq, int64_t Lk, int64_t d, float scale, void *workspace,
+                 uint64_t workspace_bytes, void *stream) {
+    bool noop = false;
+    int rc = check_common(q, k, v, tq, tk, tv, o, to, B, H, Lq, Lk, d, scale, &noop);
+    if (rc != AJVP_OK) return rc;
+    const int64_t BH = B * H;
+    const cudaStream_t st = (cudaStream_t)stream;
+    if (noop) {
+        // no query rows: the key-side gradients are zero; nothing else to write
+        if (BH == 0) return AJVP_OK;
+        if (!dk || !dv || !dtk || !dtv) return AJVP_ERR_INVALID_ARG;
+        if (BH * Lk >= (int64_t(1) << 31)) return AJVP_ERR_TOO_LARGE;
+        const size_t bytes = (size_t)(BH * Lk * d) * 2u;
+        for (void *g : {dk, dv, dtk, dtv}) {
+            cudaError_t e = cudaMemsetAsync(g, 0, bytes, st);
+            if (e != cudaSuccess) return fail_cuda(e);
+        }
+        return AJVP_OK;
+    }
+    if (d != ajvp::bwd::HD) return AJVP_ERR_UNSUPPORTED_DIM;
+    const void *ptrs[18] = {q, k, v, tq, tk, tv, o, to, lse, mu, dout, dtout, dq, dk, dv, dtq, dtk, dtv};
+    for (int i = 0; i < 18; ++i) {
+        if (!ptrs[i]) return AJVP_ERR_INVALID_ARG;
+        if (!aligned(ptrs[i], 16)) return AJVP_ERR_MISALIGNED;
+    }
+    if (((Lq + 127) / 128) * BH >= (int64_t(1) << 31) || ((Lk + 127) / 128) * BH >= (int64_t(1) << 31) ||
+        BH * Lq + ajvp::bwd::BN >= (int64_t(1) << 40))
+        return AJVP_ERR_TOO_LARGE;
+    if (!workspace || !aligned(workspace, 256) || workspace_bytes < bwd_stats_bytes(BH, Lq))
+        return AJVP_ERR_WORKSPACE;
+    int dev = 0;
+    if ((rc = device_setup(&dev)) != AJVP_OK) return rc;
+    if ((rc = get_encoder()) != AJVP_OK) return rc;
+
+    const long long rows = (long long)(BH * Lq);
+    const unsigned grid = (unsigned)std::min<long long>((rows + 7) / 8, 148LL * 16);
+    ajvp::bwd::bwd_rowstats_kernel<<<grid, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16 *>(o), static_cast<const __nv_bfloat16 *>(to),
+        static_cast<const __nv_bfloat16 *>(dout), static_cast<const __nv_bfloat16 *>(dtout), lse, mu,
+        static_cast<float4 *>(workspace), rows);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail_cuda(e);
+    using namespace ajvp::bwd;
+    {   // dQ, dtQ: rows = queries, streamed keys
+        const void *r[4] = {q, tq, dtout, dout}, *c[4] = {k, tk, v, tv};
+        if ((rc = launch_bwd_role<ROLE_Q>(r, c, dq, dtq, workspace, BH, Lq, Lk, Lq, d, scale, scale, st)) != AJVP_OK)
+            return rc;
+    }
+    {   // dK, dtK: rows = keys, streamed queries
+        const void *r[4] = {k, tk, v, tv}, *c[4] = {q, tq, dtout, dout};
+        if ((rc = launch_bwd_role<ROLE_K>(r, c, dk, dtk, workspace, BH, Lk, Lq, Lq, d, scale, scale, st)) != AJVP_OK)
+            return rc;
+    }
+    {   // dV, dtV: rows = keys, streamed queries
+        const void *r[4] = {k, tk, nullptr, nullptr}, *c[4] = {q, tq, dout, dtout};
+        if ((rc = launch_bwd_role<ROLE_V>(r, c, dv, dtv, workspace, BH, Lk, Lq, Lq, d, scale, 1.0f, st)) != AJVP_OK)
+            return rc;
+    }
+    return AJVP_OK;
 }
 
 uint64_t attn_jvp_host_workspace_bytes(int64_t Lq, int64_t Lk, int64_t d, int64_t heads_per_chunk) {
@@ -365,6 +491,7 @@ const char *attn_jvp_strerror(int status) {
         case AJVP_ERR_CUDA: return "CUDA runtime or driver error";
         case AJVP_ERR_TOO_LARGE: return "a size exceeds the supported maximum";
         case AJVP_ERR_WORKSPACE: return "device workspace missing, not 256-byte aligned or too small";
+        case AJVP_ERR_DEVICE_LAYOUT: return "a kernel found its shared memory misaligned and did nothing";
         default: return "unknown status";
     }
 }
@@ -381,7 +508,7 @@ int attn_jvp_check_device_status(void *stream) {
         const int zero = 0;
         e = cudaMemcpyToSymbol(ajvp::g_status_word, &zero, sizeof(int));
         if (e != cudaSuccess) return fail_cuda(e);
-        return AJVP_ERR_TIMEOUT;
+        return (word & 2) ? AJVP_ERR_DEVICE_LAYOUT : AJVP_ERR_TIMEOUT;
     }
     return AJVP_OK;
 }

@@ -100,6 +100,7 @@ struct Params {
     CUtensorMap tm_q, tm_tq, tm_k, tm_tk, tm_v, tm_tv, tm_o, tm_to;
     float *o_f32, *to_f32;  // kSplit: fp32 outputs [B*H][Lq][128] (tm_o / tm_to unused)
     float *lse;
+    float *mu;  // optional [B*H][Lq]: mu_i = sum_j P_ij s dS'_ij (saved for the backward)
     int Lq, Lk, n_qtiles;  // n_qtiles: 128-row query tiles per (batch, head)
     float scale;           // s
     float scale_log2;      // s * log2(e)
@@ -533,6 +534,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                 p.lse[(size_t)bh * (size_t)p.Lq + (size_t)(q0 + row)] =
                     (m_ref + __log2f(lt)) * 0.69314718055994531f;
             }
+            if (grp == 1 && p.mu != nullptr && q0 + row < p.Lq) p.mu[(size_t)bh * (size_t)p.Lq + (size_t)(q0 + row)] = mu;
         }
         fence_proxy_async_smem();
         named_bar_sync(NB_EPI, SOFTMAX_THREADS);  // staging complete (every softmax thread gets here)

@@ -126,6 +126,20 @@ def make_inputs(w: Workload | str, seed: int = 0, device="cpu", dtype=None):
     return out
 
 
+def make_cotangents(w: Workload | str, seed: int = 1, device="cpu", dtype=None):
+    """Cotangents dO, dtO of the outputs (for the backward pass): standard
+    normal [B, H, Lq, d] tensors, drawn in that order from their own seeded
+    generator (the pages give no training signal to imitate)."""
+    if isinstance(w, str):
+        w = WORKLOADS[w]
+    out_dtype = dtype if dtype is not None else w.torch_dtype
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    shape = (w.B, w.H, w.Lq, w.d)
+    return {n: torch.randn(shape, generator=g, device=device, dtype=torch.float32).to(out_dtype).contiguous()
+            for n in ("dout", "dtout")}
+
+
 def sample_rows(Lq: int, n: int, seed: int = 0, tile: int = 128):
     """A seeded subset of query rows that always contains the first and last
     rows, both sides of every 128-row tile boundary it can reach and the

@@ -27,8 +27,9 @@
  *
  * Ownership and execution: all pointers are DEVICE pointers owned by the
  * caller (except the data pointers of attn_jvp_fwd_host and
- * attn_jvp_fwd_host_noalloc, which are host pointers).  The library allocates no device memory per call and keeps no
- * per-call state.  Calls are stream-ordered and asynchronous: they return
+ * attn_jvp_fwd_host_noalloc, which are host pointers).  The library
+ * allocates no device memory per call and keeps no per-call state.  Calls
+ * are stream-ordered and asynchronous: they return
  * after enqueueing work on `stream` (a cudaStream_t; NULL = legacy default
  * stream) and do not synchronise.  Calls are thread-safe.  Inputs must not
  * alias outputs.  Non-finite inputs give unspecified (but memory-safe)
@@ -66,7 +67,8 @@ typedef enum {
     AJVP_ERR_TIMEOUT = -5,            /* a kernel wait ran past its bound (device status word) */
     AJVP_ERR_CUDA = -6,               /* a CUDA runtime/driver call failed */
     AJVP_ERR_TOO_LARGE = -7,          /* a size exceeds the documented maximum */
-    AJVP_ERR_WORKSPACE = -8           /* workspace missing, misaligned or too small */
+    AJVP_ERR_WORKSPACE = -8,          /* workspace missing, misaligned or too small */
+    AJVP_ERR_DEVICE_LAYOUT = -9       /* a kernel found its shared memory misaligned (device status word) */
 } ajvp_status;
 
 /*
@@ -111,6 +113,58 @@ AJVP_API int attn_jvp_fwd_f32out(const void *q, const void *k, const void *v,
                         float *o, float *to, float *lse,
                         int64_t B, int64_t H, int64_t Lq, int64_t Lk, int64_t d,
                         float scale, void *stream);
+
+/*
+ * attn_jvp_fwd_stats -- attn_jvp_fwd that also saves, per query row, the
+ * statistic mu_i = sum_j P_ij dS_ij (fp32 [B][H][Lq]) that attn_jvp_bwd needs
+ * beside lse.  lse and mu are required (non-NULL, 16-byte aligned); all
+ * other arguments and rules as attn_jvp_fwd.
+ */
+AJVP_API int attn_jvp_fwd_stats(const void *q, const void *k, const void *v,
+                       const void *tq, const void *tk, const void *tv,
+                       void *o, void *to, float *lse, float *mu,
+                       int64_t B, int64_t H, int64_t Lq, int64_t Lk, int64_t d,
+                       float scale, void *stream);
+
+/*
+ * attn_jvp_bwd -- backward pass of attn_jvp_fwd: the gradients of
+ *
+ *     L = sum <dout, O> + sum <dtout, tO>
+ *
+ * with respect to q, k, v and the tangents tq, tk, tv (rCM trains through
+ * its fused attention + JVP kernel; the pages describe its forward pass
+ * only, and this is the gradient of that forward definition).
+ *
+ *   q, k, v, tq, tk, tv : the forward's bf16 inputs (layouts as attn_jvp_fwd)
+ *   o, to               : the forward's bf16 outputs [B][H][Lq][d]
+ *   lse, mu             : the forward's float row statistics [B][H][Lq]
+ *                         (attn_jvp_fwd_stats)
+ *   dout, dtout         : bf16 cotangents of O and tO, [B][H][Lq][d]
+ *   dq, dtq             : bf16 [B][H][Lq][d] (written)
+ *   dk, dv, dtk, dtv    : bf16 [B][H][Lk][d] (written)
+ *   workspace           : DEVICE memory owned by the caller, 256-byte aligned,
+ *                         at least attn_jvp_bwd_workspace_bytes(B, H, Lq)
+ *                         bytes; nothing in it needs to start at zero
+ *
+ * Four kernels on `stream`: per-row statistics into the workspace, then the
+ * query-side, key-side and value-side gradient kernels (tcgen05), each
+ * owning its outputs (no atomics: results are deterministic).  Gradients are
+ * accumulated in fp32 and rounded to bf16 (round-to-nearest-even).
+ * Supported: d == 128, every pointer non-NULL and 16-byte aligned, sizes as
+ * attn_jvp_fwd.  B*H == 0 is a no-op; Lq == 0 writes zeros to dk, dv, dtk,
+ * dtv.  Outputs must not alias inputs.  Errors as attn_jvp_fwd plus
+ * AJVP_ERR_WORKSPACE.
+ */
+AJVP_API int attn_jvp_bwd(const void *q, const void *k, const void *v,
+                 const void *tq, const void *tk, const void *tv,
+                 const void *o, const void *to, const float *lse, const float *mu,
+                 const void *dout, const void *dtout,
+                 void *dq, void *dk, void *dv, void *dtq, void *dtk, void *dtv,
+                 int64_t B, int64_t H, int64_t Lq, int64_t Lk, int64_t d,
+                 float scale, void *workspace, uint64_t workspace_bytes, void *stream);
+
+/* Device workspace, in bytes, that attn_jvp_bwd needs (0 for invalid sizes). */
+AJVP_API uint64_t attn_jvp_bwd_workspace_bytes(int64_t B, int64_t H, int64_t Lq);
 
 /*
  * attn_jvp_fwd_f32 -- fp32 I/O, fp32 arithmetic (CUDA-core kernel), for the
@@ -205,7 +259,9 @@ AJVP_API int attn_jvp_last_cuda_error(void);
 /*
  * Synchronise `stream`, then read and clear the device status word of the
  * current device.  Returns AJVP_OK, AJVP_ERR_TIMEOUT (some kernel wait ran
- * past its bound since the last check) or AJVP_ERR_CUDA.
+ * past its bound since the last check), AJVP_ERR_DEVICE_LAYOUT (a backward
+ * kernel found its dynamic shared memory not 1024-byte aligned and returned
+ * without work) or AJVP_ERR_CUDA.
  */
 AJVP_API int attn_jvp_check_device_status(void *stream);
 
