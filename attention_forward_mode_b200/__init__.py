@@ -18,6 +18,7 @@ from ._binding import (  # noqa: F401
     AJVP_ERR_UNSUPPORTED_DIM,
     AJVP_ERR_WORKSPACE,
     AJVP_OK,
+    GRAD_NAMES,
     AttnJvpError,
     attn_jvp,
     attn_jvp_bwd,

@@ -28,7 +28,7 @@ AJVP_ERR_WORKSPACE = -8
 AJVP_ERR_DEVICE_LAYOUT = -9
 
 # every symbol the header declares
-EXPORTED = ("attn_jvp_fwd", "attn_jvp_fwd_f32out", "attn_jvp_fwd_stats", "attn_jvp_bwd",
+EXPORTED = ("attn_jvp_fwd", "attn_jvp_fwd_f32out", "attn_jvp_fwd_stats", "attn_jvp_bwd", "attn_jvp_bwd_step",
             "attn_jvp_bwd_workspace_bytes", "attn_jvp_fwd_f32", "attn_jvp_fwd_host",
             "attn_jvp_fwd_host_noalloc", "attn_jvp_host_workspace_bytes", "attn_jvp_strerror",
             "attn_jvp_last_cuda_error",
@@ -67,6 +67,8 @@ def load_library(path: str = LIB_PATH):
         lib.attn_jvp_fwd_stats.restype = ctypes.c_int
         lib.attn_jvp_bwd.argtypes = [vp] * 18 + [i64] * 5 + [f32, vp, ctypes.c_uint64, vp]
         lib.attn_jvp_bwd.restype = ctypes.c_int
+        lib.attn_jvp_bwd_step.argtypes = [ctypes.c_int] + [vp] * 18 + [i64] * 5 + [f32, vp, ctypes.c_uint64, vp]
+        lib.attn_jvp_bwd_step.restype = ctypes.c_int
         lib.attn_jvp_bwd_workspace_bytes.argtypes = [i64] * 3
         lib.attn_jvp_bwd_workspace_bytes.restype = ctypes.c_uint64
         lib.attn_jvp_fwd_host.argtypes = [vp] * 9 + [i64] * 5 + [f32, vp, ctypes.c_uint64, vp]
@@ -201,12 +203,13 @@ GRAD_NAMES = ("dq", "dk", "dv", "dtq", "dtk", "dtv")
 
 
 def attn_jvp_bwd(q, k, v, tq, tk, tv, o, to, lse, mu, dout, dtout, scale=None, grads=None, workspace=None,
-                 stream=None):
+                 stream=None, step=None):
     """Gradients of <dout, O> + <dtout, tO> with respect to q, k, v, tq, tk,
     tv, through the C ABI's ``attn_jvp_bwd`` (bf16, d = 128).  o, to, lse,
     mu are the outputs of ``attn_jvp_fwd_stats`` on the same inputs.
     ``grads``: optional dict of preallocated outputs.  Returns a dict
-    dq, dk, dv, dtq, dtk, dtv.  Asynchronous on ``stream``."""
+    dq, dk, dv, dtq, dtk, dtv.  Asynchronous on ``stream``.  ``step`` (0-3)
+    runs one of the four kernels only (``attn_jvp_bwd_step``)."""
     _, _, _, (B, H, Lq, Lk, d) = _prepare(q, k, v, tq, tk, tv, o, to, lse, torch.bfloat16, True)
     for name, x, shp, dt in (("mu", mu, (B, H, Lq), torch.float32), ("dout", dout, q.shape, torch.bfloat16),
                              ("dtout", dtout, q.shape, torch.bfloat16)):
@@ -228,10 +231,13 @@ def attn_jvp_bwd(q, k, v, tq, tk, tv, o, to, lse, mu, dout, dtout, scale=None, g
     if not workspace.is_cuda or workspace.dtype != torch.uint8 or not workspace.is_contiguous():
         raise ValueError("workspace must be a contiguous CUDA uint8 tensor")
     lib = load_library()
-    rc = lib.attn_jvp_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(tq), _ptr(tk), _ptr(tv), _ptr(o), _ptr(to), _ptr(lse),
-                          _ptr(mu), _ptr(dout), _ptr(dtout), *(_ptr(grads[n]) for n in GRAD_NAMES), B, H, Lq, Lk, d,
-                          float(scale), _ptr(workspace), workspace.numel(), _stream_handle(stream))
-    _check(rc, "attn_jvp_bwd")
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(tq), _ptr(tk), _ptr(tv), _ptr(o), _ptr(to), _ptr(lse), _ptr(mu),
+            _ptr(dout), _ptr(dtout), *(_ptr(grads[n]) for n in GRAD_NAMES), B, H, Lq, Lk, d, float(scale),
+            _ptr(workspace), workspace.numel(), _stream_handle(stream))
+    if step is None:
+        _check(lib.attn_jvp_bwd(*args), "attn_jvp_bwd")
+    else:
+        _check(lib.attn_jvp_bwd_step(int(step), *args), "attn_jvp_bwd_step")
     return grads
 
 

@@ -315,11 +315,16 @@ uint64_t attn_jvp_bwd_workspace_bytes(int64_t B, int64_t H, int64_t Lq) {
     return bwd_stats_bytes(B * H, Lq);
 }
 
-int attn_jvp_bwd(const void *q, const void *k, const void *v, const void *tq, const void *tk, const void *tv,
-                 const void *o, const void *to, const float *lse, const float *mu, const void *dout,
-                 const void *dtout, void *dq, void *dk, void *dv, void *dtq, void *dtk, void *dtv, int64_t B,
-                 int64_t H, int64_t Lq, int64_t Lk, int64_t d, float scale, void *workspace,
-                 uint64_t workspace_bytes, void *stream) {
+}  // extern "C"
+
+namespace {
+// Steps first..last of the backward (0 row statistics, 1 dQ/dtQ, 2 dK/dtK,
+// 3 dV/dtV) after the full argument check.
+int bwd_steps(int first, int last, const void *q, const void *k, const void *v, const void *tq, const void *tk,
+              const void *tv, const void *o, const void *to, const float *lse, const float *mu, const void *dout,
+              const void *dtout, void *dq, void *dk, void *dv, void *dtq, void *dtk, void *dtv, int64_t B, int64_t H,
+              int64_t Lq, int64_t Lk, int64_t d, float scale, void *workspace, uint64_t workspace_bytes,
+              void *stream) {
     bool noop = false;
     int rc = check_common(q, k, v, tq, tk, tv, o, to, B, H, Lq, Lk, d, scale, &noop);
     if (rc != AJVP_OK) return rc;
@@ -331,8 +336,11 @@ int attn_jvp_bwd(const void *q, const void *k, const void *v, const void *tq, co
         if (!dk || !dv || !dtk || !dtv) return AJVP_ERR_INVALID_ARG;
         if (BH * Lk >= (int64_t(1) << 31)) return AJVP_ERR_TOO_LARGE;
         const size_t bytes = (size_t)(BH * Lk * d) * 2u;
-        for (void *g : {dk, dv, dtk, dtv}) {
-            cudaError_t e = cudaMemsetAsync(g, 0, bytes, st);
+        void *zero_k[2] = {dk, dtk}, *zero_v[2] = {dv, dtv};
+        for (int i = 0; i < 2; ++i) {
+            cudaError_t e = cudaSuccess;
+            if (first <= 2 && last >= 2) e = cudaMemsetAsync(zero_k[i], 0, bytes, st);
+            if (e == cudaSuccess && first <= 3 && last >= 3) e = cudaMemsetAsync(zero_v[i], 0, bytes, st);
             if (e != cudaSuccess) return fail_cuda(e);
         }
         return AJVP_OK;
@@ -352,31 +360,55 @@ int attn_jvp_bwd(const void *q, const void *k, const void *v, const void *tq, co
     if ((rc = device_setup(&dev)) != AJVP_OK) return rc;
     if ((rc = get_encoder()) != AJVP_OK) return rc;
 
-    const long long rows = (long long)(BH * Lq);
-    const unsigned grid = (unsigned)std::min<long long>((rows + 7) / 8, 148LL * 16);
-    ajvp::bwd::bwd_rowstats_kernel<<<grid, 256, 0, st>>>(
-        static_cast<const __nv_bfloat16 *>(o), static_cast<const __nv_bfloat16 *>(to),
-        static_cast<const __nv_bfloat16 *>(dout), static_cast<const __nv_bfloat16 *>(dtout), lse, mu,
-        static_cast<float4 *>(workspace), rows);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return fail_cuda(e);
     using namespace ajvp::bwd;
-    {   // dQ, dtQ: rows = queries, streamed keys
+    if (first <= 0 && last >= 0) {
+        const long long rows = (long long)(BH * Lq);
+        const unsigned grid = (unsigned)std::min<long long>((rows + 7) / 8, 148LL * 16);
+        bwd_rowstats_kernel<<<grid, 256, 0, st>>>(
+            static_cast<const __nv_bfloat16 *>(o), static_cast<const __nv_bfloat16 *>(to),
+            static_cast<const __nv_bfloat16 *>(dout), static_cast<const __nv_bfloat16 *>(dtout), lse, mu,
+            static_cast<float4 *>(workspace), rows);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return fail_cuda(e);
+    }
+    if (first <= 1 && last >= 1) {  // dQ, dtQ: rows = queries, streamed keys
         const void *r[4] = {q, tq, dtout, dout}, *c[4] = {k, tk, v, tv};
         if ((rc = launch_bwd_role<ROLE_Q>(r, c, dq, dtq, workspace, BH, Lq, Lk, Lq, d, scale, scale, st)) != AJVP_OK)
             return rc;
     }
-    {   // dK, dtK: rows = keys, streamed queries
+    if (first <= 2 && last >= 2) {  // dK, dtK: rows = keys, streamed queries
         const void *r[4] = {k, tk, v, tv}, *c[4] = {q, tq, dtout, dout};
         if ((rc = launch_bwd_role<ROLE_K>(r, c, dk, dtk, workspace, BH, Lk, Lq, Lq, d, scale, scale, st)) != AJVP_OK)
             return rc;
     }
-    {   // dV, dtV: rows = keys, streamed queries
+    if (first <= 3 && last >= 3) {  // dV, dtV: rows = keys, streamed queries
         const void *r[4] = {k, tk, nullptr, nullptr}, *c[4] = {q, tq, dout, dtout};
         if ((rc = launch_bwd_role<ROLE_V>(r, c, dv, dtv, workspace, BH, Lk, Lq, Lq, d, scale, 1.0f, st)) != AJVP_OK)
             return rc;
     }
     return AJVP_OK;
+}
+}  // namespace
+
+extern "C" {
+
+int attn_jvp_bwd(const void *q, const void *k, const void *v, const void *tq, const void *tk, const void *tv,
+                 const void *o, const void *to, const float *lse, const float *mu, const void *dout,
+                 const void *dtout, void *dq, void *dk, void *dv, void *dtq, void *dtk, void *dtv, int64_t B,
+                 int64_t H, int64_t Lq, int64_t Lk, int64_t d, float scale, void *workspace,
+                 uint64_t workspace_bytes, void *stream) {
+    return bwd_steps(0, 3, q, k, v, tq, tk, tv, o, to, lse, mu, dout, dtout, dq, dk, dv, dtq, dtk, dtv, B, H, Lq, Lk,
+                     d, scale, workspace, workspace_bytes, stream);
+}
+
+int attn_jvp_bwd_step(int step, const void *q, const void *k, const void *v, const void *tq, const void *tk,
+                      const void *tv, const void *o, const void *to, const float *lse, const float *mu,
+                      const void *dout, const void *dtout, void *dq, void *dk, void *dv, void *dtq, void *dtk,
+                      void *dtv, int64_t B, int64_t H, int64_t Lq, int64_t Lk, int64_t d, float scale,
+                      void *workspace, uint64_t workspace_bytes, void *stream) {
+    if (step < 0 || step > 3) return AJVP_ERR_INVALID_ARG;
+    return bwd_steps(step, step, q, k, v, tq, tk, tv, o, to, lse, mu, dout, dtout, dq, dk, dv, dtq, dtk, dtv, B, H,
+                     Lq, Lk, d, scale, workspace, workspace_bytes, stream);
 }
 
 uint64_t attn_jvp_host_workspace_bytes(int64_t Lq, int64_t Lk, int64_t d, int64_t heads_per_chunk) {

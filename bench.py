@@ -41,6 +41,13 @@ METRIC = "attention+JVP TFLOP/s (12·Lq·Lk·d/head) and % of B200 BF16 tensor p
 FALLBACK_BF16_TFLOPS = 1590.0
 KERNEL_SOURCES = ["attention_forward_mode_b200/csrc/jvp_sm100.cuh", "attention_forward_mode_b200/csrc/ptx_sm100.cuh"]
 TRAFFIC_FILE = "profiles/attn_jvp_fwd_kernel.video_selfattn_b1h12_l32760.md"
+BWD_METRIC = "attention+JVP backward TFLOP/s (30·Lq·Lk·d/head) and % of B200 BF16 tensor peak"
+BWD_KERNEL_SOURCES = ["attention_forward_mode_b200/csrc/jvp_bwd_sm100.cuh",
+                      "attention_forward_mode_b200/csrc/ptx_sm100.cuh"]
+BWD_TRAFFIC_FILE = "profiles/attn_jvp_bwd_kernel.video_selfattn_b1h12_l32760.md"
+# backward kernels (steps of attn_jvp_bwd): name, contraction FLOPs per (Lq*Lk*d) per head
+BWD_STEPS = [("bwd_rowstats_kernel", 0.0), ("attn_jvp_bwd_kernel<ROLE_Q> (dQ, dtQ)", 18.0),
+             ("attn_jvp_bwd_kernel<ROLE_K> (dK, dtK)", 18.0), ("attn_jvp_bwd_kernel<ROLE_V> (dV, dtV)", 12.0)]
 L2_BYTES = 126 * 1024 * 1024
 
 
@@ -87,18 +94,18 @@ def measured_peaks():
         return FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
 
 
-def kernel_source_sha() -> str:
+def kernel_source_sha(sources=None) -> str:
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in sources or KERNEL_SOURCES:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def committed_traffic():
+def committed_traffic(traffic_file=TRAFFIC_FILE, sources=None):
     """DRAM bytes per launch from the committed ncu summary, if it was taken
     on the kernel source as it stands (else None)."""
-    path = os.path.join(ROOT, TRAFFIC_FILE)
+    path = os.path.join(ROOT, traffic_file)
     if not os.path.exists(path):
         return None
     fields = {}
@@ -106,7 +113,7 @@ def committed_traffic():
         if ":" in line and line.strip().startswith(("traffic_bytes_per_launch", "kernel_source_sha")):
             k, v = line.split(":", 1)
             fields[k.strip()] = v.strip().strip("`")
-    if fields.get("kernel_source_sha") != kernel_source_sha():
+    if fields.get("kernel_source_sha") != kernel_source_sha(sources):
         return None
     try:
         return float(fields["traffic_bytes_per_launch"])
@@ -381,6 +388,194 @@ def run_ours(args, w):
     return 0
 
 
+# ------------------------------------------------------------- backward
+def bwd_flops(w) -> float:
+    """Backward contraction FLOPs of one (batch, head) set: 15 products of
+    2 Lq Lk d each (S, two score-tangent terms, dtO V^T, dO V^T, dtO tV^T,
+    two each for dV, dK, dQ and one each for dtV, dtK, dtQ)."""
+    return 30.0 * w.B * w.H * w.Lq * w.Lk * w.d
+
+
+def oracle_bwd_sample(w, full_cpu_head, seconds: float, seed: int = 0):
+    """Time the fp64 backward oracle on a prefix sub-problem of one head: the
+    first n query rows with every key (a complete backward of an n-row
+    problem, 30 n Lk d FLOPs), n sized to about ``seconds``."""
+    import oracle
+    x = full_cpu_head
+    probe = max(4, 2 * oracle.num_threads())
+
+    def run(n):
+        t0 = time.perf_counter()
+        oracle.attn_jvp_bwd(x["q"][None, :n], x["k"][None], x["v"][None], x["tq"][None, :n], x["tk"][None],
+                            x["tv"][None], x["dout"][None, :n], x["dtout"][None, :n], w.scale)
+        return time.perf_counter() - t0
+
+    per_row = max(run(probe) / probe, 1e-6)
+    n = int(max(1, min(x["q"].shape[0], seconds / per_row)))
+    el = run(n)
+    return 30.0 * n * w.Lk * w.d / el / 1e12, n, el, oracle.num_threads()
+
+
+def bwd_head0_cpu(inp, cot):
+    return {n: t[0, 0].detach().cpu() for n, t in {**inp, **cot}.items()}
+
+
+def run_reference_bwd(args, w):
+    rank, world, local = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+    from attention_forward_mode_b200.workloads import make_cotangents
+    oracle.build()
+    head = bwd_head0_cpu(make_inputs(w, seed=0, device="cpu"), make_cotangents(w, device="cpu"))
+    per_step = max(0.5, args.reference_seconds / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        oracle_bwd_sample(w, head, per_step)
+    rows_total, el_total, threads = 0, 0.0, oracle.num_threads()
+    for _ in range(args.steps):
+        _, n, el, threads = oracle_bwd_sample(w, head, per_step)
+        rows_total += n
+        el_total += el
+    value = 30.0 * rows_total * w.Lk * w.d / el_total / 1e12
+    sample = (f"backward of the first query rows of head 0 with all {w.Lk} keys, {rows_total} rows over "
+              f"{args.steps} steps, {el_total:.1f} s of fp64 oracle time")
+    line = {"impl": "reference", "metric": BWD_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * el_total / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": dict(workload_config(w, world), entry="attn_jvp_bwd"),
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours_bwd(args, w):
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    init_dist(world, local)
+    import attention_forward_mode_b200 as ajvp
+    from attention_forward_mode_b200.workloads import make_cotangents
+    ajvp.load_library()
+    names = ("q", "k", "v", "tq", "tk", "tv")
+    inp = make_inputs(w, seed=rank, device=dev)
+    cot = make_cotangents(w, seed=1000 + rank, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    o, to, lse, mu = ajvp.attn_jvp_fwd_stats(*(inp[n] for n in names), w.scale, stream=stream)
+    grads = {n: torch.empty_like(inp["q"] if n in ("dq", "dtq") else inp["k"]) for n in ajvp.GRAD_NAMES}
+    ws = torch.empty(ajvp.bwd_workspace_bytes(w.B, w.H, w.Lq), dtype=torch.uint8, device=dev)
+    in_bytes = sum(t.numel() * t.element_size() for t in list(inp.values()) + list(cot.values()) + [o, to])
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev) if in_bytes <= L2_BYTES else None
+
+    def step(which=None):
+        if flush is not None:
+            flush.zero_()
+        ajvp.attn_jvp_bwd(*(inp[n] for n in names), o, to, lse, mu, cot["dout"], cot["dtout"], w.scale,
+                          grads=grads, workspace=ws, stream=stream, step=which)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if ajvp.check_device_status(stream) != ajvp.AJVP_OK:
+        raise RuntimeError("kernel wait bound exceeded during warm-up")
+
+    dist = __import__("torch.distributed", fromlist=["barrier"])
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clocks:
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    ms = ev0.elapsed_time(ev1)
+    ms_max = max_over_ranks(ms, world, dev)
+    if ajvp.check_device_status(stream) != ajvp.AJVP_OK:
+        raise RuntimeError("kernel wait bound exceeded")
+    flops = bwd_flops(w)
+    value = aggregate_value(flops, args.steps, world, ms_max / 1e3)
+
+    # each of the four kernels alone, K launches each, events on the stream
+    per_kernel = []
+    nk = max(3, args.steps // 2)
+    for i, (kname, fl) in enumerate(BWD_STEPS):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        step(i)
+        torch.cuda.synchronize(dev)
+        a.record(stream)
+        for _ in range(nk):
+            step(i)
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        kms = a.elapsed_time(b) / nk
+        kfl = fl * w.B * w.H * w.Lq * w.Lk * w.d
+        per_kernel.append({"kernel": kname, "ms": kms, "flops": kfl, "tflops": kfl / (kms / 1e3) / 1e12 if fl else None})
+    dom = max(per_kernel, key=lambda r: r["ms"])
+
+    # end to end: pinned host inputs -> device -> attn_jvp_bwd -> host gradients, every step
+    dev_in = {**{n: inp[n] for n in names}, "o": o, "to": to, "lse": lse, "mu": mu, **cot}
+    host_in = {n: t.detach().to("cpu").pin_memory() for n, t in dev_in.items()}
+    host_g = {n: torch.empty(g.shape, dtype=g.dtype).pin_memory() for n, g in grads.items()}
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_g.values())
+
+    def e2e_step():
+        for n in dev_in:
+            dev_in[n].copy_(host_in[n], non_blocking=True)
+        step()
+        for n in grads:
+            host_g[n].copy_(grads[n], non_blocking=True)
+
+    e2e_steps = max(1, min(args.steps, args.e2e_steps))
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    ev2, ev3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev2.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    ev3.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(ev2.elapsed_time(ev3), world, dev)
+    e2e_value = aggregate_value(flops, e2e_steps, world, e2e_ms / 1e3)
+
+    line = None
+    if rank == 0:
+        burst, _, src = measured_peaks()
+        achieved = dom["flops"] / (dom["ms"] / 1e3) / 1e12
+        line = {"metric": BWD_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": dict(workload_config(w, world), entry="attn_jvp_bwd",
+                               flops_per_step="30·Lq·Lk·d per head (minimal contraction count)"),
+                "pct_of_bf16_peak": 100.0 * value / world / burst,
+                "roofline": {"bound": "tensor", "achieved": achieved, "peak": burst, "unit": "TFLOP/s",
+                             "frac": achieved / burst,
+                             "traffic": committed_traffic(BWD_TRAFFIC_FILE, BWD_KERNEL_SOURCES),
+                             "peak_source": f"{src} bf16 dense (burst) from MEASURED_PEAKS.json"
+                             if src == "measured" else "fallback 1.59 PFLOP/s",
+                             "kernel": dom["kernel"], "algorithmic_flops_per_launch": dom["flops"],
+                             "launch_ms": dom["ms"]},
+                "kernels": per_kernel,
+                "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                        "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps,
+                        "path": "copy in, attn_jvp_bwd, copy out (serial on one stream)"},
+                "gpu_launches": 4 * args.steps, "clocks": clocks.summary()}
+        if world == 1 and not args.no_cpu_baseline:
+            v, n, el, threads = oracle_bwd_sample(w, bwd_head0_cpu(inp, cot), args.cpu_seconds)
+            line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                                    "sample": f"backward of the first {n} query rows of head 0 with all {w.Lk} keys "
+                                              f"({el:.1f} s, fp64, OpenMP)"}
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def eager_reference(w, inp, chunk: int = 8192):
     """torch.func.jvp of softmax(s q k^T) v in the I/O dtype on the GPU,
     looped over heads and 8192-row query chunks (what fits in memory);
@@ -424,8 +619,9 @@ def main(argv=None):
     ap.add_argument("--reference-seconds", type=float, default=90.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-eager", action="store_true")
-    ap.add_argument("--entry", choices=["bf16", "f32out"], default="bf16",
-                    help="f32out: time attn_jvp_fwd_f32out (fp32 outputs, split-bf16 probabilities)")
+    ap.add_argument("--entry", choices=["bf16", "f32out", "bwd"], default="bf16",
+                    help="f32out: time attn_jvp_fwd_f32out (fp32 outputs, split-bf16 probabilities); "
+                         "bwd: time the backward pass attn_jvp_bwd")
     ap.add_argument("--heads", type=int, default=None,
                     help="override H (small profiling captures); the JSON config shows the H used")
     args = ap.parse_args(argv)
@@ -436,6 +632,8 @@ def main(argv=None):
         w = dataclasses.replace(w, H=args.heads, name=f"{w.name}_h{args.heads}")
     if w.dtype != "bf16" and args.impl == "ours":
         ap.error("the benchmark times the bf16 tensor-core path")
+    if args.entry == "bwd":
+        return run_reference_bwd(args, w) if args.impl == "reference" else run_ours_bwd(args, w)
     if args.impl == "reference":
         return run_reference(args, w)
     return run_ours(args, w)

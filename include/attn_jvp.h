@@ -163,6 +163,24 @@ AJVP_API int attn_jvp_bwd(const void *q, const void *k, const void *v,
                  int64_t B, int64_t H, int64_t Lq, int64_t Lk, int64_t d,
                  float scale, void *workspace, uint64_t workspace_bytes, void *stream);
 
+/*
+ * attn_jvp_bwd_step -- one of attn_jvp_bwd's four kernels, for callers that
+ * schedule them (or time them) separately: step 0 writes the row
+ * statistics into the workspace, step 1 dq and dtq, step 2 dk and dtk,
+ * step 3 dv and dtv.  Steps 1-3 read the workspace step 0 wrote (same
+ * inputs, same workspace, ordered after it); they are independent of each
+ * other.  Arguments, checks and errors as attn_jvp_bwd (every pointer is
+ * checked, even those a step does not touch); AJVP_ERR_INVALID_ARG for a
+ * step outside 0..3.
+ */
+AJVP_API int attn_jvp_bwd_step(int step, const void *q, const void *k, const void *v,
+                      const void *tq, const void *tk, const void *tv,
+                      const void *o, const void *to, const float *lse, const float *mu,
+                      const void *dout, const void *dtout,
+                      void *dq, void *dk, void *dv, void *dtq, void *dtk, void *dtv,
+                      int64_t B, int64_t H, int64_t Lq, int64_t Lk, int64_t d,
+                      float scale, void *workspace, uint64_t workspace_bytes, void *stream);
+
 /* Device workspace, in bytes, that attn_jvp_bwd needs (0 for invalid sizes). */
 AJVP_API uint64_t attn_jvp_bwd_workspace_bytes(int64_t B, int64_t H, int64_t Lq);
 

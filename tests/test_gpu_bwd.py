@@ -126,3 +126,18 @@ def test_image_workload_sampled():
     print(w.name, err)
     for n, e in err.items():
         assert e <= TOL, f"{n}: {e:.3e} ({err})"
+
+
+def test_steps_equal_all_in_one():
+    w = custom(2, 2, 300, 270, 128)
+    inp = gpu_inputs(w, seed=12)
+    cot = make_cotangents(w, seed=13, device="cuda")
+    full, (o, to, lse, mu) = run(inp, cot, w.scale)
+    ws = torch.empty(ajvp.bwd_workspace_bytes(w.B, w.H, w.Lq), dtype=torch.uint8, device="cuda")
+    grads = None
+    for step in (0, 3, 1, 2):  # steps 1-3 only need step 0 before them
+        grads = ajvp.attn_jvp_bwd(*(inp[n] for n in NAMES), o, to, lse, mu, cot["dout"], cot["dtout"], w.scale,
+                                  grads=grads, workspace=ws, step=step)
+    torch.cuda.synchronize()
+    for n in full:
+        assert torch.equal(full[n], grads[n]), n
