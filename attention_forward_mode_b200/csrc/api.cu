@@ -8,6 +8,7 @@
 
 #include <algorithm>
 #include <atomic>
+#include <initializer_list>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -46,6 +47,12 @@ int fail_cuda(cudaError_t e) {
     return AJVP_ERR_CUDA;
 }
 
+template <int VAR>
+cudaError_t set_bwd_smem() {
+    return cudaFuncSetAttribute(ajvp::bwd::attn_jvp_bwd_kernel<VAR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)ajvp::bwd::Var<VAR>::SMEM_BYTES);
+}
+
 int device_setup(int *dev_out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -71,15 +78,11 @@ int device_setup(int *dev_out) {
         if (e3 == cudaSuccess)
             e3 = cudaFuncSetAttribute(ajvp::sm100::attn_jvp_fwd_kernel<true>,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ajvp::sm100::SMEM_BYTES);
-        if (e3 == cudaSuccess)
-            e3 = cudaFuncSetAttribute(ajvp::bwd::attn_jvp_bwd_kernel<ajvp::bwd::ROLE_Q>,
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ajvp::bwd::SMEM_BYTES);
-        if (e3 == cudaSuccess)
-            e3 = cudaFuncSetAttribute(ajvp::bwd::attn_jvp_bwd_kernel<ajvp::bwd::ROLE_K>,
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ajvp::bwd::SMEM_BYTES);
-        if (e3 == cudaSuccess)
-            e3 = cudaFuncSetAttribute(ajvp::bwd::attn_jvp_bwd_kernel<ajvp::bwd::ROLE_V>,
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ajvp::bwd::SMEM_BYTES);
+        if (e3 == cudaSuccess) e3 = set_bwd_smem<ajvp::bwd::V_DQ>();
+        if (e3 == cudaSuccess) e3 = set_bwd_smem<ajvp::bwd::V_DTQ>();
+        if (e3 == cudaSuccess) e3 = set_bwd_smem<ajvp::bwd::V_DK>();
+        if (e3 == cudaSuccess) e3 = set_bwd_smem<ajvp::bwd::V_DKT>();
+        if (e3 == cudaSuccess) e3 = set_bwd_smem<ajvp::bwd::V_DV>();
         cudaError_t e4 = cudaFuncSetAttribute(ajvp::f32::attn_jvp_fwd_f32_kernel,
                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
                                               (int)ajvp::f32::smem_bytes(ajvp::f32::DMAX));
@@ -200,22 +203,32 @@ uint64_t bwd_stats_bytes(int64_t BH, int64_t Lq) {
     return ((uint64_t)(BH * Lq + ajvp::bwd::BN) * 16u + 255u) / 256u * 256u;
 }
 
-template <int ROLE>
-int launch_bwd_role(const void *const r[4], const void *const c[4], void *out0, void *out1, const void *stats,
-                    int64_t BH, int64_t Lrow, int64_t Lcol, int64_t Lq, int64_t d, float scale, float out_scale,
-                    cudaStream_t stream) {
+// One backward variant: resident tensors r (row side, Lrow rows), streamed
+// tensors l (the long ring) and sh (the short stage), Lcol rows; outputs
+// out[] (Lrow rows) scaled by sc[].
+template <int VAR>
+int launch_bwd_var(std::initializer_list<const void *> r, std::initializer_list<const void *> l,
+                   std::initializer_list<const void *> sh, std::initializer_list<void *> out,
+                   std::initializer_list<float> sc, const void *stats, int64_t BH, int64_t Lrow, int64_t Lcol,
+                   int64_t Lq, int64_t d, float scale, cudaStream_t stream) {
     using namespace ajvp::bwd;
     int rc;
     Params p;
     std::memset(&p, 0, sizeof(p));
-    const int nr = ROLE == ROLE_V ? 2 : 4;
-    for (int i = 0; i < 4; ++i) {
-        const void *rp = i < nr ? r[i] : r[0];  // ROLE_V leaves R2, R3 unused
-        if ((rc = encode_3d(&p.tm_r[i], rp, d, Lrow, BH, 128)) != AJVP_OK) return rc;
-        if ((rc = encode_3d(&p.tm_c[i], c[i], d, Lcol, BH, 64)) != AJVP_OK) return rc;
-    }
-    if ((rc = encode_3d(&p.tm_out[0], out0, d, Lrow, BH, 128)) != AJVP_OK) return rc;
-    if ((rc = encode_3d(&p.tm_out[1], out1, d, Lrow, BH, 128)) != AJVP_OK) return rc;
+    int i = 0;
+    for (const void *x : r)
+        if ((rc = encode_3d(&p.tm_r[i++], x, d, Lrow, BH, 128)) != AJVP_OK) return rc;
+    i = 0;
+    for (const void *x : l)
+        if ((rc = encode_3d(&p.tm_l[i++], x, d, Lcol, BH, 64)) != AJVP_OK) return rc;
+    i = 0;
+    for (const void *x : sh)
+        if ((rc = encode_3d(&p.tm_s[i++], x, d, Lcol, BH, 64)) != AJVP_OK) return rc;
+    i = 0;
+    for (void *x : out)
+        if ((rc = encode_3d(&p.tm_out[i++], x, d, Lrow, BH, 128)) != AJVP_OK) return rc;
+    i = 0;
+    for (float f : sc) p.out_scale[i++] = f;
     const int64_t n_rtiles = (Lrow + BM - 1) / BM;
     p.stats = static_cast<const float4 *>(stats);
     p.Lrow = (int)Lrow;
@@ -224,9 +237,8 @@ int launch_bwd_role(const void *const r[4], const void *const c[4], void *out0, 
     p.n_rtiles = (int)n_rtiles;
     p.scale = scale;
     p.scale_log2 = scale * 1.4426950408889634f;
-    p.out_scale = out_scale;
     p.bound_ns = g_bound_ns.load();
-    attn_jvp_bwd_kernel<ROLE><<<(unsigned)(n_rtiles * BH), NTHREADS, SMEM_BYTES, stream>>>(p);
+    attn_jvp_bwd_kernel<VAR><<<(unsigned)(n_rtiles * BH), NTHREADS, Var<VAR>::SMEM_BYTES, stream>>>(p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail_cuda(e);
     return AJVP_OK;
@@ -318,8 +330,8 @@ uint64_t attn_jvp_bwd_workspace_bytes(int64_t B, int64_t H, int64_t Lq) {
 }  // extern "C"
 
 namespace {
-// Steps first..last of the backward (0 row statistics, 1 dQ/dtQ, 2 dK/dtK,
-// 3 dV/dtV) after the full argument check.
+// Kernels first..last of the backward (0 row statistics, 1 dQ, 2 dtQ, 3 dK,
+// 4 dtK and dtV, 5 dV) after the full argument check.
 int bwd_steps(int first, int last, const void *q, const void *k, const void *v, const void *tq, const void *tk,
               const void *tv, const void *o, const void *to, const float *lse, const float *mu, const void *dout,
               const void *dtout, void *dq, void *dk, void *dv, void *dtq, void *dtk, void *dtv, int64_t B, int64_t H,
@@ -336,11 +348,12 @@ int bwd_steps(int first, int last, const void *q, const void *k, const void *v, 
         if (!dk || !dv || !dtk || !dtv) return AJVP_ERR_INVALID_ARG;
         if (BH * Lk >= (int64_t(1) << 31)) return AJVP_ERR_TOO_LARGE;
         const size_t bytes = (size_t)(BH * Lk * d) * 2u;
-        void *zero_k[2] = {dk, dtk}, *zero_v[2] = {dv, dtv};
-        for (int i = 0; i < 2; ++i) {
-            cudaError_t e = cudaSuccess;
-            if (first <= 2 && last >= 2) e = cudaMemsetAsync(zero_k[i], 0, bytes, st);
-            if (e == cudaSuccess && first <= 3 && last >= 3) e = cudaMemsetAsync(zero_v[i], 0, bytes, st);
+        // the kernels that would write them: dk 3, dtk and dtv 4, dv 5
+        void *zero[4] = {dk, dtk, dtv, dv};
+        const int kern[4] = {3, 4, 4, 5};
+        for (int i = 0; i < 4; ++i) {
+            if (first > kern[i] || last < kern[i]) continue;
+            cudaError_t e = cudaMemsetAsync(zero[i], 0, bytes, st);
             if (e != cudaSuccess) return fail_cuda(e);
         }
         return AJVP_OK;
@@ -371,21 +384,25 @@ int bwd_steps(int first, int last, const void *q, const void *k, const void *v, 
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return fail_cuda(e);
     }
-    if (first <= 1 && last >= 1) {  // dQ, dtQ: rows = queries, streamed keys
-        const void *r[4] = {q, tq, dtout, dout}, *c[4] = {k, tk, v, tv};
-        if ((rc = launch_bwd_role<ROLE_Q>(r, c, dq, dtq, workspace, BH, Lq, Lk, Lq, d, scale, scale, st)) != AJVP_OK)
-            return rc;
-    }
-    if (first <= 2 && last >= 2) {  // dK, dtK: rows = keys, streamed queries
-        const void *r[4] = {k, tk, v, tv}, *c[4] = {q, tq, dtout, dout};
-        if ((rc = launch_bwd_role<ROLE_K>(r, c, dk, dtk, workspace, BH, Lk, Lq, Lq, d, scale, scale, st)) != AJVP_OK)
-            return rc;
-    }
-    if (first <= 3 && last >= 3) {  // dV, dtV: rows = keys, streamed queries
-        const void *r[4] = {k, tk, nullptr, nullptr}, *c[4] = {q, tq, dout, dtout};
-        if ((rc = launch_bwd_role<ROLE_V>(r, c, dv, dtv, workspace, BH, Lk, Lq, Lq, d, scale, 1.0f, st)) != AJVP_OK)
-            return rc;
-    }
+    auto want = [&](int k) { return first <= k && last >= k; };
+    const float s1 = scale;
+    // rows = queries, streamed keys
+    if (want(1) && (rc = launch_bwd_var<V_DQ>({q, tq, dtout, dout}, {k, tk}, {v, tv}, {dq}, {s1}, workspace, BH, Lq,
+                                              Lk, Lq, d, scale, st)) != AJVP_OK)
+        return rc;
+    if (want(2) && (rc = launch_bwd_var<V_DTQ>({q, dtout}, {k}, {v}, {dtq}, {s1}, workspace, BH, Lq, Lk, Lq, d, scale,
+                                               st)) != AJVP_OK)
+        return rc;
+    // rows = keys, streamed queries
+    if (want(3) && (rc = launch_bwd_var<V_DK>({k, tk, v, tv}, {q, tq}, {dtout, dout}, {dk}, {s1}, workspace, BH, Lk,
+                                              Lq, Lq, d, scale, st)) != AJVP_OK)
+        return rc;
+    if (want(4) && (rc = launch_bwd_var<V_DKT>({k, v}, {q, dtout}, {}, {dtk, dtv}, {s1, 1.0f}, workspace, BH, Lk, Lq,
+                                               Lq, d, scale, st)) != AJVP_OK)
+        return rc;
+    if (want(5) && (rc = launch_bwd_var<V_DV>({k, tk}, {dout, dtout}, {q, tq}, {dv}, {1.0f}, workspace, BH, Lk, Lq,
+                                              Lq, d, scale, st)) != AJVP_OK)
+        return rc;
     return AJVP_OK;
 }
 }  // namespace
@@ -397,7 +414,7 @@ int attn_jvp_bwd(const void *q, const void *k, const void *v, const void *tq, co
                  const void *dtout, void *dq, void *dk, void *dv, void *dtq, void *dtk, void *dtv, int64_t B,
                  int64_t H, int64_t Lq, int64_t Lk, int64_t d, float scale, void *workspace,
                  uint64_t workspace_bytes, void *stream) {
-    return bwd_steps(0, 3, q, k, v, tq, tk, tv, o, to, lse, mu, dout, dtout, dq, dk, dv, dtq, dtk, dtv, B, H, Lq, Lk,
+    return bwd_steps(0, 5, q, k, v, tq, tk, tv, o, to, lse, mu, dout, dtout, dq, dk, dv, dtq, dtk, dtv, B, H, Lq, Lk,
                      d, scale, workspace, workspace_bytes, stream);
 }
 
@@ -406,7 +423,7 @@ int attn_jvp_bwd_step(int step, const void *q, const void *k, const void *v, con
                       const void *dout, const void *dtout, void *dq, void *dk, void *dv, void *dtq, void *dtk,
                       void *dtv, int64_t B, int64_t H, int64_t Lq, int64_t Lk, int64_t d, float scale,
                       void *workspace, uint64_t workspace_bytes, void *stream) {
-    if (step < 0 || step > 3) return AJVP_ERR_INVALID_ARG;
+    if (step < 0 || step > 5) return AJVP_ERR_INVALID_ARG;
     return bwd_steps(step, step, q, k, v, tq, tk, tv, o, to, lse, mu, dout, dtout, dq, dk, dv, dtq, dtk, dtv, B, H,
                      Lq, Lk, d, scale, workspace, workspace_bytes, stream);
 }

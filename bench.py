@@ -45,10 +45,11 @@ BWD_METRIC = "attention+JVP backward TFLOP/s (30·Lq·Lk·d/head) and % of B200 
 BWD_KERNEL_SOURCES = ["attention_forward_mode_b200/csrc/jvp_bwd_sm100.cuh",
                       "attention_forward_mode_b200/csrc/ptx_sm100.cuh"]
 BWD_TRAFFIC_FILE = "profiles/attn_jvp_bwd_kernel.video_selfattn_b1h12_l32760.md"
-# backward kernels (steps of attn_jvp_bwd): name, contraction FLOPs per (Lq*Lk*d) per head
-BWD_STEPS = [("bwd_rowstats_kernel", 0.0), ("attn_jvp_bwd_kernel<ROLE_Q> (dQ, dtQ)", 18.0),
-             ("attn_jvp_bwd_kernel<ROLE_K> (dK, dtK)", 18.0), ("attn_jvp_bwd_kernel<ROLE_V> (dV, dtV)", 12.0)]
 L2_BYTES = 126 * 1024 * 1024
+# backward kernels (steps of attn_jvp_bwd): name, contraction FLOPs per (Lq*Lk*d) per head
+BWD_STEPS = [("bwd_rowstats_kernel", 0.0), ("attn_jvp_bwd_kernel<V_DQ> (dQ)", 16.0),
+             ("attn_jvp_bwd_kernel<V_DTQ> (dtQ)", 6.0), ("attn_jvp_bwd_kernel<V_DK> (dK)", 16.0),
+             ("attn_jvp_bwd_kernel<V_DKT> (dtK, dtV)", 8.0), ("attn_jvp_bwd_kernel<V_DV> (dV)", 10.0)]
 
 
 # ------------------------------------------------------------------ helpers
@@ -566,7 +567,7 @@ def run_ours_bwd(args, w):
                 "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                         "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps,
                         "path": "copy in, attn_jvp_bwd, copy out (serial on one stream)"},
-                "gpu_launches": 4 * args.steps, "clocks": clocks.summary()}
+                "gpu_launches": len(BWD_STEPS) * args.steps, "clocks": clocks.summary()}
         if world == 1 and not args.no_cpu_baseline:
             v, n, el, threads = oracle_bwd_sample(w, bwd_head0_cpu(inp, cot), args.cpu_seconds)
             line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
