@@ -81,7 +81,9 @@ enum : int {
     B_G2_DONE = 17,  // + long stage: the tile's G2 products complete (the stage is free again)
     B_ACC_FULL = 21,
     B_MMA_DRAIN = 22,
-    N_BARS = 23
+    B_R1_READY = 23,  // single-buffer variants: R1 written into tensor memory (256 arrivals)
+    B_ST_FULL = 24,   // + slot: V_DK's own two-slot ring of column statistics
+    N_BARS = 26
 };
 constexpr uint32_t OFF_TMEM_SLOT = 8 * N_BARS;
 constexpr uint32_t OFF_ABORT = OFF_TMEM_SLOT + 4;
@@ -90,6 +92,7 @@ constexpr uint32_t NB_EPI = 1;
 struct Params {
     CUtensorMap tm_r[4], tm_l[2], tm_s[2], tm_out[2];
     const float4 *stats;  // [B*H][Lq] {lse*log2(e), mu, a, D}, plus BN rows of padding
+    const __nv_bfloat16 *r1;  // single-buffer variants: R1 ([B*H][Lrow][128]), staged into tensor memory
     int Lrow, Lcol;       // row-side and streamed lengths
     int Lq;               // query rows per (batch, head): the stats row stride
     int n_rtiles;         // 128-row tiles per (batch, head)
@@ -154,7 +157,14 @@ struct Var {
     // streamed-tile rings: "long" (tiles G2 reads, freed when G2 completes) and
     // "short" (tiles only G1 reads, freed when G1 completes), as deep as shared
     // memory allows so that loads run well ahead of the products
-    static constexpr int kLS = (kSingle || VAR == V_DV) ? 2 : 4;
+    // single-buffer variants keep R1 in tensor memory (an A operand read from
+    // there) and use its shared-memory slot as a third long-ring stage
+    static constexpr bool kR1T = kSingle;
+    static constexpr int kLS = kSingle ? 3 : (VAR == V_DV ? 2 : 4);
+    // column statistics in shared memory: with the long-ring stage (double-buffer
+    // variants), or in a two-slot ring of their own freed by the elementwise warps (V_DK)
+    static constexpr bool kStatsSmem = kColStats;
+    static constexpr bool kStatsRing = kColStats && kSingle;
     static constexpr int kSS = kNS == 0 ? 0 : (kSingle ? 1 : (VAR == V_DV ? 3 : 4));
     static constexpr int kSSd = kSS > 0 ? kSS : 1;  // divisor for short-ring indices
     // a stage holds one or two [64 rows][128] tiles as [x c0 | y c0 | x c1 | y c1]
@@ -162,9 +172,12 @@ struct Var {
     static constexpr uint32_t L_CH = (kL1 ? 2u : 1u) * CHUNK_C, S_CH = (kNS > 1 ? 2u : 1u) * CHUNK_C;
     static constexpr uint32_t L_BYTES = 2 * L_CH, S_BYTES = 2 * S_CH;
     static constexpr uint32_t SM_L = SM_R + kNR * R_TILE;
-    static constexpr uint32_t SM_S = SM_L + kLS * L_BYTES;
+    static constexpr uint32_t SM_S = SM_L + (kR1T ? kLS - 1 : kLS) * L_BYTES;
     static constexpr uint32_t SM_ST = SM_S + kSS * S_BYTES;  // statistics of the long-ring tiles
-    static constexpr uint32_t SM_BAR = SM_ST + (kColStats ? kLS * STATS_TILE : 0u);
+    static constexpr uint32_t SM_BAR = SM_ST + (kStatsRing ? 2 * STATS_TILE : (kStatsSmem ? kLS * STATS_TILE : 0u));
+    __device__ static uint32_t long_off(int s) {  // offset of long-ring stage s
+        return (kR1T && s == kLS - 1) ? SM_R + R_TILE : SM_L + (uint32_t)s * L_BYTES;
+    }
     static constexpr uint32_t SMEM_BYTES = SM_BAR + 256;  // the base is 1024-byte aligned (checked)
     static_assert(SMEM_BYTES <= 232448, "exceeds the opt-in shared memory of one CTA");
     static_assert(8 * N_BARS + 8 <= 256, "barrier area");
@@ -173,6 +186,7 @@ struct Var {
     static constexpr uint32_t BUF_COLS = kSingle ? 256u : 128u;
     static constexpr uint32_t X = 0, Y = 64, Z = kSingle ? 128u : 64u, W = 192;  // inside a buffer
     static constexpr uint32_t E1 = BUF0 + 256u, E2 = BUF0 + 288u;               // single only
+    static constexpr uint32_t R1T = BUF0 + 320u;                                  // single only: R1 (64 columns)
 };
 
 template <int VAR>
@@ -209,6 +223,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
         }
         for (int b = 0; b < 2; ++b) mbar_init(BAR(B_G1_DONE + b), 1);
         mbar_init(BAR(B_X_FREE), EW_THREADS);
+        mbar_init(BAR(B_R1_READY), EW_THREADS);
+        mbar_init(BAR(B_ST_FULL), 1);
+        mbar_init(BAR(B_ST_FULL + 1), 1);
         mbar_init(BAR(B_E_DONE), EW_THREADS);
         mbar_init(BAR(B_ACC_FULL), 1);
         mbar_init(BAR(B_MMA_DRAIN), 1);
@@ -236,10 +253,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
         const bool lp = warp == 0;
         if (lane == 0 && (lp || C::kSS > 0)) {
             bool ok = true;
-            int l_last[4] = {-1, -1, -1, -1}, s_last[4] = {-1, -1, -1, -1};
+            int l_last[4] = {-1, -1, -1, -1}, s_last[4] = {-1, -1, -1, -1}, st_last = -1;
             if (lp) {
-                mbar_arrive_expect_tx(BAR(B_R_FULL), C::kNR * R_TILE);
+                mbar_arrive_expect_tx(BAR(B_R_FULL), (C::kNR - (C::kR1T ? 1 : 0)) * R_TILE);
                 for (int i = 0; i < C::kNR; ++i) {
+                    if (C::kR1T && i == 1) continue;  // R1 goes to tensor memory (elementwise warps)
                     tma_load_3d(base + SM_R + i * R_TILE, &p.tm_r[i], BAR(B_R_FULL), 0, r0, bh);
                     tma_load_3d(base + SM_R + i * R_TILE + CHUNK_R, &p.tm_r[i], BAR(B_R_FULL), 64, r0, bh);
                 }
@@ -253,16 +271,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
                         ok = false;
                         break;
                     }
-                    const uint32_t st = base + C::SM_L + s * C::L_BYTES;
+                    const uint32_t st = base + C::long_off(s);
                     const uint32_t fb = BAR(B_L_FULL + s);
-                    mbar_arrive_expect_tx(fb, (C::kL1 ? 4 : 2) * CHUNK_C + (C::kColStats ? STATS_TILE : 0));
+                    constexpr bool kWithStats = C::kStatsSmem && !C::kStatsRing;
+                    mbar_arrive_expect_tx(fb, (C::kL1 ? 4 : 2) * CHUNK_C + (kWithStats ? STATS_TILE : 0));
                     tma_load_3d(st, &p.tm_l[0], fb, 0, y, bh);
                     tma_load_3d(st + C::L_CH, &p.tm_l[0], fb, 64, y, bh);
                     if (C::kL1) {
                         tma_load_3d(st + CHUNK_C, &p.tm_l[1], fb, 0, y, bh);
                         tma_load_3d(st + C::L_CH + CHUNK_C, &p.tm_l[1], fb, 64, y, bh);
                     }
-                    if (C::kColStats)  // padded by BN rows past the last head: never out of bounds
+                    if (kWithStats)  // padded by BN rows past the last head: never out of bounds
                         bulk_load(base + C::SM_ST + s * STATS_TILE, p.stats + (size_t)bh * p.Lq + y, STATS_TILE, fb);
                     l_last[s] = t;
                 }
@@ -283,6 +302,18 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
                         tma_load_3d(st + C::S_CH + CHUNK_C, &p.tm_s[1], fb, 64, y, bh);
                     }
                     s_last[ss] = t;
+                    if (C::kStatsRing) {
+                        // statistics slot t % 2: free once the elementwise warps finished tile t - 2
+                        // (E_DONE phases are waited in order, so the parity is unambiguous)
+                        if (t >= 2 && !mbar_wait(BAR(B_E_DONE), (t - 2) & 1, abort_flag, bound)) {
+                            ok = false;
+                            break;
+                        }
+                        const uint32_t sb = BAR(B_ST_FULL + (t & 1));
+                        mbar_arrive_expect_tx(sb, STATS_TILE);  // padded by BN rows: never out of bounds
+                        bulk_load(base + C::SM_ST + (t & 1) * STATS_TILE, p.stats + (size_t)bh * p.Lq + y, STATS_TILE, sb);
+                        st_last = t;
+                    }
                 }
             }
             // every copy already issued lands before shared memory is released
@@ -291,6 +322,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
                 if (l_last[s] >= 0) mbar_wait_drain(BAR(B_L_FULL + s), (l_last[s] / C::kLS) & 1, bound);
             for (int s = 0; s < C::kSS; ++s)
                 if (s_last[s] >= 0) mbar_wait_drain(BAR(B_S_FULL + s), (s_last[s] / C::kSSd) & 1, bound);
+            for (int u = st_last - 1; u <= st_last; ++u)  // the last two statistics copies
+                if (C::kStatsRing && u >= 0) mbar_wait_drain(BAR(B_ST_FULL + (u & 1)), (u >> 1) & 1, bound);
         }
         __syncwarp();
     } else if (warp == 1) {
@@ -321,12 +354,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
             auto issue_g1 = [&](int j) -> bool {
                 const int b = j % C::kNB, s = j % C::kLS, ss = j % C::kSSd;
                 const uint32_t tb = tbase + C::BUF0 + (uint32_t)b * C::BUF_COLS;
-                const uint64_t dl = smem_desc_sw128(base + C::SM_L + s * C::L_BYTES, 16, 1024);
+                const uint64_t dl = smem_desc_sw128(base + C::long_off(s), 16, 1024);
                 const uint64_t ds = smem_desc_sw128(base + C::SM_S + ss * C::S_BYTES, 16, 1024);
                 if (VAR != V_DV && !wait_full(B_L_FULL, j, C::kLS)) return false;  // V_DV: G1 reads no long tile
                 if (VAR == V_DQ || VAR == V_DK) {
                     g1(tb + C::X, dr[0], dl, LC, ID_W, false);  // [X | Y] = R0 [L0; L1]^T
-                    g1(tb + C::Y, dr[1], dl, LC, ID_N, true);   // Y += R1 L0^T
+#pragma unroll
+                    for (int kk = 0; kk < HD / 16; ++kk)  // Y += R1 L0^T, R1 from tensor memory
+                        mma_ts(tb + C::Y, tbase + C::R1T + 8u * kk,
+                               desc_add(dl, (kk >> 2) * LC + (kk & 3) * 32), ID_N, 1u);
                     // the short stage is needed only now: its load overlaps the products above
                     if (!wait_full(B_S_FULL, j, C::kSSd)) return false;
                     g1(tb + C::Z, dr[2], ds, SC, ID_W, false);  // [Z | W] = R2 [S0; S1]^T
@@ -353,7 +389,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
                 const int b = j % C::kNB, s = j % C::kLS;
                 const uint32_t tb = tbase + C::BUF0 + (uint32_t)b * C::BUF_COLS;
                 // MN-major views of the long-ring tiles: chunks L_CH apart (LBO), 8 rows 1024 B apart
-                const uint64_t m0 = smem_desc_sw128(base + C::SM_L + s * C::L_BYTES, C::L_CH, 1024);
+                const uint64_t m0 = smem_desc_sw128(base + C::long_off(s), C::L_CH, 1024);
                 const uint64_t m1 = desc_add(m0, CHUNK_C);
                 const uint32_t e1 = C::kSingle ? tbase + C::E1 : tb + C::X;
                 const uint32_t e2 = C::kSingle ? tbase + C::E2 : tb + (VAR == V_DKT ? C::Z : C::Y);
@@ -379,6 +415,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
                 return true;
             };
             bool ok = mbar_wait(BAR(B_R_FULL), 0, abort_flag, bound);
+            if (ok && C::kR1T) ok = wait_full(B_R1_READY, 0, 1);
             if (ok) ok = issue_g1(0);
             for (int j = 0; j < nt && ok; ++j) {
                 if (j + 1 < nt) {
@@ -405,15 +442,43 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
         float4 rs = make_float4(0.f, 0.f, 0.f, 0.f);  // row statistics {lse2, mu, a, D} (query rows)
         if (!C::kColStats && r0 + row < p.Lrow) rs = p.stats[(size_t)bh * p.Lq + (size_t)(r0 + row)];
         bool failed = false;
+        if (C::kR1T) {
+            // R1 row `row` into tensor memory as bf16 pairs (column c = features 2c, 2c+1),
+            // the layout of an A operand; group grp writes features 64*grp .. 64*grp+63
+            uint32_t w[32];
+            if (r0 + row < p.Lrow) {
+                const uint4 *src = reinterpret_cast<const uint4 *>(
+                    p.r1 + ((size_t)bh * (size_t)p.Lrow + (size_t)(r0 + row)) * HD + 64u * (uint32_t)grp);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const uint4 v4 = __ldg(src + u);
+                    w[4 * u] = v4.x;
+                    w[4 * u + 1] = v4.y;
+                    w[4 * u + 2] = v4.z;
+                    w[4 * u + 3] = v4.w;
+                }
+            } else {
+#pragma unroll
+                for (int u = 0; u < 32; ++u) w[u] = 0u;
+            }
+            tmem_st32(tbase + lane_off + C::R1T + 32u * (uint32_t)grp, w);
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(BAR(B_R1_READY));
+        }
 
         // one pair of columns (c, c + 1 of this group): x scores, y score tangent,
         // z A, w B -> r1, r2 (see the variant table)
+        const float4 *cst = p.stats;  // column statistics of the current tile (read through L1)
         auto pair = [&](int c, int valid, uint32_t st_base, uint32_t xa, uint32_t xb, uint32_t ya, uint32_t yb,
                         uint32_t za, uint32_t zb, uint32_t wa, uint32_t wb, float2 &r1, float2 &r2) {
             float4 sa = rs, sb = rs;  // statistics of columns c and c + 1
-            if (C::kColStats) {
+            if (C::kStatsSmem) {
                 sa = ld_shared_f4(st_base + 16u * c);
                 sb = ld_shared_f4(st_base + 16u * (c + 1));
+            } else if (C::kColStats) {
+                sa = __ldg(cst + c);
+                sb = __ldg(cst + c + 1);
             }
             const float2 x = make_float2(__uint_as_float(xa), __uint_as_float(xb));
             const float2 t = __ffma2_rn(x, c2, make_float2(-sa.x, -sb.x));
@@ -450,12 +515,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
             const int b = j % C::kNB, s = j % C::kLS;
             if (!failed) failed = !mbar_wait_warp(BAR(B_G1_DONE + b), (j / C::kNB) & 1, abort_flag, bound);
             // the statistics came with the long-ring stage (bulk copy): observe its barrier too
-            if (C::kColStats && !failed)
+            if (C::kStatsRing && !failed)
+                failed = !mbar_wait_warp(BAR(B_ST_FULL + (j & 1)), (j >> 1) & 1, abort_flag, bound);
+            else if (C::kStatsSmem && !failed)
                 failed = !mbar_wait_warp(BAR(B_L_FULL + s), (j / C::kLS) & 1, abort_flag, bound);
             if (failed) continue;
             tc_fence_after();
+            cst = p.stats + (size_t)bh * p.Lq + (size_t)j * BN + col0;  // padded: never out of bounds
             const int valid = p.Lcol - j * BN - (int)col0;  // this group's columns inside the tensor
-            const uint32_t st_base = base + C::SM_ST + (uint32_t)s * STATS_TILE + col0 * 16u;
+            const uint32_t st_base =
+                base + C::SM_ST + (uint32_t)(C::kStatsRing ? (j & 1) : s) * STATS_TILE + col0 * 16u;
             const uint32_t tb = tbase + lane_off + C::BUF0 + (uint32_t)b * C::BUF_COLS;
             uint32_t e1[16], e2[16];
             if (C::kSingle) {
