@@ -32,9 +32,12 @@ _SRC = os.path.join(_HERE, "attn_jvp_oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
 _BWD_SRC = os.path.join(_HERE, "attn_jvp_bwd_oracle.c")
 _BWD_LIB = os.path.join(_HERE, "liboracle_bwd.so")
+_MSK_SRC = os.path.join(_HERE, "attn_jvp_masked_oracle.c")
+_MSK_LIB = os.path.join(_HERE, "liboracle_masked.so")
 _lock = threading.Lock()
 _lib = None
 _bwd_lib = None
+_msk_lib = None
 
 
 def _compile(src: str, lib: str, force: bool) -> str:
@@ -53,6 +56,7 @@ def build(force: bool = False) -> str:
     No -ffast-math: the oracle keeps IEEE fp64 semantics.
     """
     _compile(_BWD_SRC, _BWD_LIB, force)
+    _compile(_MSK_SRC, _MSK_LIB, force)
     return _compile(_SRC, _LIB, force)
 
 
@@ -74,6 +78,11 @@ def source_text() -> str:
 
 def bwd_source_text() -> str:
     with open(_BWD_SRC) as f:
+        return f.read()
+
+
+def masked_source_text() -> str:
+    with open(_MSK_SRC) as f:
         return f.read()
 
 
@@ -117,6 +126,30 @@ def _get_bwd():
             build()
             _bwd_lib = _bind_bwd(_BWD_LIB)
         return _bwd_lib
+
+
+def _bind_masked(path: str):
+    lib = ctypes.CDLL(path)
+    dp = ctypes.POINTER(ctypes.c_double)
+    ip = ctypes.POINTER(ctypes.c_int64)
+    lib.oracle_attn_jvp_masked_f64.argtypes = ([dp] * 9 + [ctypes.c_int64] * 4 + [ctypes.c_double, ip, ip,
+                                                                               ctypes.c_int64, ctypes.c_int])
+    lib.oracle_attn_jvp_masked_f64.restype = ctypes.c_int
+    return lib
+
+
+def _get_masked():
+    global _msk_lib
+    with _lock:
+        if _msk_lib is None:
+            build()
+            _msk_lib = _bind_masked(_MSK_LIB)
+        return _msk_lib
+
+
+def load_masked_variant(path: str):
+    """ctypes handle of a separately compiled masked-oracle build."""
+    return _bind_masked(path)
 
 
 def load_bwd_variant(path: str):
@@ -219,3 +252,46 @@ def attn_jvp_bwd(q, k, v, tq, tk, tv, dout, dtout, scale: float, qrows=None, kro
     if rc != 0:
         raise RuntimeError(f"oracle_attn_jvp_bwd_f64 failed with {rc}")
     return out
+
+
+def attn_jvp_packed(q, k, v, tq, tk, tv, scale: float, cu_q, cu_k, causal: bool, lib=None):
+    """Packed (variable-length) attention + JVP, optionally causal.
+
+    q, tq: [H, Tq, d]; k, v, tk, tv: [H, Tk, d]; cu_q, cu_k: cumulative
+    sequence starts (length nseq + 1, first 0, last Tq / Tk).  Causal means
+    key j of a sequence is visible to its query row i iff j <= i + (Lk - Lq).
+    Rows with no visible key give O = tO = 0, lse = -inf.  Returns fp64 numpy
+    (O [H, Tq, d], tO [H, Tq, d], lse [H, Tq]).
+    """
+    q, k, v, tq, tk, tv = (_f64(x) for x in (q, k, v, tq, tk, tv))
+    H, Tq, d = q.shape
+    Tk = k.shape[1]
+    cq = np.ascontiguousarray(np.asarray(cu_q, dtype=np.int64))
+    ck = np.ascontiguousarray(np.asarray(cu_k, dtype=np.int64))
+    o = np.empty((H, Tq, d))
+    to = np.empty_like(o)
+    lse = np.empty((H, Tq))
+    dp = ctypes.POINTER(ctypes.c_double)
+    ip = ctypes.POINTER(ctypes.c_int64)
+    ptr = lambda a: a.ctypes.data_as(dp)  # noqa: E731
+    handle = lib if lib is not None else _get_masked()
+    rc = handle.oracle_attn_jvp_masked_f64(ptr(q), ptr(k), ptr(v), ptr(tq), ptr(tk), ptr(tv), ptr(o), ptr(to),
+                                           ptr(lse), H, Tq, Tk, d, float(scale), cq.ctypes.data_as(ip),
+                                           ck.ctypes.data_as(ip), len(cq) - 1, int(bool(causal)))
+    if rc != 0:
+        raise RuntimeError(f"oracle_attn_jvp_masked_f64 failed with {rc}")
+    return o, to, lse
+
+
+def attn_jvp_causal(q, k, v, tq, tk, tv, scale: float, lib=None):
+    """Causal attention + JVP for dense [..., L, d] tensors (one sequence per
+    leading index; bottom-right aligned when Lq != Lk)."""
+    q, k, v, tq, tk, tv = (_f64(x) for x in (q, k, v, tq, tk, tv))
+    lead = q.shape[:-2]
+    Lq, d = q.shape[-2], q.shape[-1]
+    Lk = k.shape[-2]
+    BH = int(np.prod(lead)) if lead else 1
+    f = lambda x, L: x.reshape(BH, L, d)  # noqa: E731
+    o, to, lse = attn_jvp_packed(f(q, Lq), f(k, Lk), f(v, Lk), f(tq, Lq), f(tk, Lk), f(tv, Lk), scale,
+                                 [0, Lq], [0, Lk], True, lib=lib)
+    return o.reshape(q.shape), to.reshape(q.shape), lse.reshape(tuple(lead) + (Lq,))
