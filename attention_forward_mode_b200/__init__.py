@@ -23,11 +23,13 @@ from ._binding import (  # noqa: F401
     attn_jvp,
     attn_jvp_bwd,
     attn_jvp_fwd,
+    attn_jvp_fwd_causal,
     attn_jvp_fwd_f32,
     attn_jvp_fwd_f32out,
     attn_jvp_fwd_host,
     attn_jvp_fwd_host_noalloc,
     attn_jvp_fwd_stats,
+    attn_jvp_fwd_varlen,
     bwd_workspace_bytes,
     check_device_status,
     default_heads_per_chunk,
@@ -40,7 +42,7 @@ from ._binding import (  # noqa: F401
 )
 
 __all__ = [
-    "attn_jvp", "attn_jvp_bwd", "attn_jvp_fwd_stats", "bwd_workspace_bytes", "attn_jvp_fwd", "attn_jvp_fwd_f32", "attn_jvp_fwd_f32out", "attn_jvp_fwd_host", "attn_jvp_fwd_host_noalloc", "check_device_status",
+    "attn_jvp", "attn_jvp_bwd", "attn_jvp_fwd_causal", "attn_jvp_fwd_varlen", "attn_jvp_fwd_stats", "bwd_workspace_bytes", "attn_jvp_fwd", "attn_jvp_fwd_f32", "attn_jvp_fwd_f32out", "attn_jvp_fwd_host", "attn_jvp_fwd_host_noalloc", "check_device_status",
     "default_heads_per_chunk", "host_workspace_bytes", "load_library",
     "selftest_wait_timeout", "set_wait_bound_ns", "strerror", "version", "AttnJvpError",
 ]

@@ -28,7 +28,7 @@ AJVP_ERR_WORKSPACE = -8
 AJVP_ERR_DEVICE_LAYOUT = -9
 
 # every symbol the header declares
-EXPORTED = ("attn_jvp_fwd", "attn_jvp_fwd_f32out", "attn_jvp_fwd_stats", "attn_jvp_bwd", "attn_jvp_bwd_step",
+EXPORTED = ("attn_jvp_fwd", "attn_jvp_fwd_causal", "attn_jvp_fwd_varlen", "attn_jvp_fwd_f32out", "attn_jvp_fwd_stats", "attn_jvp_bwd", "attn_jvp_bwd_step",
             "attn_jvp_bwd_workspace_bytes", "attn_jvp_fwd_f32", "attn_jvp_fwd_host",
             "attn_jvp_fwd_host_noalloc", "attn_jvp_host_workspace_bytes", "attn_jvp_strerror",
             "attn_jvp_last_cuda_error",
@@ -63,6 +63,10 @@ def load_library(path: str = LIB_PATH):
         lib.attn_jvp_fwd_f32.restype = ctypes.c_int
         lib.attn_jvp_fwd_f32out.argtypes = fwd_args
         lib.attn_jvp_fwd_f32out.restype = ctypes.c_int
+        lib.attn_jvp_fwd_causal.argtypes = fwd_args
+        lib.attn_jvp_fwd_causal.restype = ctypes.c_int
+        lib.attn_jvp_fwd_varlen.argtypes = [vp] * 11 + [i64] * 6 + [f32, ctypes.c_int, vp]
+        lib.attn_jvp_fwd_varlen.restype = ctypes.c_int
         lib.attn_jvp_fwd_stats.argtypes = [vp] * 10 + [i64] * 5 + [f32, vp]
         lib.attn_jvp_fwd_stats.restype = ctypes.c_int
         lib.attn_jvp_bwd.argtypes = [vp] * 18 + [i64] * 5 + [f32, vp, ctypes.c_uint64, vp]
@@ -174,6 +178,60 @@ def attn_jvp_fwd_f32out(q, k, v, tq, tk, tv, scale=None, o=None, to=None, lse=No
     rc = lib.attn_jvp_fwd_f32out(_ptr(q), _ptr(k), _ptr(v), _ptr(tq), _ptr(tk), _ptr(tv), _ptr(o), _ptr(to),
                                  _ptr(lse), B, H, Lq, Lk, d, float(scale), _stream_handle(stream))
     _check(rc, "attn_jvp_fwd_f32out")
+    return o, to, lse
+
+
+def attn_jvp_fwd_causal(q, k, v, tq, tk, tv, scale=None, o=None, to=None, lse=None, stream=None, want_lse=True):
+    """``attn_jvp_fwd`` with a causal mask (key j visible to query row i iff
+    j <= i + Lk - Lq); rows that see no key give zeros and lse = -inf."""
+    o, to, lse, (B, H, Lq, Lk, d) = _prepare(q, k, v, tq, tk, tv, o, to, lse, torch.bfloat16, want_lse)
+    if scale is None:
+        scale = d ** -0.5
+    lib = load_library()
+    rc = lib.attn_jvp_fwd_causal(_ptr(q), _ptr(k), _ptr(v), _ptr(tq), _ptr(tk), _ptr(tv), _ptr(o), _ptr(to),
+                                 _ptr(lse), B, H, Lq, Lk, d, float(scale), _stream_handle(stream))
+    _check(rc, "attn_jvp_fwd_causal")
+    return o, to, lse
+
+
+def attn_jvp_fwd_varlen(q, k, v, tq, tk, tv, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, scale=None, causal=False,
+                        o=None, to=None, lse=None, stream=None, want_lse=True):
+    """Packed variable-length sequences: q, tq [H, total_q, d], k, v, tk, tv
+    [H, total_k, d] bf16 CUDA tensors; cu_seqlens_q / _k int32 CUDA tensors of
+    n_seq + 1 offsets.  Returns (o, to, lse) with o, to [H, total_q, d] and
+    lse [H, total_q]."""
+    for name, x in (("q", q), ("k", k), ("v", v), ("tq", tq), ("tk", tk), ("tv", tv)):
+        if not isinstance(x, torch.Tensor) or not x.is_cuda or x.dtype != torch.bfloat16 or x.dim() != 3 \
+                or not x.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA bf16 [H, total, d] tensor")
+    H, Tq, d = q.shape
+    Tk = k.shape[1]
+    if tq.shape != q.shape or any(x.shape != (H, Tk, d) for x in (k, v, tk, tv)):
+        raise ValueError("q, tq must be [H, total_q, d] and k, v, tk, tv [H, total_k, d]")
+    for name, c in (("cu_seqlens_q", cu_seqlens_q), ("cu_seqlens_k", cu_seqlens_k)):
+        if not isinstance(c, torch.Tensor) or not c.is_cuda or c.dtype != torch.int32 or c.dim() != 1 \
+                or not c.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA int32 vector")
+    if cu_seqlens_q.numel() != cu_seqlens_k.numel() or cu_seqlens_q.numel() < 1:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must have the same length n_seq + 1 >= 1")
+    if o is None:
+        o = torch.empty_like(q)
+    if to is None:
+        to = torch.empty_like(q)
+    if want_lse and lse is None:
+        lse = torch.empty((H, Tq), device=q.device, dtype=torch.float32)
+    for name, x in (("o", o), ("to", to)):
+        if x.shape != q.shape or x.dtype != torch.bfloat16 or not x.is_contiguous() or not x.is_cuda:
+            raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor of shape {tuple(q.shape)}")
+    if lse is not None and (lse.shape != (H, Tq) or lse.dtype != torch.float32 or not lse.is_contiguous()):
+        raise ValueError("lse must be a contiguous float32 [H, total_q] tensor")
+    if scale is None:
+        scale = d ** -0.5
+    lib = load_library()
+    rc = lib.attn_jvp_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(tq), _ptr(tk), _ptr(tv), _ptr(o), _ptr(to),
+                                 _ptr(lse), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), cu_seqlens_q.numel() - 1, H, Tq,
+                                 Tk, int(max_seqlen_q), d, float(scale), int(bool(causal)), _stream_handle(stream))
+    _check(rc, "attn_jvp_fwd_varlen")
     return o, to, lse
 
 

@@ -47,6 +47,12 @@ int fail_cuda(cudaError_t e) {
     return AJVP_ERR_CUDA;
 }
 
+template <bool kSplit, int MASK>
+cudaError_t set_fwd_smem() {
+    return cudaFuncSetAttribute(ajvp::sm100::attn_jvp_fwd_kernel<kSplit, MASK>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ajvp::sm100::SMEM_BYTES);
+}
+
 template <int VAR>
 cudaError_t set_bwd_smem() {
     return cudaFuncSetAttribute(ajvp::bwd::attn_jvp_bwd_kernel<VAR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -78,6 +84,9 @@ int device_setup(int *dev_out) {
         if (e3 == cudaSuccess)
             e3 = cudaFuncSetAttribute(ajvp::sm100::attn_jvp_fwd_kernel<true>,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ajvp::sm100::SMEM_BYTES);
+        if (e3 == cudaSuccess) e3 = set_fwd_smem<false, 1>();
+        if (e3 == cudaSuccess) e3 = set_fwd_smem<false, 2>();
+        if (e3 == cudaSuccess) e3 = set_fwd_smem<false, 3>();
         if (e3 == cudaSuccess) e3 = set_bwd_smem<ajvp::bwd::V_DQ>();
         if (e3 == cudaSuccess) e3 = set_bwd_smem<ajvp::bwd::V_DTQ>();
         if (e3 == cudaSuccess) e3 = set_bwd_smem<ajvp::bwd::V_DK>();
@@ -142,12 +151,16 @@ int check_common(const void *q, const void *k, const void *v, const void *tq, co
     return AJVP_OK;
 }
 
-// Shared host path of the two tensor-core entry points (kSplit: fp32 outputs,
-// split-bf16 probability operands).
-template <bool kSplit>
+// Shared host path of the tensor-core forward entry points (kSplit: fp32
+// outputs, split-bf16 probability operands; MASK: causal and/or packed
+// sequences -- packed calls pass B = 1, H, the total row counts as Lq, Lk and
+// the sequence offsets).
+template <bool kSplit, int MASK = 0>
 int launch_sm100(const void *q, const void *k, const void *v, const void *tq, const void *tk, const void *tv,
                  void *o, void *to, float *lse, int64_t B, int64_t H, int64_t Lq, int64_t Lk, int64_t d,
-                 float scale, void *stream, float *mu = nullptr) {
+                 float scale, void *stream, float *mu = nullptr, const int *cu_q = nullptr,
+                 const int *cu_k = nullptr, int64_t n_seq = 0, int64_t max_qtiles = 0) {
+    constexpr bool kPacked = (MASK & ajvp::sm100::MASK_PACKED) != 0;
     bool noop = false;
     int rc = check_common(q, k, v, tq, tk, tv, o, to, B, H, Lq, Lk, d, scale, &noop);
     if (rc != AJVP_OK || noop) return rc;
@@ -156,8 +169,10 @@ int launch_sm100(const void *q, const void *k, const void *v, const void *tq, co
     for (int i = 0; i < 10; ++i)
         if (ptrs[i] && !aligned(ptrs[i], 16)) return AJVP_ERR_MISALIGNED;
     const int64_t BH = B * H;
-    const int64_t n_qtiles = (Lq + ajvp::sm100::BR - 1) / ajvp::sm100::BR;
-    if (n_qtiles * BH >= (int64_t(1) << 31)) return AJVP_ERR_TOO_LARGE;
+    const int64_t n_qtiles = kPacked ? max_qtiles : (Lq + ajvp::sm100::BR - 1) / ajvp::sm100::BR;
+    const int64_t n_cta = n_qtiles * BH * (kPacked ? n_seq : 1);
+    if (n_cta >= (int64_t(1) << 31)) return AJVP_ERR_TOO_LARGE;
+    if (n_cta == 0) return AJVP_OK;
 
     int dev = 0;
     rc = device_setup(&dev);
@@ -182,6 +197,14 @@ int launch_sm100(const void *q, const void *k, const void *v, const void *tq, co
     }
     p.lse = lse;
     p.mu = mu;
+    if (!kSplit) {
+        p.o_bf = static_cast<__nv_bfloat16 *>(o);
+        p.to_bf = static_cast<__nv_bfloat16 *>(to);
+    }
+    p.cu_q = cu_q;
+    p.cu_k = cu_k;
+    p.n_seq = (int)n_seq;
+    p.BH = (int)BH;
     p.Lq = (int)Lq;
     p.Lk = (int)Lk;
     p.n_qtiles = (int)n_qtiles;
@@ -189,8 +212,8 @@ int launch_sm100(const void *q, const void *k, const void *v, const void *tq, co
     p.scale_log2 = scale * 1.4426950408889634f;
     p.bound_ns = g_bound_ns.load();
 
-    ajvp::sm100::attn_jvp_fwd_kernel<kSplit><<<(unsigned)(n_qtiles * BH), ajvp::sm100::NTHREADS,
-                                               ajvp::sm100::SMEM_BYTES, (cudaStream_t)stream>>>(p);
+    ajvp::sm100::attn_jvp_fwd_kernel<kSplit, MASK><<<(unsigned)n_cta, ajvp::sm100::NTHREADS,
+                                                     ajvp::sm100::SMEM_BYTES, (cudaStream_t)stream>>>(p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail_cuda(e);
     return AJVP_OK;
@@ -314,6 +337,36 @@ int attn_jvp_fwd_f32out(const void *q, const void *k, const void *v, const void 
                         const void *tv, float *o, float *to, float *lse, int64_t B, int64_t H, int64_t Lq,
                         int64_t Lk, int64_t d, float scale, void *stream) {
     return launch_sm100<true>(q, k, v, tq, tk, tv, o, to, lse, B, H, Lq, Lk, d, scale, stream);
+}
+
+int attn_jvp_fwd_causal(const void *q, const void *k, const void *v, const void *tq, const void *tk, const void *tv,
+                        void *o, void *to, float *lse, int64_t B, int64_t H, int64_t Lq, int64_t Lk, int64_t d,
+                        float scale, void *stream) {
+    return launch_sm100<false, ajvp::sm100::MASK_CAUSAL>(q, k, v, tq, tk, tv, o, to, lse, B, H, Lq, Lk, d, scale,
+                                                          stream);
+}
+
+int attn_jvp_fwd_varlen(const void *q, const void *k, const void *v, const void *tq, const void *tk, const void *tv,
+                        void *o, void *to, float *lse, const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                        int64_t n_seq, int64_t H, int64_t total_q, int64_t total_k, int64_t max_seqlen_q, int64_t d,
+                        float scale, int causal, void *stream) {
+    if (n_seq < 0 || max_seqlen_q < 0) return AJVP_ERR_INVALID_ARG;
+    if (n_seq == 0 || max_seqlen_q == 0) {
+        // nothing to compute; the size checks still apply
+        if (H < 0 || total_q < 0 || total_k < 1 || d < 1 || !std::isfinite(scale)) return AJVP_ERR_INVALID_ARG;
+        return AJVP_OK;
+    }
+    if (!cu_seqlens_q || !cu_seqlens_k) return AJVP_ERR_INVALID_ARG;
+    if (!aligned(cu_seqlens_q, 4) || !aligned(cu_seqlens_k, 4)) return AJVP_ERR_MISALIGNED;
+    if (n_seq >= (int64_t(1) << 31) || max_seqlen_q > total_q) return AJVP_ERR_INVALID_ARG;
+    const int64_t max_qtiles = (max_seqlen_q + ajvp::sm100::BR - 1) / ajvp::sm100::BR;
+    if (causal)
+        return launch_sm100<false, ajvp::sm100::MASK_PACKED | ajvp::sm100::MASK_CAUSAL>(
+            q, k, v, tq, tk, tv, o, to, lse, 1, H, total_q, total_k, d, scale, stream, nullptr, cu_seqlens_q,
+            cu_seqlens_k, n_seq, max_qtiles);
+    return launch_sm100<false, ajvp::sm100::MASK_PACKED>(q, k, v, tq, tk, tv, o, to, lse, 1, H, total_q, total_k, d,
+                                                          scale, stream, nullptr, cu_seqlens_q, cu_seqlens_k, n_seq,
+                                                          max_qtiles);
 }
 
 int attn_jvp_fwd_stats(const void *q, const void *k, const void *v, const void *tq, const void *tk, const void *tv,

@@ -101,18 +101,32 @@ struct Params {
     float *o_f32, *to_f32;  // kSplit: fp32 outputs [B*H][Lq][128] (tm_o / tm_to unused)
     float *lse;
     float *mu;  // optional [B*H][Lq]: mu_i = sum_j P_ij s dS'_ij (saved for the backward)
-    int Lq, Lk, n_qtiles;  // n_qtiles: 128-row query tiles per (batch, head)
+    __nv_bfloat16 *o_bf, *to_bf;  // bf16 outputs as plain pointers (packed rows, empty tiles)
+    const int *cu_q, *cu_k;       // packed sequences: starts of each sequence's rows (n_seq + 1)
+    int n_seq;                    // packed sequences per head
+    int BH;                       // dense: B*H; packed: H (the tensors' outermost extent)
+    int Lq, Lk, n_qtiles;  // rows per (batch, head) -- packed: total rows; n_qtiles: 128-row tiles
+                           // per (batch, head) -- packed: tiles of the longest sequence
     float scale;           // s
     float scale_log2;      // s * log2(e)
     unsigned long long bound_ns;
 };
 
+// Key masks (MASK bits): 1 causal -- key j is visible to query i of a sequence
+// iff j <= i + (Lk - Lq), bottom-right aligned; 2 packed -- the tensors are
+// [H][total][128] and sequence b owns rows cu_q[b] .. cu_q[b+1]-1 (queries)
+// and cu_k[b] .. cu_k[b+1]-1 (keys).  Rows with no visible key give zeros and
+// lse = -inf.
+constexpr int MASK_CAUSAL = 1, MASK_PACKED = 2;
+
 // kSplit = false: bf16 P and P.*s dS' operands, bf16 outputs.
 // kSplit = true : P and P.*s dS' are each split into bf16 hi + lo parts
 //                 (x = hi + lo to ~16 significant bits), both multiplied into
 //                 O and T, and O, tO are written in fp32; 1.5x the MMA work.
-template <bool kSplit>
+template <bool kSplit, int MASK = 0>
 __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_constant__ Params p) {
+    static_assert(!kSplit || MASK == 0, "the fp32-output variant has no masks");
+    constexpr bool kCausal = (MASK & MASK_CAUSAL) != 0, kPacked = (MASK & MASK_PACKED) != 0;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -120,10 +134,48 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int qt = blockIdx.x % p.n_qtiles;
-    const int bh = blockIdx.x / p.n_qtiles;
+    // this CTA's tile: outermost tensor index bh, local rows q0.. of a sequence whose
+    // rows start at tensor row yq - q0 and keys at yk0, with Lq_s rows and Lk_s keys
+    int qt, bh, Lq_s = p.Lq, Lk_s = p.Lk, yk0 = 0, yq0 = 0;
+    if (kPacked) {
+        // longest-first: the last tiles of every (sequence, head) go in the first wave
+        bh = blockIdx.x % p.BH;
+        const int rest = blockIdx.x / p.BH;
+        const int b = rest % p.n_seq;
+        qt = p.n_qtiles - 1 - rest / p.n_seq;
+        // clamped into the tensors, so that bad offsets stay memory-safe
+        const int a0 = min(max(p.cu_q[b], 0), p.Lq), a1 = min(max(p.cu_q[b + 1], a0), p.Lq);
+        const int k0 = min(max(p.cu_k[b], 0), p.Lk), k1 = min(max(p.cu_k[b + 1], k0), p.Lk);
+        yq0 = a0;
+        Lq_s = a1 - a0;
+        yk0 = k0;
+        Lk_s = k1 - k0;
+    } else if (kCausal) {
+        bh = blockIdx.x % p.BH;
+        qt = p.n_qtiles - 1 - blockIdx.x / p.BH;  // heavy (late) query tiles first
+    } else {
+        qt = blockIdx.x % p.n_qtiles;
+        bh = blockIdx.x / p.n_qtiles;
+    }
     const int q0 = qt * BR;
-    const int nk = (p.Lk + BC - 1) / BC;
+    const int yq = yq0 + q0;
+    if (kPacked && q0 >= Lq_s) return;  // past the end of this sequence (uniform for the CTA)
+    const int koff = Lk_s - Lq_s;        // causal offset of the diagonal
+    int kend = Lk_s;                     // keys any row of this tile may see
+    if (kCausal) kend = max(0, min(Lk_s, q0 + BR + koff));
+    const int nk = (kend + BC - 1) / BC;
+    if (MASK != 0 && nk == 0) {
+        // no row of the tile sees a key: zeros and lse = -inf, no pipeline at all
+        for (int r = threadIdx.x; r < BR && q0 + r < Lq_s; r += blockDim.x) {
+            const size_t row = (size_t)bh * (size_t)p.Lq + (size_t)(yq + r);
+            uint4 *po = reinterpret_cast<uint4 *>(p.o_bf + row * HD);
+            uint4 *pt = reinterpret_cast<uint4 *>(p.to_bf + row * HD);
+            for (int u = 0; u < HD / 8; ++u) po[u] = pt[u] = make_uint4(0u, 0u, 0u, 0u);
+            if (p.lse) p.lse[row] = -INFINITY;
+            if (p.mu) p.mu[row] = 0.f;
+        }
+        return;
+    }
     const uint64_t bound = p.bound_ns;
 
     const uint32_t bars = base + SM_BAR;
@@ -171,10 +223,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
             int kt_last[STAGES], vt_last[STAGES];
             for (int s = 0; s < STAGES; ++s) kt_last[s] = vt_last[s] = -1;
             mbar_arrive_expect_tx(BAR(B_Q_FULL), 4 * CHUNK_Q);
-            tma_load_3d(base + SM_Q, &p.tm_q, BAR(B_Q_FULL), 0, q0, bh);
-            tma_load_3d(base + SM_Q + CHUNK_Q, &p.tm_q, BAR(B_Q_FULL), 64, q0, bh);
-            tma_load_3d(base + SM_TQ, &p.tm_tq, BAR(B_Q_FULL), 0, q0, bh);
-            tma_load_3d(base + SM_TQ + CHUNK_Q, &p.tm_tq, BAR(B_Q_FULL), 64, q0, bh);
+            tma_load_3d(base + SM_Q, &p.tm_q, BAR(B_Q_FULL), 0, yq, bh);
+            tma_load_3d(base + SM_Q + CHUNK_Q, &p.tm_q, BAR(B_Q_FULL), 64, yq, bh);
+            tma_load_3d(base + SM_TQ, &p.tm_tq, BAR(B_Q_FULL), 0, yq, bh);
+            tma_load_3d(base + SM_TQ + CHUNK_Q, &p.tm_tq, BAR(B_Q_FULL), 64, yq, bh);
             // order of use by the MMA warp: KT_0, KT_1, VT_0, KT_2, VT_1, ...
             for (int t = 0; t <= nk && ok; ++t) {
                 if (t < nk) {
@@ -186,7 +238,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                     }
                     const uint32_t st = base + SM_KT + s * KT_STAGE;
                     const uint32_t fb = BAR(B_KT_FULL + s);
-                    const int y = t * BC;
+                    const int y = yk0 + t * BC;
                     mbar_arrive_expect_tx(fb, KT_STAGE);
                     // chunk c: K rows then tK rows, so [K | tK] is one N = 128 operand
                     tma_load_3d(st, &p.tm_k, fb, 0, y, bh);
@@ -204,7 +256,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                     }
                     const uint32_t st = base + SM_VT + s * VT_STAGE;
                     const uint32_t fb = BAR(B_VT_FULL + s);
-                    const int y = i * BC;
+                    const int y = yk0 + i * BC;
                     mbar_arrive_expect_tx(fb, VT_STAGE);
                     // [V c0 | V c1 | tV c0 | tV c1]: N-chunks 64 columns apart (LBO)
                     tma_load_3d(st, &p.tm_v, fb, 0, y, bh);
@@ -321,13 +373,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
         float *xch = reinterpret_cast<float *>(gbase + SM_XCH);
         float m_ref = -INFINITY, l = 0.f, g = 0.f;
         bool failed = false;
+        // keys this row sees (a prefix of the sequence's keys; may be <= 0 when causal)
+        const int kcount = kCausal ? min(Lk_s, q0 + row + koff + 1) : Lk_s;
 
         for (int j = 0; j < nk; ++j) {
             const int b = j & 1;
             const uint32_t t_s = tbase + lane_off + TM_BUF + 128u * b;
             if (!failed) failed = !mbar_wait_warp(BAR(B_SD_FULL + b), (j >> 1) & 1, abort_flag, bound);
             uint32_t xs[32], xd[32];
-            const int valid = p.Lk - j * BC - (int)col0;  // keys of this group inside Lk (may be <= 0)
+            const int valid = kcount - j * BC - (int)col0;  // visible keys of this group (may be <= 0)
             float part = sentinel;
             if (!failed) {
                 tc_fence_after();
@@ -469,7 +523,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
             tc_fence_after();
             const float lt = l + lg[(0 * 2 + (grp ^ 1)) * 128 + row];
             const float gt = g + lg[(1 * 2 + (grp ^ 1)) * 128 + row];
-            const float inv_l = 1.f / lt;
+            // a row that saw no key (masks only) has lt = 0: zeros, lse = -inf
+            const float inv_l = (MASK != 0 && !(lt > 0.f)) ? 0.f : 1.f / lt;
             const float mu = gt * inv_l;
             // group grp writes output columns 64*grp .. 64*grp+63
             if (kSplit) {
@@ -519,6 +574,20 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                     wo[i] = pack_bf16x2(o0, o1);
                     wt[i] = pack_bf16x2(t0, t1);
                 }
+                if (kPacked) {
+                    // rows past the sequence belong to the next one: plain guarded stores
+                    if (q0 + row < Lq_s) {
+                        const size_t off = ((size_t)bh * (size_t)p.Lq + (size_t)(yq + row)) * HD + 64u * grp + 32u * h;
+                        uint4 *po = reinterpret_cast<uint4 *>(p.o_bf + off);
+                        uint4 *pt = reinterpret_cast<uint4 *>(p.to_bf + off);
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            po[u] = make_uint4(wo[4 * u], wo[4 * u + 1], wo[4 * u + 2], wo[4 * u + 3]);
+                            pt[u] = make_uint4(wt[4 * u], wt[4 * u + 1], wt[4 * u + 2], wt[4 * u + 3]);
+                        }
+                    }
+                    continue;
+                }
                 const uint32_t chunk_off = (uint32_t)grp * CHUNK_Q + (uint32_t)row * 128u;
                 const uint32_t unit0 = (uint32_t)h * 4u;
 #pragma unroll
@@ -530,19 +599,20 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                                  wt[4 * u + 3]);
                 }
             }
-            if (grp == 0 && p.lse != nullptr && q0 + row < p.Lq) {
-                p.lse[(size_t)bh * (size_t)p.Lq + (size_t)(q0 + row)] =
-                    (m_ref + __log2f(lt)) * 0.69314718055994531f;
+            if (grp == 0 && p.lse != nullptr && q0 + row < Lq_s) {
+                p.lse[(size_t)bh * (size_t)p.Lq + (size_t)(yq + row)] =
+                    (MASK != 0 && !(lt > 0.f)) ? -INFINITY : (m_ref + __log2f(lt)) * 0.69314718055994531f;
             }
-            if (grp == 1 && p.mu != nullptr && q0 + row < p.Lq) p.mu[(size_t)bh * (size_t)p.Lq + (size_t)(q0 + row)] = mu;
+            if (grp == 1 && p.mu != nullptr && q0 + row < Lq_s)
+                p.mu[(size_t)bh * (size_t)p.Lq + (size_t)(yq + row)] = mu;
         }
         fence_proxy_async_smem();
         named_bar_sync(NB_EPI, SOFTMAX_THREADS);  // staging complete (every softmax thread gets here)
-        if (!kSplit && warp == 4 && lane == 0 && !any_failed && *abort_flag == 0) {
-            tma_store_3d(&p.tm_o, base + SM_Q, 0, q0, bh);
-            tma_store_3d(&p.tm_o, base + SM_Q + CHUNK_Q, 64, q0, bh);
-            tma_store_3d(&p.tm_to, base + SM_TQ, 0, q0, bh);
-            tma_store_3d(&p.tm_to, base + SM_TQ + CHUNK_Q, 64, q0, bh);
+        if (!kSplit && !kPacked && warp == 4 && lane == 0 && !any_failed && *abort_flag == 0) {
+            tma_store_3d(&p.tm_o, base + SM_Q, 0, yq, bh);
+            tma_store_3d(&p.tm_o, base + SM_Q + CHUNK_Q, 64, yq, bh);
+            tma_store_3d(&p.tm_to, base + SM_TQ, 0, yq, bh);
+            tma_store_3d(&p.tm_to, base + SM_TQ + CHUNK_Q, 64, yq, bh);
             tma_store_commit();
             tma_store_wait_all();
         }

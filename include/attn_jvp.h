@@ -115,6 +115,52 @@ AJVP_API int attn_jvp_fwd_f32out(const void *q, const void *k, const void *v,
                         float scale, void *stream);
 
 /*
+ * attn_jvp_fwd_causal -- attn_jvp_fwd with a causal mask: key j is visible to
+ * query row i iff j <= i + (Lk - Lq), i.e. the lower-triangular mask when
+ * Lq == Lk and bottom-right aligned otherwise.  Rows that see no key (only
+ * when Lq > Lk) get O = tO = 0 and lse = -infinity.  The pages do not
+ * describe masks; the arguments, layout and rules are those of
+ * attn_jvp_fwd.
+ */
+AJVP_API int attn_jvp_fwd_causal(const void *q, const void *k, const void *v,
+                        const void *tq, const void *tk, const void *tv,
+                        void *o, void *to, float *lse,
+                        int64_t B, int64_t H, int64_t Lq, int64_t Lk, int64_t d,
+                        float scale, void *stream);
+
+/*
+ * attn_jvp_fwd_varlen -- packed variable-length sequences (for example text
+ * conditions of different lengths in one batch), optionally causal.
+ *
+ *   q, tq, o, to        : __nv_bfloat16 [H][total_q][d]
+ *   k, v, tk, tv        : __nv_bfloat16 [H][total_k][d]
+ *   lse                 : float [H][total_q], or NULL
+ *   cu_seqlens_q / _k   : DEVICE int32 arrays of n_seq + 1 non-decreasing
+ *                         offsets, first 0, last total_q / total_k: sequence
+ *                         b is query rows cu_seqlens_q[b] .. cu_seqlens_q[b+1]-1
+ *                         and keys cu_seqlens_k[b] .. cu_seqlens_k[b+1]-1 of
+ *                         every head
+ *   max_seqlen_q        : at least the longest query sequence (sets the grid;
+ *                         rows of longer sequences would not be computed)
+ *   causal              : 0, or the causal rule of attn_jvp_fwd_causal inside
+ *                         each sequence
+ *
+ * Attention never crosses sequences.  A sequence with no keys (or a causal
+ * row with none visible) gives O = tO = 0 and lse = -infinity.  Offsets
+ * outside [0, total] are clamped in the kernel (memory-safe; the results of
+ * such a call are unspecified).  Supported: d == 128, total_k >= 1, the
+ * tensors 16-byte and the offset arrays 4-byte aligned; other rules as
+ * attn_jvp_fwd.  n_seq == 0, max_seqlen_q == 0 or total_q == 0 is a no-op.
+ */
+AJVP_API int attn_jvp_fwd_varlen(const void *q, const void *k, const void *v,
+                        const void *tq, const void *tk, const void *tv,
+                        void *o, void *to, float *lse,
+                        const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                        int64_t n_seq, int64_t H, int64_t total_q, int64_t total_k,
+                        int64_t max_seqlen_q, int64_t d, float scale, int causal,
+                        void *stream);
+
+/*
  * attn_jvp_fwd_stats -- attn_jvp_fwd that also saves, per query row, the
  * statistic mu_i = sum_j P_ij dS_ij (fp32 [B][H][Lq]) that attn_jvp_bwd needs
  * beside lse.  lse and mu are required (non-NULL, 16-byte aligned); all

@@ -120,3 +120,19 @@ def test_binding_raises_without_cuda_tensors(lib):
     x = torch.zeros(1, 1, 4, 128, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         B.attn_jvp_fwd(x, x, x, x, x, x)
+
+
+def test_varlen_host_rejections(lib):
+    f = lib.attn_jvp_fwd_varlen
+    vp = ctypes.c_void_p
+    p = vp(16)
+
+    def call(cu=vp(64), n_seq=2, total_q=100, total_k=90, max_q=60, d=128):
+        return f(p, p, p, p, p, p, p, p, None, cu, cu, n_seq, 2, total_q, total_k, max_q, d, 0.1, 0, None)
+
+    assert call(n_seq=0) == B.AJVP_OK and call(max_q=0) == B.AJVP_OK  # nothing to compute
+    assert call(cu=None) == B.AJVP_ERR_INVALID_ARG
+    assert call(cu=vp(66)) == B.AJVP_ERR_MISALIGNED
+    assert call(max_q=101) == B.AJVP_ERR_INVALID_ARG  # longer than the packed tensor
+    assert call(total_k=0) == B.AJVP_ERR_INVALID_ARG
+    assert call(d=64) == B.AJVP_ERR_UNSUPPORTED_DIM
