@@ -41,6 +41,7 @@ METRIC = "attention+JVP TFLOP/s (12·Lq·Lk·d/head) and % of B200 BF16 tensor p
 FALLBACK_BF16_TFLOPS = 1590.0
 KERNEL_SOURCES = ["attention_forward_mode_b200/csrc/jvp_sm100.cuh", "attention_forward_mode_b200/csrc/ptx_sm100.cuh"]
 TRAFFIC_FILE = "profiles/attn_jvp_fwd_kernel.video_selfattn_b1h12_l32760.md"
+MASKED_METRIC = "attention+JVP TFLOP/s (12·d per visible query-key pair) and % of B200 BF16 tensor peak"
 BWD_METRIC = "attention+JVP backward TFLOP/s (30·Lq·Lk·d/head) and % of B200 BF16 tensor peak"
 BWD_KERNEL_SOURCES = ["attention_forward_mode_b200/csrc/jvp_bwd_sm100.cuh",
                       "attention_forward_mode_b200/csrc/ptx_sm100.cuh"]
@@ -203,6 +204,39 @@ def oracle_sample(w, inputs_cpu_head, seconds: float, seed: int = 0):
     return flops / el / 1e12, rows, el, oracle.num_threads()
 
 
+def causal_flops(w) -> float:
+    """12 d FLOPs per visible (query, key) pair of the causal mask (key j
+    visible to query i iff j <= i + Lk - Lq), summed over the heads."""
+    i = torch.arange(w.Lq, dtype=torch.float64)
+    vis = torch.clamp(i + (w.Lk - w.Lq) + 1, 0, w.Lk).sum().item()
+    return 12.0 * w.d * w.B * w.H * vis
+
+
+def oracle_sample_causal(w, inputs_cpu_head, seconds: float):
+    """Time the fp64 masked oracle on the causal sub-problem made of the first
+    n query rows and the first n + Lk - Lq keys of one head (complete, so its
+    FLOPs are those of an n-row causal problem), n sized to about ``seconds``."""
+    import oracle
+    q, k, v, tq, tk, tv = inputs_cpu_head
+    off = w.Lk - w.Lq
+
+    def run(n):
+        nk = max(1, min(w.Lk, n + off))
+        t0 = time.perf_counter()
+        oracle.attn_jvp_causal(q[:n][None], k[:nk][None], v[:nk][None], tq[:n][None], tk[:nk][None],
+                               tv[:nk][None], w.scale)
+        el = time.perf_counter() - t0
+        i = torch.arange(n, dtype=torch.float64)
+        vis = torch.clamp(i + (nk - n) + 1, 0, nk).sum().item()
+        return el, 12.0 * w.d * vis
+
+    n0 = min(w.Lq, 512)
+    el0, _ = run(n0)
+    n = int(min(w.Lq, max(n0, n0 * (seconds / max(el0, 1e-6)) ** 0.5)))
+    el, fl = run(n)
+    return fl / el / 1e12, n, el, oracle.num_threads()
+
+
 def head0_cpu(inp):
     return tuple(inp[n][0, 0].detach().cpu() for n in ("q", "k", "v", "tq", "tk", "tv"))
 
@@ -261,9 +295,27 @@ def run_ours(args, w):
     ajvp.load_library()
 
     inp = make_inputs(w, seed=rank, device=dev)
-    # entry point: attn_jvp_fwd (bf16 outputs) or attn_jvp_fwd_f32out (fp32 outputs)
-    fwd = ajvp.attn_jvp_fwd if args.entry == "bf16" else ajvp.attn_jvp_fwd_f32out
-    out_dtype = torch.bfloat16 if args.entry == "bf16" else torch.float32
+    # entry point: attn_jvp_fwd (bf16 outputs), attn_jvp_fwd_f32out (fp32 outputs) or
+    # attn_jvp_fwd_causal (causal mask: FLOPs counted over the visible pairs only)
+    # or attn_jvp_fwd_varlen (the heads' tokens packed as 8 sequences of seeded lengths)
+    entry_name = {"bf16": "attn_jvp_fwd", "f32out": "attn_jvp_fwd_f32out", "causal": "attn_jvp_fwd_causal",
+                  "varlen": "attn_jvp_fwd_varlen"}[args.entry]
+    flops = causal_flops(w) if args.entry == "causal" else w.flops
+    seq_lens = None
+    if args.entry == "varlen":
+        import numpy as np
+        cuts = np.sort(np.random.default_rng(0).choice(np.arange(1, w.Lq), size=7, replace=False))
+        seq_lens = np.diff(np.concatenate([[0], cuts, [w.Lq]])).astype(int).tolist()
+        cu = torch.tensor(np.concatenate([[0], np.cumsum(seq_lens)]), dtype=torch.int32, device=dev)
+        flops = 12.0 * w.d * w.B * w.H * float(sum(n * n for n in seq_lens))
+
+        def fwd(q, k, v, tq, tk, tv, scale, o, to, lse, stream):
+            ajvp.attn_jvp_fwd_varlen(q[0], k[0], v[0], tq[0], tk[0], tv[0], cu, cu, max(seq_lens), scale,
+                                     o=o[0], to=to[0], lse=lse[0], stream=stream)
+    else:
+        fwd = {"bf16": ajvp.attn_jvp_fwd, "f32out": ajvp.attn_jvp_fwd_f32out,
+               "causal": ajvp.attn_jvp_fwd_causal}[args.entry]
+    out_dtype = torch.float32 if args.entry == "f32out" else torch.bfloat16
     o = torch.empty(inp["q"].shape, device=dev, dtype=out_dtype)
     to = torch.empty(inp["q"].shape, device=dev, dtype=out_dtype)
     lse = torch.empty((w.B, w.H, w.Lq), device=dev, dtype=torch.float32)
@@ -303,9 +355,9 @@ def run_ours(args, w):
     status = ajvp.check_device_status(stream)
     if status != ajvp.AJVP_OK:
         raise RuntimeError(f"kernel reported {ajvp.strerror(status)}")
-    value = aggregate_value(w.flops, args.steps, world, ms_max / 1e3)
+    value = aggregate_value(flops, args.steps, world, ms_max / 1e3)
     per_launch_s = ms / 1e3 / args.steps
-    achieved = w.flops / per_launch_s / 1e12
+    achieved = flops / per_launch_s / 1e12
 
     # ---- end to end: pinned host inputs -> device -> C ABI -> host, every step
     host_in = {n: t.detach().to("cpu").pin_memory() for n, t in inp.items()}
@@ -327,7 +379,7 @@ def run_ours(args, w):
                                    host_in["tv"], w.scale, o=host_o, to=host_to, lse=host_lse, workspace=ws,
                                    stream=stream)
     else:
-        e2e_path = "copy in, attn_jvp_fwd_f32out, copy out (serial on one stream)"
+        e2e_path = f"copy in, {entry_name}, copy out (serial on one stream)"
 
         def e2e_step():
             for n in inp:
@@ -350,23 +402,27 @@ def run_ours(args, w):
     ev3.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = max_over_ranks(ev2.elapsed_time(ev3), world, dev)
-    e2e_value = aggregate_value(w.flops, e2e_steps, world, e2e_ms / 1e3)
+    e2e_value = aggregate_value(flops, e2e_steps, world, e2e_ms / 1e3)
 
     line = None
     if rank == 0:
         burst, sustained, src = measured_peaks()
         clk = clocks.summary()
-        line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        line = {"metric": MASKED_METRIC if args.entry in ("causal", "varlen") else METRIC, "value": value,
+                "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-                "config": dict(workload_config(w, world), entry=("attn_jvp_fwd" if args.entry == "bf16"
-                                                                 else "attn_jvp_fwd_f32out")),
+                "config": dict(workload_config(w, world), entry=entry_name,
+                               **({"flops_per_step": "12·d per visible (query, key) pair"}
+                                  if args.entry in ("causal", "varlen") else {}),
+                               **({"sequence_lengths": seq_lens} if seq_lens else {})),
                 "pct_of_bf16_peak": 100.0 * value / world / burst,
                 "roofline": {"bound": "tensor", "achieved": achieved, "peak": burst, "unit": "TFLOP/s",
-                             "frac": achieved / burst, "traffic": committed_traffic(),
+                             "frac": achieved / burst,
+                             "traffic": committed_traffic() if args.entry == "bf16" else None,
                              "peak_source": f"{src} bf16 dense (burst) from MEASURED_PEAKS.json"
                              if src == "measured" else "fallback 1.59 PFLOP/s",
-                             "kernel": "attn_jvp_fwd_kernel", "algorithmic_flops_per_launch": w.flops,
+                             "kernel": "attn_jvp_fwd_kernel", "algorithmic_flops_per_launch": flops,
                              "algorithmic_bytes_per_launch": w.io_bytes},
                 "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                         "d2h_bytes_per_step": d2h, "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps,
@@ -374,12 +430,26 @@ def run_ours(args, w):
                 "gpu_launches": args.steps,
                 "clocks": clk}
         # CPU oracle next to the kernel: rank 0 at N = 1 only
-        if world == 1 and not args.no_cpu_baseline:
+        if world == 1 and not args.no_cpu_baseline and args.entry == "causal":
+            v, n, el, threads = oracle_sample_causal(w, head0_cpu(inp), args.cpu_seconds)
+            line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                                    "sample": f"causal sub-problem of the first {n} query rows and keys of head 0 "
+                                              f"({el:.1f} s, fp64, OpenMP)"}
+        elif world == 1 and not args.no_cpu_baseline and args.entry == "varlen":
+            import dataclasses
+            b0 = max(range(len(seq_lens)), key=lambda b: seq_lens[b])  # the longest sequence
+            a0, n0 = sum(seq_lens[:b0]), seq_lens[b0]
+            w0 = dataclasses.replace(w, Lq=n0, Lk=n0)
+            v, rows, el, threads = oracle_sample(w0, tuple(x[a0:a0 + n0] for x in head0_cpu(inp)), args.cpu_seconds)
+            line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                                    "sample": f"{rows} random query rows of sequence {b0} ({n0} tokens) of head 0 "
+                                              f"against its keys ({el:.1f} s, fp64, OpenMP)"}
+        elif world == 1 and not args.no_cpu_baseline:
             v, rows, el, threads = oracle_sample(w, head0_cpu(inp), args.cpu_seconds)
             line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                                     "sample": f"{rows} random query rows of head 0 against all {w.Lk} keys "
                                               f"({el:.1f} s, fp64, OpenMP)"}
-        if world == 1 and not args.no_eager:
+        if world == 1 and not args.no_eager and args.entry not in ("causal", "varlen"):
             line["eager_torch_jvp"] = eager_reference(w, inp)
     if world > 1:
         dist.barrier()
@@ -620,8 +690,9 @@ def main(argv=None):
     ap.add_argument("--reference-seconds", type=float, default=90.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-eager", action="store_true")
-    ap.add_argument("--entry", choices=["bf16", "f32out", "bwd"], default="bf16",
+    ap.add_argument("--entry", choices=["bf16", "f32out", "causal", "varlen", "bwd"], default="bf16",
                     help="f32out: time attn_jvp_fwd_f32out (fp32 outputs, split-bf16 probabilities); "
+                         "causal: attn_jvp_fwd_causal; varlen: attn_jvp_fwd_varlen on 8 packed sequences; "
                          "bwd: time the backward pass attn_jvp_bwd")
     ap.add_argument("--heads", type=int, default=None,
                     help="override H (small profiling captures); the JSON config shows the H used")
