@@ -141,3 +141,26 @@ def test_steps_equal_all_in_one():
     torch.cuda.synchronize()
     for n in full:
         assert torch.equal(full[n], grads[n]), n
+
+
+def test_video_workload_query_side_sampled():
+    # the bench's backward configuration (B=1, H=12, L=32760): dQ and dtQ rows can be
+    # computed by the oracle one by one (each needs all keys of its head, no other rows)
+    w = WORKLOADS["video_selfattn_b1h12_l32760_d128"]
+    inp = gpu_inputs(w)
+    cot = make_cotangents(w, device="cuda")
+    got, _ = run(inp, cot, w.scale)
+    rows = sample_rows(w.Lq, 12)
+    err = {"dq": 0.0, "dtq": 0.0}
+    for h in (0, 7, w.B * w.H - 1):
+        fl = {n: t.reshape(-1, t.shape[-2], t.shape[-1])[h] for n, t in {**inp, **cot}.items()}
+        ref = oracle.attn_jvp_bwd(*(fl[n][None] for n in NAMES), fl["dout"][None], fl["dtout"][None], w.scale,
+                                  qrows=rows, krows=[])
+        for n in ("dq", "dtq"):
+            e = max_rel(got[n].reshape(-1, w.Lq, w.d)[h][rows].float().cpu().numpy(), ref[n][0])
+            err[n] = max(err[n], e)
+    print(w.name, err)
+    for n, e in err.items():
+        assert e <= TOL, f"{n}: {e:.3e}"
+    del inp, cot, got
+    torch.cuda.empty_cache()

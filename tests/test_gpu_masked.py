@@ -123,3 +123,52 @@ def test_many_short_sequences():
     ref = oracle.attn_jvp_packed(*(x[n] for n in NAMES), s, cq.cpu().numpy(), ck.cpu().numpy(), True)
     seen = np.concatenate([np.arange(a) + (b - a) >= 0 for a, b in zip(lq, lk)])[None]
     check(got, ref, seen, "many short")
+
+
+def test_causal_video_workload_sampled():
+    # the bench configuration of --entry causal: rows checked one by one on their visible prefix
+    w = WORKLOADS["video_selfattn_b1h12_l32760_d128"]
+    inp = gpu_inputs(w)
+    o, to, lse = ajvp.attn_jvp_fwd_causal(*(inp[n] for n in NAMES), w.scale)
+    torch.cuda.synchronize()
+    rows = sample_rows(w.Lq, 16)
+    fl = {n: t.reshape(-1, t.shape[-2], t.shape[-1]) for n, t in inp.items()}
+    worst = {"o": 0.0, "to": 0.0, "lse": 0.0}
+    for h in (0, w.B * w.H - 1):
+        for i in rows:
+            r = oracle.attn_jvp(*(fl[n][h][i:i + 1][None] if n in ("q", "tq") else fl[n][h][:i + 1][None]
+                                  for n in NAMES), w.scale)
+            got = (o.reshape(-1, w.Lq, w.d)[h, i], to.reshape(-1, w.Lq, w.d)[h, i], lse.reshape(-1, w.Lq)[h, i])
+            for g, rr, key in zip(got, r, ("o", "to", "lse")):
+                worst[key] = max(worst[key], max_rel(g.float().cpu().numpy(), rr[0, 0]))
+    print(worst)
+    for key, e in worst.items():
+        assert e <= BOUND[key], (key, e)
+    del inp, o, to, lse
+    torch.cuda.empty_cache()
+
+
+def test_varlen_bench_configuration_sampled():
+    # the bench configuration of --entry varlen: the 12 heads' 32760 tokens as 8 sequences
+    w = WORKLOADS["video_selfattn_b1h12_l32760_d128"]
+    inp = gpu_inputs(w)
+    cuts = np.sort(np.random.default_rng(0).choice(np.arange(1, w.Lq), size=7, replace=False))
+    bounds = np.concatenate([[0], cuts, [w.Lq]]).astype(np.int64)
+    cu = torch.tensor(bounds, dtype=torch.int32, device="cuda")
+    x = {n: t[0] for n, t in inp.items()}
+    o, to, lse = ajvp.attn_jvp_fwd_varlen(*(x[n] for n in NAMES), cu, cu, int(np.diff(bounds).max()), w.scale)
+    torch.cuda.synchronize()
+    worst = {"o": 0.0, "to": 0.0, "lse": 0.0}
+    for h in (0, w.H - 1):
+        for b in (0, 3, 7):
+            a0, a1 = int(bounds[b]), int(bounds[b + 1])
+            rows = sorted({a0, a1 - 1, (a0 + a1) // 2})
+            ks = slice(a0, a1)
+            for r in rows:
+                ref = oracle.attn_jvp(*(x[n][h, r:r + 1][None] if n in ("q", "tq") else x[n][h, ks][None]
+                                        for n in NAMES), w.scale)
+                for g, rr, key in zip((o[h, r], to[h, r], lse[h, r]), ref, ("o", "to", "lse")):
+                    worst[key] = max(worst[key], max_rel(g.float().cpu().numpy(), rr[0, 0]))
+    print(worst)
+    for key, e in worst.items():
+        assert e <= BOUND[key], (key, e)
