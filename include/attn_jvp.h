@@ -31,8 +31,10 @@
  * allocates no device memory per call and keeps no per-call state.  Calls
  * are stream-ordered and asynchronous: they return
  * after enqueueing work on `stream` (a cudaStream_t; NULL = legacy default
- * stream) and do not synchronise.  Calls are thread-safe.  Inputs must not
- * alias outputs.  Non-finite inputs give unspecified (but memory-safe)
+ * stream) and do not synchronise.  The device-buffer calls enqueue kernels
+ * only (attn_jvp_bwd with Lq == 0: memsets), so after one eager call on a
+ * device (which does its one-time set-up) they can be captured into a CUDA
+ * graph.  Calls are thread-safe.  Inputs must not alias outputs.  Non-finite inputs give unspecified (but memory-safe)
  * results.
  *
  * Errors: argument checks run on the host before any launch and return a
