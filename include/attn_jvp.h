@@ -16,9 +16,10 @@
  *   lse = ln sum_j exp(S_ij)          (natural log, fp32)
  *
  * computed in one pass over the keys with an online softmax: P and dS are
- * never written to memory.  Non-causal, no mask, no dropout; Lq may differ
- * from Lk (cross-attention).  s is a constant (no derivative with respect to
- * it).
+ * never written to memory.  No dropout; Lq may differ from Lk
+ * (cross-attention); attn_jvp_fwd_causal and attn_jvp_fwd_varlen add a
+ * causal mask and packed variable-length sequences, attn_jvp_bwd the
+ * backward pass.  s is a constant (no derivative with respect to it).
  *
  * Layout: every tensor is a contiguous row-major [B][H][L][d] array (the
  * layout of a PyTorch [B, H, L, d] tensor); the tangents tQ, tK, tV share the
@@ -34,8 +35,8 @@
  * stream) and do not synchronise.  The device-buffer calls enqueue kernels
  * only (attn_jvp_bwd with Lq == 0: memsets), so after one eager call on a
  * device (which does its one-time set-up) they can be captured into a CUDA
- * graph.  Calls are thread-safe.  Inputs must not alias outputs.  Non-finite inputs give unspecified (but memory-safe)
- * results.
+ * graph.  Calls are thread-safe.  Inputs must not alias outputs.  Non-finite
+ * inputs give unspecified (but memory-safe) results.
  *
  * Errors: argument checks run on the host before any launch and return a
  * negative ajvp_status; nothing is enqueued then.  A failed launch returns
