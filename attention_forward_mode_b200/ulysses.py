@@ -19,6 +19,11 @@ packed all-to-all, the outputs in one more (plus one for lse).  The exchange
 uses torch.distributed (NCCL on GPUs); the attention itself is the library's
 kernel (``local_fn``, by default the C ABI entry point for the inputs'
 dtype).
+
+``ulysses_attn_jvp_train`` / ``ulysses_attn_jvp_bwd`` add the backward: the
+forward keeps its head-sharded inputs and outputs, the backward sends the
+cotangents dO, dtO to head shards, runs the local backward there and returns
+the six gradients to sequence shards.
 """
 from __future__ import annotations
 
@@ -79,3 +84,60 @@ def ulysses_attn_jvp(q, k, v, tq, tk, tv, scale=None, group=None, local_fn=None)
     lse_s = _to_sequence(lse.unsqueeze(0).unsqueeze(-1).contiguous(), world, group)[0, ..., 0]
     assert out.shape[3] == Lqs and ks.shape[3] == Lks * world
     return out[0], out[1], lse_s
+
+
+def ulysses_attn_jvp_train(q, k, v, tq, tk, tv, scale=None, group=None, local_fwd=None):
+    """Forward of ``ulysses_attn_jvp`` that also keeps what the backward needs.
+
+    Returns (o, to, lse, ctx): the sequence-sharded outputs as
+    ``ulysses_attn_jvp`` gives them, and ``ctx`` for ``ulysses_attn_jvp_bwd``
+    holding the head-sharded inputs and the forward's head-sharded O, tO, lse
+    and mu.  ``local_fwd(q, k, v, tq, tk, tv, scale) -> (o, to, lse, mu)``
+    defaults to the library's ``attn_jvp_fwd_stats``.
+    """
+    from ._binding import attn_jvp_fwd_stats
+    grouped = dist.is_initialized()
+    world = dist.get_world_size(group) if grouped else 1
+    B, H, Lqs, d = q.shape
+    if H % world != 0:
+        raise ValueError(f"heads ({H}) must divide by the group size ({world})")
+    if scale is None:
+        scale = d ** -0.5
+    fn = local_fwd if local_fwd is not None else attn_jvp_fwd_stats
+    if not grouped:
+        o, to, lse, mu = fn(q, k, v, tq, tk, tv, scale)
+        ctx = dict(inputs=(q, k, v, tq, tk, tv), outputs=(o, to, lse, mu), scale=scale, world=1)
+        return o, to, lse, ctx
+    qs = _to_heads(torch.stack((q, tq)), world, group)        # [2, B, H/P, Lq, d]
+    ks = _to_heads(torch.stack((k, v, tk, tv)), world, group)  # [4, B, H/P, Lk, d]
+    inputs = (qs[0].contiguous(), ks[0].contiguous(), ks[1].contiguous(), qs[1].contiguous(), ks[2].contiguous(),
+              ks[3].contiguous())
+    o, to, lse, mu = fn(*inputs, scale)
+    out = _to_sequence(torch.stack((o, to)), world, group)
+    lse_s = _to_sequence(lse.unsqueeze(0).unsqueeze(-1).contiguous(), world, group)[0, ..., 0]
+    ctx = dict(inputs=inputs, outputs=(o, to, lse, mu), scale=scale, world=world)
+    return out[0], out[1], lse_s, ctx
+
+
+def ulysses_attn_jvp_bwd(ctx, dout, dtout, group=None, local_bwd=None):
+    """Backward of ``ulysses_attn_jvp_train``: the gradients of
+    <dout, O> + <dtout, tO> with respect to the six sequence-sharded inputs.
+
+    ``dout``, ``dtout``: sequence-sharded cotangents [B, H, Lq/P, d].  They go
+    to head shards (one packed all-to-all), the local backward runs on the
+    head-sharded tensors the forward kept, and the gradients return to
+    sequence shards (one all-to-all for the query side, one for the key
+    side).  ``local_bwd(q, k, v, tq, tk, tv, o, to, lse, mu, dout, dtout,
+    scale) -> dict`` defaults to the library's ``attn_jvp_bwd``.  Returns a
+    dict dq, dk, dv, dtq, dtk, dtv shaped like the inputs.
+    """
+    from ._binding import attn_jvp_bwd
+    fn = local_bwd if local_bwd is not None else attn_jvp_bwd
+    world = ctx["world"]
+    if world == 1:
+        return fn(*ctx["inputs"], *ctx["outputs"], dout, dtout, ctx["scale"])
+    cot = _to_heads(torch.stack((dout, dtout)), world, group)  # [2, B, H/P, Lq, d]
+    g = fn(*ctx["inputs"], *ctx["outputs"], cot[0].contiguous(), cot[1].contiguous(), ctx["scale"])
+    qside = _to_sequence(torch.stack((g["dq"], g["dtq"])), world, group)
+    kside = _to_sequence(torch.stack((g["dk"], g["dv"], g["dtk"], g["dtv"])), world, group)
+    return {"dq": qside[0], "dtq": qside[1], "dk": kside[0], "dv": kside[1], "dtk": kside[2], "dtv": kside[3]}

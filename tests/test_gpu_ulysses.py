@@ -1,6 +1,8 @@
 """The Ulysses wrapper on the GPU through NCCL: with a one-rank NCCL group the
 two all-to-all exchanges run for real (as identity exchanges) around the CUDA
-kernel, and the result must equal a direct attn_jvp_fwd call bit for bit.
+kernel, and the result must equal a direct attn_jvp_fwd call bit for bit; the
+same for the training path (forward keeping its head shards, backward
+exchanges around attn_jvp_bwd).
 (Exchanges across several ranks are checked on CPU over gloo.)"""
 import datetime
 import os
@@ -33,5 +35,18 @@ def test_one_rank_nccl_equals_direct_call():
         torch.cuda.synchronize()
         for x, y in zip(a, b):
             assert torch.equal(x, y)
+        # training path: forward keeping its head shards, then the backward exchanges
+        from attention_forward_mode_b200.ulysses import ulysses_attn_jvp_bwd, ulysses_attn_jvp_train
+        from attention_forward_mode_b200.workloads import make_cotangents
+        names = ("q", "k", "v", "tq", "tk", "tv")
+        cot = make_cotangents(w, seed=4, device="cuda")
+        o, to, lse, ctx = ulysses_attn_jvp_train(*(inp[n] for n in names), scale=w.scale)
+        g = ulysses_attn_jvp_bwd(ctx, cot["dout"], cot["dtout"])
+        ro, rto, rlse, rmu = ajvp.attn_jvp_fwd_stats(*(inp[n] for n in names), w.scale)
+        rg = ajvp.attn_jvp_bwd(*(inp[n] for n in names), ro, rto, rlse, rmu, cot["dout"], cot["dtout"], w.scale)
+        torch.cuda.synchronize()
+        assert torch.equal(o, ro) and torch.equal(to, rto) and torch.equal(lse, rlse)
+        for n in ajvp.GRAD_NAMES:
+            assert torch.equal(g[n], rg[n]), n
     finally:
         dist.destroy_process_group()

@@ -95,3 +95,72 @@ def test_heads_must_divide():
             ulysses.ulysses_attn_jvp(t["q"], t["k"], t["v"], t["tq"], t["tk"], t["tv"], local_fn=_oracle_fn)
     finally:
         ulysses.dist.is_initialized, ulysses.dist.get_world_size = orig
+
+
+def _oracle_fwd_train(q, k, v, tq, tk, tv, scale):
+    o, to, lse = _oracle_fn(q, k, v, tq, tk, tv, scale)
+    return o, to, lse, torch.zeros_like(lse)  # the oracle backward recomputes everything it needs
+
+
+def _oracle_bwd(q, k, v, tq, tk, tv, o, to, lse, mu, dout, dtout, scale):
+    import oracle
+    g = oracle.attn_jvp_bwd(q, k, v, tq, tk, tv, dout, dtout, scale)
+    return {n: torch.from_numpy(x) for n, x in g.items()}
+
+
+def _bwd_worker(rank, world, port, shape, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from attention_forward_mode_b200.ulysses import ulysses_attn_jvp_bwd, ulysses_attn_jvp_train
+        B, H, Lq, Lk, d = shape
+        full = _inputs(B, H, Lq, Lk, d, seed=11)
+        g = torch.Generator().manual_seed(12)
+        cot = {n: torch.randn((B, H, Lq, d), generator=g, dtype=torch.float64) for n in ("dout", "dtout")}
+        sq, sk = Lq // world, Lk // world
+        qsl, ksl = slice(rank * sq, (rank + 1) * sq), slice(rank * sk, (rank + 1) * sk)
+        shard = {n: (t[:, :, qsl] if n in ("q", "tq") else t[:, :, ksl]).contiguous() for n, t in full.items()}
+        o, to, lse, ctx = ulysses_attn_jvp_train(*(shard[n] for n in ("q", "k", "v", "tq", "tk", "tv")), scale=0.3,
+                                                 local_fwd=_oracle_fwd_train)
+        grads = ulysses_attn_jvp_bwd(ctx, cot["dout"][:, :, qsl].contiguous(), cot["dtout"][:, :, qsl].contiguous(),
+                                     local_bwd=_oracle_bwd)
+        ref = _oracle_bwd(*(full[n] for n in ("q", "k", "v", "tq", "tk", "tv")), None, None, None, None,
+                          cot["dout"], cot["dtout"], 0.3)
+        eq = {n: bool(torch.equal(grads[n], ref[n][:, :, qsl if n in ("dq", "dtq") else ksl])) for n in ref}
+        out[rank] = (eq, {n: tuple(t.shape) for n, t in grads.items()})
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.timeout(300)
+@pytest.mark.parametrize("world,shape", [(2, (1, 4, 16, 24, 8)),   # cross-attention shapes
+                                         (4, (1, 8, 32, 32, 4))])  # four ranks
+def test_ulysses_backward_matches_unsharded(world, shape):
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as m:
+        out = m.dict()
+        procs = [ctx.Process(target=_bwd_worker, args=(r, world, port, shape, out)) for r in range(world)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(240)
+        assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
+        res = dict(out)
+    B, H, Lq, Lk, d = shape
+    for r in range(world):
+        eq, shapes = res[r]
+        assert all(eq.values()), (r, eq)
+        assert shapes["dq"] == (B, H, Lq // world, d) and shapes["dk"] == (B, H, Lk // world, d)
+
+
+def test_single_rank_backward_is_the_local_call():
+    from attention_forward_mode_b200.ulysses import ulysses_attn_jvp_bwd, ulysses_attn_jvp_train
+    t = _inputs(1, 2, 8, 6, 4, seed=3)
+    names = ("q", "k", "v", "tq", "tk", "tv")
+    _, _, _, ctx = ulysses_attn_jvp_train(*(t[n] for n in names), scale=0.5, local_fwd=_oracle_fwd_train)
+    dout, dtout = torch.ones(1, 2, 8, 4, dtype=torch.float64), torch.full((1, 2, 8, 4), 0.5, dtype=torch.float64)
+    a = ulysses_attn_jvp_bwd(ctx, dout, dtout, local_bwd=_oracle_bwd)
+    b = _oracle_bwd(*(t[n] for n in names), None, None, None, None, dout, dtout, 0.5)
+    for n in b:
+        assert torch.equal(a[n], b[n])
