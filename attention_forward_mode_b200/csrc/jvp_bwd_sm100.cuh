@@ -332,9 +332,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
             constexpr uint32_t ID_W = idesc_bf16_f32(128, 128, 0);  // R [Cx; Cy]^T
             constexpr uint32_t ID_N = idesc_bf16_f32(128, 64, 0);   // R Cx^T
             constexpr uint32_t ID_G2 = idesc_bf16_f32(128, 128, 1);  // E C (C read MN-major)
-            uint64_t dr[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) dr[i] = smem_desc_sw128(base + SM_R + i * R_TILE, 16, 1024);
+            // descriptors of the resident tiles, as scalars (an array captured by the
+            // lambdas below would live in local memory and delay every MMA issue)
+            const uint64_t dr0 = smem_desc_sw128(base + SM_R, 16, 1024);
+            const uint64_t dr1 = desc_add(dr0, R_TILE), dr2 = desc_add(dr0, 2 * R_TILE), dr3 = desc_add(dr0, 3 * R_TILE);
             // K-x-K products over d = 128: 8 K-steps; a tile's two 64-column chunks are
             // CHUNK_R (resident) and ch (streamed stage) apart
             auto g1 = [&](uint32_t d, uint64_t a, uint64_t b, uint32_t ch, uint32_t id, bool acc) {
@@ -358,26 +359,26 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
                 const uint64_t ds = smem_desc_sw128(base + C::SM_S + ss * C::S_BYTES, 16, 1024);
                 if (VAR != V_DV && !wait_full(B_L_FULL, j, C::kLS)) return false;  // V_DV: G1 reads no long tile
                 if (VAR == V_DQ || VAR == V_DK) {
-                    g1(tb + C::X, dr[0], dl, LC, ID_W, false);  // [X | Y] = R0 [L0; L1]^T
+                    g1(tb + C::X, dr0, dl, LC, ID_W, false);  // [X | Y] = R0 [L0; L1]^T
 #pragma unroll
                     for (int kk = 0; kk < HD / 16; ++kk)  // Y += R1 L0^T, R1 from tensor memory
                         mma_ts(tb + C::Y, tbase + C::R1T + 8u * kk,
                                desc_add(dl, (kk >> 2) * LC + (kk & 3) * 32), ID_N, 1u);
                     // the short stage is needed only now: its load overlaps the products above
                     if (!wait_full(B_S_FULL, j, C::kSSd)) return false;
-                    g1(tb + C::Z, dr[2], ds, SC, ID_W, false);  // [Z | W] = R2 [S0; S1]^T
-                    g1(tb + C::W, dr[3], ds, SC, ID_N, true);   // W += R3 S0^T
+                    g1(tb + C::Z, dr2, ds, SC, ID_W, false);  // [Z | W] = R2 [S0; S1]^T
+                    g1(tb + C::W, dr3, ds, SC, ID_N, true);   // W += R3 S0^T
                 } else if (VAR == V_DTQ) {
-                    g1(tb + C::X, dr[0], dl, LC, ID_N, false);  // X = R0 L0^T
+                    g1(tb + C::X, dr0, dl, LC, ID_N, false);  // X = R0 L0^T
                     if (!wait_full(B_S_FULL, j, C::kSSd)) return false;
-                    g1(tb + C::Z, dr[1], ds, SC, ID_N, false);  // Z = R1 S0^T
+                    g1(tb + C::Z, dr1, ds, SC, ID_N, false);  // Z = R1 S0^T
                 } else if (VAR == V_DKT) {
-                    g1(tb + C::X, dr[0], dl, LC, ID_N, false);                     // X = R0 L0^T
-                    g1(tb + C::Z, dr[1], desc_add(dl, CHUNK_C), LC, ID_N, false);  // Z = R1 L1^T
+                    g1(tb + C::X, dr0, dl, LC, ID_N, false);                     // X = R0 L0^T
+                    g1(tb + C::Z, dr1, desc_add(dl, CHUNK_C), LC, ID_N, false);  // Z = R1 L1^T
                 } else {  // V_DV
                     if (!wait_full(B_S_FULL, j, C::kSSd)) return false;
-                    g1(tb + C::X, dr[0], ds, SC, ID_W, false);  // [X | Y] = R0 [S0; S1]^T
-                    g1(tb + C::Y, dr[1], ds, SC, ID_N, true);   // Y += R1 S0^T
+                    g1(tb + C::X, dr0, ds, SC, ID_W, false);  // [X | Y] = R0 [S0; S1]^T
+                    g1(tb + C::Y, dr1, ds, SC, ID_N, true);   // Y += R1 S0^T
                 }
                 mma_commit(BAR(B_G1_DONE + b));
                 if (C::kSS > 0) mma_commit(BAR(B_S_EMPTY + ss));
@@ -416,14 +417,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
             };
             bool ok = mbar_wait(BAR(B_R_FULL), 0, abort_flag, bound);
             if (ok && C::kR1T) ok = wait_full(B_R1_READY, 0, 1);
-            if (ok) ok = issue_g1(0);
-            for (int j = 0; j < nt && ok; ++j) {
+            // one call site per issue routine: G1 of tile j + 1, then G2 of tile j
+            for (int j = -1; j < nt && ok; ++j) {
                 if (j + 1 < nt) {
                     // single buffer: the elementwise warps must have read tile j's X..W first
-                    if (C::kSingle && !(ok = mbar_wait(BAR(B_X_FREE), j & 1, abort_flag, bound))) break;
+                    if (C::kSingle && j >= 0 && !(ok = mbar_wait(BAR(B_X_FREE), j & 1, abort_flag, bound))) break;
                     if (!(ok = issue_g1(j + 1))) break;
                 }
-                ok = issue_g2(j);
+                if (j >= 0) ok = issue_g2(j);
             }
             if (ok) mma_commit(BAR(B_ACC_FULL));
             mma_commit(BAR(B_MMA_DRAIN));
