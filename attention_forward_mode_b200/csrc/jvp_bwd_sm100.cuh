@@ -147,9 +147,6 @@ struct Var {
     static constexpr bool kSingle = VAR == V_DQ || VAR == V_DK;  // one score buffer, E region of its own
     static constexpr bool kTwoAcc = VAR == V_DKT;
     static constexpr bool kColStats = VAR == V_DK || VAR == V_DKT || VAR == V_DV;
-    static constexpr bool kY = VAR == V_DQ || VAR == V_DK || VAR == V_DV;  // score tangent needed
-    static constexpr bool kZ = VAR != V_DV;                                // A needed
-    static constexpr bool kW = kSingle;                                    // B needed
     static constexpr bool kL1 = VAR != V_DTQ;                              // second long-ring tensor
     static constexpr int kNS = VAR == V_DKT ? 0 : (VAR == V_DTQ ? 1 : 2);  // short-stage tensors
     static constexpr int kNR = kSingle ? 4 : 2;        // resident tiles R0..R(kNR-1)
