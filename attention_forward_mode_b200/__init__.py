@@ -18,6 +18,7 @@ from ._binding import (  # noqa: F401
     AJVP_ERR_UNSUPPORTED_DIM,
     AJVP_ERR_WORKSPACE,
     AJVP_OK,
+    DEFAULT_PERSISTENT_KEY_TILES,
     GRAD_NAMES,
     AttnJvpError,
     attn_jvp,
@@ -36,6 +37,7 @@ from ._binding import (  # noqa: F401
     host_workspace_bytes,
     load_library,
     selftest_wait_timeout,
+    set_persistent_key_tiles,
     set_wait_bound_ns,
     strerror,
     version,
@@ -47,5 +49,5 @@ __all__ = [
     "AttnJvpFunction", "attn_jvp_autograd",
     "attn_jvp", "attn_jvp_bwd", "attn_jvp_fwd_causal", "attn_jvp_fwd_varlen", "attn_jvp_fwd_stats", "bwd_workspace_bytes", "attn_jvp_fwd", "attn_jvp_fwd_f32", "attn_jvp_fwd_f32out", "attn_jvp_fwd_host", "attn_jvp_fwd_host_noalloc", "check_device_status",
     "default_heads_per_chunk", "host_workspace_bytes", "load_library",
-    "selftest_wait_timeout", "set_wait_bound_ns", "strerror", "version", "AttnJvpError",
+    "selftest_wait_timeout", "set_persistent_key_tiles", "DEFAULT_PERSISTENT_KEY_TILES", "set_wait_bound_ns", "strerror", "version", "AttnJvpError",
 ]

@@ -32,7 +32,7 @@ EXPORTED = ("attn_jvp_fwd", "attn_jvp_fwd_causal", "attn_jvp_fwd_varlen", "attn_
             "attn_jvp_bwd_workspace_bytes", "attn_jvp_fwd_f32", "attn_jvp_fwd_host",
             "attn_jvp_fwd_host_noalloc", "attn_jvp_host_workspace_bytes", "attn_jvp_strerror",
             "attn_jvp_last_cuda_error",
-            "attn_jvp_check_device_status", "attn_jvp_set_wait_bound_ns",
+            "attn_jvp_check_device_status", "attn_jvp_set_wait_bound_ns", "attn_jvp_set_persistent_key_tiles",
             "attn_jvp_selftest_wait_timeout", "attn_jvp_version")
 
 _lock = threading.Lock()
@@ -89,6 +89,8 @@ def load_library(path: str = LIB_PATH):
         lib.attn_jvp_check_device_status.restype = ctypes.c_int
         lib.attn_jvp_set_wait_bound_ns.argtypes = [ctypes.c_uint64]
         lib.attn_jvp_set_wait_bound_ns.restype = ctypes.c_int
+        lib.attn_jvp_set_persistent_key_tiles.argtypes = [ctypes.c_int64]
+        lib.attn_jvp_set_persistent_key_tiles.restype = ctypes.c_int
         lib.attn_jvp_selftest_wait_timeout.argtypes = [ctypes.c_uint64, vp]
         lib.attn_jvp_selftest_wait_timeout.restype = ctypes.c_int
         lib.attn_jvp_version.argtypes = []
@@ -424,6 +426,16 @@ def check_device_status(stream=None) -> int:
 
 def set_wait_bound_ns(ns: int) -> None:
     _check(load_library().attn_jvp_set_wait_bound_ns(int(ns)), "attn_jvp_set_wait_bound_ns")
+
+
+DEFAULT_PERSISTENT_KEY_TILES = 32
+
+
+def set_persistent_key_tiles(max_key_tiles: int) -> None:
+    """Key sequences of at most ``max_key_tiles`` 64-key tiles use the
+    persistent form of the unmasked bf16 forward (0: never).  Process-wide."""
+    _check(load_library().attn_jvp_set_persistent_key_tiles(int(max_key_tiles)),
+           "attn_jvp_set_persistent_key_tiles")
 
 
 def selftest_wait_timeout(bound_ns: int, stream=None) -> None:

@@ -33,6 +33,7 @@ struct DeviceState {
     std::once_flag once;
     int status = AJVP_OK;
     int cuda_error = 0;
+    int sm_count = 0;
 };
 DeviceState g_dev[kMaxDevices];
 
@@ -47,9 +48,16 @@ int fail_cuda(cudaError_t e) {
     return AJVP_ERR_CUDA;
 }
 
-template <bool kSplit, int MASK>
+// Short key sequences (at most this many 64-key tiles) take the persistent
+// form of the unmasked bf16 kernel: with few key tiles per query tile, the
+// per-tile pipeline fill, drain and epilogue are a large share of a CTA's
+// time, and the persistent CTA overlaps them with the next tile's work.
+constexpr int64_t kDefaultPersistKeyTiles = 32;
+std::atomic<int64_t> g_persist_key_tiles{kDefaultPersistKeyTiles};
+
+template <bool kSplit, int MASK, bool kPersist = false>
 cudaError_t set_fwd_smem() {
-    return cudaFuncSetAttribute(ajvp::sm100::attn_jvp_fwd_kernel<kSplit, MASK>,
+    return cudaFuncSetAttribute(ajvp::sm100::attn_jvp_fwd_kernel<kSplit, MASK, kPersist>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ajvp::sm100::SMEM_BYTES);
 }
 
@@ -78,12 +86,19 @@ int device_setup(int *dev_out) {
             st.status = AJVP_ERR_UNSUPPORTED_DEVICE;
             return;
         }
+        cudaError_t e0 = cudaDeviceGetAttribute(&st.sm_count, cudaDevAttrMultiProcessorCount, dev);
+        if (e0 != cudaSuccess || st.sm_count < 1) {
+            st.status = AJVP_ERR_CUDA;
+            st.cuda_error = (int)e0;
+            return;
+        }
         cudaError_t e3 = cudaFuncSetAttribute(ajvp::sm100::attn_jvp_fwd_kernel<false>,
                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
                                               (int)ajvp::sm100::SMEM_BYTES);
         if (e3 == cudaSuccess)
             e3 = cudaFuncSetAttribute(ajvp::sm100::attn_jvp_fwd_kernel<true>,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ajvp::sm100::SMEM_BYTES);
+        if (e3 == cudaSuccess) e3 = set_fwd_smem<false, 0, true>();
         if (e3 == cudaSuccess) e3 = set_fwd_smem<false, 1>();
         if (e3 == cudaSuccess) e3 = set_fwd_smem<false, 2>();
         if (e3 == cudaSuccess) e3 = set_fwd_smem<false, 3>();
@@ -211,9 +226,18 @@ int launch_sm100(const void *q, const void *k, const void *v, const void *tq, co
     p.scale = scale;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.bound_ns = g_bound_ns.load();
+    p.n_units = (int)n_cta;
 
-    ajvp::sm100::attn_jvp_fwd_kernel<kSplit, MASK><<<(unsigned)n_cta, ajvp::sm100::NTHREADS,
-                                                     ajvp::sm100::SMEM_BYTES, (cudaStream_t)stream>>>(p);
+    const int sm_count = g_dev[dev].sm_count;
+    const int64_t nk = (Lk + ajvp::sm100::BC - 1) / ajvp::sm100::BC;
+    if (!kSplit && MASK == 0 && nk <= g_persist_key_tiles.load() && n_cta > sm_count) {
+        // one CTA per SM walks the query tiles
+        ajvp::sm100::attn_jvp_fwd_kernel<false, 0, true><<<(unsigned)sm_count, ajvp::sm100::NTHREADS,
+                                                          ajvp::sm100::SMEM_BYTES, (cudaStream_t)stream>>>(p);
+    } else {
+        ajvp::sm100::attn_jvp_fwd_kernel<kSplit, MASK><<<(unsigned)n_cta, ajvp::sm100::NTHREADS,
+                                                         ajvp::sm100::SMEM_BYTES, (cudaStream_t)stream>>>(p);
+    }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail_cuda(e);
     return AJVP_OK;
@@ -618,6 +642,12 @@ int attn_jvp_check_device_status(void *stream) {
 
 int attn_jvp_set_wait_bound_ns(uint64_t ns) {
     g_bound_ns.store(ns == 0 ? kDefaultBoundNs : ns);
+    return AJVP_OK;
+}
+
+int attn_jvp_set_persistent_key_tiles(int64_t max_key_tiles) {
+    if (max_key_tiles < 0) return AJVP_ERR_INVALID_ARG;
+    g_persist_key_tiles.store(max_key_tiles);
     return AJVP_OK;
 }
 

@@ -41,6 +41,17 @@
 // own 32 columns (group 0 at +0, group 1 at +32), so neither group overwrites
 // values the other still has to read.  They are the A operands of the
 // second MMA pair: 16 keys = 8 TMEM columns per K-step.
+//
+// Persistent form (kPersist, unmasked bf16 only; chosen for short key
+// sequences such as cross-attention to a few hundred text tokens, where a CTA
+// runs only a handful of key tiles): one CTA per SM walks the units
+// (query tile, batch*head) blockIdx.x, blockIdx.x + gridDim.x, ..., and every
+// ring, buffer and barrier phase follows one CTA-wide tile counter G = n*nk + j
+// (unit n, key tile j).  The epilogue writes O and tO straight from registers,
+// so Q / tQ shared memory is refilled for unit n+1 as soon as the last S/dS'
+// products of unit n are complete, and the next unit's first score products
+// run while the softmax warps finish the epilogue; the next unit's first
+// P.V waits for the epilogue to have read O / T (B_OT_FREE).
 #pragma once
 
 #include "ptx_sm100.cuh"
@@ -68,7 +79,10 @@ constexpr uint32_t SM_BAR = SM_VT + STAGES * VT_STAGE;
 constexpr uint32_t SM_XCH = SM_BAR + 256;  // fp32 [2 buffers][2 groups][128 rows] partial maxima,
                                            // then [l, g][2 groups][128 rows] final sums
 constexpr uint32_t XCH_FLOATS = 2 * 2 * 128 + 2 * 2 * 128;
-constexpr uint32_t SMEM_BYTES = SM_XCH + 4 * XCH_FLOATS + 1024;  // + alignment slack
+constexpr uint32_t STG_SLOT = 32 * 64;                 // one softmax warp's 32 rows x 32 bf16 columns
+constexpr uint32_t SM_STG = SM_XCH + 4 * XCH_FLOATS;  // 8 staging slots for the plain-store epilogue
+constexpr uint32_t SMEM_BYTES = SM_STG + 8 * STG_SLOT + 1024;  // + alignment slack
+static_assert(SMEM_BYTES <= 232448, "dynamic shared memory above the sm_100 per-CTA limit");
 
 // barrier slots (8 bytes each).  Two MMA commits per key tile:
 //   B_SD_FULL[j % 2]  S_j / dS'_j complete: the softmax may read them, and
@@ -82,9 +96,10 @@ enum : int {
     B_VT_EMPTY = 5,  // + stage
     B_SD_FULL = 7,   // + buffer (= K-side stage)
     B_P_FULL = 9,    // + buffer
-    B_O_FULL = 11,   // single use: every MMA of the tile has completed
+    B_O_FULL = 11,   // every MMA of the unit has completed (one phase per unit)
     B_MMA_DRAIN = 12,
-    N_BARS = 13
+    B_OT_FREE = 13,  // persistent: the epilogue has read O / T (256 arrivals per unit)
+    N_BARS = 14
 };
 static_assert(STAGES == 2, "the K-side ring reuses the two S/dS' buffer barriers");
 constexpr uint32_t OFF_TMEM_SLOT = 8 * N_BARS;     // u32
@@ -107,10 +122,33 @@ struct Params {
     int BH;                       // dense: B*H; packed: H (the tensors' outermost extent)
     int Lq, Lk, n_qtiles;  // rows per (batch, head) -- packed: total rows; n_qtiles: 128-row tiles
                            // per (batch, head) -- packed: tiles of the longest sequence
+    int n_units;           // persistent: n_qtiles * BH query tiles shared out over the grid
     float scale;           // s
     float scale_log2;      // s * log2(e)
     unsigned long long bound_ns;
 };
+
+// Coalesced store of one warp's 32 rows x 32 bf16 columns (lane = row, w = its
+// 64 bytes): through the warp's 2 KB shared-memory slot, 16-byte chunk c of row
+// r at r*64 + ((c ^ ((r >> 1) & 3)) << 4) (conflict-free for both the row-wise
+// writes and the chunk-wise reads), then 8 rows x 64 contiguous bytes per
+// global store instruction instead of 32 rows x 16 bytes.  Rows >= rows_left
+// are not written; dst: the warp's row 0 at its first column, rows HD apart.
+__device__ __forceinline__ void store_rows_32x32(uint32_t slot, const uint32_t (&w)[16], __nv_bfloat16 *dst,
+                                                 int rows_left, uint32_t lane) {
+#pragma unroll
+    for (uint32_t c = 0; c < 4; ++c)
+        st_shared_v4(slot + lane * 64u + ((c ^ ((lane >> 1) & 3u)) << 4), w[4 * c], w[4 * c + 1], w[4 * c + 2],
+                     w[4 * c + 3]);
+    __syncwarp();
+#pragma unroll
+    for (uint32_t k = 0; k < 4; ++k) {
+        const uint32_t r = 8u * k + (lane >> 2), c = lane & 3u;
+        const uint4 v = ld_shared_u4(slot + r * 64u + ((c ^ ((r >> 1) & 3u)) << 4));
+        if ((int)r < rows_left) *reinterpret_cast<uint4 *>(dst + (size_t)r * HD + 8u * c) = v;
+    }
+    __syncwarp();  // the slot is free again
+}
 
 // Key masks (MASK bits): 1 causal -- key j is visible to query i of a sequence
 // iff j <= i + (Lk - Lq), bottom-right aligned; 2 packed -- the tensors are
@@ -123,9 +161,10 @@ constexpr int MASK_CAUSAL = 1, MASK_PACKED = 2;
 // kSplit = true : P and P.*s dS' are each split into bf16 hi + lo parts
 //                 (x = hi + lo to ~16 significant bits), both multiplied into
 //                 O and T, and O, tO are written in fp32; 1.5x the MMA work.
-template <bool kSplit, int MASK = 0>
+template <bool kSplit, int MASK = 0, bool kPersist = false>
 __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_constant__ Params p) {
     static_assert(!kSplit || MASK == 0, "the fp32-output variant has no masks");
+    static_assert(!kPersist || (!kSplit && MASK == 0), "the persistent form is the unmasked bf16 kernel");
     constexpr bool kCausal = (MASK & MASK_CAUSAL) != 0, kPacked = (MASK & MASK_PACKED) != 0;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -177,6 +216,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
         return;
     }
     const uint64_t bound = p.bound_ns;
+    // persistent: the n-th unit of this CTA (unit 0 is blockIdx.x, decoded above);
+    // false past the last one, else its query tile and outer index
+    auto next_unit = [&](int n, int &qt_n, int &bh_n) -> bool {
+        const long long u = (long long)blockIdx.x + (long long)n * (long long)gridDim.x;
+        if (u >= (long long)p.n_units) return false;
+        qt_n = (int)(u % p.n_qtiles);
+        bh_n = (int)(u / p.n_qtiles);
+        return true;
+    };
 
     const uint32_t bars = base + SM_BAR;
     auto BAR = [&](int i) -> uint32_t { return bars + 8u * (uint32_t)i; };
@@ -196,6 +244,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
         }
         mbar_init(BAR(B_O_FULL), 1);
         mbar_init(BAR(B_MMA_DRAIN), 1);
+        mbar_init(BAR(B_OT_FREE), SOFTMAX_THREADS);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -220,54 +269,66 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
         // ------------------------------------------------------ TMA producer
         if (lane == 0) {
             bool ok = true;
-            int kt_last[STAGES], vt_last[STAGES];
+            int kt_last[STAGES], vt_last[STAGES], q_last = -1;
             for (int s = 0; s < STAGES; ++s) kt_last[s] = vt_last[s] = -1;
-            mbar_arrive_expect_tx(BAR(B_Q_FULL), 4 * CHUNK_Q);
-            tma_load_3d(base + SM_Q, &p.tm_q, BAR(B_Q_FULL), 0, yq, bh);
-            tma_load_3d(base + SM_Q + CHUNK_Q, &p.tm_q, BAR(B_Q_FULL), 64, yq, bh);
-            tma_load_3d(base + SM_TQ, &p.tm_tq, BAR(B_Q_FULL), 0, yq, bh);
-            tma_load_3d(base + SM_TQ + CHUNK_Q, &p.tm_tq, BAR(B_Q_FULL), 64, yq, bh);
-            // order of use by the MMA warp: KT_0, KT_1, VT_0, KT_2, VT_1, ...
-            for (int t = 0; t <= nk && ok; ++t) {
-                if (t < nk) {
-                    const int s = t % STAGES;
-                    // stage s is free once S/dS' of tile t - 2 are complete
-                    if (!mbar_wait(BAR(B_SD_FULL + s), ((t / STAGES) & 1) ^ 1, abort_flag, bound)) {
-                        ok = false;
-                        break;
-                    }
-                    const uint32_t st = base + SM_KT + s * KT_STAGE;
-                    const uint32_t fb = BAR(B_KT_FULL + s);
-                    const int y = yk0 + t * BC;
-                    mbar_arrive_expect_tx(fb, KT_STAGE);
-                    // chunk c: K rows then tK rows, so [K | tK] is one N = 128 operand
-                    tma_load_3d(st, &p.tm_k, fb, 0, y, bh);
-                    tma_load_3d(st + CHUNK_K, &p.tm_tk, fb, 0, y, bh);
-                    tma_load_3d(st + 2 * CHUNK_K, &p.tm_k, fb, 64, y, bh);
-                    tma_load_3d(st + 3 * CHUNK_K, &p.tm_tk, fb, 64, y, bh);
-                    kt_last[s] = t;
+            int n = 0, qt_n = qt, bh_n = bh;
+            do {
+                const int G0 = n * nk;  // CTA-wide index of this unit's first key tile
+                const int yq_n = yq0 + qt_n * BR;
+                // Q / tQ are free once every S / dS' product of the previous unit is complete
+                if (n > 0 && !mbar_wait(BAR(B_SD_FULL + ((G0 - 1) & 1)), ((G0 - 1) >> 1) & 1, abort_flag, bound)) {
+                    ok = false;
+                    break;
                 }
-                if (t >= 1) {
-                    const int i = t - 1;
-                    const int s = i % STAGES;
-                    if (!mbar_wait(BAR(B_VT_EMPTY + s), ((i / STAGES) & 1) ^ 1, abort_flag, bound)) {
-                        ok = false;
-                        break;
+                mbar_arrive_expect_tx(BAR(B_Q_FULL), 4 * CHUNK_Q);
+                tma_load_3d(base + SM_Q, &p.tm_q, BAR(B_Q_FULL), 0, yq_n, bh_n);
+                tma_load_3d(base + SM_Q + CHUNK_Q, &p.tm_q, BAR(B_Q_FULL), 64, yq_n, bh_n);
+                tma_load_3d(base + SM_TQ, &p.tm_tq, BAR(B_Q_FULL), 0, yq_n, bh_n);
+                tma_load_3d(base + SM_TQ + CHUNK_Q, &p.tm_tq, BAR(B_Q_FULL), 64, yq_n, bh_n);
+                q_last = n;
+                // order of use by the MMA warp: KT_0, KT_1, VT_0, KT_2, VT_1, ...
+                for (int t = 0; t <= nk && ok; ++t) {
+                    if (t < nk) {
+                        const int G = G0 + t;
+                        const int s = G % STAGES;
+                        // stage s is free once S/dS' of tile G - 2 are complete
+                        if (!mbar_wait(BAR(B_SD_FULL + s), ((G / STAGES) & 1) ^ 1, abort_flag, bound)) {
+                            ok = false;
+                            break;
+                        }
+                        const uint32_t st = base + SM_KT + s * KT_STAGE;
+                        const uint32_t fb = BAR(B_KT_FULL + s);
+                        const int y = yk0 + t * BC;
+                        mbar_arrive_expect_tx(fb, KT_STAGE);
+                        // chunk c: K rows then tK rows, so [K | tK] is one N = 128 operand
+                        tma_load_3d(st, &p.tm_k, fb, 0, y, bh_n);
+                        tma_load_3d(st + CHUNK_K, &p.tm_tk, fb, 0, y, bh_n);
+                        tma_load_3d(st + 2 * CHUNK_K, &p.tm_k, fb, 64, y, bh_n);
+                        tma_load_3d(st + 3 * CHUNK_K, &p.tm_tk, fb, 64, y, bh_n);
+                        kt_last[s] = G;
                     }
-                    const uint32_t st = base + SM_VT + s * VT_STAGE;
-                    const uint32_t fb = BAR(B_VT_FULL + s);
-                    const int y = yk0 + i * BC;
-                    mbar_arrive_expect_tx(fb, VT_STAGE);
-                    // [V c0 | V c1 | tV c0 | tV c1]: N-chunks 64 columns apart (LBO)
-                    tma_load_3d(st, &p.tm_v, fb, 0, y, bh);
-                    tma_load_3d(st + CHUNK_K, &p.tm_v, fb, 64, y, bh);
-                    tma_load_3d(st + 2 * CHUNK_K, &p.tm_tv, fb, 0, y, bh);
-                    tma_load_3d(st + 3 * CHUNK_K, &p.tm_tv, fb, 64, y, bh);
-                    vt_last[s] = i;
+                    if (t >= 1) {
+                        const int i = G0 + t - 1;
+                        const int s = i % STAGES;
+                        if (!mbar_wait(BAR(B_VT_EMPTY + s), ((i / STAGES) & 1) ^ 1, abort_flag, bound)) {
+                            ok = false;
+                            break;
+                        }
+                        const uint32_t st = base + SM_VT + s * VT_STAGE;
+                        const uint32_t fb = BAR(B_VT_FULL + s);
+                        const int y = yk0 + (t - 1) * BC;
+                        mbar_arrive_expect_tx(fb, VT_STAGE);
+                        // [V c0 | V c1 | tV c0 | tV c1]: N-chunks 64 columns apart (LBO)
+                        tma_load_3d(st, &p.tm_v, fb, 0, y, bh_n);
+                        tma_load_3d(st + CHUNK_K, &p.tm_v, fb, 64, y, bh_n);
+                        tma_load_3d(st + 2 * CHUNK_K, &p.tm_tv, fb, 0, y, bh_n);
+                        tma_load_3d(st + 3 * CHUNK_K, &p.tm_tv, fb, 64, y, bh_n);
+                        vt_last[s] = i;
+                    }
                 }
-            }
+            } while (kPersist && ok && next_unit(++n, qt_n, bh_n));
             // let every copy already issued land before shared memory is released
-            mbar_wait_drain(BAR(B_Q_FULL), 0, bound);
+            if (q_last >= 0) mbar_wait_drain(BAR(B_Q_FULL), q_last & 1, bound);
             for (int s = 0; s < STAGES; ++s) {
                 if (kt_last[s] >= 0) mbar_wait_drain(BAR(B_KT_FULL + s), (kt_last[s] / STAGES) & 1, bound);
                 if (vt_last[s] >= 0) mbar_wait_drain(BAR(B_VT_FULL + s), (vt_last[s] / STAGES) & 1, bound);
@@ -287,11 +348,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
             const uint64_t dtq = smem_desc_sw128(base + SM_TQ, 16, 1024);
             const uint64_t dk0 = smem_desc_sw128(base + SM_KT, 16, 1024);
             const uint64_t dv0 = smem_desc_sw128(base + SM_VT, CHUNK_K, 1024);
-            bool ok = mbar_wait(BAR(B_Q_FULL), 0, abort_flag, bound);
-            auto issue_sd = [&](int j) -> bool {
-                const int s = j % STAGES;
-                const int b = j & 1;
-                if (!mbar_wait(BAR(B_KT_FULL + s), (j / STAGES) & 1, abort_flag, bound)) return false;
+            bool ok = true;
+            // G: CTA-wide key-tile index (ring stage, buffer and phase)
+            auto issue_sd = [&](int G) -> bool {
+                const int s = G % STAGES;
+                const int b = G & 1;
+                if (!mbar_wait(BAR(B_KT_FULL + s), (G / STAGES) & 1, abort_flag, bound)) return false;
                 tc_fence_after();
                 const uint64_t dk = desc_add(dk0, s * KT_STAGE);
                 const uint32_t t_s = tbase + TM_BUF + 128u * b;
@@ -310,11 +372,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                 mma_commit(BAR(B_SD_FULL + b));
                 return true;
             };
-            auto issue_pv = [&](int i) -> bool {
-                const int s = i % STAGES;
-                const int b = i & 1;
-                if (!mbar_wait(BAR(B_P_FULL + b), (i >> 1) & 1, abort_flag, bound)) return false;
-                if (!mbar_wait(BAR(B_VT_FULL + s), (i / STAGES) & 1, abort_flag, bound)) return false;
+            // first: the unit's first tile (overwrites O / T); n: the unit
+            auto issue_pv = [&](int G, bool first, int n) -> bool {
+                const int s = G % STAGES;
+                const int b = G & 1;
+                if (!mbar_wait(BAR(B_P_FULL + b), (G >> 1) & 1, abort_flag, bound)) return false;
+                if (!mbar_wait(BAR(B_VT_FULL + s), (G / STAGES) & 1, abort_flag, bound)) return false;
+                // the previous unit's epilogue must have read O / T before they are overwritten
+                if (kPersist && first && n > 0 && !mbar_wait(BAR(B_OT_FREE), (n - 1) & 1, abort_flag, bound))
+                    return false;
                 tc_fence_after();
                 const uint64_t dv = desc_add(dv0, s * VT_STAGE);
                 const uint32_t t_s = tbase + TM_BUF + 128u * b;
@@ -322,7 +388,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                 for (int kk = 0; kk < BC / 16; ++kk) {
                     // keys 16kk..16kk+15: group kk/2's columns, 8 columns per K-step
                     const uint32_t a_col = (kk >> 1) * 32 + (kk & 1) * 8;
-                    mma_ts(tbase + TM_O, t_s + a_col, desc_add(dv, kk * 2048), ID_OT, (i > 0 || kk > 0) ? 1u : 0u);
+                    mma_ts(tbase + TM_O, t_s + a_col, desc_add(dv, kk * 2048), ID_OT, (!first || kk > 0) ? 1u : 0u);
                 }
 #pragma unroll
                 for (int kk = 0; kk < BC / 16; ++kk) {
@@ -344,15 +410,20 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                 mma_commit(BAR(B_VT_EMPTY + s));
                 return true;
             };
-            if (ok) ok = issue_sd(0);
-            for (int j = 1; j < nk && ok; ++j) {
-                ok = issue_sd(j);
-                if (ok) ok = issue_pv(j - 1);
-            }
-            if (ok) ok = issue_pv(nk - 1);
-            // O and T are final once everything issued so far completes (a dedicated
-            // barrier: a parity wait on a per-tile barrier could be ambiguous here)
-            if (ok) mma_commit(BAR(B_O_FULL));
+            int n = 0, qt_n = qt, bh_n = bh;
+            do {
+                const int G0 = n * nk;
+                ok = mbar_wait(BAR(B_Q_FULL), n & 1, abort_flag, bound);
+                if (ok) ok = issue_sd(G0);
+                for (int j = 1; j < nk && ok; ++j) {
+                    ok = issue_sd(G0 + j);
+                    if (ok) ok = issue_pv(G0 + j - 1, j == 1, n);
+                }
+                if (ok) ok = issue_pv(G0 + nk - 1, nk == 1, n);
+                // O and T are final once everything issued so far completes (a barrier
+                // of its own: a parity wait on a per-tile barrier could be ambiguous here)
+                if (ok) mma_commit(BAR(B_O_FULL));
+            } while (kPersist && ok && next_unit(++n, qt_n, bh_n));
             // every MMA issued must finish before tensor memory is released
             mma_commit(BAR(B_MMA_DRAIN));
             mbar_wait_drain(BAR(B_MMA_DRAIN), 0, bound);
@@ -371,251 +442,262 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
         const bool up = c >= 0.f;  // row max of c*S is c * max(S) (min(S) for c < 0)
         const float sentinel = up ? -INFINITY : INFINITY;
         float *xch = reinterpret_cast<float *>(gbase + SM_XCH);
-        float m_ref = -INFINITY, l = 0.f, g = 0.f;
         bool failed = false;
-        // keys this row sees (a prefix of the sequence's keys; may be <= 0 when causal)
-        const int kcount = kCausal ? min(Lk_s, q0 + row + koff + 1) : Lk_s;
+        int n = 0, qt_n = qt, bh_n = bh;
+        do {
+            const int G0 = n * nk;  // CTA-wide index of this unit's first key tile
+            const int q0_n = qt_n * BR, yq_n = yq0 + q0_n;
+            float m_ref = -INFINITY, l = 0.f, g = 0.f;
+            // keys this row sees (a prefix of the sequence's keys; may be <= 0 when causal)
+            const int kcount = kCausal ? min(Lk_s, q0_n + row + koff + 1) : Lk_s;
 
-        for (int j = 0; j < nk; ++j) {
-            const int b = j & 1;
-            const uint32_t t_s = tbase + lane_off + TM_BUF + 128u * b;
-            if (!failed) failed = !mbar_wait_warp(BAR(B_SD_FULL + b), (j >> 1) & 1, abort_flag, bound);
-            uint32_t xs[32], xd[32];
-            const int valid = kcount - j * BC - (int)col0;  // visible keys of this group (may be <= 0)
-            float part = sentinel;
-            if (!failed) {
-                tc_fence_after();
-                tmem_ld32(t_s + col0, xs);
-                tmem_ld32(t_s + 64 + col0, xd);
-                tmem_wait_ld();
-                if (valid < 32) {
+            for (int j = 0; j < nk; ++j) {
+                const int G = G0 + j;  // CTA-wide tile index
+                const int b = G & 1;
+                const uint32_t t_s = tbase + lane_off + TM_BUF + 128u * b;
+                if (!failed) failed = !mbar_wait_warp(BAR(B_SD_FULL + b), (G >> 1) & 1, abort_flag, bound);
+                uint32_t xs[32], xd[32];
+                const int valid = kcount - j * BC - (int)col0;  // visible keys of this group (may be <= 0)
+                float part = sentinel;
+                if (!failed) {
+                    tc_fence_after();
+                    tmem_ld32(t_s + col0, xs);
+                    tmem_ld32(t_s + 64 + col0, xd);
+                    tmem_wait_ld();
+                    if (valid < 32) {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        if (i >= valid) xs[i] = __float_as_uint(sentinel);
-                }
-                float m4[4];
-#pragma unroll
-                for (int k = 0; k < 4; ++k) m4[k] = __uint_as_float(xs[k]);
-                if (up) {
-#pragma unroll
-                    for (int i = 4; i < 28; i += 8)
-#pragma unroll
-                        for (int k = 0; k < 4; ++k)
-                            m4[k] = fmax3(m4[k], __uint_as_float(xs[i + k]), __uint_as_float(xs[i + 4 + k]));
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) m4[k] = fmaxf(m4[k], __uint_as_float(xs[28 + k]));
-                    part = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]);
-                } else {
-#pragma unroll
-                    for (int i = 4; i < 28; i += 8)
-#pragma unroll
-                        for (int k = 0; k < 4; ++k)
-                            m4[k] = fmin3(m4[k], __uint_as_float(xs[i + k]), __uint_as_float(xs[i + 4 + k]));
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) m4[k] = fminf(m4[k], __uint_as_float(xs[28 + k]));
-                    part = fminf(fmin3(m4[0], m4[1], m4[2]), m4[3]);
-                }
-                xch[(b * 2 + grp) * 128 + row] = part;
-            }
-            // both groups' partial maxima are in shared memory; every softmax
-            // thread reaches this barrier each tile, and a failure anywhere
-            // ends the loop for all of them together
-            if (named_bar_or(NB_TILE, SOFTMAX_THREADS, failed)) {
-                failed = true;
-                break;
-            }
-            const float other = xch[(b * 2 + (grp ^ 1)) * 128 + row];
-            const float m_tile = (up ? fmaxf(part, other) : fminf(part, other)) * c;
-            if (j == 0) {
-                m_ref = m_tile;
-            } else {
-                const bool need = m_tile > m_ref + RESCALE_THRESHOLD;
-                if (__any_sync(0xffffffffu, need)) {
-                    float alpha = 1.f;
-                    if (need) {
-                        alpha = ex2_approx(m_ref - m_tile);
-                        m_ref = m_tile;
+                        for (int i = 0; i < 32; ++i)
+                            if (i >= valid) xs[i] = __float_as_uint(sentinel);
                     }
-                    l *= alpha;
-                    g *= alpha;
-                    // O and T may only be touched once the P.V products of tile j-1
-                    // are complete (the V-side barrier of its stage); group 0
-                    // rescales O, group 1 rescales T
-                    failed = !mbar_wait_warp(BAR(B_VT_EMPTY + ((j - 1) & 1)), ((j - 1) >> 1) & 1, abort_flag, bound);
-                    if (!failed) {
-                        tc_fence_after();
-#pragma unroll 1
-                        for (int cc = 0; cc < 4; ++cc) {
-                            uint32_t r[32];
-                            const uint32_t ta = tbase + lane_off + 128u * (uint32_t)grp + 32u * cc;
-                            tmem_ld32(ta, r);
-                            tmem_wait_ld();
+                    float m4[4];
 #pragma unroll
-                            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-                            tmem_st32(ta, r);
+                    for (int k = 0; k < 4; ++k) m4[k] = __uint_as_float(xs[k]);
+                    if (up) {
+#pragma unroll
+                        for (int i = 4; i < 28; i += 8)
+#pragma unroll
+                            for (int k = 0; k < 4; ++k)
+                                m4[k] = fmax3(m4[k], __uint_as_float(xs[i + k]), __uint_as_float(xs[i + 4 + k]));
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) m4[k] = fmaxf(m4[k], __uint_as_float(xs[28 + k]));
+                        part = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]);
+                    } else {
+#pragma unroll
+                        for (int i = 4; i < 28; i += 8)
+#pragma unroll
+                            for (int k = 0; k < 4; ++k)
+                                m4[k] = fmin3(m4[k], __uint_as_float(xs[i + k]), __uint_as_float(xs[i + 4 + k]));
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) m4[k] = fminf(m4[k], __uint_as_float(xs[28 + k]));
+                        part = fminf(fmin3(m4[0], m4[1], m4[2]), m4[3]);
+                    }
+                    xch[(b * 2 + grp) * 128 + row] = part;
+                }
+                // both groups' partial maxima are in shared memory; every softmax
+                // thread reaches this barrier each tile, and a failure anywhere
+                // ends the loop for all of them together
+                if (named_bar_or(NB_TILE, SOFTMAX_THREADS, failed)) {
+                    failed = true;
+                    break;
+                }
+                const float other = xch[(b * 2 + (grp ^ 1)) * 128 + row];
+                const float m_tile = (up ? fmaxf(part, other) : fminf(part, other)) * c;
+                if (j == 0) {
+                    m_ref = m_tile;
+                } else {
+                    const bool need = m_tile > m_ref + RESCALE_THRESHOLD;
+                    if (__any_sync(0xffffffffu, need)) {
+                        float alpha = 1.f;
+                        if (need) {
+                            alpha = ex2_approx(m_ref - m_tile);
+                            m_ref = m_tile;
+                        }
+                        l *= alpha;
+                        g *= alpha;
+                        // O and T may only be touched once the P.V products of tile j-1
+                        // are complete (the V-side barrier of its stage); group 0
+                        // rescales O, group 1 rescales T
+                        failed = !mbar_wait_warp(BAR(B_VT_EMPTY + ((G - 1) & 1)), ((G - 1) >> 1) & 1, abort_flag, bound);
+                        if (!failed) {
+                            tc_fence_after();
+#pragma unroll 1
+                            for (int cc = 0; cc < 4; ++cc) {
+                                uint32_t r[32];
+                                const uint32_t ta = tbase + lane_off + 128u * (uint32_t)grp + 32u * cc;
+                                tmem_ld32(ta, r);
+                                tmem_wait_ld();
+#pragma unroll
+                                for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+                                tmem_st32(ta, r);
+                            }
                         }
                     }
                 }
-            }
-            if (failed) continue;  // the next tile's barrier carries the failure to everyone
-            const float2 nm2 = make_float2(-m_ref, -m_ref);
-            float pv[32];
+                if (failed) continue;  // the next tile's barrier carries the failure to everyone
+                const float2 nm2 = make_float2(-m_ref, -m_ref);
+                float pv[32];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const float2 y =
-                    __ffma2_rn(make_float2(__uint_as_float(xs[2 * i]), __uint_as_float(xs[2 * i + 1])), c2, nm2);
-                pv[2 * i] = ex2_approx(y.x);
-                pv[2 * i + 1] = ex2_approx(y.y);
-            }
-            if (valid < 32) {
-#pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    if (i >= valid) pv[i] = 0.f;
-            }
-            float2 ls2a = make_float2(0.f, 0.f), ls2b = ls2a, gs2a = ls2a, gs2b = ls2a;
-            uint32_t pk[16], pd[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const float2 pp = make_float2(pv[2 * i], pv[2 * i + 1]);
-                const float2 dd = make_float2(__uint_as_float(xd[2 * i]), __uint_as_float(xd[2 * i + 1]));
-                const float2 t = __fmul2_rn(__fmul2_rn(pp, dd), s2);  // p * s dS'
-                if (i & 1) {
-                    ls2b = __fadd2_rn(ls2b, pp);
-                    gs2b = __fadd2_rn(gs2b, t);
-                } else {
-                    ls2a = __fadd2_rn(ls2a, pp);
-                    gs2a = __fadd2_rn(gs2a, t);
+                for (int i = 0; i < 16; ++i) {
+                    const float2 y =
+                        __ffma2_rn(make_float2(__uint_as_float(xs[2 * i]), __uint_as_float(xs[2 * i + 1])), c2, nm2);
+                    pv[2 * i] = ex2_approx(y.x);
+                    pv[2 * i + 1] = ex2_approx(y.y);
                 }
-                pk[i] = pack_bf16x2(pp.x, pp.y);
-                pd[i] = pack_bf16x2(t.x, t.y);
-            }
-            tmem_st16(t_s + col0, pk);       // P over this group's S columns
-            tmem_st16(t_s + 64 + col0, pd);  // P.*s dS' over this group's dS' columns
-            if (kSplit) {
-                // lo = x - hi, rounded to bf16: hi + lo carries ~16 significant bits
+                if (valid < 32) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (i >= valid) pv[i] = 0.f;
+                }
+                float2 ls2a = make_float2(0.f, 0.f), ls2b = ls2a, gs2a = ls2a, gs2b = ls2a;
+                uint32_t pk[16], pd[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const float2 pp = make_float2(pv[2 * i], pv[2 * i + 1]);
                     const float2 dd = make_float2(__uint_as_float(xd[2 * i]), __uint_as_float(xd[2 * i + 1]));
-                    const float2 t = __fmul2_rn(__fmul2_rn(pp, dd), s2);
-                    const uint32_t ph = pack_bf16x2(pp.x, pp.y), th = pack_bf16x2(t.x, t.y);
-                    pk[i] = pack_bf16x2(pp.x - __uint_as_float(ph << 16), pp.y - __uint_as_float(ph & 0xffff0000u));
-                    pd[i] = pack_bf16x2(t.x - __uint_as_float(th << 16), t.y - __uint_as_float(th & 0xffff0000u));
+                    const float2 t = __fmul2_rn(__fmul2_rn(pp, dd), s2);  // p * s dS'
+                    if (i & 1) {
+                        ls2b = __fadd2_rn(ls2b, pp);
+                        gs2b = __fadd2_rn(gs2b, t);
+                    } else {
+                        ls2a = __fadd2_rn(ls2a, pp);
+                        gs2a = __fadd2_rn(gs2a, t);
+                    }
+                    pk[i] = pack_bf16x2(pp.x, pp.y);
+                    pd[i] = pack_bf16x2(t.x, t.y);
                 }
-                tmem_st16(t_s + col0 + 16, pk);
-                tmem_st16(t_s + 64 + col0 + 16, pd);
+                tmem_st16(t_s + col0, pk);       // P over this group's S columns
+                tmem_st16(t_s + 64 + col0, pd);  // P.*s dS' over this group's dS' columns
+                if (kSplit) {
+                    // lo = x - hi, rounded to bf16: hi + lo carries ~16 significant bits
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const float2 pp = make_float2(pv[2 * i], pv[2 * i + 1]);
+                        const float2 dd = make_float2(__uint_as_float(xd[2 * i]), __uint_as_float(xd[2 * i + 1]));
+                        const float2 t = __fmul2_rn(__fmul2_rn(pp, dd), s2);
+                        const uint32_t ph = pack_bf16x2(pp.x, pp.y), th = pack_bf16x2(t.x, t.y);
+                        pk[i] = pack_bf16x2(pp.x - __uint_as_float(ph << 16), pp.y - __uint_as_float(ph & 0xffff0000u));
+                        pd[i] = pack_bf16x2(t.x - __uint_as_float(th << 16), t.y - __uint_as_float(th & 0xffff0000u));
+                    }
+                    tmem_st16(t_s + col0 + 16, pk);
+                    tmem_st16(t_s + 64 + col0 + 16, pd);
+                }
+                l += (ls2a.x + ls2b.x) + (ls2a.y + ls2b.y);
+                g += (gs2a.x + gs2b.x) + (gs2a.y + gs2b.y);
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(BAR(B_P_FULL + b));
             }
-            l += (ls2a.x + ls2b.x) + (ls2a.y + ls2b.y);
-            g += (gs2a.x + gs2b.x) + (gs2a.y + gs2b.y);
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(BAR(B_P_FULL + b));
-        }
 
-        if (!failed) failed = !mbar_wait_warp(BAR(B_O_FULL), 0, abort_flag, bound);
-        float *lg = xch + 2 * 2 * 128;  // [l, g][group][row]
-        if (!failed) {
-            lg[(0 * 2 + grp) * 128 + row] = l;
-            lg[(1 * 2 + grp) * 128 + row] = g;
-        }
-        const bool any_failed = named_bar_or(NB_EPI, SOFTMAX_THREADS, failed);
-        if (!any_failed) {
-            tc_fence_after();
-            const float lt = l + lg[(0 * 2 + (grp ^ 1)) * 128 + row];
-            const float gt = g + lg[(1 * 2 + (grp ^ 1)) * 128 + row];
-            // a row that saw no key (masks only) has lt = 0: zeros, lse = -inf
-            const float inv_l = (MASK != 0 && !(lt > 0.f)) ? 0.f : 1.f / lt;
-            const float mu = gt * inv_l;
-            // group grp writes output columns 64*grp .. 64*grp+63
-            if (kSplit) {
-                // fp32 outputs straight from registers, 16 bytes per store
-                const bool row_ok = q0 + row < p.Lq;
-                const size_t off = ((size_t)bh * (size_t)p.Lq + (size_t)(q0 + row)) * HD + 64u * (uint32_t)grp;
+            if (!failed) failed = !mbar_wait_warp(BAR(B_O_FULL), n & 1, abort_flag, bound);
+            float *lg = xch + 2 * 2 * 128;  // [l, g][group][row]
+            if (!failed) {
+                lg[(0 * 2 + grp) * 128 + row] = l;
+                lg[(1 * 2 + grp) * 128 + row] = g;
+            }
+            const bool any_failed = named_bar_or(NB_EPI, SOFTMAX_THREADS, failed);
+            if (!any_failed) {
+                tc_fence_after();
+                const float lt = l + lg[(0 * 2 + (grp ^ 1)) * 128 + row];
+                const float gt = g + lg[(1 * 2 + (grp ^ 1)) * 128 + row];
+                // a row that saw no key (masks only) has lt = 0: zeros, lse = -inf
+                const float inv_l = (MASK != 0 && !(lt > 0.f)) ? 0.f : 1.f / lt;
+                const float mu = gt * inv_l;
+                // group grp writes output columns 64*grp .. 64*grp+63
+                if (kSplit) {
+                    // fp32 outputs straight from registers, 16 bytes per store
+                    const bool row_ok = q0_n + row < p.Lq;
+                    const size_t off = ((size_t)bh_n * (size_t)p.Lq + (size_t)(q0_n + row)) * HD + 64u * (uint32_t)grp;
 #pragma unroll 1
-                for (int h = 0; h < 2; ++h) {
+                    for (int h = 0; h < 2; ++h) {
+                        const int pc = 2 * grp + h;
+                        uint32_t ro[32], rt[32];
+                        tmem_ld32(tbase + lane_off + TM_O + 32u * pc, ro);
+                        tmem_ld32(tbase + lane_off + TM_T + 32u * pc, rt);
+                        tmem_wait_ld();
+                        if (row_ok) {
+                            float4 *po = reinterpret_cast<float4 *>(p.o_f32 + off + 32 * h);
+                            float4 *pt = reinterpret_cast<float4 *>(p.to_f32 + off + 32 * h);
+#pragma unroll
+                            for (int u = 0; u < 8; ++u) {
+                                float o4[4], t4[4];
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    o4[e] = __uint_as_float(ro[4 * u + e]) * inv_l;
+                                    t4[e] = fmaf(-mu, o4[e], __uint_as_float(rt[4 * u + e]) * inv_l);
+                                }
+                                po[u] = make_float4(o4[0], o4[1], o4[2], o4[3]);
+                                pt[u] = make_float4(t4[0], t4[1], t4[2], t4[3]);
+                            }
+                        }
+                    }
+                }
+                // bf16 outputs: O into the Q tile's shared memory, tO into tQ's, in
+                // the 128-byte-swizzled layout of the store tensor maps (packed rows and
+                // the persistent form: plain stores from registers)
+#pragma unroll 1
+                for (int h = 0; h < (kSplit ? 0 : 2); ++h) {
                     const int pc = 2 * grp + h;
                     uint32_t ro[32], rt[32];
                     tmem_ld32(tbase + lane_off + TM_O + 32u * pc, ro);
                     tmem_ld32(tbase + lane_off + TM_T + 32u * pc, rt);
                     tmem_wait_ld();
-                    if (row_ok) {
-                        float4 *po = reinterpret_cast<float4 *>(p.o_f32 + off + 32 * h);
-                        float4 *pt = reinterpret_cast<float4 *>(p.to_f32 + off + 32 * h);
+                    if (kPersist && h == 1) {  // O / T read: the next unit may overwrite them
+                        tc_fence_before();
+                        mbar_arrive(BAR(B_OT_FREE));
+                    }
+                    uint32_t wo[16], wt[16];
 #pragma unroll
-                        for (int u = 0; u < 8; ++u) {
-                            float o4[4], t4[4];
+                    for (int i = 0; i < 16; ++i) {
+                        const float o0 = __uint_as_float(ro[2 * i]) * inv_l;
+                        const float o1 = __uint_as_float(ro[2 * i + 1]) * inv_l;
+                        const float t0 = fmaf(-mu, o0, __uint_as_float(rt[2 * i]) * inv_l);
+                        const float t1 = fmaf(-mu, o1, __uint_as_float(rt[2 * i + 1]) * inv_l);
+                        wo[i] = pack_bf16x2(o0, o1);
+                        wt[i] = pack_bf16x2(t0, t1);
+                    }
+                    if (kPacked || kPersist) {
+                        // plain stores, staged per warp (packed: rows past the sequence
+                        // belong to the next one and are not written)
+                        const size_t off =
+                            ((size_t)bh_n * (size_t)p.Lq + (size_t)(yq_n + wl * 32)) * HD + 64u * grp + 32u * h;
+                        const int rows_left = Lq_s - (q0_n + wl * 32);
+                        const uint32_t slot = base + SM_STG + (uint32_t)(warp - 4) * STG_SLOT;
+                        store_rows_32x32(slot, wo, p.o_bf + off, rows_left, (uint32_t)lane);
+                        store_rows_32x32(slot, wt, p.to_bf + off, rows_left, (uint32_t)lane);
+                        continue;
+                    }
+                    const uint32_t chunk_off = (uint32_t)grp * CHUNK_Q + (uint32_t)row * 128u;
+                    const uint32_t unit0 = (uint32_t)h * 4u;
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                o4[e] = __uint_as_float(ro[4 * u + e]) * inv_l;
-                                t4[e] = fmaf(-mu, o4[e], __uint_as_float(rt[4 * u + e]) * inv_l);
-                            }
-                            po[u] = make_float4(o4[0], o4[1], o4[2], o4[3]);
-                            pt[u] = make_float4(t4[0], t4[1], t4[2], t4[3]);
-                        }
+                    for (int u = 0; u < 4; ++u) {
+                        const uint32_t phys = (((unit0 + u) ^ (uint32_t)(row & 7)) * 16u);
+                        st_shared_v4(base + SM_Q + chunk_off + phys, wo[4 * u], wo[4 * u + 1], wo[4 * u + 2],
+                                     wo[4 * u + 3]);
+                        st_shared_v4(base + SM_TQ + chunk_off + phys, wt[4 * u], wt[4 * u + 1], wt[4 * u + 2],
+                                     wt[4 * u + 3]);
                     }
                 }
+                if (grp == 0 && p.lse != nullptr && q0_n + row < Lq_s) {
+                    p.lse[(size_t)bh_n * (size_t)p.Lq + (size_t)(yq_n + row)] =
+                        (MASK != 0 && !(lt > 0.f)) ? -INFINITY : (m_ref + __log2f(lt)) * 0.69314718055994531f;
+                }
+                if (grp == 1 && p.mu != nullptr && q0_n + row < Lq_s)
+                    p.mu[(size_t)bh_n * (size_t)p.Lq + (size_t)(yq_n + row)] = mu;
             }
-            // bf16 outputs: O into the Q tile's shared memory, tO into tQ's, in
-            // the 128-byte-swizzled layout of the store tensor maps
-#pragma unroll 1
-            for (int h = 0; h < (kSplit ? 0 : 2); ++h) {
-                const int pc = 2 * grp + h;
-                uint32_t ro[32], rt[32];
-                tmem_ld32(tbase + lane_off + TM_O + 32u * pc, ro);
-                tmem_ld32(tbase + lane_off + TM_T + 32u * pc, rt);
-                tmem_wait_ld();
-                uint32_t wo[16], wt[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const float o0 = __uint_as_float(ro[2 * i]) * inv_l;
-                    const float o1 = __uint_as_float(ro[2 * i + 1]) * inv_l;
-                    const float t0 = fmaf(-mu, o0, __uint_as_float(rt[2 * i]) * inv_l);
-                    const float t1 = fmaf(-mu, o1, __uint_as_float(rt[2 * i + 1]) * inv_l);
-                    wo[i] = pack_bf16x2(o0, o1);
-                    wt[i] = pack_bf16x2(t0, t1);
-                }
-                if (kPacked) {
-                    // rows past the sequence belong to the next one: plain guarded stores
-                    if (q0 + row < Lq_s) {
-                        const size_t off = ((size_t)bh * (size_t)p.Lq + (size_t)(yq + row)) * HD + 64u * grp + 32u * h;
-                        uint4 *po = reinterpret_cast<uint4 *>(p.o_bf + off);
-                        uint4 *pt = reinterpret_cast<uint4 *>(p.to_bf + off);
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            po[u] = make_uint4(wo[4 * u], wo[4 * u + 1], wo[4 * u + 2], wo[4 * u + 3]);
-                            pt[u] = make_uint4(wt[4 * u], wt[4 * u + 1], wt[4 * u + 2], wt[4 * u + 3]);
-                        }
-                    }
-                    continue;
-                }
-                const uint32_t chunk_off = (uint32_t)grp * CHUNK_Q + (uint32_t)row * 128u;
-                const uint32_t unit0 = (uint32_t)h * 4u;
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const uint32_t phys = (((unit0 + u) ^ (uint32_t)(row & 7)) * 16u);
-                    st_shared_v4(base + SM_Q + chunk_off + phys, wo[4 * u], wo[4 * u + 1], wo[4 * u + 2],
-                                 wo[4 * u + 3]);
-                    st_shared_v4(base + SM_TQ + chunk_off + phys, wt[4 * u], wt[4 * u + 1], wt[4 * u + 2],
-                                 wt[4 * u + 3]);
+            if (!kPersist) {
+                fence_proxy_async_smem();
+                named_bar_sync(NB_EPI, SOFTMAX_THREADS);  // staging complete (every softmax thread gets here)
+                if (!kSplit && !kPacked && warp == 4 && lane == 0 && !any_failed && *abort_flag == 0) {
+                    tma_store_3d(&p.tm_o, base + SM_Q, 0, yq_n, bh_n);
+                    tma_store_3d(&p.tm_o, base + SM_Q + CHUNK_Q, 64, yq_n, bh_n);
+                    tma_store_3d(&p.tm_to, base + SM_TQ, 0, yq_n, bh_n);
+                    tma_store_3d(&p.tm_to, base + SM_TQ + CHUNK_Q, 64, yq_n, bh_n);
+                    tma_store_commit();
+                    tma_store_wait_all();
                 }
             }
-            if (grp == 0 && p.lse != nullptr && q0 + row < Lq_s) {
-                p.lse[(size_t)bh * (size_t)p.Lq + (size_t)(yq + row)] =
-                    (MASK != 0 && !(lt > 0.f)) ? -INFINITY : (m_ref + __log2f(lt)) * 0.69314718055994531f;
-            }
-            if (grp == 1 && p.mu != nullptr && q0 + row < Lq_s)
-                p.mu[(size_t)bh * (size_t)p.Lq + (size_t)(yq + row)] = mu;
-        }
-        fence_proxy_async_smem();
-        named_bar_sync(NB_EPI, SOFTMAX_THREADS);  // staging complete (every softmax thread gets here)
-        if (!kSplit && !kPacked && warp == 4 && lane == 0 && !any_failed && *abort_flag == 0) {
-            tma_store_3d(&p.tm_o, base + SM_Q, 0, yq, bh);
-            tma_store_3d(&p.tm_o, base + SM_Q + CHUNK_Q, 64, yq, bh);
-            tma_store_3d(&p.tm_to, base + SM_TQ, 0, yq, bh);
-            tma_store_3d(&p.tm_to, base + SM_TQ + CHUNK_Q, 64, yq, bh);
-            tma_store_commit();
-            tma_store_wait_all();
-        }
+            if (any_failed) break;  // uniform: an OR over every softmax thread
+        } while (kPersist && next_unit(++n, qt_n, bh_n));
         __syncwarp();
     }
 

@@ -340,6 +340,19 @@ AJVP_API int attn_jvp_check_device_status(void *stream);
 AJVP_API int attn_jvp_set_wait_bound_ns(uint64_t ns);
 
 /*
+ * Scheduling of the bf16 forward entry points without masks (attn_jvp_fwd,
+ * attn_jvp_fwd_stats, the host entries): when the keys span at most
+ * `max_key_tiles` tiles of 64 and there are more 128-row query tiles than
+ * SMs, one persistent CTA per SM walks the query tiles and overlaps each
+ * tile's epilogue with the next tile's loads and score products (short key
+ * sequences, e.g. cross-attention to a few hundred text tokens).  Results are
+ * bit-identical either way.  Default 32; 0 turns the persistent form off;
+ * negative values are rejected (AJVP_ERR_INVALID_ARG).  Applies to launches
+ * made after the call, process-wide.
+ */
+AJVP_API int attn_jvp_set_persistent_key_tiles(int64_t max_key_tiles);
+
+/*
  * Failure-detection self test: enqueue a one-warp kernel that waits, through
  * the same bounded-wait routine the attention kernel uses, on a barrier that
  * nothing ever completes, with a bound of `bound_ns`.  The kernel gives up,

@@ -136,3 +136,11 @@ def test_varlen_host_rejections(lib):
     assert call(max_q=101) == B.AJVP_ERR_INVALID_ARG  # longer than the packed tensor
     assert call(total_k=0) == B.AJVP_ERR_INVALID_ARG
     assert call(d=64) == B.AJVP_ERR_UNSUPPORTED_DIM
+
+
+def test_persistent_key_tiles_setting(lib):
+    """The scheduling knob accepts 0 (off) and positive tile counts, rejects
+    negative ones, and needs no GPU."""
+    assert lib.attn_jvp_set_persistent_key_tiles(-1) == B.AJVP_ERR_INVALID_ARG
+    assert lib.attn_jvp_set_persistent_key_tiles(0) == B.AJVP_OK
+    assert lib.attn_jvp_set_persistent_key_tiles(B.DEFAULT_PERSISTENT_KEY_TILES) == B.AJVP_OK
