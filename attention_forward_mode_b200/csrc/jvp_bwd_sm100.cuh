@@ -77,13 +77,13 @@ enum : int {
     B_S_EMPTY = 9,   // + short stage: the G1 products that read it are complete
     B_G1_DONE = 13,  // + score buffer: X..W of the tile complete
     B_X_FREE = 15,   // single-buffer variants: the elementwise warps have read X..W (256 arrivals)
-    B_E_DONE = 16,   // E1, E2 written (256 arrivals)
-    B_G2_DONE = 17,  // + long stage: the tile's G2 products complete (the stage is free again)
-    B_ACC_FULL = 21,
-    B_MMA_DRAIN = 22,
-    B_R1_READY = 23,  // single-buffer variants: R1 written into tensor memory (256 arrivals)
-    B_ST_FULL = 24,   // + slot: V_DK's own two-slot ring of column statistics
-    N_BARS = 26
+    B_E_DONE = 16,   // + score buffer: E1, E2 of the tile written (256 arrivals)
+    B_G2_DONE = 18,  // + long stage: the tile's G2 products complete (the stage is free again)
+    B_ACC_FULL = 22,
+    B_MMA_DRAIN = 23,
+    B_R1_READY = 24,  // single-buffer variants: R1 written into tensor memory (256 arrivals)
+    B_ST_FULL = 25,   // + slot: V_DK's own two-slot ring of column statistics
+    N_BARS = 27
 };
 constexpr uint32_t OFF_TMEM_SLOT = 8 * N_BARS;
 constexpr uint32_t OFF_ABORT = OFF_TMEM_SLOT + 4;
@@ -218,12 +218,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
             mbar_init(BAR(B_S_EMPTY + s), 1);
             mbar_init(BAR(B_G2_DONE + s), 1);
         }
-        for (int b = 0; b < 2; ++b) mbar_init(BAR(B_G1_DONE + b), 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(BAR(B_G1_DONE + b), 1);
+            mbar_init(BAR(B_E_DONE + b), EW_THREADS);
+        }
         mbar_init(BAR(B_X_FREE), EW_THREADS);
         mbar_init(BAR(B_R1_READY), EW_THREADS);
         mbar_init(BAR(B_ST_FULL), 1);
         mbar_init(BAR(B_ST_FULL + 1), 1);
-        mbar_init(BAR(B_E_DONE), EW_THREADS);
         mbar_init(BAR(B_ACC_FULL), 1);
         mbar_init(BAR(B_MMA_DRAIN), 1);
         *abort_flag = 0;
@@ -382,7 +384,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
                 return true;
             };
             auto issue_g2 = [&](int j) -> bool {
-                if (!wait_full(B_E_DONE, j, 1)) return false;
+                // one E_DONE barrier per score buffer, so the parity is unambiguous: the
+                // next phase of buffer j % 2 needs G1 of tile j + 2, issued after this wait
+                // (single buffer: the elementwise warps wait for G2 of tile j first)
+                if (!wait_full(B_E_DONE, j, C::kNB)) return false;
                 if (VAR == V_DV && !wait_full(B_L_FULL, j, C::kLS)) return false;
                 const int b = j % C::kNB, s = j % C::kLS;
                 const uint32_t tb = tbase + C::BUF0 + (uint32_t)b * C::BUF_COLS;
@@ -572,7 +577,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
             }
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(BAR(B_E_DONE));
+            mbar_arrive(BAR(B_E_DONE + b));
         }
 
         if (!failed) failed = !mbar_wait_warp(BAR(B_ACC_FULL), 0, abort_flag, bound);
