@@ -177,14 +177,54 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
     // rows start at tensor row yq - q0 and keys at yk0, with Lq_s rows and Lk_s keys
     int qt, bh, Lq_s = p.Lq, Lk_s = p.Lk, yk0 = 0, yq0 = 0;
     if (kPacked) {
-        // longest-first: the last tiles of every (sequence, head) go in the first wave
-        bh = blockIdx.x % p.BH;
-        const int rest = blockIdx.x / p.BH;
-        const int b = rest % p.n_seq;
-        qt = p.n_qtiles - 1 - rest / p.n_seq;
-        // clamped into the tensors, so that bad offsets stay memory-safe
-        const int a0 = min(max(p.cu_q[b], 0), p.Lq), a1 = min(max(p.cu_q[b + 1], a0), p.Lq);
-        const int k0 = min(max(p.cu_k[b], 0), p.Lk), k1 = min(max(p.cu_k[b + 1], k0), p.Lk);
+        // sequence b's rows and keys, clamped into the tensors so that bad offsets stay memory-safe
+        auto q_begin = [&](int b) { return min(max(p.cu_q[b], 0), p.Lq); };
+        auto k_begin = [&](int b) { return min(max(p.cu_k[b], 0), p.Lk); };
+        int b;
+        if (!kCausal && p.n_seq <= 32) {
+            // without the causal mask a unit costs its sequence's key count whatever its
+            // query tile, so the units go out longest sequence first (ties: lower index),
+            // which leaves the short ones for the last wave.  Every warp ranks the
+            // sequences itself, one per lane; consecutive CTAs take the query tiles of
+            // one (sequence, head), which share its keys in L2.
+            const int l = threadIdx.x & 31;
+            int units = 0, cost = -1;  // lanes past the last sequence: no units, ranked last
+            if (l < p.n_seq) {
+                const int a0 = q_begin(l), a1 = max(q_begin(l + 1), a0);
+                const int k0 = k_begin(l), k1 = max(k_begin(l + 1), k0);
+                units = (a1 - a0 + BR - 1) / BR * p.BH;
+                cost = k1 - k0;
+            }
+            int rank = 0;
+#pragma unroll 4
+            for (int m = 0; m < 32; ++m) {
+                const int cm = __shfl_sync(0xffffffffu, cost, m);
+                rank += (cm > cost || (cm == cost && m < l)) ? 1 : 0;
+            }
+            int first = 0;  // units of the sequences ranked before this one
+#pragma unroll 4
+            for (int m = 0; m < 32; ++m) {
+                const int rm = __shfl_sync(0xffffffffu, rank, m), um = __shfl_sync(0xffffffffu, units, m);
+                first += rm < rank ? um : 0;
+            }
+            const int i = (int)blockIdx.x;
+            const unsigned own = __ballot_sync(0xffffffffu, i >= first && i < first + units);
+            if (own == 0u) return;  // past the last unit (the same for the whole CTA)
+            b = __ffs(own) - 1;
+            const int local = i - __shfl_sync(0xffffffffu, first, b);
+            const int nq = __shfl_sync(0xffffffffu, units, b) / p.BH;
+            bh = local / nq;
+            qt = local % nq;
+        } else {
+            // heaviest first for the causal mask: the last tiles of every (sequence, head)
+            // go in the first wave
+            bh = blockIdx.x % p.BH;
+            const int rest = blockIdx.x / p.BH;
+            b = rest % p.n_seq;
+            qt = p.n_qtiles - 1 - rest / p.n_seq;
+        }
+        const int a0 = q_begin(b), a1 = max(q_begin(b + 1), a0);
+        const int k0 = k_begin(b), k1 = max(k_begin(b + 1), k0);
         yq0 = a0;
         Lq_s = a1 - a0;
         yk0 = k0;

@@ -36,7 +36,8 @@ def host_run(inp, scale, pinned=True, heads_per_chunk=None, want_lse=True):
                                              (2, 3, 300, 700, None),    # 6 heads in chunks of 2
                                              (1, 7, 129, 257, 2),       # ragged last chunk
                                              (1, 5, 640, 512, 1),       # one head per chunk
-                                             (2, 2, 200, 64, 4)])       # all heads in one chunk
+                                             (2, 2, 200, 64, 4),        # all heads in one chunk
+                                             (1, 3, 20000, 512, 1)])    # persistent kernel per chunk
 def test_host_equals_device(B, H, Lq, Lk, chunk):
     w = custom(B, H, Lq, Lk, 128)
     inp = gpu_inputs(w, seed=B * 100 + H * 10 + Lq)

@@ -111,18 +111,25 @@ def test_unmasked_paths_agree_bitwise():
         assert torch.equal(a[0], b)
 
 
-def test_many_short_sequences():
-    # 64 sequences of 1..200 tokens (one head): the grid has many empty tiles
-    rng = np.random.default_rng(3)
-    lq = [int(v) for v in rng.integers(1, 200, size=64)]
-    lk = [int(v) for v in rng.integers(1, 200, size=64)]
-    x, cq, ck = _packed_inputs(1, lq, lk, seed=9)
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("n", [32, 33, 64])
+def test_many_short_sequences(n, causal):
+    # n sequences of 1..300 tokens (two heads): the grid has many empty tiles.  Without
+    # the mask, up to 32 sequences go out longest first (ranked inside the kernel), more
+    # in the causal order
+    rng = np.random.default_rng(n)
+    lq = [int(v) for v in rng.integers(1, 300, size=n)]
+    lk = [int(v) for v in rng.integers(1, 300, size=n)]
+    x, cq, ck = _packed_inputs(2, lq, lk, seed=9)
     s = 0.1
-    got = ajvp.attn_jvp_fwd_varlen(*(x[n] for n in NAMES), cq, ck, max(lq), s, causal=True)
+    got = ajvp.attn_jvp_fwd_varlen(*(x[n_] for n_ in NAMES), cq, ck, max(lq), s, causal=causal)
     torch.cuda.synchronize()
-    ref = oracle.attn_jvp_packed(*(x[n] for n in NAMES), s, cq.cpu().numpy(), ck.cpu().numpy(), True)
-    seen = np.concatenate([np.arange(a) + (b - a) >= 0 for a, b in zip(lq, lk)])[None]
-    check(got, ref, seen, "many short")
+    ref = oracle.attn_jvp_packed(*(x[n_] for n_ in NAMES), s, cq.cpu().numpy(), ck.cpu().numpy(), causal)
+    if causal:
+        seen = np.concatenate([np.arange(a) + (b - a) >= 0 for a, b in zip(lq, lk)])
+    else:
+        seen = np.ones(sum(lq), dtype=bool)
+    check(got, ref, np.broadcast_to(seen[None], (2, sum(lq))), f"{n} short, causal={causal}")
 
 
 def test_causal_video_workload_sampled():
