@@ -276,6 +276,7 @@ int launch_bwd_var(std::initializer_list<const void *> r, std::initializer_list<
         if ((rc = encode_3d(&p.tm_out[i++], x, d, Lrow, BH, 128)) != AJVP_OK) return rc;
     i = 0;
     for (float f : sc) p.out_scale[i++] = f;
+    p.r0 = static_cast<const __nv_bfloat16 *>(*r.begin());
     if (r.size() > 1) p.r1 = static_cast<const __nv_bfloat16 *>(*(r.begin() + 1));
     const int64_t n_rtiles = (Lrow + BM - 1) / BM;
     p.stats = static_cast<const float4 *>(stats);

@@ -42,7 +42,10 @@
 //   set of X, Y, Z, W: their elementwise warps release it as soon as they
 //   have read it (so G1 of the next tile runs while they compute) and write
 //   E1, E2 to a region of their own.  The other variants double-buffer their
-//   score tiles and write E1, E2 over them, as the forward kernel does.
+//   score tiles and write E1, E2 over them, as the forward kernel does.  The
+//   resident tile R1 (V_DQ, V_DK) or R0 and R1 (V_DTQ, V_DV) are G1's A
+//   operands straight from tensor memory, written there once by the
+//   elementwise warps; the others are read from shared memory.
 //
 // Warp roles (384 threads): warp 0 TMA producer, warp 1 MMA issuer, warp 2
 // tensor-memory allocation, warps 4-11 elementwise in two groups of four
@@ -81,7 +84,7 @@ enum : int {
     B_G2_DONE = 18,  // + long stage: the tile's G2 products complete (the stage is free again)
     B_ACC_FULL = 22,
     B_MMA_DRAIN = 23,
-    B_R1_READY = 24,  // single-buffer variants: R1 written into tensor memory (256 arrivals)
+    B_R1_READY = 24,  // R1 (and R0) written into tensor memory (256 arrivals)
     B_ST_FULL = 25,   // + slot: V_DK's own two-slot ring of column statistics
     N_BARS = 27
 };
@@ -92,7 +95,7 @@ constexpr uint32_t NB_EPI = 1;
 struct Params {
     CUtensorMap tm_r[4], tm_l[2], tm_s[2], tm_out[2];
     const float4 *stats;  // [B*H][Lq] {lse*log2(e), mu, a, D}, plus BN rows of padding
-    const __nv_bfloat16 *r1;  // single-buffer variants: R1 ([B*H][Lrow][128]), staged into tensor memory
+    const __nv_bfloat16 *r0, *r1;  // R0 / R1 ([B*H][Lrow][128]) where they are staged into tensor memory
     int Lrow, Lcol;       // row-side and streamed lengths
     int Lq;               // query rows per (batch, head): the stats row stride
     int n_rtiles;         // 128-row tiles per (batch, head)
@@ -154,9 +157,13 @@ struct Var {
     // streamed-tile rings: "long" (tiles G2 reads, freed when G2 completes) and
     // "short" (tiles only G1 reads, freed when G1 completes), as deep as shared
     // memory allows so that loads run well ahead of the products
-    // single-buffer variants keep R1 in tensor memory (an A operand read from
-    // there) and use its shared-memory slot as a third long-ring stage
-    static constexpr bool kR1T = kSingle;
+    // resident A operands read from tensor memory instead of shared memory (the
+    // score products then read only their streamed B tile there): R1 in every
+    // variant with 64 free columns, R0 too where 128 are free (dtQ, dV)
+    static constexpr bool kR0T = VAR == V_DTQ || VAR == V_DV;
+    static constexpr bool kR1T = kSingle || kR0T;
+    // single-buffer variants use R1's shared-memory slot as a third long-ring stage
+    static constexpr bool kR1Stage = kSingle;
     static constexpr int kLS = kSingle ? 3 : (VAR == V_DV ? 2 : 4);
     // column statistics in shared memory: with the long-ring stage (double-buffer
     // variants), or in a two-slot ring of their own freed by the elementwise warps (V_DK)
@@ -169,11 +176,11 @@ struct Var {
     static constexpr uint32_t L_CH = (kL1 ? 2u : 1u) * CHUNK_C, S_CH = (kNS > 1 ? 2u : 1u) * CHUNK_C;
     static constexpr uint32_t L_BYTES = 2 * L_CH, S_BYTES = 2 * S_CH;
     static constexpr uint32_t SM_L = SM_R + kNR * R_TILE;
-    static constexpr uint32_t SM_S = SM_L + (kR1T ? kLS - 1 : kLS) * L_BYTES;
+    static constexpr uint32_t SM_S = SM_L + (kR1Stage ? kLS - 1 : kLS) * L_BYTES;
     static constexpr uint32_t SM_ST = SM_S + kSS * S_BYTES;  // statistics of the long-ring tiles
     static constexpr uint32_t SM_BAR = SM_ST + (kStatsRing ? 2 * STATS_TILE : (kStatsSmem ? kLS * STATS_TILE : 0u));
     __device__ static uint32_t long_off(int s) {  // offset of long-ring stage s
-        return (kR1T && s == kLS - 1) ? SM_R + R_TILE : SM_L + (uint32_t)s * L_BYTES;
+        return (kR1Stage && s == kLS - 1) ? SM_R + R_TILE : SM_L + (uint32_t)s * L_BYTES;
     }
     static constexpr uint32_t SMEM_BYTES = SM_BAR + 256;  // the base is 1024-byte aligned (checked)
     static_assert(SMEM_BYTES <= 232448, "exceeds the opt-in shared memory of one CTA");
@@ -183,7 +190,9 @@ struct Var {
     static constexpr uint32_t BUF_COLS = kSingle ? 256u : 128u;
     static constexpr uint32_t X = 0, Y = 64, Z = kSingle ? 128u : 64u, W = 192;  // inside a buffer
     static constexpr uint32_t E1 = BUF0 + 256u, E2 = BUF0 + 288u;               // single only
-    static constexpr uint32_t R1T = BUF0 + 320u;                                  // single only: R1 (64 columns)
+    static constexpr uint32_t R0T = 384u, R1T = 448u;  // R0, R1 as bf16 pairs (64 columns each)
+    static_assert(!kR0T || BUF0 + kNB * BUF_COLS <= R0T, "R0 overlaps the score buffers");
+    static_assert(!kR1T || (kSingle ? E2 + 32u : BUF0 + kNB * BUF_COLS) <= R1T, "R1 overlaps");
 };
 
 template <int VAR>
@@ -254,9 +263,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
             bool ok = true;
             int l_last[4] = {-1, -1, -1, -1}, s_last[4] = {-1, -1, -1, -1}, st_last = -1;
             if (lp) {
-                mbar_arrive_expect_tx(BAR(B_R_FULL), (C::kNR - (C::kR1T ? 1 : 0)) * R_TILE);
+                // (a phase that expects no bytes completes on this arrival alone)
+                mbar_arrive_expect_tx(BAR(B_R_FULL), (C::kNR - (C::kR1T ? 1 : 0) - (C::kR0T ? 1 : 0)) * R_TILE);
                 for (int i = 0; i < C::kNR; ++i) {
-                    if (C::kR1T && i == 1) continue;  // R1 goes to tensor memory (elementwise warps)
+                    // R0 / R1 in tensor memory are written by the elementwise warps
+                    if ((C::kR1T && i == 1) || (C::kR0T && i == 0)) continue;
                     tma_load_3d(base + SM_R + i * R_TILE, &p.tm_r[i], BAR(B_R_FULL), 0, r0, bh);
                     tma_load_3d(base + SM_R + i * R_TILE + CHUNK_R, &p.tm_r[i], BAR(B_R_FULL), 64, r0, bh);
                 }
@@ -345,6 +356,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
                     mma_ss(d, desc_add(a, offr), desc_add(b, offc), id, (acc || kk > 0) ? 1u : 0u);
                 }
             };
+            // the same with the A operand in tensor memory (column a_col, 8 columns per K-step)
+            auto g1t = [&](uint32_t d, uint32_t a_col, uint64_t b, uint32_t ch, uint32_t id, bool acc) {
+#pragma unroll
+                for (int kk = 0; kk < HD / 16; ++kk)
+                    mma_ts(d, tbase + a_col + 8u * kk, desc_add(b, (kk >> 2) * ch + (kk & 3) * 32), id,
+                           (acc || kk > 0) ? 1u : 0u);
+            };
             auto wait_full = [&](int bar, int j, int stages) -> bool {
                 if (!mbar_wait(BAR(bar + j % stages), (j / stages) & 1, abort_flag, bound)) return false;
                 tc_fence_after();
@@ -358,26 +376,23 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
                 const uint64_t ds = smem_desc_sw128(base + C::SM_S + ss * C::S_BYTES, 16, 1024);
                 if (VAR != V_DV && !wait_full(B_L_FULL, j, C::kLS)) return false;  // V_DV: G1 reads no long tile
                 if (VAR == V_DQ || VAR == V_DK) {
-                    g1(tb + C::X, dr0, dl, LC, ID_W, false);  // [X | Y] = R0 [L0; L1]^T
-#pragma unroll
-                    for (int kk = 0; kk < HD / 16; ++kk)  // Y += R1 L0^T, R1 from tensor memory
-                        mma_ts(tb + C::Y, tbase + C::R1T + 8u * kk,
-                               desc_add(dl, (kk >> 2) * LC + (kk & 3) * 32), ID_N, 1u);
+                    g1(tb + C::X, dr0, dl, LC, ID_W, false);   // [X | Y] = R0 [L0; L1]^T
+                    g1t(tb + C::Y, C::R1T, dl, LC, ID_N, true);  // Y += R1 L0^T, R1 from tensor memory
                     // the short stage is needed only now: its load overlaps the products above
                     if (!wait_full(B_S_FULL, j, C::kSSd)) return false;
                     g1(tb + C::Z, dr2, ds, SC, ID_W, false);  // [Z | W] = R2 [S0; S1]^T
                     g1(tb + C::W, dr3, ds, SC, ID_N, true);   // W += R3 S0^T
-                } else if (VAR == V_DTQ) {
-                    g1(tb + C::X, dr0, dl, LC, ID_N, false);  // X = R0 L0^T
+                } else if (VAR == V_DTQ) {  // both A operands from tensor memory
+                    g1t(tb + C::X, C::R0T, dl, LC, ID_N, false);  // X = R0 L0^T
                     if (!wait_full(B_S_FULL, j, C::kSSd)) return false;
-                    g1(tb + C::Z, dr1, ds, SC, ID_N, false);  // Z = R1 S0^T
+                    g1t(tb + C::Z, C::R1T, ds, SC, ID_N, false);  // Z = R1 S0^T
                 } else if (VAR == V_DKT) {
                     g1(tb + C::X, dr0, dl, LC, ID_N, false);                     // X = R0 L0^T
                     g1(tb + C::Z, dr1, desc_add(dl, CHUNK_C), LC, ID_N, false);  // Z = R1 L1^T
-                } else {  // V_DV
+                } else {  // V_DV, both A operands from tensor memory
                     if (!wait_full(B_S_FULL, j, C::kSSd)) return false;
-                    g1(tb + C::X, dr0, ds, SC, ID_W, false);  // [X | Y] = R0 [S0; S1]^T
-                    g1(tb + C::Y, dr1, ds, SC, ID_N, true);   // Y += R1 S0^T
+                    g1t(tb + C::X, C::R0T, ds, SC, ID_W, false);  // [X | Y] = R0 [S0; S1]^T
+                    g1t(tb + C::Y, C::R1T, ds, SC, ID_N, true);   // Y += R1 S0^T
                 }
                 mma_commit(BAR(B_G1_DONE + b));
                 if (C::kSS > 0) mma_commit(BAR(B_S_EMPTY + ss));
@@ -446,25 +461,30 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
         if (!C::kColStats && r0 + row < p.Lrow) rs = p.stats[(size_t)bh * p.Lq + (size_t)(r0 + row)];
         bool failed = false;
         if (C::kR1T) {
-            // R1 row `row` into tensor memory as bf16 pairs (column c = features 2c, 2c+1),
-            // the layout of an A operand; group grp writes features 64*grp .. 64*grp+63
-            uint32_t w[32];
-            if (r0 + row < p.Lrow) {
-                const uint4 *src = reinterpret_cast<const uint4 *>(
-                    p.r1 + ((size_t)bh * (size_t)p.Lrow + (size_t)(r0 + row)) * HD + 64u * (uint32_t)grp);
+            // R1 (and R0) row `row` into tensor memory as bf16 pairs (column c = features
+            // 2c, 2c+1), the layout of an A operand; group grp writes features 64*grp ..
+            // 64*grp+63 (rows past the tensor: zeros)
+            auto stage_row = [&](const __nv_bfloat16 *src_t, uint32_t col) {
+                uint32_t w[32];
+                if (r0 + row < p.Lrow) {
+                    const uint4 *src = reinterpret_cast<const uint4 *>(
+                        src_t + ((size_t)bh * (size_t)p.Lrow + (size_t)(r0 + row)) * HD + 64u * (uint32_t)grp);
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const uint4 v4 = __ldg(src + u);
-                    w[4 * u] = v4.x;
-                    w[4 * u + 1] = v4.y;
-                    w[4 * u + 2] = v4.z;
-                    w[4 * u + 3] = v4.w;
+                    for (int u = 0; u < 8; ++u) {
+                        const uint4 v4 = __ldg(src + u);
+                        w[4 * u] = v4.x;
+                        w[4 * u + 1] = v4.y;
+                        w[4 * u + 2] = v4.z;
+                        w[4 * u + 3] = v4.w;
+                    }
+                } else {
+#pragma unroll
+                    for (int u = 0; u < 32; ++u) w[u] = 0u;
                 }
-            } else {
-#pragma unroll
-                for (int u = 0; u < 32; ++u) w[u] = 0u;
-            }
-            tmem_st32(tbase + lane_off + C::R1T + 32u * (uint32_t)grp, w);
+                tmem_st32(tbase + lane_off + col + 32u * (uint32_t)grp, w);
+            };
+            stage_row(p.r1, C::R1T);
+            if (C::kR0T) stage_row(p.r0, C::R0T);
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(BAR(B_R1_READY));
