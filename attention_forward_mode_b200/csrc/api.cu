@@ -102,11 +102,9 @@ int device_setup(int *dev_out) {
         if (e3 == cudaSuccess) e3 = set_fwd_smem<false, 1>();
         if (e3 == cudaSuccess) e3 = set_fwd_smem<false, 2>();
         if (e3 == cudaSuccess) e3 = set_fwd_smem<false, 3>();
-        if (e3 == cudaSuccess) e3 = set_bwd_smem<ajvp::bwd::V_DQ>();
-        if (e3 == cudaSuccess) e3 = set_bwd_smem<ajvp::bwd::V_DTQ>();
-        if (e3 == cudaSuccess) e3 = set_bwd_smem<ajvp::bwd::V_DK>();
-        if (e3 == cudaSuccess) e3 = set_bwd_smem<ajvp::bwd::V_DKT>();
-        if (e3 == cudaSuccess) e3 = set_bwd_smem<ajvp::bwd::V_DV>();
+        if (e3 == cudaSuccess) e3 = set_bwd_smem<ajvp::bwd::V_Q>();
+        if (e3 == cudaSuccess) e3 = set_bwd_smem<ajvp::bwd::V_K>();
+        if (e3 == cudaSuccess) e3 = set_bwd_smem<ajvp::bwd::V_V>();
         cudaError_t e4 = cudaFuncSetAttribute(ajvp::f32::attn_jvp_fwd_f32_kernel,
                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
                                               (int)ajvp::f32::smem_bytes(ajvp::f32::DMAX));
@@ -276,8 +274,6 @@ int launch_bwd_var(std::initializer_list<const void *> r, std::initializer_list<
         if ((rc = encode_3d(&p.tm_out[i++], x, d, Lrow, BH, 128)) != AJVP_OK) return rc;
     i = 0;
     for (float f : sc) p.out_scale[i++] = f;
-    p.r0 = static_cast<const __nv_bfloat16 *>(*r.begin());
-    if (r.size() > 1) p.r1 = static_cast<const __nv_bfloat16 *>(*(r.begin() + 1));
     const int64_t n_rtiles = (Lrow + BM - 1) / BM;
     p.stats = static_cast<const float4 *>(stats);
     p.Lrow = (int)Lrow;
@@ -427,9 +423,9 @@ int bwd_steps(int first, int last, const void *q, const void *k, const void *v, 
         if (!dk || !dv || !dtk || !dtv) return AJVP_ERR_INVALID_ARG;
         if (BH * Lk >= (int64_t(1) << 31)) return AJVP_ERR_TOO_LARGE;
         const size_t bytes = (size_t)(BH * Lk * d) * 2u;
-        // the kernels that would write them: dk 3, dtk and dtv 4, dv 5
-        void *zero[4] = {dk, dtk, dtv, dv};
-        const int kern[4] = {3, 4, 4, 5};
+        // the steps that would write them: dk and dtk 2, dv and dtv 3
+        void *zero[4] = {dk, dtk, dv, dtv};
+        const int kern[4] = {2, 2, 3, 3};
         for (int i = 0; i < 4; ++i) {
             if (first > kern[i] || last < kern[i]) continue;
             cudaError_t e = cudaMemsetAsync(zero[i], 0, bytes, st);
@@ -465,22 +461,16 @@ int bwd_steps(int first, int last, const void *q, const void *k, const void *v, 
     }
     auto want = [&](int k) { return first <= k && last >= k; };
     const float s1 = scale;
-    // rows = queries, streamed keys
-    if (want(1) && (rc = launch_bwd_var<V_DQ>({q, tq, dtout, dout}, {k, tk}, {v, tv}, {dq}, {s1}, workspace, BH, Lq,
-                                              Lk, Lq, d, scale, st)) != AJVP_OK)
+    // rows = queries, streamed keys: dq, dtq
+    if (want(1) && (rc = launch_bwd_var<V_Q>({q, tq, dtout, dout}, {k, tk}, {v, tv}, {dq, dtq}, {s1, s1}, workspace,
+                                             BH, Lq, Lk, Lq, d, scale, st)) != AJVP_OK)
         return rc;
-    if (want(2) && (rc = launch_bwd_var<V_DTQ>({q, dtout}, {k}, {v}, {dtq}, {s1}, workspace, BH, Lq, Lk, Lq, d, scale,
-                                               st)) != AJVP_OK)
+    // rows = keys, streamed queries: dk, dtk; dv, dtv
+    if (want(2) && (rc = launch_bwd_var<V_K>({k, tk, v, tv}, {q, tq}, {dtout, dout}, {dk, dtk}, {s1, s1}, workspace,
+                                             BH, Lk, Lq, Lq, d, scale, st)) != AJVP_OK)
         return rc;
-    // rows = keys, streamed queries
-    if (want(3) && (rc = launch_bwd_var<V_DK>({k, tk, v, tv}, {q, tq}, {dtout, dout}, {dk}, {s1}, workspace, BH, Lk,
-                                              Lq, Lq, d, scale, st)) != AJVP_OK)
-        return rc;
-    if (want(4) && (rc = launch_bwd_var<V_DKT>({k, v}, {q, dtout}, {}, {dtk, dtv}, {s1, 1.0f}, workspace, BH, Lk, Lq,
-                                               Lq, d, scale, st)) != AJVP_OK)
-        return rc;
-    if (want(5) && (rc = launch_bwd_var<V_DV>({k, tk}, {dout, dtout}, {q, tq}, {dv}, {1.0f}, workspace, BH, Lk, Lq,
-                                              Lq, d, scale, st)) != AJVP_OK)
+    if (want(3) && (rc = launch_bwd_var<V_V>({k, tk}, {dout, dtout}, {q, tq}, {dv, dtv}, {1.0f, 1.0f}, workspace, BH,
+                                             Lk, Lq, Lq, d, scale, st)) != AJVP_OK)
         return rc;
     return AJVP_OK;
 }
@@ -493,7 +483,7 @@ int attn_jvp_bwd(const void *q, const void *k, const void *v, const void *tq, co
                  const void *dtout, void *dq, void *dk, void *dv, void *dtq, void *dtk, void *dtv, int64_t B,
                  int64_t H, int64_t Lq, int64_t Lk, int64_t d, float scale, void *workspace,
                  uint64_t workspace_bytes, void *stream) {
-    return bwd_steps(0, 5, q, k, v, tq, tk, tv, o, to, lse, mu, dout, dtout, dq, dk, dv, dtq, dtk, dtv, B, H, Lq, Lk,
+    return bwd_steps(0, 3, q, k, v, tq, tk, tv, o, to, lse, mu, dout, dtout, dq, dk, dv, dtq, dtk, dtv, B, H, Lq, Lk,
                      d, scale, workspace, workspace_bytes, stream);
 }
 
@@ -502,7 +492,7 @@ int attn_jvp_bwd_step(int step, const void *q, const void *k, const void *v, con
                       const void *dout, const void *dtout, void *dq, void *dk, void *dv, void *dtq, void *dtk,
                       void *dtv, int64_t B, int64_t H, int64_t Lq, int64_t Lk, int64_t d, float scale,
                       void *workspace, uint64_t workspace_bytes, void *stream) {
-    if (step < 0 || step > 5) return AJVP_ERR_INVALID_ARG;
+    if (step < 0 || step > 3) return AJVP_ERR_INVALID_ARG;
     return bwd_steps(step, step, q, k, v, tq, tk, tv, o, to, lse, mu, dout, dtout, dq, dk, dv, dtq, dtk, dtv, B, H,
                      Lq, Lk, d, scale, workspace, workspace_bytes, stream);
 }

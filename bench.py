@@ -52,9 +52,8 @@ BWD_KERNEL_SOURCES = ["attention_forward_mode_b200/csrc/jvp_bwd_sm100.cuh",
 BWD_TRAFFIC_FILE = "profiles/attn_jvp_bwd_kernel.video_selfattn_b1h12_l32760.md"
 L2_BYTES = 126 * 1024 * 1024
 # backward kernels (steps of attn_jvp_bwd): name, contraction FLOPs per (Lq*Lk*d) per head
-BWD_STEPS = [("bwd_rowstats_kernel", 0.0), ("attn_jvp_bwd_kernel<V_DQ> (dQ)", 16.0),
-             ("attn_jvp_bwd_kernel<V_DTQ> (dtQ)", 6.0), ("attn_jvp_bwd_kernel<V_DK> (dK)", 16.0),
-             ("attn_jvp_bwd_kernel<V_DKT> (dtK, dtV)", 8.0), ("attn_jvp_bwd_kernel<V_DV> (dV)", 10.0)]
+BWD_STEPS = [("bwd_rowstats_kernel", 0.0), ("attn_jvp_bwd_kernel<V_Q> (dQ, dtQ)", 18.0),
+             ("attn_jvp_bwd_kernel<V_K> (dK, dtK)", 18.0), ("attn_jvp_bwd_kernel<V_V> (dV, dtV)", 12.0)]
 
 
 # ------------------------------------------------------------------ helpers

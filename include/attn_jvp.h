@@ -195,9 +195,9 @@ AJVP_API int attn_jvp_fwd_stats(const void *q, const void *k, const void *v,
  *                         at least attn_jvp_bwd_workspace_bytes(B, H, Lq)
  *                         bytes; nothing in it needs to start at zero
  *
- * Six kernels on `stream`: per-row statistics into the workspace, then five
- * gradient kernels (tcgen05: dq; dtq; dk; dtk and dtv; dv), each owning its
- * outputs (no atomics: results are deterministic).  Gradients are
+ * Four kernels on `stream`: per-row statistics into the workspace, then
+ * three gradient kernels (tcgen05: dq and dtq; dk and dtk; dv and dtv), each
+ * owning its outputs (no atomics: results are deterministic).  Gradients are
  * accumulated in fp32 and rounded to bf16 (round-to-nearest-even).
  * Supported: d == 128, every pointer non-NULL and 16-byte aligned, sizes as
  * attn_jvp_fwd.  B*H == 0 is a no-op; Lq == 0 writes zeros to dk, dv, dtk,
@@ -213,14 +213,14 @@ AJVP_API int attn_jvp_bwd(const void *q, const void *k, const void *v,
                  float scale, void *workspace, uint64_t workspace_bytes, void *stream);
 
 /*
- * attn_jvp_bwd_step -- one of attn_jvp_bwd's six kernels, for callers that
+ * attn_jvp_bwd_step -- one of attn_jvp_bwd's four kernels, for callers that
  * schedule them (or time them) separately: step 0 writes the row
- * statistics into the workspace, step 1 dq, step 2 dtq, step 3 dk, step 4
- * dtk and dtv, step 5 dv.  Steps 1-5 read the workspace step 0 wrote (same
+ * statistics into the workspace, step 1 dq and dtq, step 2 dk and dtk,
+ * step 3 dv and dtv.  Steps 1-3 read the workspace step 0 wrote (same
  * inputs, same workspace, ordered after it); they are independent of each
  * other.  Arguments, checks and errors as attn_jvp_bwd (every pointer is
  * checked, even those a step does not touch); AJVP_ERR_INVALID_ARG for a
- * step outside 0..5.
+ * step outside 0..3.
  */
 AJVP_API int attn_jvp_bwd_step(int step, const void *q, const void *k, const void *v,
                       const void *tq, const void *tk, const void *tv,

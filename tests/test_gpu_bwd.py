@@ -135,7 +135,7 @@ def test_steps_equal_all_in_one():
     full, (o, to, lse, mu) = run(inp, cot, w.scale)
     ws = torch.empty(ajvp.bwd_workspace_bytes(w.B, w.H, w.Lq), dtype=torch.uint8, device="cuda")
     grads = None
-    for step in (0, 5, 3, 1, 4, 2):  # steps 1-5 only need step 0 before them
+    for step in (0, 3, 1, 2):  # steps 1-3 only need step 0 before them
         grads = ajvp.attn_jvp_bwd(*(inp[n] for n in NAMES), o, to, lse, mu, cot["dout"], cot["dtout"], w.scale,
                                   grads=grads, workspace=ws, step=step)
     torch.cuda.synchronize()
