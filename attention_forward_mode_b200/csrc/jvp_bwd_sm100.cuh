@@ -78,8 +78,8 @@ enum : int {
     B_S_FULL = 5,    // + short stage (up to 4)
     B_S_EMPTY = 9,   // + short stage: the G1 products that read it are complete
     B_G1_DONE = 13,  // + score buffer: X..W of the tile complete
-    B_X_FREE = 15,   // V_Q, V_K: the elementwise warps have read X..W (256 arrivals)
-    B_E_DONE = 16,   // + score buffer: E1, E2 of the tile written (256 arrivals)
+    B_X_FREE = 15,   // V_Q, V_K: the elementwise warps have read X..W (one arrival per warp)
+    B_E_DONE = 16,   // + score buffer: E1, E2 of the tile written (one arrival per warp)
     B_G2_DONE = 18,  // + long stage: the tile's G2 products complete (the stage is free again)
     B_ACC_FULL = 22,
     B_MMA_DRAIN = 23,
@@ -212,9 +212,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(BAR(B_G1_DONE + b), 1);
-            mbar_init(BAR(B_E_DONE + b), EW_THREADS);
+            mbar_init(BAR(B_E_DONE + b), EW_THREADS / 32);  // one arrival per elementwise warp
         }
-        mbar_init(BAR(B_X_FREE), EW_THREADS);
+        mbar_init(BAR(B_X_FREE), EW_THREADS / 32);
         mbar_init(BAR(B_ST_FULL), 1);
         mbar_init(BAR(B_ST_FULL + 1), 1);
         mbar_init(BAR(B_ACC_FULL), 1);
@@ -482,8 +482,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
                 tmem_ld32(tb + col0 + C::Z, zr);
                 tmem_ld32(tb + col0 + C::W, wr);
                 tmem_wait_ld();
-                tc_fence_before();
-                mbar_arrive(BAR(B_X_FREE));
+                warp_arrive_after_tc(BAR(B_X_FREE));
 #pragma unroll
                 for (int i = 0; i < 32; i += 2) {
                     float2 r1, r2;
@@ -510,8 +509,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
             tmem_st16(tb + col0 + C::E1, e1);
             tmem_st16(tb + col0 + C::E2, e2);
             tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(BAR(B_E_DONE + b));
+            warp_arrive_after_tc(BAR(B_E_DONE + b));
         }
 
         if (!failed) failed = !mbar_wait_warp(BAR(B_ACC_FULL), 0, abort_flag, bound);

@@ -98,7 +98,7 @@ enum : int {
     B_P_FULL = 9,    // + buffer
     B_O_FULL = 11,   // every MMA of the unit has completed (one phase per unit)
     B_MMA_DRAIN = 12,
-    B_OT_FREE = 13,  // persistent: the epilogue has read O / T (256 arrivals per unit)
+    B_OT_FREE = 13,  // persistent: the epilogue has read O / T (one arrival per softmax warp)
     N_BARS = 14
 };
 static_assert(STAGES == 2, "the K-side ring reuses the two S/dS' buffer barriers");
@@ -280,11 +280,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(BAR(B_SD_FULL + b), 1);
-            mbar_init(BAR(B_P_FULL + b), SOFTMAX_THREADS);
+            mbar_init(BAR(B_P_FULL + b), SOFTMAX_THREADS / 32);  // one arrival per softmax warp
         }
         mbar_init(BAR(B_O_FULL), 1);
         mbar_init(BAR(B_MMA_DRAIN), 1);
-        mbar_init(BAR(B_OT_FREE), SOFTMAX_THREADS);
+        mbar_init(BAR(B_OT_FREE), SOFTMAX_THREADS / 32);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -624,8 +624,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                 l += (ls2a.x + ls2b.x) + (ls2a.y + ls2b.y);
                 g += (gs2a.x + gs2b.x) + (gs2a.y + gs2b.y);
                 tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(BAR(B_P_FULL + b));
+                warp_arrive_after_tc(BAR(B_P_FULL + b));
             }
 
             if (!failed) failed = !mbar_wait_warp(BAR(B_O_FULL), n & 1, abort_flag, bound);
@@ -681,10 +680,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                     tmem_ld32(tbase + lane_off + TM_O + 32u * pc, ro);
                     tmem_ld32(tbase + lane_off + TM_T + 32u * pc, rt);
                     tmem_wait_ld();
-                    if (kPersist && h == 1) {  // O / T read: the next unit may overwrite them
-                        tc_fence_before();
-                        mbar_arrive(BAR(B_OT_FREE));
-                    }
+                    if (kPersist && h == 1)  // O / T read: the next unit may overwrite them
+                        warp_arrive_after_tc(BAR(B_OT_FREE));
                     uint32_t wo[16], wt[16];
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {

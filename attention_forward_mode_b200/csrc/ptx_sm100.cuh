@@ -321,4 +321,14 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                  : "memory");
 }
 
+// One arrival per warp on a barrier whose count is in warps: every lane orders
+// its tensor-memory accesses before the warp synchronisation, then lane 0
+// arrives (release semantics) for the whole warp, so eight arrivals stand for
+// 256 threads.  All 32 lanes must call it.
+__device__ __forceinline__ void warp_arrive_after_tc(uint32_t bar) {
+    tc_fence_before();
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
+
 }  // namespace ajvp

@@ -164,3 +164,25 @@ def test_video_workload_query_side_sampled():
         assert e <= TOL, f"{n}: {e:.3e}"
     del inp, cot, got
     torch.cuda.empty_cache()
+
+
+def test_video_workload_key_side_sampled():
+    # the same configuration's key-side kernels (dK+dtK, dV+dtV): the oracle's gradient
+    # of a key needs every query row of its head, so one head and 8 keys, including
+    # both sides of the first row-tile boundaries and the ragged last tile
+    w = WORKLOADS["video_selfattn_b1h12_l32760_d128"]
+    inp = gpu_inputs(w)
+    cot = make_cotangents(w, device="cuda")
+    got, _ = run(inp, cot, w.scale)
+    h = 5
+    keys = sample_rows(w.Lk, 8, seed=1)
+    fl = {n: t.reshape(-1, t.shape[-2], t.shape[-1])[h].cpu() for n, t in {**inp, **cot}.items()}
+    ref = oracle.attn_jvp_bwd(*(fl[n][None] for n in NAMES), fl["dout"][None], fl["dtout"][None], w.scale,
+                              qrows=[], krows=keys)
+    err = {n: max_rel(got[n].reshape(-1, w.Lk, w.d)[h][keys].float().cpu().numpy(), ref[n][0])
+           for n in ("dk", "dv", "dtk", "dtv")}
+    print(w.name, keys, err)
+    for n, e in err.items():
+        assert e <= TOL, f"{n}: {e:.3e}"
+    del inp, cot, got
+    torch.cuda.empty_cache()
