@@ -39,8 +39,8 @@
 //   tensor-memory columns per tile; Pd = P .* (u - mu); the elementwise
 //   results E1, E2 are bf16, the A operands of G2.)  V_Q and V_K hold one
 //   set of X, Y, Z, W next to their accumulators: the elementwise warps read
-//   all four at once and release them, so that the next tile's [Z|W]
-//   products run while they compute; each group writes its E1, E2 over its
+//   Z and W first and release them, so that the next tile's [Z|W] products
+//   run while they read X, Y and compute; each group writes its E1, E2 over its
 //   own 32 columns of X (16 packed columns each), so the next
 //   tile's [X|Y] products are issued after this tile's G2 (tensor-core
 //   operations run in issue order).  V_V double-buffers its two score tiles
@@ -78,7 +78,7 @@ enum : int {
     B_S_FULL = 5,    // + short stage (up to 4)
     B_S_EMPTY = 9,   // + short stage: the G1 products that read it are complete
     B_G1_DONE = 13,  // + score buffer: X..W of the tile complete
-    B_X_FREE = 15,   // V_Q, V_K: the elementwise warps have read X..W (one arrival per warp)
+    B_X_FREE = 15,   // V_Q, V_K: the elementwise warps have read Z, W (one arrival per warp)
     B_E_DONE = 16,   // + score buffer: E1, E2 of the tile written (one arrival per warp)
     B_G2_DONE = 18,  // + long stage: the tile's G2 products complete (the stage is free again)
     B_ACC_FULL = 22,
@@ -144,7 +144,7 @@ __global__ void __launch_bounds__(256) bwd_rowstats_kernel(const __nv_bfloat16 *
 // Compile-time shape of one variant.
 template <int VAR>
 struct Var {
-    static constexpr bool kSingle = VAR != V_V;     // one set of X..W (E1, E2 written over W)
+    static constexpr bool kSingle = VAR != V_V;     // one set of X..W (E1, E2 written over X)
     static constexpr bool kColStats = VAR != V_Q;   // statistics per streamed query
     static constexpr int kNR = kSingle ? 4 : 2;     // resident tiles R0..R(kNR-1)
     static constexpr int kNB = kSingle ? 1 : 2;     // score buffers
@@ -399,7 +399,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
             };
             bool ok = mbar_wait(BAR(B_R_FULL), 0, abort_flag, bound);
             // one call site per issue routine.  V_Q, V_K: [Z|W] of tile j + 1 once the
-            // elementwise warps have read tile j's X..W, G2 of tile j, then [X|Y] of tile
+            // elementwise warps have read tile j's Z and W, G2 of tile j, then [X|Y] of tile
             // j + 1.  V_V: G1 of tile j + 1, then G2 of tile j.
             for (int j = -1; j < nt && ok; ++j) {
                 if (j + 1 < nt) {
@@ -474,15 +474,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
             const uint32_t tb = tbase + lane_off + C::BUF0 + (uint32_t)b * C::BUF_COLS;
             uint32_t e1[16], e2[16];
             if (C::kSingle) {
-                // all of this group's X..W (4 x 32 columns) at once, so that the buffer
-                // is released for the next tile's G1 before any arithmetic
+                // this group's Z and W first: the next tile's [Z|W] products overwrite only
+                // them and start once they are read; X and Y follow (the next [X|Y] products
+                // come after this tile's G2, which waits for E_DONE)
                 uint32_t xr[32], yr[32], zr[32], wr[32];
-                tmem_ld32(tb + col0 + C::X, xr);
-                tmem_ld32(tb + col0 + C::Y, yr);
                 tmem_ld32(tb + col0 + C::Z, zr);
                 tmem_ld32(tb + col0 + C::W, wr);
                 tmem_wait_ld();
                 warp_arrive_after_tc(BAR(B_X_FREE));
+                tmem_ld32(tb + col0 + C::X, xr);
+                tmem_ld32(tb + col0 + C::Y, yr);
+                tmem_wait_ld();
 #pragma unroll
                 for (int i = 0; i < 32; i += 2) {
                     float2 r1, r2;
