@@ -30,7 +30,8 @@ AJVP_ERR_DEVICE_LAYOUT = -9
 # every symbol the header declares
 EXPORTED = ("attn_jvp_fwd", "attn_jvp_fwd_causal", "attn_jvp_fwd_varlen", "attn_jvp_fwd_f32out", "attn_jvp_fwd_stats", "attn_jvp_bwd", "attn_jvp_bwd_step",
             "attn_jvp_bwd_workspace_bytes", "attn_jvp_fwd_f32", "attn_jvp_fwd_host",
-            "attn_jvp_fwd_host_noalloc", "attn_jvp_host_workspace_bytes", "attn_jvp_strerror",
+            "attn_jvp_fwd_host_noalloc", "attn_jvp_host_workspace_bytes", "attn_jvp_bwd_host",
+            "attn_jvp_bwd_host_workspace_bytes", "attn_jvp_strerror",
             "attn_jvp_last_cuda_error",
             "attn_jvp_check_device_status", "attn_jvp_set_wait_bound_ns", "attn_jvp_set_persistent_key_tiles",
             "attn_jvp_selftest_wait_timeout", "attn_jvp_version")
@@ -75,6 +76,10 @@ def load_library(path: str = LIB_PATH):
         lib.attn_jvp_bwd_step.restype = ctypes.c_int
         lib.attn_jvp_bwd_workspace_bytes.argtypes = [i64] * 3
         lib.attn_jvp_bwd_workspace_bytes.restype = ctypes.c_uint64
+        lib.attn_jvp_bwd_host.argtypes = [vp] * 18 + [i64] * 5 + [f32, vp, ctypes.c_uint64, vp]
+        lib.attn_jvp_bwd_host.restype = ctypes.c_int
+        lib.attn_jvp_bwd_host_workspace_bytes.argtypes = [i64] * 4
+        lib.attn_jvp_bwd_host_workspace_bytes.restype = ctypes.c_uint64
         lib.attn_jvp_fwd_host.argtypes = [vp] * 9 + [i64] * 5 + [f32, vp, ctypes.c_uint64, vp]
         lib.attn_jvp_fwd_host.restype = ctypes.c_int
         lib.attn_jvp_fwd_host_noalloc.argtypes = fwd_args
@@ -298,6 +303,66 @@ def attn_jvp_bwd(q, k, v, tq, tk, tv, o, to, lse, mu, dout, dtout, scale=None, g
         _check(lib.attn_jvp_bwd(*args), "attn_jvp_bwd")
     else:
         _check(lib.attn_jvp_bwd_step(int(step), *args), "attn_jvp_bwd_step")
+    return grads
+
+
+def bwd_host_workspace_bytes(Lq: int, Lk: int, d: int, heads_per_chunk: int = 1) -> int:
+    """Device workspace bytes for ``attn_jvp_bwd_host`` with chunks of
+    ``heads_per_chunk`` (batch, head) slabs."""
+    return int(load_library().attn_jvp_bwd_host_workspace_bytes(Lq, Lk, d, heads_per_chunk))
+
+
+def default_bwd_heads_per_chunk(bh: int, Lq: int, Lk: int, d: int, target_bytes: int = 320 << 20) -> int:
+    """Heads per staged backward chunk: about ``target_bytes`` of staged
+    inputs, gradients and statistics, at least one head, at most a quarter of
+    ``bh`` (so that copies overlap kernels)."""
+    per_head = (8 * Lq + 8 * Lk) * d * 2 + 24 * Lq
+    return max(1, min((bh + 3) // 4, target_bytes // per_head))
+
+
+def attn_jvp_bwd_host(q, k, v, tq, tk, tv, o, to, lse, mu, dout, dtout, scale=None, grads=None, workspace=None,
+                      stream=None):
+    """``attn_jvp_bwd`` on HOST tensors (pinned for overlap): the library
+    stages head chunks through a device workspace and overlaps the copies with
+    the kernels.  Inputs as ``attn_jvp_bwd`` but in host memory; ``grads``: an
+    optional dict of preallocated host outputs.  ``workspace`` is a CUDA uint8
+    tensor (allocated for ``default_bwd_heads_per_chunk`` heads when
+    omitted).  Asynchronous on ``stream``; synchronise it before reading the
+    gradients.  Returns a dict dq, dk, dv, dtq, dtk, dtv."""
+    for name, x in (("q", q), ("k", k), ("v", v), ("tq", tq), ("tk", tk), ("tv", tv)):
+        if not isinstance(x, torch.Tensor) or x.is_cuda or x.dtype != torch.bfloat16 or x.dim() != 4 \
+                or not x.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous bf16 [B, H, L, d] host tensor")
+    B, H, Lq, d = q.shape
+    Lk = k.shape[2]
+    if tq.shape != q.shape or any(x.shape != (B, H, Lk, d) for x in (k, v, tk, tv)):
+        raise ValueError("q, tq must be [B, H, Lq, d] and k, v, tk, tv [B, H, Lk, d]")
+    for name, x, shp, dt in (("o", o, q.shape, torch.bfloat16), ("to", to, q.shape, torch.bfloat16),
+                             ("dout", dout, q.shape, torch.bfloat16), ("dtout", dtout, q.shape, torch.bfloat16),
+                             ("lse", lse, (B, H, Lq), torch.float32), ("mu", mu, (B, H, Lq), torch.float32)):
+        if not isinstance(x, torch.Tensor) or x.is_cuda or x.shape != shp or x.dtype != dt or not x.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous {dt} host tensor of shape {tuple(shp)}")
+    pin = q.is_pinned()
+    grads = dict(grads or {})
+    for name in GRAD_NAMES:
+        like = q if name in ("dq", "dtq") else k
+        if grads.get(name) is None:
+            grads[name] = torch.empty(like.shape, dtype=torch.bfloat16, pin_memory=pin)
+        g = grads[name]
+        if g.is_cuda or g.shape != like.shape or g.dtype != torch.bfloat16 or not g.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous bf16 host tensor of shape {tuple(like.shape)}")
+    if scale is None:
+        scale = d ** -0.5
+    if workspace is None:
+        nh = default_bwd_heads_per_chunk(B * H, Lq, Lk, d)
+        workspace = torch.empty(max(1, bwd_host_workspace_bytes(Lq, Lk, d, nh)), dtype=torch.uint8, device="cuda")
+    if not workspace.is_cuda or workspace.dtype != torch.uint8 or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA uint8 tensor")
+    lib = load_library()
+    rc = lib.attn_jvp_bwd_host(_ptr(q), _ptr(k), _ptr(v), _ptr(tq), _ptr(tk), _ptr(tv), _ptr(o), _ptr(to), _ptr(lse),
+                               _ptr(mu), _ptr(dout), _ptr(dtout), *(_ptr(grads[n]) for n in GRAD_NAMES), B, H, Lq, Lk,
+                               d, float(scale), _ptr(workspace), workspace.numel(), _stream_handle(stream))
+    _check(rc, "attn_jvp_bwd_host")
     return grads
 
 

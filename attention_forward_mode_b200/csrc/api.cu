@@ -316,7 +316,33 @@ StageLayout stage_layout(int64_t Lq, int64_t Lk, int64_t d, int64_t nh) {
     return s;
 }
 
-// Streams and events of one attn_jvp_fwd_host call, released on scope exit
+// The backward's staging buffer for `nh` slabs: its twelve inputs (q, tq, o,
+// to, dout, dtout with Lq rows; k, v, tk, tv with Lk rows; lse, mu), its six
+// gradients (dq, dtq; dk, dv, dtk, dtv) and the row-statistics workspace.
+struct BwdStageLayout {
+    uint64_t in[12], out[6], stats, stats_bytes, bytes;
+};
+
+BwdStageLayout bwd_stage_layout(int64_t Lq, int64_t Lk, int64_t d, int64_t nh) {
+    BwdStageLayout s;
+    const uint64_t qb = round_up((uint64_t)(nh * Lq * d * 2)), kb = round_up((uint64_t)(nh * Lk * d * 2));
+    const uint64_t lb = round_up((uint64_t)(nh * Lq * 4));
+    uint64_t off = 0;
+    for (int t = 0; t < 12; ++t) {
+        s.in[t] = off;
+        off += t < 6 ? qb : (t < 10 ? kb : lb);
+    }
+    for (int t = 0; t < 6; ++t) {
+        s.out[t] = off;
+        off += t < 2 ? qb : kb;
+    }
+    s.stats = off;
+    s.stats_bytes = bwd_stats_bytes(nh, Lq);
+    s.bytes = round_up(off + s.stats_bytes);
+    return s;
+}
+
+// Streams and events of one host-entry call, released on scope exit
 // (the driver defers the release of objects with work still pending).
 // Chunk c uses staging buffer c % kBuffers and compute stream 1 + c % 2, so
 // consecutive chunk kernels may overlap (the next one fills the SMs the
@@ -405,8 +431,8 @@ uint64_t attn_jvp_bwd_workspace_bytes(int64_t B, int64_t H, int64_t Lq) {
 }  // extern "C"
 
 namespace {
-// Kernels first..last of the backward (0 row statistics, 1 dQ, 2 dtQ, 3 dK,
-// 4 dtK and dtV, 5 dV) after the full argument check.
+// Kernels first..last of the backward (0 row statistics, 1 dQ and dtQ, 2 dK
+// and dtK, 3 dV and dtV) after the full argument check.
 int bwd_steps(int first, int last, const void *q, const void *k, const void *v, const void *tq, const void *tk,
               const void *tv, const void *o, const void *to, const float *lse, const float *mu, const void *dout,
               const void *dtout, void *dq, void *dk, void *dv, void *dtq, void *dtk, void *dtv, int64_t B, int64_t H,
@@ -568,6 +594,97 @@ int attn_jvp_fwd_host(const void *q, const void *k, const void *v, const void *t
         if ((e = cudaEventRecord(pipe.out(b), pipe.st[3])) != cudaSuccess) return fail_cuda(e);
     }
     // the caller's stream continues once the last chunk (and so every chunk) is copied out
+    if ((e = cudaStreamWaitEvent(caller, pipe.out((int)((nchunks - 1) % kBuffers)), 0)) != cudaSuccess)
+        return fail_cuda(e);
+    return AJVP_OK;
+}
+
+uint64_t attn_jvp_bwd_host_workspace_bytes(int64_t Lq, int64_t Lk, int64_t d, int64_t heads_per_chunk) {
+    if (Lq < 1 || Lk < 1 || d < 1 || heads_per_chunk < 1) return 0;
+    return kBuffers * bwd_stage_layout(Lq, Lk, d, heads_per_chunk).bytes;
+}
+
+int attn_jvp_bwd_host(const void *q, const void *k, const void *v, const void *tq, const void *tk, const void *tv,
+                      const void *o, const void *to, const float *lse, const float *mu, const void *dout,
+                      const void *dtout, void *dq, void *dk, void *dv, void *dtq, void *dtk, void *dtv, int64_t B,
+                      int64_t H, int64_t Lq, int64_t Lk, int64_t d, float scale, void *workspace,
+                      uint64_t workspace_bytes, void *stream) {
+    bool noop = false;
+    int rc = check_common(q, k, v, tq, tk, tv, o, to, B, H, Lq, Lk, d, scale, &noop);
+    if (rc != AJVP_OK) return rc;
+    const int64_t BH = B * H;
+    if (noop) {
+        // no query rows: the key-side gradients are zero (written once the caller's
+        // stream has reached this call, like the device entry's memsets)
+        if (BH == 0) return AJVP_OK;
+        if (!dk || !dv || !dtk || !dtv) return AJVP_ERR_INVALID_ARG;
+        cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+        if (e != cudaSuccess) return fail_cuda(e);
+        const size_t bytes = (size_t)(BH * Lk * d) * 2u;
+        for (void *g : {dk, dv, dtk, dtv}) std::memset(g, 0, bytes);
+        return AJVP_OK;
+    }
+    if (d != ajvp::bwd::HD) return AJVP_ERR_UNSUPPORTED_DIM;
+    const void *ptrs[18] = {q, k, v, tq, tk, tv, o, to, lse, mu, dout, dtout, dq, dk, dv, dtq, dtk, dtv};
+    for (int i = 0; i < 18; ++i)
+        if (!ptrs[i]) return AJVP_ERR_INVALID_ARG;
+    const uint64_t one = bwd_stage_layout(Lq, Lk, d, 1).bytes;
+    if (!workspace || !aligned(workspace, kStageAlign) || workspace_bytes < kBuffers * one) return AJVP_ERR_WORKSPACE;
+    // heads per chunk: as many as the workspace holds, at most a quarter of B*H
+    int64_t nh = std::min<int64_t>((int64_t)(workspace_bytes / (kBuffers * one)), (BH + 3) / 4);
+    while (nh > 1 && kBuffers * bwd_stage_layout(Lq, Lk, d, nh).bytes > workspace_bytes) --nh;
+    nh = std::max<int64_t>(nh, 1);
+    const BwdStageLayout L = bwd_stage_layout(Lq, Lk, d, nh);
+    int dev = 0;
+    if ((rc = device_setup(&dev)) != AJVP_OK) return rc;
+
+    HostPipe pipe;
+    cudaError_t e = pipe.create();
+    if (e != cudaSuccess) return fail_cuda(e);
+    const cudaStream_t caller = (cudaStream_t)stream;
+    if ((e = cudaEventRecord(pipe.start(), caller)) != cudaSuccess) return fail_cuda(e);
+    for (cudaStream_t s : pipe.st)
+        if ((e = cudaStreamWaitEvent(s, pipe.start(), 0)) != cudaSuccess) return fail_cuda(e);
+
+    // bytes per (b, h) slab of each array, in the layout's order
+    const uint64_t qrow = (uint64_t)(Lq * d * 2), krow = (uint64_t)(Lk * d * 2), srow = (uint64_t)(Lq * 4);
+    const void *src[12] = {q, tq, o, to, dout, dtout, k, v, tk, tv, lse, mu};
+    const uint64_t in_row[12] = {qrow, qrow, qrow, qrow, qrow, qrow, krow, krow, krow, krow, srow, srow};
+    void *dst[6] = {dq, dtq, dk, dv, dtk, dtv};
+    const uint64_t out_row[6] = {qrow, qrow, krow, krow, krow, krow};
+    const int64_t nchunks = (BH + nh - 1) / nh;
+    for (int64_t c = 0; c < nchunks; ++c) {
+        const int b = (int)(c % kBuffers);
+        const int64_t h0 = c * nh, n = std::min<int64_t>(nh, BH - h0);
+        uint8_t *buf = static_cast<uint8_t *>(workspace) + (uint64_t)b * L.bytes;
+        // copy in, once the chunk that last used this buffer has been copied out
+        if (c >= kBuffers && (e = cudaStreamWaitEvent(pipe.st[0], pipe.out(b), 0)) != cudaSuccess)
+            return fail_cuda(e);
+        for (int t = 0; t < 12; ++t) {
+            e = cudaMemcpyAsync(buf + L.in[t], static_cast<const uint8_t *>(src[t]) + (uint64_t)h0 * in_row[t],
+                                (uint64_t)n * in_row[t], cudaMemcpyHostToDevice, pipe.st[0]);
+            if (e != cudaSuccess) return fail_cuda(e);
+        }
+        if ((e = cudaEventRecord(pipe.in(b), pipe.st[0])) != cudaSuccess) return fail_cuda(e);
+        // compute: the four backward kernels on the chunk's n (batch, head) slabs
+        const cudaStream_t cs = pipe.st[1 + (c & 1)];
+        if ((e = cudaStreamWaitEvent(cs, pipe.in(b), 0)) != cudaSuccess) return fail_cuda(e);
+        rc = bwd_steps(0, 3, buf + L.in[0], buf + L.in[6], buf + L.in[7], buf + L.in[1], buf + L.in[8],
+                       buf + L.in[9], buf + L.in[2], buf + L.in[3], reinterpret_cast<const float *>(buf + L.in[10]),
+                       reinterpret_cast<const float *>(buf + L.in[11]), buf + L.in[4], buf + L.in[5],
+                       buf + L.out[0], buf + L.out[2], buf + L.out[3], buf + L.out[1], buf + L.out[4],
+                       buf + L.out[5], 1, n, Lq, Lk, d, scale, buf + L.stats, L.stats_bytes, cs);
+        if (rc != AJVP_OK) return rc;
+        if ((e = cudaEventRecord(pipe.comp(b), cs)) != cudaSuccess) return fail_cuda(e);
+        // copy out (in chunk order on one stream)
+        if ((e = cudaStreamWaitEvent(pipe.st[3], pipe.comp(b), 0)) != cudaSuccess) return fail_cuda(e);
+        for (int t = 0; t < 6; ++t) {
+            e = cudaMemcpyAsync(static_cast<uint8_t *>(dst[t]) + (uint64_t)h0 * out_row[t], buf + L.out[t],
+                                (uint64_t)n * out_row[t], cudaMemcpyDeviceToHost, pipe.st[3]);
+            if (e != cudaSuccess) return fail_cuda(e);
+        }
+        if ((e = cudaEventRecord(pipe.out(b), pipe.st[3])) != cudaSuccess) return fail_cuda(e);
+    }
     if ((e = cudaStreamWaitEvent(caller, pipe.out((int)((nchunks - 1) % kBuffers)), 0)) != cudaSuccess)
         return fail_cuda(e);
     return AJVP_OK;

@@ -597,19 +597,20 @@ def run_ours_bwd(args, w):
         per_kernel.append({"kernel": kname, "ms": kms, "flops": kfl, "tflops": kfl / (kms / 1e3) / 1e12 if fl else None})
     dom = max(per_kernel, key=lambda r: r["ms"])
 
-    # end to end: pinned host inputs -> device -> attn_jvp_bwd -> host gradients, every step
+    # end to end: pinned host inputs -> attn_jvp_bwd_host (head chunks staged through a
+    # device workspace, copies overlapped with the kernels) -> host gradients, every step
     dev_in = {**{n: inp[n] for n in names}, "o": o, "to": to, "lse": lse, "mu": mu, **cot}
     host_in = {n: t.detach().to("cpu").pin_memory() for n, t in dev_in.items()}
     host_g = {n: torch.empty(g.shape, dtype=g.dtype).pin_memory() for n, g in grads.items()}
     h2d = sum(t.numel() * t.element_size() for t in host_in.values())
     d2h = sum(t.numel() * t.element_size() for t in host_g.values())
+    nh = ajvp.default_bwd_heads_per_chunk(w.B * w.H, w.Lq, w.Lk, w.d)
+    host_ws = torch.empty(ajvp.bwd_host_workspace_bytes(w.Lq, w.Lk, w.d, nh), dtype=torch.uint8, device=dev)
 
     def e2e_step():
-        for n in dev_in:
-            dev_in[n].copy_(host_in[n], non_blocking=True)
-        step()
-        for n in grads:
-            host_g[n].copy_(grads[n], non_blocking=True)
+        ajvp.attn_jvp_bwd_host(*(host_in[n] for n in names), host_in["o"], host_in["to"], host_in["lse"],
+                               host_in["mu"], host_in["dout"], host_in["dtout"], w.scale, grads=host_g,
+                               workspace=host_ws, stream=stream)
 
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
     e2e_step()
@@ -645,7 +646,7 @@ def run_ours_bwd(args, w):
                 "kernels": per_kernel,
                 "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                         "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps,
-                        "path": "copy in, attn_jvp_bwd, copy out (serial on one stream)"},
+                        "path": f"attn_jvp_bwd_host (pipelined, chunks of {nh} head(s))"},
                 "gpu_launches": len(BWD_STEPS) * args.steps, "clocks": clocks.summary()}
         if world == 1 and not args.no_cpu_baseline:
             v, n, el, threads = oracle_bwd_sample(w, bwd_head0_cpu(inp, cot), args.cpu_seconds)

@@ -234,6 +234,37 @@ AJVP_API int attn_jvp_bwd_step(int step, const void *q, const void *k, const voi
 AJVP_API uint64_t attn_jvp_bwd_workspace_bytes(int64_t B, int64_t H, int64_t Lq);
 
 /*
+ * attn_jvp_bwd_host -- attn_jvp_bwd on HOST buffers: every tensor argument
+ * (the twelve inputs, lse and mu included, and the six gradients) is host
+ * memory in the layouts of attn_jvp_bwd; pinned memory gives overlapped
+ * transfers, pageable memory works but copies synchronously.  (batch, head)
+ * slabs are processed in chunks through `workspace`, DEVICE memory owned by
+ * the caller, 256-byte aligned, at least
+ * attn_jvp_bwd_host_workspace_bytes(Lq, Lk, d, 1) bytes (a larger one allows
+ * chunks of several heads, at most a quarter of B*H): each chunk is copied in
+ * on one internal stream, its four backward kernels run on one of two
+ * others, and its gradients are copied back on a fourth, so copies overlap
+ * the kernels of neighbouring chunks.  Results are identical to attn_jvp_bwd
+ * on the same data.  Stream-ordered with respect to `stream` (the call
+ * returns once everything is enqueued; the host buffers must stay valid and
+ * unchanged until `stream` reaches that point).  Lq == 0 writes zeros to dk,
+ * dv, dtk, dtv on the host after synchronising `stream`.  Errors as
+ * attn_jvp_bwd; AJVP_ERR_WORKSPACE for a missing, misaligned or too small
+ * workspace.
+ */
+AJVP_API int attn_jvp_bwd_host(const void *q, const void *k, const void *v,
+                      const void *tq, const void *tk, const void *tv,
+                      const void *o, const void *to, const float *lse, const float *mu,
+                      const void *dout, const void *dtout,
+                      void *dq, void *dk, void *dv, void *dtq, void *dtk, void *dtv,
+                      int64_t B, int64_t H, int64_t Lq, int64_t Lk, int64_t d,
+                      float scale, void *workspace, uint64_t workspace_bytes, void *stream);
+
+/* Device workspace, in bytes, for attn_jvp_bwd_host with chunks of
+ * `heads_per_chunk` (batch, head) slabs (0 for invalid sizes). */
+AJVP_API uint64_t attn_jvp_bwd_host_workspace_bytes(int64_t Lq, int64_t Lk, int64_t d, int64_t heads_per_chunk);
+
+/*
  * attn_jvp_fwd_f32 -- fp32 I/O, fp32 arithmetic (CUDA-core kernel), for the
  * accuracy-critical configuration.  Same math, layout and error rules as
  * attn_jvp_fwd, with float tensors.  Supported: 1 <= d <= 256; pointers

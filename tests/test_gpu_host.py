@@ -79,3 +79,68 @@ def test_workspace_too_small_is_rejected():
     with pytest.raises(ajvp.AttnJvpError) as ei:
         ajvp.attn_jvp_fwd_host(*(inp[n] for n in NAMES), w.scale, workspace=ws)
     assert ei.value.status == ajvp.AJVP_ERR_WORKSPACE
+
+
+def _bwd_case(w, seed):
+    from attention_forward_mode_b200.workloads import make_cotangents
+    inp = gpu_inputs(w, seed=seed)
+    cot = make_cotangents(w, seed=seed + 1, device="cuda")
+    o, to, lse, mu = ajvp.attn_jvp_fwd_stats(*(inp[n] for n in NAMES), w.scale)
+    ref = ajvp.attn_jvp_bwd(*(inp[n] for n in NAMES), o, to, lse, mu, cot["dout"], cot["dtout"], w.scale)
+    torch.cuda.synchronize()
+    dev = {**inp, "o": o, "to": to, "lse": lse, "mu": mu, **cot}
+    return dev, {n: g.cpu() for n, g in ref.items()}
+
+
+def _bwd_host(dev, scale, pinned=True, workspace=None):
+    h = {n: (t.cpu().pin_memory() if pinned else t.cpu()) for n, t in dev.items()}
+    got = ajvp.attn_jvp_bwd_host(*(h[n] for n in NAMES), h["o"], h["to"], h["lse"], h["mu"], h["dout"], h["dtout"],
+                                 scale, workspace=workspace)
+    torch.cuda.synchronize()
+    return got
+
+
+@pytest.mark.parametrize("B,H,Lq,Lk,chunk", [(1, 1, 64, 64, None),       # one head, one chunk
+                                             (2, 3, 300, 700, 2),        # 6 heads in chunks of 2
+                                             (1, 7, 129, 257, 2),        # ragged last chunk
+                                             (1, 5, 640, 512, 1),        # one head per chunk
+                                             (2, 2, 200, 64, 4)])        # all heads in one chunk
+def test_bwd_host_equals_device(B, H, Lq, Lk, chunk):
+    """attn_jvp_bwd_host runs the same kernels on each chunk's slabs: the
+    gradients equal attn_jvp_bwd's bit for bit."""
+    w = custom(B, H, Lq, Lk, 128)
+    dev, ref = _bwd_case(w, seed=B * 100 + H * 10 + Lq)
+    ws = None
+    if chunk is not None:
+        ws = torch.empty(ajvp.bwd_host_workspace_bytes(Lq, Lk, 128, chunk), dtype=torch.uint8, device="cuda")
+    got = _bwd_host(dev, w.scale, workspace=ws)
+    for n in ajvp.GRAD_NAMES:
+        assert not got[n].is_cuda
+        assert torch.equal(got[n], ref[n]), n
+
+
+def test_bwd_host_pageable_memory_and_small_workspace_rejected():
+    w = custom(1, 3, 200, 260, 128)
+    dev, ref = _bwd_case(w, seed=21)
+    got = _bwd_host(dev, w.scale, pinned=False)
+    for n in ajvp.GRAD_NAMES:
+        assert torch.equal(got[n], ref[n]), n
+    small = torch.empty(ajvp.bwd_host_workspace_bytes(200, 260, 128, 1) - 256, dtype=torch.uint8, device="cuda")
+    with pytest.raises(ajvp.AttnJvpError):
+        _bwd_host(dev, w.scale, workspace=small)
+
+
+def test_bwd_host_without_query_rows_zeroes_key_gradients():
+    w = custom(1, 2, 0, 96, 128)
+    h = {n: torch.zeros((1, 2, 0 if n in ("q", "tq", "o", "to", "dout", "dtout") else 96, 128), dtype=torch.bfloat16)
+         for n in ("q", "k", "v", "tq", "tk", "tv", "o", "to", "dout", "dtout")}
+    h["lse"] = torch.zeros((1, 2, 0), dtype=torch.float32)
+    h["mu"] = torch.zeros((1, 2, 0), dtype=torch.float32)
+    grads = {n: torch.full((1, 2, 0 if n in ("dq", "dtq") else 96, 128), 7.0, dtype=torch.bfloat16)
+             for n in ajvp.GRAD_NAMES}
+    ws = torch.empty(1 << 20, dtype=torch.uint8, device="cuda")
+    out = ajvp.attn_jvp_bwd_host(*(h[n] for n in NAMES), h["o"], h["to"], h["lse"], h["mu"], h["dout"], h["dtout"],
+                                 w.scale, grads=grads, workspace=ws)
+    torch.cuda.synchronize()
+    for n in ("dk", "dv", "dtk", "dtv"):
+        assert torch.count_nonzero(out[n]) == 0, n
