@@ -424,27 +424,7 @@ def attn_jvp_fwd_host(q, k, v, tq, tk, tv, scale=None, o=None, to=None, lse=None
     tensor (allocated for ``default_heads_per_chunk`` heads when omitted).  The
     call is asynchronous on ``stream``; synchronise it before reading o, to,
     lse."""
-    for name, x in (("q", q), ("k", k), ("v", v), ("tq", tq), ("tk", tk), ("tv", tv)):
-        if not isinstance(x, torch.Tensor) or x.is_cuda or x.dtype != torch.bfloat16 or x.dim() != 4 \
-                or not x.is_contiguous():
-            raise ValueError(f"{name} must be a contiguous bf16 [B, H, L, d] host tensor")
-    B, H, Lq, d = q.shape
-    Lk = k.shape[2]
-    if tq.shape != q.shape or any(x.shape != (B, H, Lk, d) for x in (k, v, tk, tv)):
-        raise ValueError("q, tq must be [B, H, Lq, d] and k, v, tk, tv [B, H, Lk, d]")
-    pin = q.is_pinned()
-    if o is None:
-        o = torch.empty(q.shape, dtype=torch.bfloat16, pin_memory=pin)
-    if to is None:
-        to = torch.empty(q.shape, dtype=torch.bfloat16, pin_memory=pin)
-    if want_lse and lse is None:
-        lse = torch.empty((B, H, Lq), dtype=torch.float32, pin_memory=pin)
-    for name, x in (("o", o), ("to", to)):
-        if x.is_cuda or x.shape != q.shape or x.dtype != torch.bfloat16 or not x.is_contiguous():
-            raise ValueError(f"{name} must be a contiguous bf16 host tensor of shape {tuple(q.shape)}")
-    if lse is not None and (lse.is_cuda or lse.shape != (B, H, Lq) or lse.dtype != torch.float32
-                            or not lse.is_contiguous()):
-        raise ValueError("lse must be a contiguous float32 [B, H, Lq] host tensor")
+    o, to, lse, (B, H, Lq, Lk, d) = _prepare_host(q, k, v, tq, tk, tv, o, to, lse, want_lse)
     if scale is None:
         scale = d ** -0.5
     if workspace is None:
