@@ -47,8 +47,9 @@
 // runs only a handful of key tiles): one CTA per SM walks the units
 // (query tile, batch*head) blockIdx.x, blockIdx.x + gridDim.x, ..., and every
 // ring, buffer and barrier phase follows one CTA-wide tile counter G = n*nk + j
-// (unit n, key tile j).  The epilogue writes O and tO straight from registers,
-// so Q / tQ shared memory is refilled for unit n+1 as soon as the last S/dS'
+// (unit n, key tile j).  The epilogue writes O and tO with plain stores
+// (staged per warp in a 2 KB slot of its own, not in Q / tQ), so Q / tQ
+// shared memory is refilled for unit n+1 as soon as the last S/dS'
 // products of unit n are complete, and the next unit's first score products
 // run while the softmax warps finish the epilogue; the next unit's first
 // P.V waits for the epilogue to have read O / T (B_OT_FREE).

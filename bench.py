@@ -23,6 +23,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -100,10 +101,15 @@ def measured_peaks():
 
 
 def kernel_source_sha(sources=None) -> str:
+    """Hash of the kernel sources' code: comments and whitespace are dropped, so
+    that a comment-only edit does not invalidate a committed ncu capture."""
     h = hashlib.sha256()
     for rel in sources or KERNEL_SOURCES:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, rel)) as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)  # block comments
+        text = re.sub(r"//[^\n]*", " ", text)                 # line comments
+        h.update("".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 
