@@ -84,7 +84,8 @@ enum : int {
     B_ACC_FULL = 22,
     B_MMA_DRAIN = 23,
     B_ST_FULL = 24,   // + slot: V_K's own two-slot ring of column statistics
-    N_BARS = 26
+    B_ZW_DONE = 26,   // V_Q, V_K: the tile's [Z|W] products complete
+    N_BARS = 27
 };
 constexpr uint32_t OFF_TMEM_SLOT = 8 * N_BARS;
 constexpr uint32_t OFF_ABORT = OFF_TMEM_SLOT + 4;
@@ -215,6 +216,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
             mbar_init(BAR(B_E_DONE + b), EW_THREADS / 32);  // one arrival per elementwise warp
         }
         mbar_init(BAR(B_X_FREE), EW_THREADS / 32);
+        mbar_init(BAR(B_ZW_DONE), 1);
         mbar_init(BAR(B_ST_FULL), 1);
         mbar_init(BAR(B_ST_FULL + 1), 1);
         mbar_init(BAR(B_ACC_FULL), 1);
@@ -349,6 +351,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
                 if (C::kSingle) {
                     g1(tb + C::Z, dr2, ds, SC, ID_W, false);
                     g1(tb + C::W, dr3, ds, SC, ID_N, true);
+                    mma_commit(BAR(B_ZW_DONE));
                 } else {
                     g1(tb + C::X, dr0, ds, SC, ID_W, false);
                     g1(tb + C::Y, dr1, ds, SC, ID_N, true);
@@ -358,7 +361,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
                 return true;
             };
             // G1, second part (V_Q, V_K): [X|Y] = R0 [L0; L1]^T, Y += R1 L0^T, over the X
-            // region that the previous tile's G2 read (issued after it)
+            // region that the previous tile's G2 read (issued after it) and the Y region
+            // the elementwise warps read before E_DONE
             auto issue_g1b = [&](int j) -> bool {
                 const uint32_t tb = tbase + C::BUF0;
                 const uint64_t dl = smem_desc_sw128(base + C::long_off(j % C::kLS), 16, 1024);
@@ -398,16 +402,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
                 return true;
             };
             bool ok = mbar_wait(BAR(B_R_FULL), 0, abort_flag, bound);
-            // one call site per issue routine.  V_Q, V_K: [Z|W] of tile j + 1 once the
-            // elementwise warps have read tile j's Z and W, G2 of tile j, then [X|Y] of tile
-            // j + 1.  V_V: G1 of tile j + 1, then G2 of tile j.
+            // one call site per issue routine.  V_Q, V_K: [X|Y] of tile j, [Z|W] of tile
+            // j + 1 once the elementwise warps have read tile j's Z and W (they do so as
+            // soon as tile j's [Z|W] completes, long before its [X|Y]), then G2 of tile j.
+            // V_V: G1 of tile j + 1, then G2 of tile j.
             for (int j = -1; j < nt && ok; ++j) {
+                if (C::kSingle && j >= 0 && !(ok = issue_g1b(j))) break;
                 if (j + 1 < nt) {
                     if (C::kSingle && j >= 0 && !(ok = mbar_wait(BAR(B_X_FREE), j & 1, abort_flag, bound))) break;
                     if (!(ok = issue_g1a(j + 1))) break;
                 }
                 if (j >= 0 && !(ok = issue_g2(j))) break;
-                if (C::kSingle && j + 1 < nt && !(ok = issue_g1b(j + 1))) break;
             }
             if (ok) mma_commit(BAR(B_ACC_FULL));
             mma_commit(BAR(B_MMA_DRAIN));
@@ -460,7 +465,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
 
         for (int j = 0; j < nt; ++j) {
             const int b = j % C::kNB, s = j % C::kLS;
-            if (!failed) failed = !mbar_wait_warp(BAR(B_G1_DONE + b), (j / C::kNB) & 1, abort_flag, bound);
+            // V_Q, V_K: Z and W first (complete well before X and Y)
+            const int g1bar = C::kSingle ? (int)B_ZW_DONE : (int)B_G1_DONE + b;
+            if (!failed) failed = !mbar_wait_warp(BAR(g1bar), (j / C::kNB) & 1, abort_flag, bound);
             // the statistics came with the long-ring stage (bulk copy): observe its barrier too
             if (C::kStatsRing && !failed)
                 failed = !mbar_wait_warp(BAR(B_ST_FULL + (j & 1)), (j >> 1) & 1, abort_flag, bound);
@@ -474,14 +481,20 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
             const uint32_t tb = tbase + lane_off + C::BUF0 + (uint32_t)b * C::BUF_COLS;
             uint32_t e1[16], e2[16];
             if (C::kSingle) {
-                // this group's Z and W first: the next tile's [Z|W] products overwrite only
-                // them and start once they are read; X and Y follow (the next [X|Y] products
+                // this group's Z and W as soon as the tile's [Z|W] products complete: the
+                // next tile's [Z|W] products overwrite only them and start once they are
+                // read; X and Y once the [X|Y] products complete (the next [X|Y] products
                 // come after this tile's G2, which waits for E_DONE)
                 uint32_t xr[32], yr[32], zr[32], wr[32];
                 tmem_ld32(tb + col0 + C::Z, zr);
                 tmem_ld32(tb + col0 + C::W, wr);
                 tmem_wait_ld();
                 warp_arrive_after_tc(BAR(B_X_FREE));
+                if (!mbar_wait_warp(BAR(B_G1_DONE), j & 1, abort_flag, bound)) {
+                    failed = true;
+                    continue;
+                }
+                tc_fence_after();
                 tmem_ld32(tb + col0 + C::X, xr);
                 tmem_ld32(tb + col0 + C::Y, yr);
                 tmem_wait_ld();
