@@ -34,10 +34,13 @@ _BWD_SRC = os.path.join(_HERE, "attn_jvp_bwd_oracle.c")
 _BWD_LIB = os.path.join(_HERE, "liboracle_bwd.so")
 _MSK_SRC = os.path.join(_HERE, "attn_jvp_masked_oracle.c")
 _MSK_LIB = os.path.join(_HERE, "liboracle_masked.so")
+_BMSK_SRC = os.path.join(_HERE, "attn_jvp_bwd_masked_oracle.c")
+_BMSK_LIB = os.path.join(_HERE, "liboracle_bwd_masked.so")
 _lock = threading.Lock()
 _lib = None
 _bwd_lib = None
 _msk_lib = None
+_bmsk_lib = None
 
 
 def _compile(src: str, lib: str, force: bool) -> str:
@@ -57,6 +60,7 @@ def build(force: bool = False) -> str:
     """
     _compile(_BWD_SRC, _BWD_LIB, force)
     _compile(_MSK_SRC, _MSK_LIB, force)
+    _compile(_BMSK_SRC, _BMSK_LIB, force)
     return _compile(_SRC, _LIB, force)
 
 
@@ -83,6 +87,11 @@ def bwd_source_text() -> str:
 
 def masked_source_text() -> str:
     with open(_MSK_SRC) as f:
+        return f.read()
+
+
+def bwd_masked_source_text() -> str:
+    with open(_BMSK_SRC) as f:
         return f.read()
 
 
@@ -150,6 +159,31 @@ def _get_masked():
 def load_masked_variant(path: str):
     """ctypes handle of a separately compiled masked-oracle build."""
     return _bind_masked(path)
+
+
+def _bind_bwd_masked(path: str):
+    lib = ctypes.CDLL(path)
+    dp = ctypes.POINTER(ctypes.c_double)
+    ip = ctypes.POINTER(ctypes.c_int64)
+    lib.oracle_attn_jvp_bwd_masked_f64.argtypes = ([dp] * 14 + [ctypes.c_int64] * 4 + [ctypes.c_double]
+                                                   + [ip, ip, ctypes.c_int64, ctypes.c_int]
+                                                   + [ip, ctypes.c_int64, ip, ctypes.c_int64])
+    lib.oracle_attn_jvp_bwd_masked_f64.restype = ctypes.c_int
+    return lib
+
+
+def _get_bwd_masked():
+    global _bmsk_lib
+    with _lock:
+        if _bmsk_lib is None:
+            build()
+            _bmsk_lib = _bind_bwd_masked(_BMSK_LIB)
+        return _bmsk_lib
+
+
+def load_bwd_masked_variant(path: str):
+    """ctypes handle of a separately compiled masked-backward-oracle build."""
+    return _bind_bwd_masked(path)
 
 
 def load_bwd_variant(path: str):
@@ -295,3 +329,62 @@ def attn_jvp_causal(q, k, v, tq, tk, tv, scale: float, lib=None):
     o, to, lse = attn_jvp_packed(f(q, Lq), f(k, Lk), f(v, Lk), f(tq, Lq), f(tk, Lk), f(tv, Lk), scale,
                                  [0, Lq], [0, Lk], True, lib=lib)
     return o.reshape(q.shape), to.reshape(q.shape), lse.reshape(tuple(lead) + (Lq,))
+
+
+def attn_jvp_bwd_packed(q, k, v, tq, tk, tv, dout, dtout, scale: float, cu_q, cu_k, causal: bool,
+                        qrows=None, krows=None, lib=None):
+    """Gradients of L = <dout, O> + <dtout, tO> for packed (variable-length),
+    optionally causal attention + JVP (O, tO as ``attn_jvp_packed`` defines
+    them), in fp64.
+
+    q, tq, dout, dtout: [H, Tq, d]; k, v, tk, tv: [H, Tk, d]; cu_q, cu_k as
+    for ``attn_jvp_packed``.  ``qrows`` / ``krows``: optional packed query rows
+    / key rows whose gradients are wanted (default: all); key-side sums run
+    over every query row of the key's sequence.  Returns a dict of fp64 numpy
+    arrays: dq, dtq [H, nq, d] and dk, dv, dtk, dtv [H, nk, d].
+    """
+    q, k, v, tq, tk, tv, dout, dtout = (_f64(x) for x in (q, k, v, tq, tk, tv, dout, dtout))
+    H, Tq, d = q.shape
+    Tk = k.shape[1]
+    for x, T in ((tq, Tq), (dout, Tq), (dtout, Tq), (k, Tk), (v, Tk), (tk, Tk), (tv, Tk)):
+        if x.shape != (H, T, d):
+            raise ValueError(f"shape mismatch: {x.shape} vs {(H, T, d)}")
+    cq = np.ascontiguousarray(np.asarray(cu_q, dtype=np.int64))
+    ck = np.ascontiguousarray(np.asarray(cu_k, dtype=np.int64))
+    qr = None if qrows is None else np.ascontiguousarray(np.asarray(qrows, dtype=np.int64))
+    kr = None if krows is None else np.ascontiguousarray(np.asarray(krows, dtype=np.int64))
+    nq = Tq if qr is None else len(qr)
+    nk = Tk if kr is None else len(kr)
+    out = {n: np.zeros((H, nq, d)) for n in ("dq", "dtq")}
+    out.update({n: np.zeros((H, nk, d)) for n in ("dk", "dv", "dtk", "dtv")})
+    dp = ctypes.POINTER(ctypes.c_double)
+    ip = ctypes.POINTER(ctypes.c_int64)
+    ptr = lambda a: a.ctypes.data_as(dp)  # noqa: E731
+    iptr = lambda a: None if a is None else a.ctypes.data_as(ip)  # noqa: E731
+    handle = lib if lib is not None else _get_bwd_masked()
+    rc = handle.oracle_attn_jvp_bwd_masked_f64(ptr(q), ptr(k), ptr(v), ptr(tq), ptr(tk), ptr(tv), ptr(dout),
+                                               ptr(dtout), ptr(out["dq"]), ptr(out["dk"]), ptr(out["dv"]),
+                                               ptr(out["dtq"]), ptr(out["dtk"]), ptr(out["dtv"]), H, Tq, Tk, d,
+                                               float(scale), iptr(cq), iptr(ck), len(cq) - 1, int(bool(causal)),
+                                               iptr(qr), nq, iptr(kr), nk)
+    if rc != 0:
+        raise RuntimeError(f"oracle_attn_jvp_bwd_masked_f64 failed with {rc}")
+    return out
+
+
+def attn_jvp_bwd_causal(q, k, v, tq, tk, tv, dout, dtout, scale: float, qrows=None, krows=None, lib=None):
+    """Causal backward for dense [..., L, d] tensors (one sequence per leading
+    index; bottom-right aligned when Lq != Lk).  ``qrows`` / ``krows`` index
+    rows within one sequence (the same rows for every leading index).
+    Returns dq, dtq [..., nq, d] and dk, dv, dtk, dtv [..., nk, d]."""
+    q, k, v, tq, tk, tv, dout, dtout = (_f64(x) for x in (q, k, v, tq, tk, tv, dout, dtout))
+    lead = q.shape[:-2]
+    Lq, d = q.shape[-2], q.shape[-1]
+    Lk = k.shape[-2]
+    BH = int(np.prod(lead)) if lead else 1
+    f = lambda x, L: x.reshape(BH, L, d)  # noqa: E731
+    g = attn_jvp_bwd_packed(f(q, Lq), f(k, Lk), f(v, Lk), f(tq, Lq), f(tk, Lk), f(tv, Lk), f(dout, Lq),
+                            f(dtout, Lq), scale, [0, Lq], [0, Lk], True, qrows=qrows, krows=krows, lib=lib)
+    nq = Lq if qrows is None else len(qrows)
+    nk = Lk if krows is None else len(krows)
+    return {n: a.reshape(tuple(lead) + ((nq if n in ("dq", "dtq") else nk), d)) for n, a in g.items()}
