@@ -28,7 +28,8 @@ AJVP_ERR_WORKSPACE = -8
 AJVP_ERR_DEVICE_LAYOUT = -9
 
 # every symbol the header declares
-EXPORTED = ("attn_jvp_fwd", "attn_jvp_fwd_causal", "attn_jvp_fwd_varlen", "attn_jvp_fwd_f32out", "attn_jvp_fwd_stats", "attn_jvp_bwd", "attn_jvp_bwd_step",
+EXPORTED = ("attn_jvp_fwd", "attn_jvp_fwd_causal", "attn_jvp_fwd_varlen", "attn_jvp_fwd_f32out", "attn_jvp_fwd_stats", "attn_jvp_fwd_causal_stats", "attn_jvp_bwd", "attn_jvp_bwd_step",
+            "attn_jvp_bwd_causal",
             "attn_jvp_bwd_workspace_bytes", "attn_jvp_fwd_f32", "attn_jvp_fwd_host",
             "attn_jvp_fwd_host_noalloc", "attn_jvp_host_workspace_bytes", "attn_jvp_bwd_host",
             "attn_jvp_bwd_host_workspace_bytes", "attn_jvp_strerror",
@@ -70,8 +71,12 @@ def load_library(path: str = LIB_PATH):
         lib.attn_jvp_fwd_varlen.restype = ctypes.c_int
         lib.attn_jvp_fwd_stats.argtypes = [vp] * 10 + [i64] * 5 + [f32, vp]
         lib.attn_jvp_fwd_stats.restype = ctypes.c_int
+        lib.attn_jvp_fwd_causal_stats.argtypes = [vp] * 10 + [i64] * 5 + [f32, vp]
+        lib.attn_jvp_fwd_causal_stats.restype = ctypes.c_int
         lib.attn_jvp_bwd.argtypes = [vp] * 18 + [i64] * 5 + [f32, vp, ctypes.c_uint64, vp]
         lib.attn_jvp_bwd.restype = ctypes.c_int
+        lib.attn_jvp_bwd_causal.argtypes = [vp] * 18 + [i64] * 5 + [f32, vp, ctypes.c_uint64, vp]
+        lib.attn_jvp_bwd_causal.restype = ctypes.c_int
         lib.attn_jvp_bwd_step.argtypes = [ctypes.c_int] + [vp] * 18 + [i64] * 5 + [f32, vp, ctypes.c_uint64, vp]
         lib.attn_jvp_bwd_step.restype = ctypes.c_int
         lib.attn_jvp_bwd_workspace_bytes.argtypes = [i64] * 3
@@ -245,6 +250,16 @@ def attn_jvp_fwd_varlen(q, k, v, tq, tk, tv, cu_seqlens_q, cu_seqlens_k, max_seq
 def attn_jvp_fwd_stats(q, k, v, tq, tk, tv, scale=None, o=None, to=None, lse=None, mu=None, stream=None):
     """``attn_jvp_fwd`` that also returns mu (fp32 [B, H, Lq]), the row
     statistic the backward needs beside lse.  Returns (o, to, lse, mu)."""
+    return _fwd_stats("attn_jvp_fwd_stats", q, k, v, tq, tk, tv, scale, o, to, lse, mu, stream)
+
+
+def attn_jvp_fwd_causal_stats(q, k, v, tq, tk, tv, scale=None, o=None, to=None, lse=None, mu=None, stream=None):
+    """``attn_jvp_fwd_causal`` that also returns mu (rows that see no key:
+    lse = -inf, mu = 0), for ``attn_jvp_bwd_causal``.  Returns (o, to, lse, mu)."""
+    return _fwd_stats("attn_jvp_fwd_causal_stats", q, k, v, tq, tk, tv, scale, o, to, lse, mu, stream)
+
+
+def _fwd_stats(entry, q, k, v, tq, tk, tv, scale, o, to, lse, mu, stream):
     o, to, lse, (B, H, Lq, Lk, d) = _prepare(q, k, v, tq, tk, tv, o, to, lse, torch.bfloat16, True)
     if mu is None:
         mu = torch.empty((B, H, Lq), device=q.device, dtype=torch.float32)
@@ -253,9 +268,9 @@ def attn_jvp_fwd_stats(q, k, v, tq, tk, tv, scale=None, o=None, to=None, lse=Non
     if scale is None:
         scale = d ** -0.5
     lib = load_library()
-    rc = lib.attn_jvp_fwd_stats(_ptr(q), _ptr(k), _ptr(v), _ptr(tq), _ptr(tk), _ptr(tv), _ptr(o), _ptr(to),
-                                _ptr(lse), _ptr(mu), B, H, Lq, Lk, d, float(scale), _stream_handle(stream))
-    _check(rc, "attn_jvp_fwd_stats")
+    rc = getattr(lib, entry)(_ptr(q), _ptr(k), _ptr(v), _ptr(tq), _ptr(tk), _ptr(tv), _ptr(o), _ptr(to),
+                             _ptr(lse), _ptr(mu), B, H, Lq, Lk, d, float(scale), _stream_handle(stream))
+    _check(rc, entry)
     return o, to, lse, mu
 
 
@@ -275,6 +290,20 @@ def attn_jvp_bwd(q, k, v, tq, tk, tv, o, to, lse, mu, dout, dtout, scale=None, g
     ``grads``: optional dict of preallocated outputs.  Returns a dict
     dq, dk, dv, dtq, dtk, dtv.  Asynchronous on ``stream``.  ``step`` (0-3)
     runs one of the four kernels only (``attn_jvp_bwd_step``)."""
+    return _bwd("attn_jvp_bwd" if step is None else "attn_jvp_bwd_step", q, k, v, tq, tk, tv, o, to, lse, mu,
+                dout, dtout, scale, grads, workspace, stream, step)
+
+
+def attn_jvp_bwd_causal(q, k, v, tq, tk, tv, o, to, lse, mu, dout, dtout, scale=None, grads=None, workspace=None,
+                        stream=None):
+    """Backward of ``attn_jvp_fwd_causal`` through ``attn_jvp_bwd_causal``;
+    o, to, lse, mu from ``attn_jvp_fwd_causal_stats``.  Arguments and result
+    as ``attn_jvp_bwd``."""
+    return _bwd("attn_jvp_bwd_causal", q, k, v, tq, tk, tv, o, to, lse, mu, dout, dtout, scale, grads, workspace,
+                stream, None)
+
+
+def _bwd(entry, q, k, v, tq, tk, tv, o, to, lse, mu, dout, dtout, scale, grads, workspace, stream, step):
     _, _, _, (B, H, Lq, Lk, d) = _prepare(q, k, v, tq, tk, tv, o, to, lse, torch.bfloat16, True)
     for name, x, shp, dt in (("mu", mu, (B, H, Lq), torch.float32), ("dout", dout, q.shape, torch.bfloat16),
                              ("dtout", dtout, q.shape, torch.bfloat16)):
@@ -300,7 +329,7 @@ def attn_jvp_bwd(q, k, v, tq, tk, tv, o, to, lse, mu, dout, dtout, scale=None, g
             _ptr(dout), _ptr(dtout), *(_ptr(grads[n]) for n in GRAD_NAMES), B, H, Lq, Lk, d, float(scale),
             _ptr(workspace), workspace.numel(), _stream_handle(stream))
     if step is None:
-        _check(lib.attn_jvp_bwd(*args), "attn_jvp_bwd")
+        _check(getattr(lib, entry)(*args), entry)
     else:
         _check(lib.attn_jvp_bwd_step(int(step), *args), "attn_jvp_bwd_step")
     return grads

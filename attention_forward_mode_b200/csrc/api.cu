@@ -61,10 +61,10 @@ cudaError_t set_fwd_smem() {
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ajvp::sm100::SMEM_BYTES);
 }
 
-template <int VAR>
+template <int VAR, bool kCausal = false>
 cudaError_t set_bwd_smem() {
-    return cudaFuncSetAttribute(ajvp::bwd::attn_jvp_bwd_kernel<VAR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)ajvp::bwd::Var<VAR>::SMEM_BYTES);
+    return cudaFuncSetAttribute(ajvp::bwd::attn_jvp_bwd_kernel<VAR, kCausal>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ajvp::bwd::Var<VAR>::SMEM_BYTES);
 }
 
 int device_setup(int *dev_out) {
@@ -105,6 +105,9 @@ int device_setup(int *dev_out) {
         if (e3 == cudaSuccess) e3 = set_bwd_smem<ajvp::bwd::V_Q>();
         if (e3 == cudaSuccess) e3 = set_bwd_smem<ajvp::bwd::V_K>();
         if (e3 == cudaSuccess) e3 = set_bwd_smem<ajvp::bwd::V_V>();
+        if (e3 == cudaSuccess) e3 = set_bwd_smem<ajvp::bwd::V_Q, true>();
+        if (e3 == cudaSuccess) e3 = set_bwd_smem<ajvp::bwd::V_K, true>();
+        if (e3 == cudaSuccess) e3 = set_bwd_smem<ajvp::bwd::V_V, true>();
         cudaError_t e4 = cudaFuncSetAttribute(ajvp::f32::attn_jvp_fwd_f32_kernel,
                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
                                               (int)ajvp::f32::smem_bytes(ajvp::f32::DMAX));
@@ -250,8 +253,8 @@ uint64_t bwd_stats_bytes(int64_t BH, int64_t Lq) {
 
 // One backward variant: resident tensors r (row side, Lrow rows), streamed
 // tensors l (the long ring) and sh (the short stage), Lcol rows; outputs
-// out[] (Lrow rows) scaled by sc[].
-template <int VAR>
+// out[] (Lrow rows) scaled by sc[]; kCausal: the bottom-right aligned mask.
+template <int VAR, bool kCausal = false>
 int launch_bwd_var(std::initializer_list<const void *> r, std::initializer_list<const void *> l,
                    std::initializer_list<const void *> sh, std::initializer_list<void *> out,
                    std::initializer_list<float> sc, const void *stats, int64_t BH, int64_t Lrow, int64_t Lcol,
@@ -283,7 +286,7 @@ int launch_bwd_var(std::initializer_list<const void *> r, std::initializer_list<
     p.scale = scale;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.bound_ns = g_bound_ns.load();
-    attn_jvp_bwd_kernel<VAR><<<(unsigned)(n_rtiles * BH), NTHREADS, Var<VAR>::SMEM_BYTES, stream>>>(p);
+    attn_jvp_bwd_kernel<VAR, kCausal><<<(unsigned)(n_rtiles * BH), NTHREADS, Var<VAR>::SMEM_BYTES, stream>>>(p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail_cuda(e);
     return AJVP_OK;
@@ -433,7 +436,7 @@ uint64_t attn_jvp_bwd_workspace_bytes(int64_t B, int64_t H, int64_t Lq) {
 namespace {
 // Kernels first..last of the backward (0 row statistics, 1 dQ and dtQ, 2 dK
 // and dtK, 3 dV and dtV) after the full argument check.
-int bwd_steps(int first, int last, const void *q, const void *k, const void *v, const void *tq, const void *tk,
+int bwd_steps(int first, int last, bool causal, const void *q, const void *k, const void *v, const void *tq, const void *tk,
               const void *tv, const void *o, const void *to, const float *lse, const float *mu, const void *dout,
               const void *dtout, void *dq, void *dk, void *dv, void *dtq, void *dtk, void *dtv, int64_t B, int64_t H,
               int64_t Lq, int64_t Lk, int64_t d, float scale, void *workspace, uint64_t workspace_bytes,
@@ -468,6 +471,8 @@ int bwd_steps(int first, int last, const void *q, const void *k, const void *v, 
     if (((Lq + 127) / 128) * BH >= (int64_t(1) << 31) || ((Lk + 127) / 128) * BH >= (int64_t(1) << 31) ||
         BH * Lq + ajvp::bwd::BN >= (int64_t(1) << 40))
         return AJVP_ERR_TOO_LARGE;
+    // the causal kernels form row + (Lk - Lq) sums in 32 bits
+    if (causal && (Lq >= (int64_t(1) << 30) || Lk >= (int64_t(1) << 30))) return AJVP_ERR_TOO_LARGE;
     if (!workspace || !aligned(workspace, 256) || workspace_bytes < bwd_stats_bytes(BH, Lq))
         return AJVP_ERR_WORKSPACE;
     int dev = 0;
@@ -488,15 +493,18 @@ int bwd_steps(int first, int last, const void *q, const void *k, const void *v, 
     auto want = [&](int k) { return first <= k && last >= k; };
     const float s1 = scale;
     // rows = queries, streamed keys: dq, dtq
-    if (want(1) && (rc = launch_bwd_var<V_Q>({q, tq, dtout, dout}, {k, tk}, {v, tv}, {dq, dtq}, {s1, s1}, workspace,
-                                             BH, Lq, Lk, Lq, d, scale, st)) != AJVP_OK)
+    auto vq = causal ? launch_bwd_var<V_Q, true> : launch_bwd_var<V_Q, false>;
+    if (want(1) && (rc = vq({q, tq, dtout, dout}, {k, tk}, {v, tv}, {dq, dtq}, {s1, s1}, workspace, BH, Lq, Lk, Lq,
+                            d, scale, st)) != AJVP_OK)
         return rc;
     // rows = keys, streamed queries: dk, dtk; dv, dtv
-    if (want(2) && (rc = launch_bwd_var<V_K>({k, tk, v, tv}, {q, tq}, {dtout, dout}, {dk, dtk}, {s1, s1}, workspace,
-                                             BH, Lk, Lq, Lq, d, scale, st)) != AJVP_OK)
+    auto vk = causal ? launch_bwd_var<V_K, true> : launch_bwd_var<V_K, false>;
+    if (want(2) && (rc = vk({k, tk, v, tv}, {q, tq}, {dtout, dout}, {dk, dtk}, {s1, s1}, workspace, BH, Lk, Lq, Lq,
+                            d, scale, st)) != AJVP_OK)
         return rc;
-    if (want(3) && (rc = launch_bwd_var<V_V>({k, tk}, {dout, dtout}, {q, tq}, {dv, dtv}, {1.0f, 1.0f}, workspace, BH,
-                                             Lk, Lq, Lq, d, scale, st)) != AJVP_OK)
+    auto vv = causal ? launch_bwd_var<V_V, true> : launch_bwd_var<V_V, false>;
+    if (want(3) && (rc = vv({k, tk}, {dout, dtout}, {q, tq}, {dv, dtv}, {1.0f, 1.0f}, workspace, BH, Lk, Lq, Lq, d,
+                            scale, st)) != AJVP_OK)
         return rc;
     return AJVP_OK;
 }
@@ -509,8 +517,25 @@ int attn_jvp_bwd(const void *q, const void *k, const void *v, const void *tq, co
                  const void *dtout, void *dq, void *dk, void *dv, void *dtq, void *dtk, void *dtv, int64_t B,
                  int64_t H, int64_t Lq, int64_t Lk, int64_t d, float scale, void *workspace,
                  uint64_t workspace_bytes, void *stream) {
-    return bwd_steps(0, 3, q, k, v, tq, tk, tv, o, to, lse, mu, dout, dtout, dq, dk, dv, dtq, dtk, dtv, B, H, Lq, Lk,
-                     d, scale, workspace, workspace_bytes, stream);
+    return bwd_steps(0, 3, false, q, k, v, tq, tk, tv, o, to, lse, mu, dout, dtout, dq, dk, dv, dtq, dtk, dtv, B, H,
+                     Lq, Lk, d, scale, workspace, workspace_bytes, stream);
+}
+
+int attn_jvp_fwd_causal_stats(const void *q, const void *k, const void *v, const void *tq, const void *tk,
+                              const void *tv, void *o, void *to, float *lse, float *mu, int64_t B, int64_t H,
+                              int64_t Lq, int64_t Lk, int64_t d, float scale, void *stream) {
+    if (B > 0 && H > 0 && Lq > 0 && (!lse || !mu)) return AJVP_ERR_INVALID_ARG;
+    return launch_sm100<false, ajvp::sm100::MASK_CAUSAL>(q, k, v, tq, tk, tv, o, to, lse, B, H, Lq, Lk, d, scale,
+                                                          stream, mu);
+}
+
+int attn_jvp_bwd_causal(const void *q, const void *k, const void *v, const void *tq, const void *tk,
+                        const void *tv, const void *o, const void *to, const float *lse, const float *mu,
+                        const void *dout, const void *dtout, void *dq, void *dk, void *dv, void *dtq, void *dtk,
+                        void *dtv, int64_t B, int64_t H, int64_t Lq, int64_t Lk, int64_t d, float scale,
+                        void *workspace, uint64_t workspace_bytes, void *stream) {
+    return bwd_steps(0, 3, true, q, k, v, tq, tk, tv, o, to, lse, mu, dout, dtout, dq, dk, dv, dtq, dtk, dtv, B, H,
+                     Lq, Lk, d, scale, workspace, workspace_bytes, stream);
 }
 
 int attn_jvp_bwd_step(int step, const void *q, const void *k, const void *v, const void *tq, const void *tk,
@@ -519,8 +544,8 @@ int attn_jvp_bwd_step(int step, const void *q, const void *k, const void *v, con
                       void *dtv, int64_t B, int64_t H, int64_t Lq, int64_t Lk, int64_t d, float scale,
                       void *workspace, uint64_t workspace_bytes, void *stream) {
     if (step < 0 || step > 3) return AJVP_ERR_INVALID_ARG;
-    return bwd_steps(step, step, q, k, v, tq, tk, tv, o, to, lse, mu, dout, dtout, dq, dk, dv, dtq, dtk, dtv, B, H,
-                     Lq, Lk, d, scale, workspace, workspace_bytes, stream);
+    return bwd_steps(step, step, false, q, k, v, tq, tk, tv, o, to, lse, mu, dout, dtout, dq, dk, dv, dtq, dtk, dtv,
+                     B, H, Lq, Lk, d, scale, workspace, workspace_bytes, stream);
 }
 
 uint64_t attn_jvp_host_workspace_bytes(int64_t Lq, int64_t Lk, int64_t d, int64_t heads_per_chunk) {
@@ -669,7 +694,7 @@ int attn_jvp_bwd_host(const void *q, const void *k, const void *v, const void *t
         // compute: the four backward kernels on the chunk's n (batch, head) slabs
         const cudaStream_t cs = pipe.st[1 + (c & 1)];
         if ((e = cudaStreamWaitEvent(cs, pipe.in(b), 0)) != cudaSuccess) return fail_cuda(e);
-        rc = bwd_steps(0, 3, buf + L.in[0], buf + L.in[6], buf + L.in[7], buf + L.in[1], buf + L.in[8],
+        rc = bwd_steps(0, 3, false, buf + L.in[0], buf + L.in[6], buf + L.in[7], buf + L.in[1], buf + L.in[8],
                        buf + L.in[9], buf + L.in[2], buf + L.in[3], reinterpret_cast<const float *>(buf + L.in[10]),
                        reinterpret_cast<const float *>(buf + L.in[11]), buf + L.in[4], buf + L.in[5],
                        buf + L.out[0], buf + L.out[2], buf + L.out[3], buf + L.out[1], buf + L.out[4],

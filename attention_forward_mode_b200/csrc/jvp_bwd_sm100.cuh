@@ -179,7 +179,11 @@ struct Var {
     static_assert(BUF0 + kNB * BUF_COLS == 512u, "tensor-memory layout");
 };
 
-template <int VAR>
+// kCausal: key j is visible to query i iff j <= i + (Lk - Lq) (bottom-right
+// aligned).  A CTA streams only the tiles that some row of its own sees (V_Q:
+// keys 0 .. r0 + 127 + Lk - Lq; V_K, V_V: queries from r0 - (Lk - Lq) on),
+// hidden pairs get P = 0, and a CTA whose rows see nothing writes zeros.
+template <int VAR, bool kCausal = false>
 __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_constant__ Params p) {
     using C = Var<VAR>;
     extern __shared__ __align__(1024) uint8_t bwd_smem[];
@@ -192,10 +196,25 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int rt = blockIdx.x % p.n_rtiles;
+    // causal dQ / dtQ: the late (heavy) query tiles of each head first
+    const int rt = (kCausal && VAR == V_Q) ? p.n_rtiles - 1 - (int)(blockIdx.x % p.n_rtiles)
+                                           : (int)(blockIdx.x % p.n_rtiles);
     const int bh = blockIdx.x / p.n_rtiles;
     const int r0 = rt * BM;
-    const int nt = (p.Lcol + BN - 1) / BN;
+    // streamed tiles jt0 .. jt0 + nt - 1 (local index j = 0 .. nt - 1)
+    int jt0 = 0, nt = (p.Lcol + BN - 1) / BN;
+    // kOff = Lk - Lq: the causal diagonal's offset
+    const int koff = VAR == V_Q ? p.Lcol - p.Lrow : p.Lrow - p.Lcol;
+    if (kCausal) {
+        if (VAR == V_Q) {
+            const int kend = min(p.Lcol, r0 + BM + koff);  // keys some row of the tile sees
+            nt = kend > 0 ? (kend + BN - 1) / BN : 0;
+        } else {
+            const int qbeg = max(0, r0 - koff);  // first query that sees a key of the tile
+            jt0 = qbeg / BN;
+            nt = qbeg < p.Lcol ? nt - jt0 : 0;
+        }
+    }
     const uint64_t bound = p.bound_ns;
 
     const uint32_t bars = base + C::SM_BAR;
@@ -265,7 +284,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
                 tma_load_3d(st + 3 * CHUNK_C, my, fb, 64, y, bh);
             };
             for (int t = 0; t < nt && ok; ++t) {
-                const int y = t * BN;
+                const int y = (jt0 + t) * BN;
                 if (lp) {  // long ring, stage t % kLS: free once the G2 products of tile t - kLS are complete
                     const int s = t % C::kLS;
                     if (t >= C::kLS &&
@@ -433,7 +452,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
         bool failed = false;
         // one pair of columns (c, c + 1 of this group): x scores, y score tangent,
         // z A, w B -> r1, r2 (see the variant table)
-        auto pair = [&](int c, int valid, uint32_t st_base, uint32_t xa, uint32_t xb, uint32_t ya, uint32_t yb,
+        auto pair = [&](int c, int lo, int hi, uint32_t st_base, uint32_t xa, uint32_t xb, uint32_t ya, uint32_t yb,
                         uint32_t za, uint32_t zb, uint32_t wa, uint32_t wb, float2 &r1, float2 &r2) {
             float4 sa = rs, sb = rs;  // statistics of columns c and c + 1
             if (C::kColStats) {
@@ -459,8 +478,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
                 r1 = __fmul2_rn(pp, pb);
                 r2 = dsb;
             }
-            if (c >= valid) r1.x = r2.x = 0.f;  // columns past the end of the tensor
-            if (c + 1 >= valid) r1.y = r2.y = 0.f;
+            // columns past the end of the tensor, or hidden by the causal mask
+            if (c >= hi || c < lo) r1.x = r2.x = 0.f;
+            if (c + 1 >= hi || c + 1 < lo) r1.y = r2.y = 0.f;
         };
 
         for (int j = 0; j < nt; ++j) {
@@ -475,7 +495,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
                 failed = !mbar_wait_warp(BAR(B_L_FULL + s), (j / C::kLS) & 1, abort_flag, bound);
             if (failed) continue;
             tc_fence_after();
-            const int valid = p.Lcol - j * BN - (int)col0;  // this group's columns inside the tensor
+            // this group's columns lo .. hi - 1 are inside the tensor and visible
+            const int y0 = (jt0 + j) * BN + (int)col0;  // the group's first streamed item
+            int lo = 0, hi = p.Lcol - y0;
+            if (kCausal) {
+                if (VAR == V_Q)
+                    hi = min(hi, r0 + row + koff - y0 + 1);  // keys <= query + (Lk - Lq)
+                else
+                    lo = r0 + row - koff - y0;  // queries >= key - (Lk - Lq)
+            }
             const uint32_t st_base =
                 base + C::SM_ST + (uint32_t)(C::kStatsRing ? (j & 1) : s) * STATS_TILE + col0 * 16u;
             const uint32_t tb = tbase + lane_off + C::BUF0 + (uint32_t)b * C::BUF_COLS;
@@ -501,7 +529,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
 #pragma unroll
                 for (int i = 0; i < 32; i += 2) {
                     float2 r1, r2;
-                    pair(i, valid, st_base, xr[i], xr[i + 1], yr[i], yr[i + 1], zr[i], zr[i + 1], wr[i], wr[i + 1], r1,
+                    pair(i, lo, hi, st_base, xr[i], xr[i + 1], yr[i], yr[i + 1], zr[i], zr[i + 1], wr[i], wr[i + 1], r1,
                          r2);
                     e1[i / 2] = pack_bf16x2(r1.x, r1.y);
                     e2[i / 2] = pack_bf16x2(r2.x, r2.y);
@@ -514,7 +542,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
 #pragma unroll
                 for (int i = 0; i < 32; i += 2) {
                     float2 r1, r2;
-                    pair(i, valid, st_base, xr[i], xr[i + 1], yr[i], yr[i + 1], 0u, 0u, 0u, 0u, r1, r2);
+                    pair(i, lo, hi, st_base, xr[i], xr[i + 1], yr[i], yr[i + 1], 0u, 0u, 0u, 0u, r1, r2);
                     e1[i / 2] = pack_bf16x2(r1.x, r1.y);
                     e2[i / 2] = pack_bf16x2(r2.x, r2.y);
                 }
@@ -541,8 +569,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
                 for (int h = 0; h < 2; ++h) {
                     const int pc = 2 * grp + h;
                     uint32_t ra[32];
-                    tmem_ld32(tbase + lane_off + 128u * a + 32u * pc, ra);
-                    tmem_wait_ld();
+                    if (kCausal && nt == 0) {  // no row of the tile sees anything: zeros
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) ra[i] = 0u;
+                    } else {
+                        tmem_ld32(tbase + lane_off + 128u * a + 32u * pc, ra);
+                        tmem_wait_ld();
+                    }
                     uint32_t wa[16];
 #pragma unroll
                     for (int i = 0; i < 16; ++i)

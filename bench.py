@@ -48,6 +48,8 @@ FWD_TRAFFIC_FILES = {"video_selfattn_b1h12_l32760_d128": TRAFFIC_FILE,
                          "profiles/attn_jvp_fwd_kernel_persistent.video_crossattn_b1h40_lq32760_lk512.md"}
 MASKED_METRIC = "attention+JVP TFLOP/s (12·d per visible query-key pair) and % of B200 BF16 tensor peak"
 BWD_METRIC = "attention+JVP backward TFLOP/s (30·Lq·Lk·d/head) and % of B200 BF16 tensor peak"
+BWD_CAUSAL_METRIC = ("attention+JVP causal backward TFLOP/s (30·d per visible query-key pair) and % of B200 "
+                     "BF16 tensor peak")
 BWD_KERNEL_SOURCES = ["attention_forward_mode_b200/csrc/jvp_bwd_sm100.cuh",
                       "attention_forward_mode_b200/csrc/ptx_sm100.cuh"]
 BWD_TRAFFIC_FILE = "profiles/attn_jvp_bwd_kernel.video_selfattn_b1h12_l32760.md"
@@ -502,6 +504,39 @@ def oracle_bwd_sample(w, full_cpu_head, seconds: float, seed: int = 0):
     return 30.0 * n * w.Lk * w.d / el / 1e12, n, el, oracle.num_threads()
 
 
+def bwd_causal_flops(w) -> float:
+    """30 d FLOPs per visible (query, key) pair of the causal mask, summed
+    over the heads (the backward's count of ``bwd_flops`` over visible pairs)."""
+    return causal_flops(w) * 30.0 / 12.0
+
+
+def oracle_bwd_sample_causal(w, full_cpu_head, seconds: float):
+    """Time the fp64 masked backward oracle on the causal sub-problem made of
+    the first n query rows and the first n + Lk - Lq keys of one head (a
+    complete n-row causal backward), n sized to about ``seconds``; FLOPs
+    30 d per visible pair of that sub-problem."""
+    import oracle
+    x = full_cpu_head
+    off = w.Lk - w.Lq
+
+    def run(n):
+        nk = max(1, min(w.Lk, n + off))
+        t0 = time.perf_counter()
+        oracle.attn_jvp_bwd_causal(x["q"][None, :n], x["k"][None, :nk], x["v"][None, :nk], x["tq"][None, :n],
+                                   x["tk"][None, :nk], x["tv"][None, :nk], x["dout"][None, :n],
+                                   x["dtout"][None, :n], w.scale)
+        return time.perf_counter() - t0, nk
+
+    n = 64
+    el, nk = run(n)
+    while el < seconds / 4 and n < w.Lq:  # the cost grows like n^2: double until a quarter of the budget
+        n = min(w.Lq, 2 * n)
+        el, nk = run(n)
+    i = torch.arange(n, dtype=torch.float64)
+    vis = torch.clamp(i + (nk - n) + 1, 0, nk).sum().item()
+    return 30.0 * w.d * vis / el / 1e12, n, el, oracle.num_threads()
+
+
 def bwd_head0_cpu(inp, cot):
     return {n: t[0, 0].detach().cpu() for n, t in {**inp, **cot}.items()}
 
@@ -513,22 +548,26 @@ def run_reference_bwd(args, w):
     import oracle
     from attention_forward_mode_b200.workloads import make_cotangents
     oracle.build()
+    causal = args.entry == "bwd_causal"
     head = bwd_head0_cpu(make_inputs(w, seed=0, device="cpu"), make_cotangents(w, device="cpu"))
     per_step = max(0.5, args.reference_seconds / max(1, args.steps + args.warmup))
+    sample_fn = oracle_bwd_sample_causal if causal else oracle_bwd_sample
     for _ in range(args.warmup):
-        oracle_bwd_sample(w, head, per_step)
-    rows_total, el_total, threads = 0, 0.0, oracle.num_threads()
+        sample_fn(w, head, per_step)
+    flops_total, el_total, rows_total, threads = 0.0, 0.0, 0, oracle.num_threads()
     for _ in range(args.steps):
-        _, n, el, threads = oracle_bwd_sample(w, head, per_step)
+        v, n, el, threads = sample_fn(w, head, per_step)
+        flops_total += v * 1e12 * el
         rows_total += n
         el_total += el
-    value = 30.0 * rows_total * w.Lk * w.d / el_total / 1e12
-    sample = (f"backward of the first query rows of head 0 with all {w.Lk} keys, {rows_total} rows over "
-              f"{args.steps} steps, {el_total:.1f} s of fp64 oracle time")
-    line = {"impl": "reference", "metric": BWD_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+    value = flops_total / el_total / 1e12
+    what = (f"causal backward sub-problems of the first query rows and keys of head 0" if causal else
+            f"backward of the first query rows of head 0 with all {w.Lk} keys")
+    sample = f"{what}, {rows_total} rows over {args.steps} steps, {el_total:.1f} s of fp64 oracle time"
+    line = {"impl": "reference", "metric": BWD_CAUSAL_METRIC if causal else BWD_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * el_total / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": dict(workload_config(w, world), entry="attn_jvp_bwd"),
+            "config": dict(workload_config(w, world), entry="attn_jvp_bwd_causal" if causal else "attn_jvp_bwd"),
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -545,10 +584,12 @@ def run_ours_bwd(args, w):
     from attention_forward_mode_b200.workloads import make_cotangents
     ajvp.load_library()
     names = ("q", "k", "v", "tq", "tk", "tv")
+    causal = args.entry == "bwd_causal"
     inp = make_inputs(w, seed=rank, device=dev)
     cot = make_cotangents(w, seed=1000 + rank, device=dev)
     stream = torch.cuda.current_stream(dev)
-    o, to, lse, mu = ajvp.attn_jvp_fwd_stats(*(inp[n] for n in names), w.scale, stream=stream)
+    fwd = ajvp.attn_jvp_fwd_causal_stats if causal else ajvp.attn_jvp_fwd_stats
+    o, to, lse, mu = fwd(*(inp[n] for n in names), w.scale, stream=stream)
     grads = {n: torch.empty_like(inp["q"] if n in ("dq", "dtq") else inp["k"]) for n in ajvp.GRAD_NAMES}
     ws = torch.empty(ajvp.bwd_workspace_bytes(w.B, w.H, w.Lq), dtype=torch.uint8, device=dev)
     in_bytes = sum(t.numel() * t.element_size() for t in list(inp.values()) + list(cot.values()) + [o, to])
@@ -557,8 +598,12 @@ def run_ours_bwd(args, w):
     def step(which=None):
         if flush is not None:
             flush.zero_()
-        ajvp.attn_jvp_bwd(*(inp[n] for n in names), o, to, lse, mu, cot["dout"], cot["dtout"], w.scale,
-                          grads=grads, workspace=ws, stream=stream, step=which)
+        if causal:
+            ajvp.attn_jvp_bwd_causal(*(inp[n] for n in names), o, to, lse, mu, cot["dout"], cot["dtout"], w.scale,
+                                     grads=grads, workspace=ws, stream=stream)
+        else:
+            ajvp.attn_jvp_bwd(*(inp[n] for n in names), o, to, lse, mu, cot["dout"], cot["dtout"], w.scale,
+                              grads=grads, workspace=ws, stream=stream, step=which)
 
     for _ in range(args.warmup):
         step()
@@ -583,8 +628,10 @@ def run_ours_bwd(args, w):
     ms_max = max_over_ranks(ms, world, dev)
     if ajvp.check_device_status(stream) != ajvp.AJVP_OK:
         raise RuntimeError("kernel wait bound exceeded")
-    flops = bwd_flops(w)
+    flops = bwd_causal_flops(w) if causal else bwd_flops(w)
     value = aggregate_value(flops, args.steps, world, ms_max / 1e3)
+    if causal:
+        return finish_bwd_causal(args, w, rank, world, value, flops, ms_max, clocks, inp, cot)
 
     # each of the four kernels alone, K launches each, events on the stream
     per_kernel = []
@@ -663,6 +710,37 @@ def run_ours_bwd(args, w):
     return 0
 
 
+def finish_bwd_causal(args, w, rank, world, value, flops, ms_max, clocks, inp, cot):
+    """JSON line of ``--entry bwd_causal``: the causal backward timed as one
+    step (four kernels; there is no per-kernel or host-buffer entry for it),
+    FLOPs counted over the visible pairs."""
+    if rank == 0:
+        burst, _, src = measured_peaks()
+        achieved = flops / (ms_max / args.steps / 1e3) / 1e12
+        line = {"metric": BWD_CAUSAL_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic",
+                "config": dict(workload_config(w, world), entry="attn_jvp_bwd_causal",
+                               flops_per_step="30·d per visible (query, key) pair"),
+                "pct_of_bf16_peak": 100.0 * value / world / burst,
+                "roofline": {"bound": "tensor", "achieved": achieved, "peak": burst, "unit": "TFLOP/s",
+                             "frac": achieved / burst, "traffic": None,
+                             "peak_source": f"{src} bf16 dense (burst) from MEASURED_PEAKS.json"
+                             if src == "measured" else "fallback 1.59 PFLOP/s",
+                             "kernel": "attn_jvp_bwd_causal (row statistics and three gradient kernels, one step)",
+                             "algorithmic_flops_per_launch": flops},
+                "e2e": None,
+                "gpu_launches": 4 * args.steps, "clocks": clocks.summary()}
+        if world == 1 and not args.no_cpu_baseline:
+            v, n, el, threads = oracle_bwd_sample_causal(w, bwd_head0_cpu(inp, cot), args.cpu_seconds)
+            line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                                    "sample": f"causal backward of the first {n} query rows and keys of head 0 "
+                                              f"({el:.1f} s, fp64, OpenMP)"}
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def eager_reference(w, inp, chunk: int = 8192):
     """torch.func.jvp of softmax(s q k^T) v in the I/O dtype on the GPU,
     looped over heads and 8192-row query chunks (what fits in memory);
@@ -706,10 +784,10 @@ def main(argv=None):
     ap.add_argument("--reference-seconds", type=float, default=90.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-eager", action="store_true")
-    ap.add_argument("--entry", choices=["bf16", "f32out", "causal", "varlen", "bwd"], default="bf16",
+    ap.add_argument("--entry", choices=["bf16", "f32out", "causal", "varlen", "bwd", "bwd_causal"], default="bf16",
                     help="f32out: time attn_jvp_fwd_f32out (fp32 outputs, split-bf16 probabilities); "
                          "causal: attn_jvp_fwd_causal; varlen: attn_jvp_fwd_varlen on 8 packed sequences; "
-                         "bwd: time the backward pass attn_jvp_bwd")
+                         "bwd: time the backward pass attn_jvp_bwd; bwd_causal: attn_jvp_bwd_causal")
     ap.add_argument("--heads", type=int, default=None,
                     help="override H (small profiling captures); the JSON config shows the H used")
     args = ap.parse_args(argv)
@@ -720,7 +798,7 @@ def main(argv=None):
         w = dataclasses.replace(w, H=args.heads, name=f"{w.name}_h{args.heads}")
     if w.dtype != "bf16" and args.impl == "ours":
         ap.error("the benchmark times the bf16 tensor-core path")
-    if args.entry == "bwd":
+    if args.entry in ("bwd", "bwd_causal"):
         return run_reference_bwd(args, w) if args.impl == "reference" else run_ours_bwd(args, w)
     if args.impl == "reference":
         return run_reference(args, w)

@@ -19,7 +19,8 @@
  * never written to memory.  No dropout; Lq may differ from Lk
  * (cross-attention); attn_jvp_fwd_causal and attn_jvp_fwd_varlen add a
  * causal mask and packed variable-length sequences, attn_jvp_bwd the
- * backward pass.  s is a constant (no derivative with respect to it).
+ * backward pass (attn_jvp_bwd_causal that of the causal forward).  s is a
+ * constant (no derivative with respect to it).
  *
  * Layout: every tensor is a contiguous row-major [B][H][L][d] array (the
  * layout of a PyTorch [B, H, L, d] tensor); the tangents tQ, tK, tV share the
@@ -229,6 +230,40 @@ AJVP_API int attn_jvp_bwd_step(int step, const void *q, const void *k, const voi
                       void *dq, void *dk, void *dv, void *dtq, void *dtk, void *dtv,
                       int64_t B, int64_t H, int64_t Lq, int64_t Lk, int64_t d,
                       float scale, void *workspace, uint64_t workspace_bytes, void *stream);
+
+/*
+ * attn_jvp_fwd_causal_stats -- attn_jvp_fwd_causal that also saves mu (as
+ * attn_jvp_fwd_stats does for the unmasked forward): the statistics
+ * attn_jvp_bwd_causal needs.  Rows that see no key get lse = -infinity and
+ * mu = 0.  lse and mu are required; other arguments and rules as
+ * attn_jvp_fwd_causal.
+ */
+AJVP_API int attn_jvp_fwd_causal_stats(const void *q, const void *k, const void *v,
+                       const void *tq, const void *tk, const void *tv,
+                       void *o, void *to, float *lse, float *mu,
+                       int64_t B, int64_t H, int64_t Lq, int64_t Lk, int64_t d,
+                       float scale, void *stream);
+
+/*
+ * attn_jvp_bwd_causal -- backward pass of attn_jvp_fwd_causal: the gradients
+ * of L = sum <dout, O> + sum <dtout, tO> where O, tO are the causal forward's
+ * outputs (key j visible to query row i iff j <= i + (Lk - Lq)).  The pages
+ * describe neither masks nor the backward; this is the gradient of the
+ * masked forward definition, with every sum over keys taken over the keys a
+ * row sees.  o, to, lse, mu come from attn_jvp_fwd_causal_stats.  Each
+ * gradient kernel streams only the tiles some row of its own tile sees
+ * (about half the work of attn_jvp_bwd when Lq == Lk); gradients of rows
+ * that see no key, and of keys no row sees, are zero.  Arguments, layouts,
+ * workspace, checks and errors as attn_jvp_bwd, plus AJVP_ERR_TOO_LARGE for
+ * Lq or Lk >= 2^30.
+ */
+AJVP_API int attn_jvp_bwd_causal(const void *q, const void *k, const void *v,
+                 const void *tq, const void *tk, const void *tv,
+                 const void *o, const void *to, const float *lse, const float *mu,
+                 const void *dout, const void *dtout,
+                 void *dq, void *dk, void *dv, void *dtq, void *dtk, void *dtv,
+                 int64_t B, int64_t H, int64_t Lq, int64_t Lk, int64_t d,
+                 float scale, void *workspace, uint64_t workspace_bytes, void *stream);
 
 /* Device workspace, in bytes, that attn_jvp_bwd needs (0 for invalid sizes). */
 AJVP_API uint64_t attn_jvp_bwd_workspace_bytes(int64_t B, int64_t H, int64_t Lq);
