@@ -29,7 +29,7 @@ AJVP_ERR_DEVICE_LAYOUT = -9
 
 # every symbol the header declares
 EXPORTED = ("attn_jvp_fwd", "attn_jvp_fwd_causal", "attn_jvp_fwd_varlen", "attn_jvp_fwd_f32out", "attn_jvp_fwd_stats", "attn_jvp_fwd_causal_stats", "attn_jvp_bwd", "attn_jvp_bwd_step",
-            "attn_jvp_bwd_causal",
+            "attn_jvp_bwd_causal", "attn_jvp_fwd_varlen_stats", "attn_jvp_bwd_varlen",
             "attn_jvp_bwd_workspace_bytes", "attn_jvp_fwd_f32", "attn_jvp_fwd_host",
             "attn_jvp_fwd_host_noalloc", "attn_jvp_host_workspace_bytes", "attn_jvp_bwd_host",
             "attn_jvp_bwd_host_workspace_bytes", "attn_jvp_strerror",
@@ -77,6 +77,10 @@ def load_library(path: str = LIB_PATH):
         lib.attn_jvp_bwd.restype = ctypes.c_int
         lib.attn_jvp_bwd_causal.argtypes = [vp] * 18 + [i64] * 5 + [f32, vp, ctypes.c_uint64, vp]
         lib.attn_jvp_bwd_causal.restype = ctypes.c_int
+        lib.attn_jvp_fwd_varlen_stats.argtypes = [vp] * 12 + [i64] * 6 + [f32, ctypes.c_int, vp]
+        lib.attn_jvp_fwd_varlen_stats.restype = ctypes.c_int
+        lib.attn_jvp_bwd_varlen.argtypes = ([vp] * 20 + [i64] * 7 + [f32, ctypes.c_int, vp, ctypes.c_uint64, vp])
+        lib.attn_jvp_bwd_varlen.restype = ctypes.c_int
         lib.attn_jvp_bwd_step.argtypes = [ctypes.c_int] + [vp] * 18 + [i64] * 5 + [f32, vp, ctypes.c_uint64, vp]
         lib.attn_jvp_bwd_step.restype = ctypes.c_int
         lib.attn_jvp_bwd_workspace_bytes.argtypes = [i64] * 3
@@ -212,6 +216,77 @@ def attn_jvp_fwd_varlen(q, k, v, tq, tk, tv, cu_seqlens_q, cu_seqlens_k, max_seq
     [H, total_k, d] bf16 CUDA tensors; cu_seqlens_q / _k int32 CUDA tensors of
     n_seq + 1 offsets.  Returns (o, to, lse) with o, to [H, total_q, d] and
     lse [H, total_q]."""
+    o, to, lse, (H, Tq, Tk, d) = _prepare_varlen(q, k, v, tq, tk, tv, cu_seqlens_q, cu_seqlens_k, o, to, lse,
+                                                 want_lse)
+    if scale is None:
+        scale = d ** -0.5
+    lib = load_library()
+    rc = lib.attn_jvp_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(tq), _ptr(tk), _ptr(tv), _ptr(o), _ptr(to),
+                                 _ptr(lse), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), cu_seqlens_q.numel() - 1, H, Tq,
+                                 Tk, int(max_seqlen_q), d, float(scale), int(bool(causal)), _stream_handle(stream))
+    _check(rc, "attn_jvp_fwd_varlen")
+    return o, to, lse
+
+
+def attn_jvp_fwd_varlen_stats(q, k, v, tq, tk, tv, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, scale=None,
+                              causal=False, o=None, to=None, lse=None, mu=None, stream=None):
+    """``attn_jvp_fwd_varlen`` that also returns mu (fp32 [H, total_q]; rows
+    that see no key: lse = -inf, mu = 0), for ``attn_jvp_bwd_varlen``.
+    Returns (o, to, lse, mu)."""
+    o, to, lse, (H, Tq, Tk, d) = _prepare_varlen(q, k, v, tq, tk, tv, cu_seqlens_q, cu_seqlens_k, o, to, lse, True)
+    if mu is None:
+        mu = torch.empty((H, Tq), device=q.device, dtype=torch.float32)
+    if mu.shape != (H, Tq) or mu.dtype != torch.float32 or not mu.is_contiguous() or not mu.is_cuda:
+        raise ValueError("mu must be a contiguous float32 CUDA [H, total_q] tensor")
+    if scale is None:
+        scale = d ** -0.5
+    lib = load_library()
+    rc = lib.attn_jvp_fwd_varlen_stats(_ptr(q), _ptr(k), _ptr(v), _ptr(tq), _ptr(tk), _ptr(tv), _ptr(o), _ptr(to),
+                                       _ptr(lse), _ptr(mu), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k),
+                                       cu_seqlens_q.numel() - 1, H, Tq, Tk, int(max_seqlen_q), d, float(scale),
+                                       int(bool(causal)), _stream_handle(stream))
+    _check(rc, "attn_jvp_fwd_varlen_stats")
+    return o, to, lse, mu
+
+
+def attn_jvp_bwd_varlen(q, k, v, tq, tk, tv, o, to, lse, mu, dout, dtout, cu_seqlens_q, cu_seqlens_k,
+                        max_seqlen_q, max_seqlen_k, scale=None, causal=False, grads=None, workspace=None,
+                        stream=None):
+    """Backward of ``attn_jvp_fwd_varlen`` through ``attn_jvp_bwd_varlen``: the
+    packed tensors and offsets of the forward, o, to, lse, mu from
+    ``attn_jvp_fwd_varlen_stats``, cotangents dout, dtout [H, total_q, d].
+    Returns a dict dq, dk, dv, dtq, dtk, dtv (packed like q / k)."""
+    _, _, _, (H, Tq, Tk, d) = _prepare_varlen(q, k, v, tq, tk, tv, cu_seqlens_q, cu_seqlens_k, o, to, lse, True)
+    for name, x, shp, dt in (("mu", mu, (H, Tq), torch.float32), ("dout", dout, q.shape, torch.bfloat16),
+                             ("dtout", dtout, q.shape, torch.bfloat16)):
+        if not isinstance(x, torch.Tensor) or x.shape != shp or x.dtype != dt or not x.is_contiguous() \
+                or not x.is_cuda:
+            raise ValueError(f"{name} must be a contiguous CUDA {dt} tensor of shape {tuple(shp)}")
+    grads = dict(grads or {})
+    for name in GRAD_NAMES:
+        like = q if name in ("dq", "dtq") else k
+        if grads.get(name) is None:
+            grads[name] = torch.empty_like(like)
+        g = grads[name]
+        if g.shape != like.shape or g.dtype != torch.bfloat16 or not g.is_contiguous() or not g.is_cuda:
+            raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor of shape {tuple(like.shape)}")
+    if scale is None:
+        scale = d ** -0.5
+    if workspace is None:
+        workspace = torch.empty(max(1, bwd_workspace_bytes(1, H, Tq)), dtype=torch.uint8, device=q.device)
+    if not workspace.is_cuda or workspace.dtype != torch.uint8 or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA uint8 tensor")
+    lib = load_library()
+    rc = lib.attn_jvp_bwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(tq), _ptr(tk), _ptr(tv), _ptr(o), _ptr(to),
+                                 _ptr(lse), _ptr(mu), _ptr(dout), _ptr(dtout), *(_ptr(grads[n]) for n in GRAD_NAMES),
+                                 _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), cu_seqlens_q.numel() - 1, H, Tq, Tk,
+                                 int(max_seqlen_q), int(max_seqlen_k), d, float(scale), int(bool(causal)),
+                                 _ptr(workspace), workspace.numel(), _stream_handle(stream))
+    _check(rc, "attn_jvp_bwd_varlen")
+    return grads
+
+
+def _prepare_varlen(q, k, v, tq, tk, tv, cu_seqlens_q, cu_seqlens_k, o, to, lse, want_lse):
     for name, x in (("q", q), ("k", k), ("v", v), ("tq", tq), ("tk", tk), ("tv", tv)):
         if not isinstance(x, torch.Tensor) or not x.is_cuda or x.dtype != torch.bfloat16 or x.dim() != 3 \
                 or not x.is_contiguous():
@@ -237,14 +312,7 @@ def attn_jvp_fwd_varlen(q, k, v, tq, tk, tv, cu_seqlens_q, cu_seqlens_k, max_seq
             raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor of shape {tuple(q.shape)}")
     if lse is not None and (lse.shape != (H, Tq) or lse.dtype != torch.float32 or not lse.is_contiguous()):
         raise ValueError("lse must be a contiguous float32 [H, total_q] tensor")
-    if scale is None:
-        scale = d ** -0.5
-    lib = load_library()
-    rc = lib.attn_jvp_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(tq), _ptr(tk), _ptr(tv), _ptr(o), _ptr(to),
-                                 _ptr(lse), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), cu_seqlens_q.numel() - 1, H, Tq,
-                                 Tk, int(max_seqlen_q), d, float(scale), int(bool(causal)), _stream_handle(stream))
-    _check(rc, "attn_jvp_fwd_varlen")
-    return o, to, lse
+    return o, to, lse, (H, Tq, Tk, d)
 
 
 def attn_jvp_fwd_stats(q, k, v, tq, tk, tv, scale=None, o=None, to=None, lse=None, mu=None, stream=None):

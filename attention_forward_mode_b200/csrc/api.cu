@@ -61,10 +61,20 @@ cudaError_t set_fwd_smem() {
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ajvp::sm100::SMEM_BYTES);
 }
 
-template <int VAR, bool kCausal = false>
-cudaError_t set_bwd_smem() {
-    return cudaFuncSetAttribute(ajvp::bwd::attn_jvp_bwd_kernel<VAR, kCausal>,
+template <int VAR, int MASK>
+cudaError_t set_bwd_smem_one() {
+    return cudaFuncSetAttribute(ajvp::bwd::attn_jvp_bwd_kernel<VAR, MASK>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ajvp::bwd::Var<VAR>::SMEM_BYTES);
+}
+
+// every mask instantiation (none, causal, packed, both) of one variant
+template <int VAR>
+cudaError_t set_bwd_smem() {
+    cudaError_t e = set_bwd_smem_one<VAR, 0>();
+    if (e == cudaSuccess) e = set_bwd_smem_one<VAR, 1>();
+    if (e == cudaSuccess) e = set_bwd_smem_one<VAR, 2>();
+    if (e == cudaSuccess) e = set_bwd_smem_one<VAR, 3>();
+    return e;
 }
 
 int device_setup(int *dev_out) {
@@ -105,9 +115,6 @@ int device_setup(int *dev_out) {
         if (e3 == cudaSuccess) e3 = set_bwd_smem<ajvp::bwd::V_Q>();
         if (e3 == cudaSuccess) e3 = set_bwd_smem<ajvp::bwd::V_K>();
         if (e3 == cudaSuccess) e3 = set_bwd_smem<ajvp::bwd::V_V>();
-        if (e3 == cudaSuccess) e3 = set_bwd_smem<ajvp::bwd::V_Q, true>();
-        if (e3 == cudaSuccess) e3 = set_bwd_smem<ajvp::bwd::V_K, true>();
-        if (e3 == cudaSuccess) e3 = set_bwd_smem<ajvp::bwd::V_V, true>();
         cudaError_t e4 = cudaFuncSetAttribute(ajvp::f32::attn_jvp_fwd_f32_kernel,
                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
                                               (int)ajvp::f32::smem_bytes(ajvp::f32::DMAX));
@@ -251,15 +258,29 @@ uint64_t bwd_stats_bytes(int64_t BH, int64_t Lq) {
     return ((uint64_t)(BH * Lq + ajvp::bwd::BN) * 16u + 255u) / 256u * 256u;
 }
 
+// Packed sequences of a backward call (MASK_PACKED): device offsets of the
+// query and key rows of each sequence, and the longest sequences (grid size).
+struct BwdPack {
+    const int *cu_q = nullptr, *cu_k = nullptr;
+    int64_t n_seq = 0, max_q = 0, max_k = 0;
+};
+
 // One backward variant: resident tensors r (row side, Lrow rows), streamed
 // tensors l (the long ring) and sh (the short stage), Lcol rows; outputs
-// out[] (Lrow rows) scaled by sc[]; kCausal: the bottom-right aligned mask.
-template <int VAR, bool kCausal = false>
+// out[] (Lrow rows) scaled by sc[]; MASK: causal and/or packed (cu_row /
+// cu_col the row-side / streamed offsets, max_row the longest row-side run).
+template <int VAR, int MASK>
 int launch_bwd_var(std::initializer_list<const void *> r, std::initializer_list<const void *> l,
                    std::initializer_list<const void *> sh, std::initializer_list<void *> out,
                    std::initializer_list<float> sc, const void *stats, int64_t BH, int64_t Lrow, int64_t Lcol,
-                   int64_t Lq, int64_t d, float scale, cudaStream_t stream) {
+                   int64_t Lq, int64_t d, float scale, cudaStream_t stream, const int *cu_row, const int *cu_col,
+                   int64_t n_seq, int64_t max_row) {
     using namespace ajvp::bwd;
+    constexpr bool kPacked = (MASK & MASK_PACKED) != 0;
+    const int64_t n_rtiles = ((kPacked ? max_row : Lrow) + BM - 1) / BM;
+    const int64_t n_cta = n_rtiles * BH * (kPacked ? n_seq : 1);
+    if (n_cta >= (int64_t(1) << 31)) return AJVP_ERR_TOO_LARGE;
+    if (n_cta == 0) return AJVP_OK;
     int rc;
     Params p;
     std::memset(&p, 0, sizeof(p));
@@ -276,8 +297,13 @@ int launch_bwd_var(std::initializer_list<const void *> r, std::initializer_list<
     for (void *x : out)
         if ((rc = encode_3d(&p.tm_out[i++], x, d, Lrow, BH, 128)) != AJVP_OK) return rc;
     i = 0;
+    for (void *x : out) p.out[i++] = static_cast<__nv_bfloat16 *>(x);
+    i = 0;
     for (float f : sc) p.out_scale[i++] = f;
-    const int64_t n_rtiles = (Lrow + BM - 1) / BM;
+    p.BH = (int)BH;
+    p.n_seq = (int)n_seq;
+    p.cu_row = cu_row;
+    p.cu_col = cu_col;
     p.stats = static_cast<const float4 *>(stats);
     p.Lrow = (int)Lrow;
     p.Lcol = (int)Lcol;
@@ -286,10 +312,29 @@ int launch_bwd_var(std::initializer_list<const void *> r, std::initializer_list<
     p.scale = scale;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.bound_ns = g_bound_ns.load();
-    attn_jvp_bwd_kernel<VAR, kCausal><<<(unsigned)(n_rtiles * BH), NTHREADS, Var<VAR>::SMEM_BYTES, stream>>>(p);
+    attn_jvp_bwd_kernel<VAR, MASK><<<(unsigned)n_cta, NTHREADS, Var<VAR>::SMEM_BYTES, stream>>>(p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail_cuda(e);
     return AJVP_OK;
+}
+
+// launch_bwd_var with the mask chosen at run time
+template <int VAR>
+int launch_bwd_mask(int mask, std::initializer_list<const void *> r, std::initializer_list<const void *> l,
+                    std::initializer_list<const void *> sh, std::initializer_list<void *> out,
+                    std::initializer_list<float> sc, const void *stats, int64_t BH, int64_t Lrow, int64_t Lcol,
+                    int64_t Lq, int64_t d, float scale, cudaStream_t stream, const int *cu_row, const int *cu_col,
+                    int64_t n_seq, int64_t max_row) {
+    switch (mask) {
+        case 0: return launch_bwd_var<VAR, 0>(r, l, sh, out, sc, stats, BH, Lrow, Lcol, Lq, d, scale, stream,
+                                              cu_row, cu_col, n_seq, max_row);
+        case 1: return launch_bwd_var<VAR, 1>(r, l, sh, out, sc, stats, BH, Lrow, Lcol, Lq, d, scale, stream,
+                                              cu_row, cu_col, n_seq, max_row);
+        case 2: return launch_bwd_var<VAR, 2>(r, l, sh, out, sc, stats, BH, Lrow, Lcol, Lq, d, scale, stream,
+                                              cu_row, cu_col, n_seq, max_row);
+        default: return launch_bwd_var<VAR, 3>(r, l, sh, out, sc, stats, BH, Lrow, Lcol, Lq, d, scale, stream,
+                                               cu_row, cu_col, n_seq, max_row);
+    }
 }
 
 // ---------------------------------------------------------- host pipeline
@@ -436,7 +481,7 @@ uint64_t attn_jvp_bwd_workspace_bytes(int64_t B, int64_t H, int64_t Lq) {
 namespace {
 // Kernels first..last of the backward (0 row statistics, 1 dQ and dtQ, 2 dK
 // and dtK, 3 dV and dtV) after the full argument check.
-int bwd_steps(int first, int last, bool causal, const void *q, const void *k, const void *v, const void *tq, const void *tk,
+int bwd_steps(int first, int last, int mask, const BwdPack &pk, const void *q, const void *k, const void *v, const void *tq, const void *tk,
               const void *tv, const void *o, const void *to, const float *lse, const float *mu, const void *dout,
               const void *dtout, void *dq, void *dk, void *dv, void *dtq, void *dtk, void *dtv, int64_t B, int64_t H,
               int64_t Lq, int64_t Lk, int64_t d, float scale, void *workspace, uint64_t workspace_bytes,
@@ -471,8 +516,8 @@ int bwd_steps(int first, int last, bool causal, const void *q, const void *k, co
     if (((Lq + 127) / 128) * BH >= (int64_t(1) << 31) || ((Lk + 127) / 128) * BH >= (int64_t(1) << 31) ||
         BH * Lq + ajvp::bwd::BN >= (int64_t(1) << 40))
         return AJVP_ERR_TOO_LARGE;
-    // the causal kernels form row + (Lk - Lq) sums in 32 bits
-    if (causal && (Lq >= (int64_t(1) << 30) || Lk >= (int64_t(1) << 30))) return AJVP_ERR_TOO_LARGE;
+    // the masked kernels form row + (Lk - Lq) sums in 32 bits
+    if (mask != 0 && (Lq >= (int64_t(1) << 30) || Lk >= (int64_t(1) << 30))) return AJVP_ERR_TOO_LARGE;
     if (!workspace || !aligned(workspace, 256) || workspace_bytes < bwd_stats_bytes(BH, Lq))
         return AJVP_ERR_WORKSPACE;
     int dev = 0;
@@ -493,18 +538,18 @@ int bwd_steps(int first, int last, bool causal, const void *q, const void *k, co
     auto want = [&](int k) { return first <= k && last >= k; };
     const float s1 = scale;
     // rows = queries, streamed keys: dq, dtq
-    auto vq = causal ? launch_bwd_var<V_Q, true> : launch_bwd_var<V_Q, false>;
-    if (want(1) && (rc = vq({q, tq, dtout, dout}, {k, tk}, {v, tv}, {dq, dtq}, {s1, s1}, workspace, BH, Lq, Lk, Lq,
-                            d, scale, st)) != AJVP_OK)
+    if (want(1) && (rc = launch_bwd_mask<V_Q>(mask, {q, tq, dtout, dout}, {k, tk}, {v, tv}, {dq, dtq}, {s1, s1},
+                                              workspace, BH, Lq, Lk, Lq, d, scale, st, pk.cu_q, pk.cu_k, pk.n_seq,
+                                              pk.max_q)) != AJVP_OK)
         return rc;
     // rows = keys, streamed queries: dk, dtk; dv, dtv
-    auto vk = causal ? launch_bwd_var<V_K, true> : launch_bwd_var<V_K, false>;
-    if (want(2) && (rc = vk({k, tk, v, tv}, {q, tq}, {dtout, dout}, {dk, dtk}, {s1, s1}, workspace, BH, Lk, Lq, Lq,
-                            d, scale, st)) != AJVP_OK)
+    if (want(2) && (rc = launch_bwd_mask<V_K>(mask, {k, tk, v, tv}, {q, tq}, {dtout, dout}, {dk, dtk}, {s1, s1},
+                                              workspace, BH, Lk, Lq, Lq, d, scale, st, pk.cu_k, pk.cu_q, pk.n_seq,
+                                              pk.max_k)) != AJVP_OK)
         return rc;
-    auto vv = causal ? launch_bwd_var<V_V, true> : launch_bwd_var<V_V, false>;
-    if (want(3) && (rc = vv({k, tk}, {dout, dtout}, {q, tq}, {dv, dtv}, {1.0f, 1.0f}, workspace, BH, Lk, Lq, Lq, d,
-                            scale, st)) != AJVP_OK)
+    if (want(3) && (rc = launch_bwd_mask<V_V>(mask, {k, tk}, {dout, dtout}, {q, tq}, {dv, dtv}, {1.0f, 1.0f},
+                                              workspace, BH, Lk, Lq, Lq, d, scale, st, pk.cu_k, pk.cu_q, pk.n_seq,
+                                              pk.max_k)) != AJVP_OK)
         return rc;
     return AJVP_OK;
 }
@@ -517,8 +562,8 @@ int attn_jvp_bwd(const void *q, const void *k, const void *v, const void *tq, co
                  const void *dtout, void *dq, void *dk, void *dv, void *dtq, void *dtk, void *dtv, int64_t B,
                  int64_t H, int64_t Lq, int64_t Lk, int64_t d, float scale, void *workspace,
                  uint64_t workspace_bytes, void *stream) {
-    return bwd_steps(0, 3, false, q, k, v, tq, tk, tv, o, to, lse, mu, dout, dtout, dq, dk, dv, dtq, dtk, dtv, B, H,
-                     Lq, Lk, d, scale, workspace, workspace_bytes, stream);
+    return bwd_steps(0, 3, 0, BwdPack(), q, k, v, tq, tk, tv, o, to, lse, mu, dout, dtout, dq, dk, dv, dtq, dtk,
+                     dtv, B, H, Lq, Lk, d, scale, workspace, workspace_bytes, stream);
 }
 
 int attn_jvp_fwd_causal_stats(const void *q, const void *k, const void *v, const void *tq, const void *tk,
@@ -534,8 +579,57 @@ int attn_jvp_bwd_causal(const void *q, const void *k, const void *v, const void 
                         const void *dout, const void *dtout, void *dq, void *dk, void *dv, void *dtq, void *dtk,
                         void *dtv, int64_t B, int64_t H, int64_t Lq, int64_t Lk, int64_t d, float scale,
                         void *workspace, uint64_t workspace_bytes, void *stream) {
-    return bwd_steps(0, 3, true, q, k, v, tq, tk, tv, o, to, lse, mu, dout, dtout, dq, dk, dv, dtq, dtk, dtv, B, H,
-                     Lq, Lk, d, scale, workspace, workspace_bytes, stream);
+    return bwd_steps(0, 3, ajvp::bwd::MASK_CAUSAL, BwdPack(), q, k, v, tq, tk, tv, o, to, lse, mu, dout, dtout, dq,
+                     dk, dv, dtq, dtk, dtv, B, H, Lq, Lk, d, scale, workspace, workspace_bytes, stream);
+}
+
+int attn_jvp_fwd_varlen_stats(const void *q, const void *k, const void *v, const void *tq, const void *tk,
+                              const void *tv, void *o, void *to, float *lse, float *mu,
+                              const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k, int64_t n_seq, int64_t H,
+                              int64_t total_q, int64_t total_k, int64_t max_seqlen_q, int64_t d, float scale,
+                              int causal, void *stream) {
+    if (n_seq < 0 || max_seqlen_q < 0) return AJVP_ERR_INVALID_ARG;
+    if (n_seq == 0 || max_seqlen_q == 0) {
+        if (H < 0 || total_q < 0 || total_k < 1 || d < 1 || !std::isfinite(scale)) return AJVP_ERR_INVALID_ARG;
+        return AJVP_OK;
+    }
+    if (H > 0 && total_q > 0 && (!lse || !mu)) return AJVP_ERR_INVALID_ARG;
+    if (!cu_seqlens_q || !cu_seqlens_k) return AJVP_ERR_INVALID_ARG;
+    if (!aligned(cu_seqlens_q, 4) || !aligned(cu_seqlens_k, 4)) return AJVP_ERR_MISALIGNED;
+    if (n_seq >= (int64_t(1) << 31) || max_seqlen_q > total_q) return AJVP_ERR_INVALID_ARG;
+    const int64_t max_qtiles = (max_seqlen_q + ajvp::sm100::BR - 1) / ajvp::sm100::BR;
+    if (causal)
+        return launch_sm100<false, ajvp::sm100::MASK_PACKED | ajvp::sm100::MASK_CAUSAL>(
+            q, k, v, tq, tk, tv, o, to, lse, 1, H, total_q, total_k, d, scale, stream, mu, cu_seqlens_q,
+            cu_seqlens_k, n_seq, max_qtiles);
+    return launch_sm100<false, ajvp::sm100::MASK_PACKED>(q, k, v, tq, tk, tv, o, to, lse, 1, H, total_q, total_k, d,
+                                                          scale, stream, mu, cu_seqlens_q, cu_seqlens_k, n_seq,
+                                                          max_qtiles);
+}
+
+int attn_jvp_bwd_varlen(const void *q, const void *k, const void *v, const void *tq, const void *tk,
+                        const void *tv, const void *o, const void *to, const float *lse, const float *mu,
+                        const void *dout, const void *dtout, void *dq, void *dk, void *dv, void *dtq, void *dtk,
+                        void *dtv, const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k, int64_t n_seq,
+                        int64_t H, int64_t total_q, int64_t total_k, int64_t max_seqlen_q, int64_t max_seqlen_k,
+                        int64_t d, float scale, int causal, void *workspace, uint64_t workspace_bytes,
+                        void *stream) {
+    if (n_seq < 0 || max_seqlen_q < 0 || max_seqlen_k < 0) return AJVP_ERR_INVALID_ARG;
+    if (max_seqlen_q > total_q || max_seqlen_k > total_k || n_seq >= (int64_t(1) << 31))
+        return AJVP_ERR_INVALID_ARG;
+    BwdPack pk;
+    pk.cu_q = cu_seqlens_q;
+    pk.cu_k = cu_seqlens_k;
+    pk.n_seq = n_seq;
+    pk.max_q = max_seqlen_q;
+    pk.max_k = max_seqlen_k;
+    if (n_seq > 0 && total_q > 0) {
+        if (!cu_seqlens_q || !cu_seqlens_k) return AJVP_ERR_INVALID_ARG;
+        if (!aligned(cu_seqlens_q, 4) || !aligned(cu_seqlens_k, 4)) return AJVP_ERR_MISALIGNED;
+    }
+    const int mask = ajvp::bwd::MASK_PACKED | (causal ? ajvp::bwd::MASK_CAUSAL : 0);
+    return bwd_steps(0, 3, mask, pk, q, k, v, tq, tk, tv, o, to, lse, mu, dout, dtout, dq, dk, dv, dtq, dtk, dtv, 1,
+                     H, total_q, total_k, d, scale, workspace, workspace_bytes, stream);
 }
 
 int attn_jvp_bwd_step(int step, const void *q, const void *k, const void *v, const void *tq, const void *tk,
@@ -544,8 +638,8 @@ int attn_jvp_bwd_step(int step, const void *q, const void *k, const void *v, con
                       void *dtv, int64_t B, int64_t H, int64_t Lq, int64_t Lk, int64_t d, float scale,
                       void *workspace, uint64_t workspace_bytes, void *stream) {
     if (step < 0 || step > 3) return AJVP_ERR_INVALID_ARG;
-    return bwd_steps(step, step, false, q, k, v, tq, tk, tv, o, to, lse, mu, dout, dtout, dq, dk, dv, dtq, dtk, dtv,
-                     B, H, Lq, Lk, d, scale, workspace, workspace_bytes, stream);
+    return bwd_steps(step, step, 0, BwdPack(), q, k, v, tq, tk, tv, o, to, lse, mu, dout, dtout, dq, dk, dv, dtq, dtk,
+                     dtv, B, H, Lq, Lk, d, scale, workspace, workspace_bytes, stream);
 }
 
 uint64_t attn_jvp_host_workspace_bytes(int64_t Lq, int64_t Lk, int64_t d, int64_t heads_per_chunk) {
@@ -694,7 +788,7 @@ int attn_jvp_bwd_host(const void *q, const void *k, const void *v, const void *t
         // compute: the four backward kernels on the chunk's n (batch, head) slabs
         const cudaStream_t cs = pipe.st[1 + (c & 1)];
         if ((e = cudaStreamWaitEvent(cs, pipe.in(b), 0)) != cudaSuccess) return fail_cuda(e);
-        rc = bwd_steps(0, 3, false, buf + L.in[0], buf + L.in[6], buf + L.in[7], buf + L.in[1], buf + L.in[8],
+        rc = bwd_steps(0, 3, 0, BwdPack(), buf + L.in[0], buf + L.in[6], buf + L.in[7], buf + L.in[1], buf + L.in[8],
                        buf + L.in[9], buf + L.in[2], buf + L.in[3], reinterpret_cast<const float *>(buf + L.in[10]),
                        reinterpret_cast<const float *>(buf + L.in[11]), buf + L.in[4], buf + L.in[5],
                        buf + L.out[0], buf + L.out[2], buf + L.out[3], buf + L.out[1], buf + L.out[4],

@@ -91,12 +91,22 @@ constexpr uint32_t OFF_TMEM_SLOT = 8 * N_BARS;
 constexpr uint32_t OFF_ABORT = OFF_TMEM_SLOT + 4;
 constexpr uint32_t NB_EPI = 1;
 
+// Masks (MASK bits): 1 causal -- key j is visible to query i iff
+// j <= i + (Lk - Lq) of its sequence, bottom-right aligned; 2 packed -- the
+// tensors are [H][total][128] and sequence b owns row-side rows
+// cu_row[b] .. cu_row[b+1]-1 and streamed rows cu_col[b] .. cu_col[b+1]-1.
+constexpr int MASK_CAUSAL = 1, MASK_PACKED = 2;
+
 struct Params {
     CUtensorMap tm_r[4], tm_l[2], tm_s[2], tm_out[2];
     const float4 *stats;  // [B*H][Lq] {lse*log2(e), mu, a, D}, plus BN rows of padding
-    int Lrow, Lcol;       // row-side and streamed lengths
+    int Lrow, Lcol;       // row-side and streamed lengths (packed: the tensors' totals)
     int Lq;               // query rows per (batch, head): the stats row stride
-    int n_rtiles;         // 128-row tiles per (batch, head)
+    int n_rtiles;         // 128-row tiles per (batch, head) (packed: of the longest sequence)
+    int BH;               // packed: heads (the tensors' outermost extent)
+    int n_seq;            // packed: sequences per head
+    const int *cu_row, *cu_col;  // packed: starts of each sequence's row-side / streamed rows
+    __nv_bfloat16 *out[2];       // packed: the outputs as plain pointers (guarded row stores)
     float scale;          // s
     float scale_log2;     // s * log2(e)
     float out_scale[2];   // factor applied to each accumulator at the end (s or 1)
@@ -179,13 +189,17 @@ struct Var {
     static_assert(BUF0 + kNB * BUF_COLS == 512u, "tensor-memory layout");
 };
 
-// kCausal: key j is visible to query i iff j <= i + (Lk - Lq) (bottom-right
-// aligned).  A CTA streams only the tiles that some row of its own sees (V_Q:
+// Causal: a CTA streams only the tiles that some row of its own sees (V_Q:
 // keys 0 .. r0 + 127 + Lk - Lq; V_K, V_V: queries from r0 - (Lk - Lq) on),
 // hidden pairs get P = 0, and a CTA whose rows see nothing writes zeros.
-template <int VAR, bool kCausal = false>
+// Packed: a CTA is one 128-row tile of one (sequence, head); streamed tiles
+// start at the sequence's first streamed row and columns past its end are
+// hidden; rows past the sequence's end (the tile may overhang into the next
+// sequence) are computed but not stored.
+template <int VAR, int MASK = 0>
 __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_constant__ Params p) {
     using C = Var<VAR>;
+    constexpr bool kCausal = (MASK & MASK_CAUSAL) != 0, kPacked = (MASK & MASK_PACKED) != 0;
     extern __shared__ __align__(1024) uint8_t bwd_smem[];
     const uint32_t base = smem_u32(bwd_smem);
     if (base & 1023u) {  // the tile layout needs 1024-byte alignment and leaves no slack
@@ -196,23 +210,41 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    // causal dQ / dtQ: the late (heavy) query tiles of each head first
-    const int rt = (kCausal && VAR == V_Q) ? p.n_rtiles - 1 - (int)(blockIdx.x % p.n_rtiles)
-                                           : (int)(blockIdx.x % p.n_rtiles);
-    const int bh = blockIdx.x / p.n_rtiles;
-    const int r0 = rt * BM;
+    // this CTA: local row tile rt of a sequence (dense: the whole tensor) whose row-side
+    // rows start at tensor row yr0 and streamed rows at yc0, Lrow_s and Lcol_s of them
+    int rt, bh, yr0 = 0, yc0 = 0, Lrow_s = p.Lrow, Lcol_s = p.Lcol;
+    if (kPacked) {
+        // (sequence, head) major, row tiles fastest (they share the streamed rows in
+        // L2); offsets clamped into the tensors so that bad ones stay memory-safe
+        const int u = (int)(blockIdx.x % p.n_rtiles), sh = (int)(blockIdx.x / p.n_rtiles);
+        const int b = sh / p.BH;
+        bh = sh % p.BH;
+        rt = (kCausal && VAR == V_Q) ? p.n_rtiles - 1 - u : u;  // causal dQ: late (heavy) tiles first
+        yr0 = min(max(p.cu_row[b], 0), p.Lrow);
+        Lrow_s = max(min(max(p.cu_row[b + 1], 0), p.Lrow), yr0) - yr0;
+        yc0 = min(max(p.cu_col[b], 0), p.Lcol);
+        Lcol_s = max(min(max(p.cu_col[b + 1], 0), p.Lcol), yc0) - yc0;
+    } else {
+        // causal dQ / dtQ: the late (heavy) query tiles of each head first
+        rt = (kCausal && VAR == V_Q) ? p.n_rtiles - 1 - (int)(blockIdx.x % p.n_rtiles)
+                                     : (int)(blockIdx.x % p.n_rtiles);
+        bh = blockIdx.x / p.n_rtiles;
+    }
+    const int r0 = rt * BM;  // local first row
+    if (kPacked && r0 >= Lrow_s) return;  // past the end of this sequence (uniform for the CTA)
+    const int yr = yr0 + r0;              // tensor row of the tile's first row
     // streamed tiles jt0 .. jt0 + nt - 1 (local index j = 0 .. nt - 1)
-    int jt0 = 0, nt = (p.Lcol + BN - 1) / BN;
-    // kOff = Lk - Lq: the causal diagonal's offset
-    const int koff = VAR == V_Q ? p.Lcol - p.Lrow : p.Lrow - p.Lcol;
+    int jt0 = 0, nt = (Lcol_s + BN - 1) / BN;
+    // koff = Lk - Lq of the sequence: the causal diagonal's offset
+    const int koff = VAR == V_Q ? Lcol_s - Lrow_s : Lrow_s - Lcol_s;
     if (kCausal) {
         if (VAR == V_Q) {
-            const int kend = min(p.Lcol, r0 + BM + koff);  // keys some row of the tile sees
+            const int kend = min(Lcol_s, r0 + BM + koff);  // keys some row of the tile sees
             nt = kend > 0 ? (kend + BN - 1) / BN : 0;
         } else {
             const int qbeg = max(0, r0 - koff);  // first query that sees a key of the tile
             jt0 = qbeg / BN;
-            nt = qbeg < p.Lcol ? nt - jt0 : 0;
+            nt = qbeg < Lcol_s ? nt - jt0 : 0;
         }
     }
     const uint64_t bound = p.bound_ns;
@@ -272,8 +304,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
             if (lp) {
                 mbar_arrive_expect_tx(BAR(B_R_FULL), C::kNR * R_TILE);
                 for (int i = 0; i < C::kNR; ++i) {
-                    tma_load_3d(base + SM_R + i * R_TILE, &p.tm_r[i], BAR(B_R_FULL), 0, r0, bh);
-                    tma_load_3d(base + SM_R + i * R_TILE + CHUNK_R, &p.tm_r[i], BAR(B_R_FULL), 64, r0, bh);
+                    tma_load_3d(base + SM_R + i * R_TILE, &p.tm_r[i], BAR(B_R_FULL), 0, yr, bh);
+                    tma_load_3d(base + SM_R + i * R_TILE + CHUNK_R, &p.tm_r[i], BAR(B_R_FULL), 64, yr, bh);
                 }
             }
             // a stage [x c0 | y c0 | x c1 | y c1] of two streamed tensors, rows y..y+63
@@ -284,7 +316,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
                 tma_load_3d(st + 3 * CHUNK_C, my, fb, 64, y, bh);
             };
             for (int t = 0; t < nt && ok; ++t) {
-                const int y = (jt0 + t) * BN;
+                const int y = yc0 + (jt0 + t) * BN;  // tensor row of the streamed tile
                 if (lp) {  // long ring, stage t % kLS: free once the G2 products of tile t - kLS are complete
                     const int s = t % C::kLS;
                     if (t >= C::kLS &&
@@ -448,7 +480,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
         const float2 c2 = make_float2(p.scale_log2, p.scale_log2);
         const float2 s2 = make_float2(p.scale, p.scale);
         float4 rs = make_float4(0.f, 0.f, 0.f, 0.f);  // row statistics {lse2, mu, a, D} (query rows)
-        if (!C::kColStats && r0 + row < p.Lrow) rs = p.stats[(size_t)bh * p.Lq + (size_t)(r0 + row)];
+        if (!C::kColStats && r0 + row < Lrow_s) rs = p.stats[(size_t)bh * p.Lq + (size_t)(yr + row)];
         bool failed = false;
         // one pair of columns (c, c + 1 of this group): x scores, y score tangent,
         // z A, w B -> r1, r2 (see the variant table)
@@ -497,7 +529,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
             tc_fence_after();
             // this group's columns lo .. hi - 1 are inside the tensor and visible
             const int y0 = (jt0 + j) * BN + (int)col0;  // the group's first streamed item
-            int lo = 0, hi = p.Lcol - y0;
+            int lo = 0, hi = Lcol_s - y0;
             if (kCausal) {
                 if (VAR == V_Q)
                     hi = min(hi, r0 + row + koff - y0 + 1);  // keys <= query + (Lk - Lq)
@@ -569,7 +601,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
                 for (int h = 0; h < 2; ++h) {
                     const int pc = 2 * grp + h;
                     uint32_t ra[32];
-                    if (kCausal && nt == 0) {  // no row of the tile sees anything: zeros
+                    if (MASK != 0 && nt == 0) {  // no row of the tile sees anything: zeros
 #pragma unroll
                         for (int i = 0; i < 32; ++i) ra[i] = 0u;
                     } else {
@@ -580,6 +612,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
 #pragma unroll
                     for (int i = 0; i < 16; ++i)
                         wa[i] = pack_bf16x2(__uint_as_float(ra[2 * i]) * os, __uint_as_float(ra[2 * i + 1]) * os);
+                    if (kPacked) {
+                        // rows past the sequence's end belong to the next one: not written
+                        if (r0 + row < Lrow_s) {
+                            uint4 *dst = reinterpret_cast<uint4 *>(
+                                p.out[a] + ((size_t)bh * (size_t)p.Lrow + (size_t)(yr + row)) * HD + 64u * grp + 32u * h);
+#pragma unroll
+                            for (int u = 0; u < 4; ++u)
+                                dst[u] = make_uint4(wa[4 * u], wa[4 * u + 1], wa[4 * u + 2], wa[4 * u + 3]);
+                        }
+                        continue;
+                    }
                     const uint32_t dst = base + SM_R + (uint32_t)a * R_TILE + (uint32_t)grp * CHUNK_R + (uint32_t)row * 128u;
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
@@ -591,10 +634,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
         }
         fence_proxy_async_smem();
         named_bar_sync(NB_EPI, EW_THREADS);  // staging complete
-        if (warp == 4 && lane == 0 && !any_failed && *abort_flag == 0) {
+        if (!kPacked && warp == 4 && lane == 0 && !any_failed && *abort_flag == 0) {
             for (int a = 0; a < 2; ++a) {
-                tma_store_3d(&p.tm_out[a], base + SM_R + a * R_TILE, 0, r0, bh);
-                tma_store_3d(&p.tm_out[a], base + SM_R + a * R_TILE + CHUNK_R, 64, r0, bh);
+                tma_store_3d(&p.tm_out[a], base + SM_R + a * R_TILE, 0, yr, bh);
+                tma_store_3d(&p.tm_out[a], base + SM_R + a * R_TILE + CHUNK_R, 64, yr, bh);
             }
             tma_store_commit();
             tma_store_wait_all();

@@ -19,8 +19,8 @@
  * never written to memory.  No dropout; Lq may differ from Lk
  * (cross-attention); attn_jvp_fwd_causal and attn_jvp_fwd_varlen add a
  * causal mask and packed variable-length sequences, attn_jvp_bwd the
- * backward pass (attn_jvp_bwd_causal that of the causal forward).  s is a
- * constant (no derivative with respect to it).
+ * backward pass (attn_jvp_bwd_causal and attn_jvp_bwd_varlen those of the
+ * masked forwards).  s is a constant (no derivative with respect to it).
  *
  * Layout: every tensor is a contiguous row-major [B][H][L][d] array (the
  * layout of a PyTorch [B, H, L, d] tensor); the tangents tQ, tK, tV share the
@@ -264,6 +264,56 @@ AJVP_API int attn_jvp_bwd_causal(const void *q, const void *k, const void *v,
                  void *dq, void *dk, void *dv, void *dtq, void *dtk, void *dtv,
                  int64_t B, int64_t H, int64_t Lq, int64_t Lk, int64_t d,
                  float scale, void *workspace, uint64_t workspace_bytes, void *stream);
+
+/*
+ * attn_jvp_fwd_varlen_stats -- attn_jvp_fwd_varlen that also saves mu
+ * (float [H][total_q]), the statistics attn_jvp_bwd_varlen needs beside lse.
+ * Rows that see no key get lse = -infinity and mu = 0.  lse and mu are
+ * required; other arguments and rules as attn_jvp_fwd_varlen.
+ */
+AJVP_API int attn_jvp_fwd_varlen_stats(const void *q, const void *k, const void *v,
+                       const void *tq, const void *tk, const void *tv,
+                       void *o, void *to, float *lse, float *mu,
+                       const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                       int64_t n_seq, int64_t H, int64_t total_q, int64_t total_k,
+                       int64_t max_seqlen_q, int64_t d, float scale, int causal,
+                       void *stream);
+
+/*
+ * attn_jvp_bwd_varlen -- backward pass of attn_jvp_fwd_varlen (packed
+ * variable-length sequences, optionally causal inside each sequence): the
+ * gradients of L = sum <dout, O> + sum <dtout, tO>.  The pages describe
+ * neither packed batches nor the backward; this is the gradient of the
+ * packed forward definition, attention never crossing sequences.
+ *
+ *   q, tq, o, to, dout, dtout, dq, dtq : __nv_bfloat16 [H][total_q][d]
+ *   k, v, tk, tv, dk, dv, dtk, dtv     : __nv_bfloat16 [H][total_k][d]
+ *   lse, mu             : float [H][total_q] (attn_jvp_fwd_varlen_stats)
+ *   cu_seqlens_q / _k, n_seq, causal   : as attn_jvp_fwd_varlen
+ *   max_seqlen_q / _k   : at least the longest query / key sequence (they
+ *                         set the grids; rows of longer sequences would not
+ *                         be computed)
+ *   workspace           : DEVICE memory, 256-byte aligned, at least
+ *                         attn_jvp_bwd_workspace_bytes(1, H, total_q) bytes
+ *
+ * Gradients of rows that see no key, and of keys that no row sees (a
+ * sequence without queries), are zero; rows outside every sequence are not
+ * written.  Offsets outside [0, total] are clamped in the kernels
+ * (memory-safe; such a call's results are unspecified).  total_q == 0 writes
+ * zeros to dk, dv, dtk, dtv.  Supported: d == 128, total_k >= 1, tensors
+ * 16-byte and offset arrays 4-byte aligned; workspace, checks and errors as
+ * attn_jvp_bwd, plus AJVP_ERR_TOO_LARGE for total_q or total_k >= 2^30.
+ */
+AJVP_API int attn_jvp_bwd_varlen(const void *q, const void *k, const void *v,
+                 const void *tq, const void *tk, const void *tv,
+                 const void *o, const void *to, const float *lse, const float *mu,
+                 const void *dout, const void *dtout,
+                 void *dq, void *dk, void *dv, void *dtq, void *dtk, void *dtv,
+                 const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                 int64_t n_seq, int64_t H, int64_t total_q, int64_t total_k,
+                 int64_t max_seqlen_q, int64_t max_seqlen_k, int64_t d,
+                 float scale, int causal, void *workspace, uint64_t workspace_bytes,
+                 void *stream);
 
 /* Device workspace, in bytes, that attn_jvp_bwd needs (0 for invalid sizes). */
 AJVP_API uint64_t attn_jvp_bwd_workspace_bytes(int64_t B, int64_t H, int64_t Lq);
