@@ -48,7 +48,7 @@ FWD_TRAFFIC_FILES = {"video_selfattn_b1h12_l32760_d128": TRAFFIC_FILE,
                          "profiles/attn_jvp_fwd_kernel_persistent.video_crossattn_b1h40_lq32760_lk512.md"}
 MASKED_METRIC = "attention+JVP TFLOP/s (12·d per visible query-key pair) and % of B200 BF16 tensor peak"
 BWD_METRIC = "attention+JVP backward TFLOP/s (30·Lq·Lk·d/head) and % of B200 BF16 tensor peak"
-BWD_CAUSAL_METRIC = ("attention+JVP causal backward TFLOP/s (30·d per visible query-key pair) and % of B200 "
+BWD_MASKED_METRIC = ("attention+JVP masked backward TFLOP/s (30·d per visible query-key pair) and % of B200 "
                      "BF16 tensor peak")
 BWD_KERNEL_SOURCES = ["attention_forward_mode_b200/csrc/jvp_bwd_sm100.cuh",
                       "attention_forward_mode_b200/csrc/ptx_sm100.cuh"]
@@ -315,8 +315,7 @@ def run_ours(args, w):
     seq_lens = None
     if args.entry == "varlen":
         import numpy as np
-        cuts = np.sort(np.random.default_rng(0).choice(np.arange(1, w.Lq), size=7, replace=False))
-        seq_lens = np.diff(np.concatenate([[0], cuts, [w.Lq]])).astype(int).tolist()
+        seq_lens = varlen_lengths(w)
         cu = torch.tensor(np.concatenate([[0], np.cumsum(seq_lens)]), dtype=torch.int32, device=dev)
         flops = 12.0 * w.d * w.B * w.H * float(sum(n * n for n in seq_lens))
 
@@ -504,6 +503,14 @@ def oracle_bwd_sample(w, full_cpu_head, seconds: float, seed: int = 0):
     return 30.0 * n * w.Lk * w.d / el / 1e12, n, el, oracle.num_threads()
 
 
+def varlen_lengths(w):
+    """The 8 packed sequences of ``--entry varlen`` / ``bwd_varlen``: the
+    workload's tokens cut at 7 seeded positions."""
+    import numpy as np
+    cuts = np.sort(np.random.default_rng(0).choice(np.arange(1, w.Lq), size=7, replace=False))
+    return np.diff(np.concatenate([[0], cuts, [w.Lq]])).astype(int).tolist()
+
+
 def bwd_causal_flops(w) -> float:
     """30 d FLOPs per visible (query, key) pair of the causal mask, summed
     over the heads (the backward's count of ``bwd_flops`` over visible pairs)."""
@@ -548,10 +555,19 @@ def run_reference_bwd(args, w):
     import oracle
     from attention_forward_mode_b200.workloads import make_cotangents
     oracle.build()
+    w0 = w  # the workload named in the line (a packed call's sample is one of its sequences)
     causal = args.entry == "bwd_causal"
     head = bwd_head0_cpu(make_inputs(w, seed=0, device="cpu"), make_cotangents(w, device="cpu"))
     per_step = max(0.5, args.reference_seconds / max(1, args.steps + args.warmup))
     sample_fn = oracle_bwd_sample_causal if causal else oracle_bwd_sample
+    if args.entry == "bwd_varlen":
+        # packed sequences are independent problems: the longest one stands for the pack
+        import dataclasses
+        lens = varlen_lengths(w)
+        b0 = max(range(len(lens)), key=lambda b: lens[b])
+        a0, n0 = sum(lens[:b0]), lens[b0]
+        head = {n: t[a0:a0 + n0] for n, t in head.items()}
+        w = dataclasses.replace(w, Lq=n0, Lk=n0)
     for _ in range(args.warmup):
         sample_fn(w, head, per_step)
     flops_total, el_total, rows_total, threads = 0.0, 0.0, 0, oracle.num_threads()
@@ -562,12 +578,15 @@ def run_reference_bwd(args, w):
         el_total += el
     value = flops_total / el_total / 1e12
     what = (f"causal backward sub-problems of the first query rows and keys of head 0" if causal else
-            f"backward of the first query rows of head 0 with all {w.Lk} keys")
+            f"backward of the first query rows of head 0 with all {w.Lk} keys"
+            + (" of its longest packed sequence" if args.entry == "bwd_varlen" else ""))
     sample = f"{what}, {rows_total} rows over {args.steps} steps, {el_total:.1f} s of fp64 oracle time"
-    line = {"impl": "reference", "metric": BWD_CAUSAL_METRIC if causal else BWD_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+    masked = args.entry in ("bwd_causal", "bwd_varlen")
+    line = {"impl": "reference", "metric": BWD_MASKED_METRIC if masked else BWD_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * el_total / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": dict(workload_config(w, world), entry="attn_jvp_bwd_causal" if causal else "attn_jvp_bwd"),
+            "config": dict(workload_config(w0, world), entry={"bwd": "attn_jvp_bwd", "bwd_causal": "attn_jvp_bwd_causal",
+                                                              "bwd_varlen": "attn_jvp_bwd_varlen"}[args.entry]),
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -585,12 +604,23 @@ def run_ours_bwd(args, w):
     ajvp.load_library()
     names = ("q", "k", "v", "tq", "tk", "tv")
     causal = args.entry == "bwd_causal"
+    varlen = args.entry == "bwd_varlen"
     inp = make_inputs(w, seed=rank, device=dev)
     cot = make_cotangents(w, seed=1000 + rank, device=dev)
     stream = torch.cuda.current_stream(dev)
-    fwd = ajvp.attn_jvp_fwd_causal_stats if causal else ajvp.attn_jvp_fwd_stats
-    o, to, lse, mu = fwd(*(inp[n] for n in names), w.scale, stream=stream)
+    if varlen:
+        # the (batch, head) slabs' tokens packed as 8 sequences, [H, total, d] views
+        import numpy as np
+        seq_lens = varlen_lengths(w)
+        cu = torch.tensor(np.concatenate([[0], np.cumsum(seq_lens)]), dtype=torch.int32, device=dev)
+        pk = {n: t.reshape(-1, t.shape[-2], t.shape[-1]) for n, t in {**inp, **cot}.items()}
+        o, to, lse, mu = ajvp.attn_jvp_fwd_varlen_stats(*(pk[n] for n in names), cu, cu, max(seq_lens), w.scale,
+                                                        stream=stream)
+    else:
+        fwd = ajvp.attn_jvp_fwd_causal_stats if causal else ajvp.attn_jvp_fwd_stats
+        o, to, lse, mu = fwd(*(inp[n] for n in names), w.scale, stream=stream)
     grads = {n: torch.empty_like(inp["q"] if n in ("dq", "dtq") else inp["k"]) for n in ajvp.GRAD_NAMES}
+    gpk = {n: g.reshape(-1, g.shape[-2], g.shape[-1]) for n, g in grads.items()}
     ws = torch.empty(ajvp.bwd_workspace_bytes(w.B, w.H, w.Lq), dtype=torch.uint8, device=dev)
     in_bytes = sum(t.numel() * t.element_size() for t in list(inp.values()) + list(cot.values()) + [o, to])
     flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev) if in_bytes <= L2_BYTES else None
@@ -601,6 +631,9 @@ def run_ours_bwd(args, w):
         if causal:
             ajvp.attn_jvp_bwd_causal(*(inp[n] for n in names), o, to, lse, mu, cot["dout"], cot["dtout"], w.scale,
                                      grads=grads, workspace=ws, stream=stream)
+        elif varlen:
+            ajvp.attn_jvp_bwd_varlen(*(pk[n] for n in names), o, to, lse, mu, pk["dout"], pk["dtout"], cu, cu,
+                                     max(seq_lens), max(seq_lens), w.scale, grads=gpk, workspace=ws, stream=stream)
         else:
             ajvp.attn_jvp_bwd(*(inp[n] for n in names), o, to, lse, mu, cot["dout"], cot["dtout"], w.scale,
                               grads=grads, workspace=ws, stream=stream, step=which)
@@ -628,10 +661,14 @@ def run_ours_bwd(args, w):
     ms_max = max_over_ranks(ms, world, dev)
     if ajvp.check_device_status(stream) != ajvp.AJVP_OK:
         raise RuntimeError("kernel wait bound exceeded")
-    flops = bwd_causal_flops(w) if causal else bwd_flops(w)
+    if varlen:
+        flops = 30.0 * w.d * w.B * w.H * float(sum(n * n for n in seq_lens))
+    else:
+        flops = bwd_causal_flops(w) if causal else bwd_flops(w)
     value = aggregate_value(flops, args.steps, world, ms_max / 1e3)
-    if causal:
-        return finish_bwd_causal(args, w, rank, world, value, flops, ms_max, clocks, inp, cot)
+    if causal or varlen:
+        return finish_bwd_masked(args, w, rank, world, value, flops, ms_max, clocks, inp, cot,
+                                 seq_lens if varlen else None)
 
     # each of the four kernels alone, K launches each, events on the stream
     per_kernel = []
@@ -710,29 +747,40 @@ def run_ours_bwd(args, w):
     return 0
 
 
-def finish_bwd_causal(args, w, rank, world, value, flops, ms_max, clocks, inp, cot):
-    """JSON line of ``--entry bwd_causal``: the causal backward timed as one
-    step (four kernels; there is no per-kernel or host-buffer entry for it),
-    FLOPs counted over the visible pairs."""
+def finish_bwd_masked(args, w, rank, world, value, flops, ms_max, clocks, inp, cot, seq_lens=None):
+    """JSON line of ``--entry bwd_causal`` / ``bwd_varlen``: the masked
+    backward timed as one step (four kernels; there is no per-kernel or
+    host-buffer entry for it), FLOPs counted over the visible pairs."""
+    entry = "attn_jvp_bwd_varlen" if seq_lens else "attn_jvp_bwd_causal"
     if rank == 0:
         burst, _, src = measured_peaks()
         achieved = flops / (ms_max / args.steps / 1e3) / 1e12
-        line = {"metric": BWD_CAUSAL_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        line = {"metric": BWD_MASKED_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
                 "data": "synthetic",
-                "config": dict(workload_config(w, world), entry="attn_jvp_bwd_causal",
-                               flops_per_step="30·d per visible (query, key) pair"),
+                "config": dict(workload_config(w, world), entry=entry,
+                               flops_per_step="30·d per visible (query, key) pair",
+                               **({"sequence_lengths": seq_lens} if seq_lens else {})),
                 "pct_of_bf16_peak": 100.0 * value / world / burst,
                 "roofline": {"bound": "tensor", "achieved": achieved, "peak": burst, "unit": "TFLOP/s",
                              "frac": achieved / burst, "traffic": None,
                              "peak_source": f"{src} bf16 dense (burst) from MEASURED_PEAKS.json"
                              if src == "measured" else "fallback 1.59 PFLOP/s",
-                             "kernel": "attn_jvp_bwd_causal (row statistics and three gradient kernels, one step)",
+                             "kernel": f"{entry} (row statistics and three gradient kernels, one step)",
                              "algorithmic_flops_per_launch": flops},
                 "e2e": None,
                 "gpu_launches": 4 * args.steps, "clocks": clocks.summary()}
-        if world == 1 and not args.no_cpu_baseline:
+        if world == 1 and not args.no_cpu_baseline and seq_lens:
+            import dataclasses
+            b0 = max(range(len(seq_lens)), key=lambda b: seq_lens[b])  # the longest sequence
+            a0, n0 = sum(seq_lens[:b0]), seq_lens[b0]
+            head = {n: t[a0:a0 + n0] for n, t in bwd_head0_cpu(inp, cot).items()}
+            v, n, el, threads = oracle_bwd_sample(dataclasses.replace(w, Lq=n0, Lk=n0), head, args.cpu_seconds)
+            line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                                    "sample": f"backward of the first {n} query rows of sequence {b0} ({n0} tokens) "
+                                              f"of head 0 with its keys ({el:.1f} s, fp64, OpenMP)"}
+        elif world == 1 and not args.no_cpu_baseline:
             v, n, el, threads = oracle_bwd_sample_causal(w, bwd_head0_cpu(inp, cot), args.cpu_seconds)
             line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                                     "sample": f"causal backward of the first {n} query rows and keys of head 0 "
@@ -784,10 +832,12 @@ def main(argv=None):
     ap.add_argument("--reference-seconds", type=float, default=90.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-eager", action="store_true")
-    ap.add_argument("--entry", choices=["bf16", "f32out", "causal", "varlen", "bwd", "bwd_causal"], default="bf16",
+    ap.add_argument("--entry", choices=["bf16", "f32out", "causal", "varlen", "bwd", "bwd_causal", "bwd_varlen"],
+                    default="bf16",
                     help="f32out: time attn_jvp_fwd_f32out (fp32 outputs, split-bf16 probabilities); "
                          "causal: attn_jvp_fwd_causal; varlen: attn_jvp_fwd_varlen on 8 packed sequences; "
-                         "bwd: time the backward pass attn_jvp_bwd; bwd_causal: attn_jvp_bwd_causal")
+                         "bwd: time the backward pass attn_jvp_bwd; bwd_causal: attn_jvp_bwd_causal; "
+                         "bwd_varlen: attn_jvp_bwd_varlen on the 8 packed sequences of varlen")
     ap.add_argument("--heads", type=int, default=None,
                     help="override H (small profiling captures); the JSON config shows the H used")
     args = ap.parse_args(argv)
@@ -798,7 +848,7 @@ def main(argv=None):
         w = dataclasses.replace(w, H=args.heads, name=f"{w.name}_h{args.heads}")
     if w.dtype != "bf16" and args.impl == "ours":
         ap.error("the benchmark times the bf16 tensor-core path")
-    if args.entry in ("bwd", "bwd_causal"):
+    if args.entry in ("bwd", "bwd_causal", "bwd_varlen"):
         return run_reference_bwd(args, w) if args.impl == "reference" else run_ours_bwd(args, w)
     if args.impl == "reference":
         return run_reference(args, w)
