@@ -24,6 +24,10 @@ dtype).
 forward keeps its head-sharded inputs and outputs, the backward sends the
 cotangents dO, dtO to head shards, runs the local backward there and returns
 the six gradients to sequence shards.
+
+``causal=True`` selects the causal kernels as the local step: after the
+exchange every rank holds whole sequences in their original order, so the
+mask (key j visible to query i iff j <= i + Lk - Lq) applies unchanged.
 """
 from __future__ import annotations
 
@@ -57,12 +61,13 @@ def _to_sequence(y: torch.Tensor, world: int, group) -> torch.Tensor:
     return recv.permute(1, 2, 0, 3, 4, 5).reshape(n, B, world * hp, Ls, e)
 
 
-def ulysses_attn_jvp(q, k, v, tq, tk, tv, scale=None, group=None, local_fn=None):
+def ulysses_attn_jvp(q, k, v, tq, tk, tv, scale=None, group=None, local_fn=None, causal=False):
     """O, tO, lse for sequence-sharded inputs (see the module docstring).
 
     ``local_fn(q, k, v, tq, tk, tv, scale) -> (o, to, lse)`` computes the
     attention JVP of the gathered head shard; it defaults to the CUDA kernel
-    (``attn_jvp``).  Collective calls are made in the same order on every rank.
+    (``attn_jvp``, or ``attn_jvp_fwd_causal`` with ``causal``).  Collective
+    calls are made in the same order on every rank.
     """
     grouped = dist.is_initialized()
     world = dist.get_world_size(group) if grouped else 1
@@ -72,7 +77,13 @@ def ulysses_attn_jvp(q, k, v, tq, tk, tv, scale=None, group=None, local_fn=None)
         raise ValueError(f"heads ({H}) must divide by the group size ({world})")
     if scale is None:
         scale = d ** -0.5
-    fn = local_fn if local_fn is not None else attn_jvp
+    if local_fn is not None:
+        fn = local_fn
+    elif causal:
+        from ._binding import attn_jvp_fwd_causal
+        fn = attn_jvp_fwd_causal
+    else:
+        fn = attn_jvp
     if not grouped:  # no process group: the plain local call
         return fn(q, k, v, tq, tk, tv, scale)
 
@@ -86,16 +97,17 @@ def ulysses_attn_jvp(q, k, v, tq, tk, tv, scale=None, group=None, local_fn=None)
     return out[0], out[1], lse_s
 
 
-def ulysses_attn_jvp_train(q, k, v, tq, tk, tv, scale=None, group=None, local_fwd=None):
+def ulysses_attn_jvp_train(q, k, v, tq, tk, tv, scale=None, group=None, local_fwd=None, causal=False):
     """Forward of ``ulysses_attn_jvp`` that also keeps what the backward needs.
 
     Returns (o, to, lse, ctx): the sequence-sharded outputs as
     ``ulysses_attn_jvp`` gives them, and ``ctx`` for ``ulysses_attn_jvp_bwd``
     holding the head-sharded inputs and the forward's head-sharded O, tO, lse
     and mu.  ``local_fwd(q, k, v, tq, tk, tv, scale) -> (o, to, lse, mu)``
-    defaults to the library's ``attn_jvp_fwd_stats``.
+    defaults to the library's ``attn_jvp_fwd_stats`` (``attn_jvp_fwd_causal_stats``
+    with ``causal``, which ``ulysses_attn_jvp_bwd`` then follows).
     """
-    from ._binding import attn_jvp_fwd_stats
+    from ._binding import attn_jvp_fwd_causal_stats, attn_jvp_fwd_stats
     grouped = dist.is_initialized()
     world = dist.get_world_size(group) if grouped else 1
     B, H, Lqs, d = q.shape
@@ -103,10 +115,10 @@ def ulysses_attn_jvp_train(q, k, v, tq, tk, tv, scale=None, group=None, local_fw
         raise ValueError(f"heads ({H}) must divide by the group size ({world})")
     if scale is None:
         scale = d ** -0.5
-    fn = local_fwd if local_fwd is not None else attn_jvp_fwd_stats
+    fn = local_fwd if local_fwd is not None else (attn_jvp_fwd_causal_stats if causal else attn_jvp_fwd_stats)
     if not grouped:
         o, to, lse, mu = fn(q, k, v, tq, tk, tv, scale)
-        ctx = dict(inputs=(q, k, v, tq, tk, tv), outputs=(o, to, lse, mu), scale=scale, world=1)
+        ctx = dict(inputs=(q, k, v, tq, tk, tv), outputs=(o, to, lse, mu), scale=scale, world=1, causal=causal)
         return o, to, lse, ctx
     qs = _to_heads(torch.stack((q, tq)), world, group)        # [2, B, H/P, Lq, d]
     ks = _to_heads(torch.stack((k, v, tk, tv)), world, group)  # [4, B, H/P, Lk, d]
@@ -115,7 +127,7 @@ def ulysses_attn_jvp_train(q, k, v, tq, tk, tv, scale=None, group=None, local_fw
     o, to, lse, mu = fn(*inputs, scale)
     out = _to_sequence(torch.stack((o, to)), world, group)
     lse_s = _to_sequence(lse.unsqueeze(0).unsqueeze(-1).contiguous(), world, group)[0, ..., 0]
-    ctx = dict(inputs=inputs, outputs=(o, to, lse, mu), scale=scale, world=world)
+    ctx = dict(inputs=inputs, outputs=(o, to, lse, mu), scale=scale, world=world, causal=causal)
     return out[0], out[1], lse_s, ctx
 
 
@@ -128,11 +140,12 @@ def ulysses_attn_jvp_bwd(ctx, dout, dtout, group=None, local_bwd=None):
     head-sharded tensors the forward kept, and the gradients return to
     sequence shards (one all-to-all for the query side, one for the key
     side).  ``local_bwd(q, k, v, tq, tk, tv, o, to, lse, mu, dout, dtout,
-    scale) -> dict`` defaults to the library's ``attn_jvp_bwd``.  Returns a
-    dict dq, dk, dv, dtq, dtk, dtv shaped like the inputs.
+    scale) -> dict`` defaults to the library's ``attn_jvp_bwd`` (or
+    ``attn_jvp_bwd_causal`` when the forward was causal).  Returns a dict dq,
+    dk, dv, dtq, dtk, dtv shaped like the inputs.
     """
-    from ._binding import attn_jvp_bwd
-    fn = local_bwd if local_bwd is not None else attn_jvp_bwd
+    from ._binding import attn_jvp_bwd, attn_jvp_bwd_causal
+    fn = local_bwd if local_bwd is not None else (attn_jvp_bwd_causal if ctx.get("causal") else attn_jvp_bwd)
     world = ctx["world"]
     if world == 1:
         return fn(*ctx["inputs"], *ctx["outputs"], dout, dtout, ctx["scale"])

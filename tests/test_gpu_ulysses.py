@@ -2,7 +2,7 @@
 two all-to-all exchanges run for real (as identity exchanges) around the CUDA
 kernel, and the result must equal a direct attn_jvp_fwd call bit for bit; the
 same for the training path (forward keeping its head shards, backward
-exchanges around attn_jvp_bwd).
+exchanges around attn_jvp_bwd), unmasked and causal.
 (Exchanges across several ranks are checked on CPU over gloo.)"""
 import datetime
 import os
@@ -44,6 +44,16 @@ def test_one_rank_nccl_equals_direct_call():
         g = ulysses_attn_jvp_bwd(ctx, cot["dout"], cot["dtout"])
         ro, rto, rlse, rmu = ajvp.attn_jvp_fwd_stats(*(inp[n] for n in names), w.scale)
         rg = ajvp.attn_jvp_bwd(*(inp[n] for n in names), ro, rto, rlse, rmu, cot["dout"], cot["dtout"], w.scale)
+        torch.cuda.synchronize()
+        assert torch.equal(o, ro) and torch.equal(to, rto) and torch.equal(lse, rlse)
+        for n in ajvp.GRAD_NAMES:
+            assert torch.equal(g[n], rg[n]), n
+        # the causal training path: the default local steps are the causal kernels
+        o, to, lse, ctx = ulysses_attn_jvp_train(*(inp[n] for n in names), scale=w.scale, causal=True)
+        g = ulysses_attn_jvp_bwd(ctx, cot["dout"], cot["dtout"])
+        ro, rto, rlse, rmu = ajvp.attn_jvp_fwd_causal_stats(*(inp[n] for n in names), w.scale)
+        rg = ajvp.attn_jvp_bwd_causal(*(inp[n] for n in names), ro, rto, rlse, rmu, cot["dout"], cot["dtout"],
+                                      w.scale)
         torch.cuda.synchronize()
         assert torch.equal(o, ro) and torch.equal(to, rto) and torch.equal(lse, rlse)
         for n in ajvp.GRAD_NAMES:

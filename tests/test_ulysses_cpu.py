@@ -164,3 +164,63 @@ def test_single_rank_backward_is_the_local_call():
     b = _oracle_bwd(*(t[n] for n in names), None, None, None, None, dout, dtout, 0.5)
     for n in b:
         assert torch.equal(a[n], b[n])
+
+
+def _causal_fwd_train(q, k, v, tq, tk, tv, scale):
+    import oracle
+    o, to, lse = (torch.from_numpy(x) for x in oracle.attn_jvp_causal(q, k, v, tq, tk, tv, scale))
+    return o, to, lse, torch.zeros_like(lse)  # the oracle backward recomputes everything it needs
+
+
+def _causal_bwd(q, k, v, tq, tk, tv, o, to, lse, mu, dout, dtout, scale):
+    import oracle
+    g = oracle.attn_jvp_bwd_causal(q, k, v, tq, tk, tv, dout, dtout, scale)
+    return {n: torch.from_numpy(x) for n, x in g.items()}
+
+
+def _causal_worker(rank, world, port, shape, out):
+    # the causal mask needs every row's global position: after the exchange a rank
+    # holds whole sequences in order, so the sharded result equals the unsharded one
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from attention_forward_mode_b200.ulysses import ulysses_attn_jvp_bwd, ulysses_attn_jvp_train
+        B, H, Lq, Lk, d = shape
+        names = ("q", "k", "v", "tq", "tk", "tv")
+        full = _inputs(B, H, Lq, Lk, d, seed=13)
+        g = torch.Generator().manual_seed(14)
+        cot = {n: torch.randn((B, H, Lq, d), generator=g, dtype=torch.float64) for n in ("dout", "dtout")}
+        sq, sk = Lq // world, Lk // world
+        qsl, ksl = slice(rank * sq, (rank + 1) * sq), slice(rank * sk, (rank + 1) * sk)
+        shard = {n: (t[:, :, qsl] if n in ("q", "tq") else t[:, :, ksl]).contiguous() for n, t in full.items()}
+        o, to, lse, ctx = ulysses_attn_jvp_train(*(shard[n] for n in names), scale=0.3, local_fwd=_causal_fwd_train,
+                                                 causal=True)
+        grads = ulysses_attn_jvp_bwd(ctx, cot["dout"][:, :, qsl].contiguous(), cot["dtout"][:, :, qsl].contiguous(),
+                                     local_bwd=_causal_bwd)
+        ro, rto, rlse, _ = _causal_fwd_train(*(full[n] for n in names), 0.3)
+        ref = _causal_bwd(*(full[n] for n in names), None, None, None, None, cot["dout"], cot["dtout"], 0.3)
+        eq = {n: bool(torch.equal(grads[n], ref[n][:, :, qsl if n in ("dq", "dtq") else ksl])) for n in ref}
+        eq["o"] = bool(torch.equal(o, ro[:, :, qsl]))
+        eq["to"] = bool(torch.equal(to, rto[:, :, qsl]))
+        eq["lse"] = bool(torch.equal(lse, rlse[:, :, qsl]))
+        out[rank] = eq
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.timeout(300)
+@pytest.mark.parametrize("world,shape", [(2, (1, 4, 16, 24, 8)), (4, (1, 4, 32, 16, 4))])
+def test_ulysses_causal_matches_unsharded(world, shape):
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as m:
+        out = m.dict()
+        procs = [ctx.Process(target=_causal_worker, args=(r, world, port, shape, out)) for r in range(world)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(240)
+        assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
+        res = dict(out)
+    for r in range(world):
+        assert all(res[r].values()), (r, res[r])
