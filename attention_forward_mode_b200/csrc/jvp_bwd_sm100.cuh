@@ -183,9 +183,8 @@ struct Var {
     static constexpr uint32_t BUF0 = 256u;
     static constexpr uint32_t BUF_COLS = kSingle ? 256u : 128u;
     static constexpr uint32_t X = 0, Y = 64, Z = 128, W = 192;  // inside a buffer (Z, W: V_Q, V_K)
-    // E1, E2 (16 packed columns per group): V_V over each group's own columns of X
-    // and Y; V_Q, V_K both inside each group's own 32 columns of X
-    static constexpr uint32_t E1 = X, E2 = kSingle ? X + 16u : Y;
+    // E1, E2 (16 packed columns per group) over each group's own columns of X and Y
+    static constexpr uint32_t E1 = X, E2 = Y;
     static_assert(BUF0 + kNB * BUF_COLS == 512u, "tensor-memory layout");
 };
 
@@ -539,32 +538,66 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
             const uint32_t st_base =
                 base + C::SM_ST + (uint32_t)(C::kStatsRing ? (j & 1) : s) * STATS_TILE + col0 * 16u;
             const uint32_t tb = tbase + lane_off + C::BUF0 + (uint32_t)b * C::BUF_COLS;
+            const float *stf = reinterpret_cast<const float *>(gbase + (st_base - base));
             uint32_t e1[16], e2[16];
             if (C::kSingle) {
-                // this group's Z and W as soon as the tile's [Z|W] products complete: the
+                // this group's Z and W as soon as the tile's [Z|W] products complete (the
                 // next tile's [Z|W] products overwrite only them and start once they are
-                // read; X and Y once the [X|Y] products complete (the next [X|Y] products
-                // come after this tile's G2, which waits for E_DONE)
-                uint32_t xr[32], yr[32], zr[32], wr[32];
-                tmem_ld32(tb + col0 + C::Z, zr);
-                tmem_ld32(tb + col0 + C::W, wr);
-                tmem_wait_ld();
-                warp_arrive_after_tc(BAR(B_X_FREE));
+                // read), and their statistics terms formed while [X|Y] still runs:
+                //   za = A - a,  wz = B - D - A mu,
+                // so that once X and Y arrive only P = ex2(c S - lse2), u = s Y,
+                // S_bar = P (u za + wz) and dS_bar = P za remain (the critical path of
+                // the tile: the next [X|Y] products follow this tile's G2, which waits
+                // for E_DONE)
+                float za[32], wz[32];
+                {
+                    uint32_t zr[32], wr[32];
+                    tmem_ld32(tb + col0 + C::Z, zr);
+                    tmem_ld32(tb + col0 + C::W, wr);
+                    tmem_wait_ld();
+                    warp_arrive_after_tc(BAR(B_X_FREE));
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const float4 st = C::kColStats ? ld_shared_f4(st_base + 16u * i) : rs;
+                        const float z = __uint_as_float(zr[i]);
+                        za[i] = z - st.z;
+                        wz[i] = fmaf(-z, st.y, __uint_as_float(wr[i]) - st.w);
+                    }
+                }
                 if (!mbar_wait_warp(BAR(B_G1_DONE), j & 1, abort_flag, bound)) {
                     failed = true;
                     continue;
                 }
                 tc_fence_after();
-                tmem_ld32(tb + col0 + C::X, xr);
-                tmem_ld32(tb + col0 + C::Y, yr);
-                tmem_wait_ld();
+                // X and Y in two halves of 16 columns; each half's E1, E2 (8 packed columns
+                // each) go over columns of X and Y that half has already read
 #pragma unroll
-                for (int i = 0; i < 32; i += 2) {
-                    float2 r1, r2;
-                    pair(i, lo, hi, st_base, xr[i], xr[i + 1], yr[i], yr[i + 1], zr[i], zr[i + 1], wr[i], wr[i + 1], r1,
-                         r2);
-                    e1[i / 2] = pack_bf16x2(r1.x, r1.y);
-                    e2[i / 2] = pack_bf16x2(r2.x, r2.y);
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t xr[16], yr[16], h1[8], h2[8];
+                    tmem_ld16(tb + col0 + C::X + 16u * hh, xr);
+                    tmem_ld16(tb + col0 + C::Y + 16u * hh, yr);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 16; i += 2) {
+                        const int c = 16 * hh + i;
+                        // lse2 of columns c, c + 1 (column statistics: read again from the
+                        // slot, which stays valid until E_DONE)
+                        const float2 ls = C::kColStats ? make_float2(stf[4 * c], stf[4 * c + 4]) : make_float2(rs.x, rs.x);
+                        const float2 x = make_float2(__uint_as_float(xr[i]), __uint_as_float(xr[i + 1]));
+                        const float2 tt = __ffma2_rn(x, c2, make_float2(-ls.x, -ls.y));
+                        const float2 pp = make_float2(ex2_approx(tt.x), ex2_approx(tt.y));
+                        const float2 u = __fmul2_rn(make_float2(__uint_as_float(yr[i]), __uint_as_float(yr[i + 1])), s2);
+                        const float2 zz = make_float2(za[c], za[c + 1]);
+                        const float2 pb = __ffma2_rn(u, zz, make_float2(wz[c], wz[c + 1]));
+                        float2 r1 = __fmul2_rn(pp, pb), r2 = __fmul2_rn(pp, zz);
+                        // columns past the end of the tensor, or hidden by the causal mask
+                        if (c >= hi || c < lo) r1.x = r2.x = 0.f;
+                        if (c + 1 >= hi || c + 1 < lo) r1.y = r2.y = 0.f;
+                        h1[i / 2] = pack_bf16x2(r1.x, r1.y);
+                        h2[i / 2] = pack_bf16x2(r2.x, r2.y);
+                    }
+                    tmem_st8(tb + col0 + C::E1 + 8u * hh, h1);
+                    tmem_st8(tb + col0 + C::E2 + 8u * hh, h2);
                 }
             } else {
                 uint32_t xr[32], yr[32];
@@ -579,10 +612,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
                     e2[i / 2] = pack_bf16x2(r2.x, r2.y);
                 }
             }
-            // over this group's own columns (V_Q, V_K: the buffer was read whole above, and
-            // the previous tile's G2, which read E from there, completed before this G1)
-            tmem_st16(tb + col0 + C::E1, e1);
-            tmem_st16(tb + col0 + C::E2, e2);
+            // over this group's own columns of X and Y (the previous tile's G2, which read
+            // E from there, completed before this tile's G1)
+            if (!C::kSingle) {
+                tmem_st16(tb + col0 + C::E1, e1);
+                tmem_st16(tb + col0 + C::E2, e2);
+            }
             tmem_wait_st();
             warp_arrive_after_tc(BAR(B_E_DONE + b));
         }
