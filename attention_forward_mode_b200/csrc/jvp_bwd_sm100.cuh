@@ -35,7 +35,8 @@
 //   V_V  keys     queries  dV, dtV   [X|Y] = K [Q;tQ]^T, Y += tK Q^T      P^T, Pd^T     dV  += E1 dO + E2 dtO
 //                                                                                       dtV += E1 dtO
 //
-//   (X = scores, Y = score tangent without the scale, Z = A, W = B, each 64
+//   (V_V issues its G2 as [dV | dtV] += E1 [dO | dtO], one N = 256 product, and
+//   dV += E2 dtO.  X = scores, Y = score tangent without the scale, Z = A, W = B, each 64
 //   tensor-memory columns per tile; Pd = P .* (u - mu); the elementwise
 //   results E1, E2 are bf16, the A operands of G2.)  V_Q and V_K hold one
 //   set of X, Y, Z, W next to their accumulators: the elementwise warps read
@@ -326,7 +327,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
                     const uint32_t fb = BAR(B_L_FULL + s);
                     constexpr bool kWithStats = C::kColStats && !C::kStatsRing;
                     mbar_arrive_expect_tx(fb, 4 * CHUNK_C + (kWithStats ? STATS_TILE : 0));
-                    load_pair(base + C::long_off(s), &p.tm_l[0], &p.tm_l[1], fb, y);
+                    if (VAR == V_V) {
+                        // only G2 reads it, as one N = 256 operand [x | y]: [x c0 | x c1 | y c0 | y c1]
+                        const uint32_t st = base + C::long_off(s);
+                        tma_load_3d(st, &p.tm_l[0], fb, 0, y, bh);
+                        tma_load_3d(st + CHUNK_C, &p.tm_l[0], fb, 64, y, bh);
+                        tma_load_3d(st + 2 * CHUNK_C, &p.tm_l[1], fb, 0, y, bh);
+                        tma_load_3d(st + 3 * CHUNK_C, &p.tm_l[1], fb, 64, y, bh);
+                    } else {
+                        load_pair(base + C::long_off(s), &p.tm_l[0], &p.tm_l[1], fb, y);
+                    }
                     if (kWithStats)  // padded by BN rows past the last head: never out of bounds
                         bulk_load(base + C::SM_ST + s * STATS_TILE, p.stats + (size_t)bh * p.Lq + y, STATS_TILE, fb);
                     l_last[s] = t;
@@ -371,6 +381,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
             constexpr uint32_t ID_W = idesc_bf16_f32(128, 128, 0);  // R [Cx; Cy]^T
             constexpr uint32_t ID_N = idesc_bf16_f32(128, 64, 0);   // R Cx^T
             constexpr uint32_t ID_G2 = idesc_bf16_f32(128, 128, 1);  // E C (C read MN-major)
+            constexpr uint32_t ID_G2W = idesc_bf16_f32(128, 256, 1);  // V_V: E1 [L0 | L1]
             // descriptors of the resident tiles, as scalars (an array captured by the
             // lambdas below would live in local memory and delay every MMA issue)
             const uint64_t dr0 = smem_desc_sw128(base + SM_R, 16, 1024);
@@ -429,25 +440,28 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
                 if (!C::kSingle && !wait_full(B_L_FULL, j, C::kLS)) return false;  // V_V: only G2 reads it
                 const int b = j % C::kNB, s = j % C::kLS;
                 const uint32_t tb = tbase + C::BUF0 + (uint32_t)b * C::BUF_COLS;
-                // MN-major views of the long-ring tiles: chunks L_CH apart (LBO), 8 rows 1024 B apart
-                const uint64_t m0 = smem_desc_sw128(base + C::long_off(s), C::L_CH, 1024);
-                const uint64_t m1 = desc_add(m0, CHUNK_C);
                 const uint32_t e1 = tb + C::E1, e2 = tb + C::E2;
-                auto g2 = [&](uint32_t acc, uint32_t e, uint64_t bm, bool first) {
+                auto g2 = [&](uint32_t acc, uint32_t e, uint64_t bm, uint32_t id, bool first) {
 #pragma unroll
                     for (int kk = 0; kk < BN / 16; ++kk) {
                         // streamed items 16kk..16kk+15: group kk / 2's columns, 8 packed per K-step
                         const uint32_t a_col = (kk >> 1) * 32u + (kk & 1) * 8u;
-                        mma_ts(tbase + acc, e + a_col, desc_add(bm, kk * 2048), ID_G2,
-                               (!first || j > 0 || kk > 0) ? 1u : 0u);
+                        mma_ts(tbase + acc, e + a_col, desc_add(bm, kk * 2048), id, (!first || j > 0 || kk > 0) ? 1u : 0u);
                     }
                 };
-                g2(0, e1, m0, true);       // acc0 += E1 L0
-                g2(0, e2, m1, false);      //       + E2 L1
-                if (VAR == V_V)
-                    g2(128, e1, m1, true);  // dtV += E1 L1
-                else
-                    g2(128, e2, m0, true);  // dtQ / dtK += E2 L0
+                if (VAR == V_V) {
+                    // MN-major [L0 | L1]: 64-column chunks CHUNK_C apart (LBO), 8 rows 1024 B apart
+                    const uint64_t mw = smem_desc_sw128(base + C::long_off(s), CHUNK_C, 1024);
+                    g2(0, e1, mw, ID_G2W, true);                         // [dV | dtV] += E1 [L0 | L1]
+                    g2(0, e2, desc_add(mw, 2 * CHUNK_C), ID_G2, false);  // dV += E2 L1
+                } else {
+                    // MN-major views of the long-ring tiles: chunks L_CH apart (LBO), 8 rows 1024 B apart
+                    const uint64_t m0 = smem_desc_sw128(base + C::long_off(s), C::L_CH, 1024);
+                    const uint64_t m1 = desc_add(m0, CHUNK_C);
+                    g2(0, e1, m0, ID_G2, true);    // acc0 += E1 L0
+                    g2(0, e2, m1, ID_G2, false);   //       + E2 L1
+                    g2(128, e2, m0, ID_G2, true);  // dtQ / dtK += E2 L0
+                }
                 mma_commit(BAR(B_G2_DONE + s));
                 return true;
             };
