@@ -47,12 +47,14 @@
 // runs only a handful of key tiles): one CTA per SM walks the units
 // (query tile, batch*head) blockIdx.x, blockIdx.x + gridDim.x, ..., and every
 // ring, buffer and barrier phase follows one CTA-wide tile counter G = n*nk + j
-// (unit n, key tile j).  The epilogue writes O and tO with plain stores
-// (staged per warp in a 2 KB slot of its own, not in Q / tQ), so Q / tQ
-// shared memory is refilled for unit n+1 as soon as the last S/dS'
-// products of unit n are complete, and the next unit's first score products
-// run while the softmax warps finish the epilogue; the next unit's first
-// P.V waits for the epilogue to have read O / T (B_OT_FREE).
+// (unit n, key tile j).  The epilogue stages O and tO in the V-side ring
+// (whose tiles are dead once every product of the unit is complete) and warp
+// 3 stores them with the tensor-store unit, so Q / tQ shared memory is
+// refilled for unit n+1 as soon as the last S/dS' products of unit n are
+// complete, and the next unit's first score products run during the
+// epilogue; the producer loads unit n+1's first V tiles once the stores have
+// read the staging (B_STG_FREE), and the next unit's first P.V waits for the
+// epilogue to have read O / T (B_OT_FREE).
 #pragma once
 
 #include "ptx_sm100.cuh"
@@ -99,8 +101,10 @@ enum : int {
     B_P_FULL = 9,    // + buffer
     B_O_FULL = 11,   // every MMA of the unit has completed (one phase per unit)
     B_MMA_DRAIN = 12,
-    B_OT_FREE = 13,  // persistent: the epilogue has read O / T (one arrival per softmax warp)
-    N_BARS = 14
+    B_OT_FREE = 13,   // persistent: the epilogue has read O / T (one arrival per softmax warp)
+    B_STG_FULL = 14,  // persistent: O, tO staged in the V-side ring (one arrival per softmax warp)
+    B_STG_FREE = 15,  // persistent: + 0 the stores have read O's stage, + 1 tO's as well
+    N_BARS = 17
 };
 static_assert(STAGES == 2, "the K-side ring reuses the two S/dS' buffer barriers");
 constexpr uint32_t OFF_TMEM_SLOT = 8 * N_BARS;     // u32
@@ -259,6 +263,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
     const uint64_t bound = p.bound_ns;
     // persistent: the n-th unit of this CTA (unit 0 is blockIdx.x, decoded above);
     // false past the last one, else its query tile and outer index
+    // persistent: unit n's staged O goes to the V-side stage of unit n + 1's first
+    // key tile (G = (n + 1) * nk), tO to the other stage
+    auto stage_o = [&](int n) -> uint32_t { return SM_VT + (uint32_t)(((n + 1) * nk) % STAGES) * VT_STAGE; };
     auto next_unit = [&](int n, int &qt_n, int &bh_n) -> bool {
         const long long u = (long long)blockIdx.x + (long long)n * (long long)gridDim.x;
         if (u >= (long long)p.n_units) return false;
@@ -286,6 +293,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
         mbar_init(BAR(B_O_FULL), 1);
         mbar_init(BAR(B_MMA_DRAIN), 1);
         mbar_init(BAR(B_OT_FREE), SOFTMAX_THREADS / 32);
+        mbar_init(BAR(B_STG_FULL), SOFTMAX_THREADS / 32);
+        mbar_init(BAR(B_STG_FREE), 1);
+        mbar_init(BAR(B_STG_FREE + 1), 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -352,6 +362,20 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                         const int i = G0 + t - 1;
                         const int s = i % STAGES;
                         if (!mbar_wait(BAR(B_VT_EMPTY + s), ((i / STAGES) & 1) ^ 1, abort_flag, bound)) {
+                            ok = false;
+                            break;
+                        }
+                        // persistent: the V-side ring held the previous unit's staged outputs,
+                        // O in the stage of this unit's first V tile (stored first), tO in
+                        // the other (a unit of one key tile waits for both: this unit's
+                        // epilogue stages into them only after its own P.V completes)
+                        if (kPersist && n > 0 && t <= 2 &&
+                            !mbar_wait(BAR(B_STG_FREE + (t - 1)), (n - 1) & 1, abort_flag, bound)) {
+                            ok = false;
+                            break;
+                        }
+                        if (kPersist && n > 0 && t == 1 && nk == 1 &&
+                            !mbar_wait(BAR(B_STG_FREE + 1), (n - 1) & 1, abort_flag, bound)) {
                             ok = false;
                             break;
                         }
@@ -468,6 +492,31 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
             // every MMA issued must finish before tensor memory is released
             mma_commit(BAR(B_MMA_DRAIN));
             mbar_wait_drain(BAR(B_MMA_DRAIN), 0, bound);
+        }
+        __syncwarp();
+    } else if (kPersist && warp == 3) {
+        // ------------------------------------- persistent: output tensor stores
+        // each unit's O and tO, staged by the softmax warps in the V-side ring, go out
+        // through the tensor-store unit; once the stores have read the staging the
+        // producer may load the next unit's V tiles there
+        if (lane == 0) {
+            int n = 0, qt_n = qt, bh_n = bh;
+            do {
+                if (!mbar_wait(BAR(B_STG_FULL), n & 1, abort_flag, bound) || *abort_flag != 0) break;
+                const int yq_n = yq0 + qt_n * BR;
+                const uint32_t so = stage_o(n), st = SM_VT + VT_STAGE - (so - SM_VT);
+                tma_store_3d(&p.tm_o, base + so, 0, yq_n, bh_n);
+                tma_store_3d(&p.tm_o, base + so + CHUNK_Q, 64, yq_n, bh_n);
+                tma_store_commit();
+                tma_store_3d(&p.tm_to, base + st, 0, yq_n, bh_n);
+                tma_store_3d(&p.tm_to, base + st + CHUNK_Q, 64, yq_n, bh_n);
+                tma_store_commit();
+                tma_store_wait_read_1();  // O's stage read: the next unit's first V tile may land there
+                mbar_arrive(BAR(B_STG_FREE));
+                tma_store_wait_read_all();
+                mbar_arrive(BAR(B_STG_FREE + 1));
+            } while (next_unit(++n, qt_n, bh_n));
+            tma_store_wait_all();  // the last stores complete before the CTA exits
         }
         __syncwarp();
     } else if (warp >= 4) {
@@ -693,9 +742,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                         wo[i] = pack_bf16x2(o0, o1);
                         wt[i] = pack_bf16x2(t0, t1);
                     }
-                    if (kPacked || kPersist) {
-                        // plain stores, staged per warp (packed: rows past the sequence
-                        // belong to the next one and are not written)
+                    if (kPacked) {
+                        // plain stores, staged per warp (rows past the sequence belong to
+                        // the next one and are not written)
                         const size_t off =
                             ((size_t)bh_n * (size_t)p.Lq + (size_t)(yq_n + wl * 32)) * HD + 64u * grp + 32u * h;
                         const int rows_left = Lq_s - (q0_n + wl * 32);
@@ -704,14 +753,18 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                         store_rows_32x32(slot, wt, p.to_bf + off, rows_left, (uint32_t)lane);
                         continue;
                     }
+                    // staging in the store maps' 128-byte-swizzled layout: Q / tQ shared
+                    // memory (persistent form: the V-side ring, O in stage 0, tO in stage 1)
                     const uint32_t chunk_off = (uint32_t)grp * CHUNK_Q + (uint32_t)row * 128u;
                     const uint32_t unit0 = (uint32_t)h * 4u;
+                    const uint32_t so = kPersist ? stage_o(n) : SM_Q;
+                    const uint32_t st = kPersist ? SM_VT + VT_STAGE - (so - SM_VT) : SM_TQ;
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
                         const uint32_t phys = (((unit0 + u) ^ (uint32_t)(row & 7)) * 16u);
-                        st_shared_v4(base + SM_Q + chunk_off + phys, wo[4 * u], wo[4 * u + 1], wo[4 * u + 2],
+                        st_shared_v4(base + so + chunk_off + phys, wo[4 * u], wo[4 * u + 1], wo[4 * u + 2],
                                      wo[4 * u + 3]);
-                        st_shared_v4(base + SM_TQ + chunk_off + phys, wt[4 * u], wt[4 * u + 1], wt[4 * u + 2],
+                        st_shared_v4(base + st + chunk_off + phys, wt[4 * u], wt[4 * u + 1], wt[4 * u + 2],
                                      wt[4 * u + 3]);
                     }
                 }
@@ -722,7 +775,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                 if (grp == 1 && p.mu != nullptr && q0_n + row < Lq_s)
                     p.mu[(size_t)bh_n * (size_t)p.Lq + (size_t)(yq_n + row)] = mu;
             }
-            if (!kPersist) {
+            if (kPersist) {
+                // staging complete: one arrival per warp for the storing warp
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0 && !any_failed) mbar_arrive(BAR(B_STG_FULL));
+            } else {
                 fence_proxy_async_smem();
                 named_bar_sync(NB_EPI, SOFTMAX_THREADS);  // staging complete (every softmax thread gets here)
                 if (!kSplit && !kPacked && warp == 4 && lane == 0 && !any_failed && *abort_flag == 0) {
