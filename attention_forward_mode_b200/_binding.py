@@ -30,6 +30,7 @@ AJVP_ERR_DEVICE_LAYOUT = -9
 # every symbol the header declares
 EXPORTED = ("attn_jvp_fwd", "attn_jvp_fwd_causal", "attn_jvp_fwd_varlen", "attn_jvp_fwd_f32out", "attn_jvp_fwd_stats", "attn_jvp_fwd_causal_stats", "attn_jvp_bwd", "attn_jvp_bwd_step",
             "attn_jvp_bwd_causal", "attn_jvp_fwd_varlen_stats", "attn_jvp_bwd_varlen",
+            "attn_jvp_fwd_f32out_causal", "attn_jvp_fwd_f32out_varlen",
             "attn_jvp_bwd_workspace_bytes", "attn_jvp_fwd_f32", "attn_jvp_fwd_host",
             "attn_jvp_fwd_host_noalloc", "attn_jvp_host_workspace_bytes", "attn_jvp_bwd_host",
             "attn_jvp_bwd_host_workspace_bytes", "attn_jvp_strerror",
@@ -67,6 +68,10 @@ def load_library(path: str = LIB_PATH):
         lib.attn_jvp_fwd_f32out.restype = ctypes.c_int
         lib.attn_jvp_fwd_causal.argtypes = fwd_args
         lib.attn_jvp_fwd_causal.restype = ctypes.c_int
+        lib.attn_jvp_fwd_f32out_causal.argtypes = fwd_args
+        lib.attn_jvp_fwd_f32out_causal.restype = ctypes.c_int
+        lib.attn_jvp_fwd_f32out_varlen.argtypes = [vp] * 11 + [i64] * 6 + [f32, ctypes.c_int, vp]
+        lib.attn_jvp_fwd_f32out_varlen.restype = ctypes.c_int
         lib.attn_jvp_fwd_varlen.argtypes = [vp] * 11 + [i64] * 6 + [f32, ctypes.c_int, vp]
         lib.attn_jvp_fwd_varlen.restype = ctypes.c_int
         lib.attn_jvp_fwd_stats.argtypes = [vp] * 10 + [i64] * 5 + [f32, vp]
@@ -186,14 +191,24 @@ def attn_jvp_fwd(q, k, v, tq, tk, tv, scale=None, o=None, to=None, lse=None, str
 def attn_jvp_fwd_f32out(q, k, v, tq, tk, tv, scale=None, o=None, to=None, lse=None, stream=None, want_lse=True):
     """bf16 inputs, fp32 O and tO, through ``attn_jvp_fwd_f32out`` (tcgen05
     kernel with split-bf16 probability operands; d = 128)."""
+    return _fwd_f32out("attn_jvp_fwd_f32out", q, k, v, tq, tk, tv, scale, o, to, lse, stream, want_lse)
+
+
+def attn_jvp_fwd_f32out_causal(q, k, v, tq, tk, tv, scale=None, o=None, to=None, lse=None, stream=None,
+                               want_lse=True):
+    """``attn_jvp_fwd_f32out`` with the causal mask of ``attn_jvp_fwd_causal``."""
+    return _fwd_f32out("attn_jvp_fwd_f32out_causal", q, k, v, tq, tk, tv, scale, o, to, lse, stream, want_lse)
+
+
+def _fwd_f32out(entry, q, k, v, tq, tk, tv, scale, o, to, lse, stream, want_lse):
     o, to, lse, (B, H, Lq, Lk, d) = _prepare(q, k, v, tq, tk, tv, o, to, lse, torch.bfloat16, want_lse,
                                             out_dtype=torch.float32)
     if scale is None:
         scale = d ** -0.5
     lib = load_library()
-    rc = lib.attn_jvp_fwd_f32out(_ptr(q), _ptr(k), _ptr(v), _ptr(tq), _ptr(tk), _ptr(tv), _ptr(o), _ptr(to),
-                                 _ptr(lse), B, H, Lq, Lk, d, float(scale), _stream_handle(stream))
-    _check(rc, "attn_jvp_fwd_f32out")
+    rc = getattr(lib, entry)(_ptr(q), _ptr(k), _ptr(v), _ptr(tq), _ptr(tk), _ptr(tv), _ptr(o), _ptr(to),
+                             _ptr(lse), B, H, Lq, Lk, d, float(scale), _stream_handle(stream))
+    _check(rc, entry)
     return o, to, lse
 
 
@@ -225,6 +240,27 @@ def attn_jvp_fwd_varlen(q, k, v, tq, tk, tv, cu_seqlens_q, cu_seqlens_k, max_seq
                                  _ptr(lse), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), cu_seqlens_q.numel() - 1, H, Tq,
                                  Tk, int(max_seqlen_q), d, float(scale), int(bool(causal)), _stream_handle(stream))
     _check(rc, "attn_jvp_fwd_varlen")
+    return o, to, lse
+
+
+def attn_jvp_fwd_f32out_varlen(q, k, v, tq, tk, tv, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, scale=None,
+                               causal=False, o=None, to=None, lse=None, stream=None, want_lse=True):
+    """``attn_jvp_fwd_varlen`` with fp32 O and tO (split-bf16 probability
+    operands, as ``attn_jvp_fwd_f32out``).  Returns (o, to, lse)."""
+    if o is None:
+        o = torch.empty(q.shape, device=q.device, dtype=torch.float32)
+    if to is None:
+        to = torch.empty(q.shape, device=q.device, dtype=torch.float32)
+    o, to, lse, (H, Tq, Tk, d) = _prepare_varlen(q, k, v, tq, tk, tv, cu_seqlens_q, cu_seqlens_k, o, to, lse,
+                                                 want_lse, out_dtype=torch.float32)
+    if scale is None:
+        scale = d ** -0.5
+    lib = load_library()
+    rc = lib.attn_jvp_fwd_f32out_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(tq), _ptr(tk), _ptr(tv), _ptr(o), _ptr(to),
+                                        _ptr(lse), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), cu_seqlens_q.numel() - 1,
+                                        H, Tq, Tk, int(max_seqlen_q), d, float(scale), int(bool(causal)),
+                                        _stream_handle(stream))
+    _check(rc, "attn_jvp_fwd_f32out_varlen")
     return o, to, lse
 
 
@@ -286,7 +322,7 @@ def attn_jvp_bwd_varlen(q, k, v, tq, tk, tv, o, to, lse, mu, dout, dtout, cu_seq
     return grads
 
 
-def _prepare_varlen(q, k, v, tq, tk, tv, cu_seqlens_q, cu_seqlens_k, o, to, lse, want_lse):
+def _prepare_varlen(q, k, v, tq, tk, tv, cu_seqlens_q, cu_seqlens_k, o, to, lse, want_lse, out_dtype=None):
     for name, x in (("q", q), ("k", k), ("v", v), ("tq", tq), ("tk", tk), ("tv", tv)):
         if not isinstance(x, torch.Tensor) or not x.is_cuda or x.dtype != torch.bfloat16 or x.dim() != 3 \
                 or not x.is_contiguous():
@@ -307,9 +343,10 @@ def _prepare_varlen(q, k, v, tq, tk, tv, cu_seqlens_q, cu_seqlens_k, o, to, lse,
         to = torch.empty_like(q)
     if want_lse and lse is None:
         lse = torch.empty((H, Tq), device=q.device, dtype=torch.float32)
+    out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
     for name, x in (("o", o), ("to", to)):
-        if x.shape != q.shape or x.dtype != torch.bfloat16 or not x.is_contiguous() or not x.is_cuda:
-            raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor of shape {tuple(q.shape)}")
+        if x.shape != q.shape or x.dtype != out_dtype or not x.is_contiguous() or not x.is_cuda:
+            raise ValueError(f"{name} must be a contiguous CUDA {out_dtype} tensor of shape {tuple(q.shape)}")
     if lse is not None and (lse.shape != (H, Tq) or lse.dtype != torch.float32 or not lse.is_contiguous()):
         raise ValueError("lse must be a contiguous float32 [H, total_q] tensor")
     return o, to, lse, (H, Tq, Tk, d)

@@ -112,6 +112,9 @@ int device_setup(int *dev_out) {
         if (e3 == cudaSuccess) e3 = set_fwd_smem<false, 1>();
         if (e3 == cudaSuccess) e3 = set_fwd_smem<false, 2>();
         if (e3 == cudaSuccess) e3 = set_fwd_smem<false, 3>();
+        if (e3 == cudaSuccess) e3 = set_fwd_smem<true, 1>();
+        if (e3 == cudaSuccess) e3 = set_fwd_smem<true, 2>();
+        if (e3 == cudaSuccess) e3 = set_fwd_smem<true, 3>();
         if (e3 == cudaSuccess) e3 = set_bwd_smem<ajvp::bwd::V_Q>();
         if (e3 == cudaSuccess) e3 = set_bwd_smem<ajvp::bwd::V_K>();
         if (e3 == cudaSuccess) e3 = set_bwd_smem<ajvp::bwd::V_V>();
@@ -418,6 +421,31 @@ struct HostPipe {
     }
 };
 
+// packed sequences, bf16 or fp32 outputs (kSplit), optionally causal and saving mu
+template <bool kSplit>
+int launch_varlen(const void *q, const void *k, const void *v, const void *tq, const void *tk, const void *tv,
+                  void *o, void *to, float *lse, float *mu, const int32_t *cu_seqlens_q,
+                  const int32_t *cu_seqlens_k, int64_t n_seq, int64_t H, int64_t total_q, int64_t total_k,
+                  int64_t max_seqlen_q, int64_t d, float scale, int causal, void *stream) {
+    if (n_seq < 0 || max_seqlen_q < 0) return AJVP_ERR_INVALID_ARG;
+    if (n_seq == 0 || max_seqlen_q == 0) {
+        // nothing to compute; the size checks still apply
+        if (H < 0 || total_q < 0 || total_k < 1 || d < 1 || !std::isfinite(scale)) return AJVP_ERR_INVALID_ARG;
+        return AJVP_OK;
+    }
+    if (!cu_seqlens_q || !cu_seqlens_k) return AJVP_ERR_INVALID_ARG;
+    if (!aligned(cu_seqlens_q, 4) || !aligned(cu_seqlens_k, 4)) return AJVP_ERR_MISALIGNED;
+    if (n_seq >= (int64_t(1) << 31) || max_seqlen_q > total_q) return AJVP_ERR_INVALID_ARG;
+    const int64_t max_qtiles = (max_seqlen_q + ajvp::sm100::BR - 1) / ajvp::sm100::BR;
+    if (causal)
+        return launch_sm100<kSplit, ajvp::sm100::MASK_PACKED | ajvp::sm100::MASK_CAUSAL>(
+            q, k, v, tq, tk, tv, o, to, lse, 1, H, total_q, total_k, d, scale, stream, mu, cu_seqlens_q,
+            cu_seqlens_k, n_seq, max_qtiles);
+    return launch_sm100<kSplit, ajvp::sm100::MASK_PACKED>(q, k, v, tq, tk, tv, o, to, lse, 1, H, total_q, total_k, d,
+                                                           scale, stream, mu, cu_seqlens_q, cu_seqlens_k, n_seq,
+                                                           max_qtiles);
+}
+
 }  // namespace
 
 extern "C" {
@@ -445,23 +473,24 @@ int attn_jvp_fwd_varlen(const void *q, const void *k, const void *v, const void 
                         void *o, void *to, float *lse, const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
                         int64_t n_seq, int64_t H, int64_t total_q, int64_t total_k, int64_t max_seqlen_q, int64_t d,
                         float scale, int causal, void *stream) {
-    if (n_seq < 0 || max_seqlen_q < 0) return AJVP_ERR_INVALID_ARG;
-    if (n_seq == 0 || max_seqlen_q == 0) {
-        // nothing to compute; the size checks still apply
-        if (H < 0 || total_q < 0 || total_k < 1 || d < 1 || !std::isfinite(scale)) return AJVP_ERR_INVALID_ARG;
-        return AJVP_OK;
-    }
-    if (!cu_seqlens_q || !cu_seqlens_k) return AJVP_ERR_INVALID_ARG;
-    if (!aligned(cu_seqlens_q, 4) || !aligned(cu_seqlens_k, 4)) return AJVP_ERR_MISALIGNED;
-    if (n_seq >= (int64_t(1) << 31) || max_seqlen_q > total_q) return AJVP_ERR_INVALID_ARG;
-    const int64_t max_qtiles = (max_seqlen_q + ajvp::sm100::BR - 1) / ajvp::sm100::BR;
-    if (causal)
-        return launch_sm100<false, ajvp::sm100::MASK_PACKED | ajvp::sm100::MASK_CAUSAL>(
-            q, k, v, tq, tk, tv, o, to, lse, 1, H, total_q, total_k, d, scale, stream, nullptr, cu_seqlens_q,
-            cu_seqlens_k, n_seq, max_qtiles);
-    return launch_sm100<false, ajvp::sm100::MASK_PACKED>(q, k, v, tq, tk, tv, o, to, lse, 1, H, total_q, total_k, d,
-                                                          scale, stream, nullptr, cu_seqlens_q, cu_seqlens_k, n_seq,
-                                                          max_qtiles);
+    return launch_varlen<false>(q, k, v, tq, tk, tv, o, to, lse, nullptr, cu_seqlens_q, cu_seqlens_k, n_seq, H,
+                                total_q, total_k, max_seqlen_q, d, scale, causal, stream);
+}
+
+int attn_jvp_fwd_f32out_causal(const void *q, const void *k, const void *v, const void *tq, const void *tk,
+                               const void *tv, float *o, float *to, float *lse, int64_t B, int64_t H, int64_t Lq,
+                               int64_t Lk, int64_t d, float scale, void *stream) {
+    return launch_sm100<true, ajvp::sm100::MASK_CAUSAL>(q, k, v, tq, tk, tv, o, to, lse, B, H, Lq, Lk, d, scale,
+                                                         stream);
+}
+
+int attn_jvp_fwd_f32out_varlen(const void *q, const void *k, const void *v, const void *tq, const void *tk,
+                               const void *tv, float *o, float *to, float *lse, const int32_t *cu_seqlens_q,
+                               const int32_t *cu_seqlens_k, int64_t n_seq, int64_t H, int64_t total_q,
+                               int64_t total_k, int64_t max_seqlen_q, int64_t d, float scale, int causal,
+                               void *stream) {
+    return launch_varlen<true>(q, k, v, tq, tk, tv, o, to, lse, nullptr, cu_seqlens_q, cu_seqlens_k, n_seq, H,
+                               total_q, total_k, max_seqlen_q, d, scale, causal, stream);
 }
 
 int attn_jvp_fwd_stats(const void *q, const void *k, const void *v, const void *tq, const void *tk, const void *tv,
@@ -588,23 +617,9 @@ int attn_jvp_fwd_varlen_stats(const void *q, const void *k, const void *v, const
                               const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k, int64_t n_seq, int64_t H,
                               int64_t total_q, int64_t total_k, int64_t max_seqlen_q, int64_t d, float scale,
                               int causal, void *stream) {
-    if (n_seq < 0 || max_seqlen_q < 0) return AJVP_ERR_INVALID_ARG;
-    if (n_seq == 0 || max_seqlen_q == 0) {
-        if (H < 0 || total_q < 0 || total_k < 1 || d < 1 || !std::isfinite(scale)) return AJVP_ERR_INVALID_ARG;
-        return AJVP_OK;
-    }
-    if (H > 0 && total_q > 0 && (!lse || !mu)) return AJVP_ERR_INVALID_ARG;
-    if (!cu_seqlens_q || !cu_seqlens_k) return AJVP_ERR_INVALID_ARG;
-    if (!aligned(cu_seqlens_q, 4) || !aligned(cu_seqlens_k, 4)) return AJVP_ERR_MISALIGNED;
-    if (n_seq >= (int64_t(1) << 31) || max_seqlen_q > total_q) return AJVP_ERR_INVALID_ARG;
-    const int64_t max_qtiles = (max_seqlen_q + ajvp::sm100::BR - 1) / ajvp::sm100::BR;
-    if (causal)
-        return launch_sm100<false, ajvp::sm100::MASK_PACKED | ajvp::sm100::MASK_CAUSAL>(
-            q, k, v, tq, tk, tv, o, to, lse, 1, H, total_q, total_k, d, scale, stream, mu, cu_seqlens_q,
-            cu_seqlens_k, n_seq, max_qtiles);
-    return launch_sm100<false, ajvp::sm100::MASK_PACKED>(q, k, v, tq, tk, tv, o, to, lse, 1, H, total_q, total_k, d,
-                                                          scale, stream, mu, cu_seqlens_q, cu_seqlens_k, n_seq,
-                                                          max_qtiles);
+    if (n_seq > 0 && max_seqlen_q > 0 && H > 0 && total_q > 0 && (!lse || !mu)) return AJVP_ERR_INVALID_ARG;
+    return launch_varlen<false>(q, k, v, tq, tk, tv, o, to, lse, mu, cu_seqlens_q, cu_seqlens_k, n_seq, H, total_q,
+                                total_k, max_seqlen_q, d, scale, causal, stream);
 }
 
 int attn_jvp_bwd_varlen(const void *q, const void *k, const void *v, const void *tq, const void *tk,

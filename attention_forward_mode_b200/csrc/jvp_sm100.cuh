@@ -168,7 +168,6 @@ constexpr int MASK_CAUSAL = 1, MASK_PACKED = 2;
 //                 O and T, and O, tO are written in fp32; 1.5x the MMA work.
 template <bool kSplit, int MASK = 0, bool kPersist = false>
 __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_constant__ Params p) {
-    static_assert(!kSplit || MASK == 0, "the fp32-output variant has no masks");
     static_assert(!kPersist || (!kSplit && MASK == 0), "the persistent form is the unmasked bf16 kernel");
     constexpr bool kCausal = (MASK & MASK_CAUSAL) != 0, kPacked = (MASK & MASK_PACKED) != 0;
     extern __shared__ uint8_t smem_raw[];
@@ -252,20 +251,22 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
         // no row of the tile sees a key: zeros and lse = -inf, no pipeline at all
         for (int r = threadIdx.x; r < BR && q0 + r < Lq_s; r += blockDim.x) {
             const size_t row = (size_t)bh * (size_t)p.Lq + (size_t)(yq + r);
-            uint4 *po = reinterpret_cast<uint4 *>(p.o_bf + row * HD);
-            uint4 *pt = reinterpret_cast<uint4 *>(p.to_bf + row * HD);
-            for (int u = 0; u < HD / 8; ++u) po[u] = pt[u] = make_uint4(0u, 0u, 0u, 0u);
+            // 16-byte words per output row: 128 bf16 or 128 fp32
+            constexpr int kWords = kSplit ? HD / 4 : HD / 8;
+            uint4 *po = kSplit ? reinterpret_cast<uint4 *>(p.o_f32 + row * HD) : reinterpret_cast<uint4 *>(p.o_bf + row * HD);
+            uint4 *pt = kSplit ? reinterpret_cast<uint4 *>(p.to_f32 + row * HD) : reinterpret_cast<uint4 *>(p.to_bf + row * HD);
+            for (int u = 0; u < kWords; ++u) po[u] = pt[u] = make_uint4(0u, 0u, 0u, 0u);
             if (p.lse) p.lse[row] = -INFINITY;
             if (p.mu) p.mu[row] = 0.f;
         }
         return;
     }
     const uint64_t bound = p.bound_ns;
-    // persistent: the n-th unit of this CTA (unit 0 is blockIdx.x, decoded above);
-    // false past the last one, else its query tile and outer index
     // persistent: unit n's staged O goes to the V-side stage of unit n + 1's first
     // key tile (G = (n + 1) * nk), tO to the other stage
     auto stage_o = [&](int n) -> uint32_t { return SM_VT + (uint32_t)(((n + 1) * nk) % STAGES) * VT_STAGE; };
+    // persistent: the n-th unit of this CTA (unit 0 is blockIdx.x, decoded above);
+    // false past the last one, else its query tile and outer index
     auto next_unit = [&](int n, int &qt_n, int &bh_n) -> bool {
         const long long u = (long long)blockIdx.x + (long long)n * (long long)gridDim.x;
         if (u >= (long long)p.n_units) return false;
@@ -694,8 +695,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                 // group grp writes output columns 64*grp .. 64*grp+63
                 if (kSplit) {
                     // fp32 outputs straight from registers, 16 bytes per store
-                    const bool row_ok = q0_n + row < p.Lq;
-                    const size_t off = ((size_t)bh_n * (size_t)p.Lq + (size_t)(q0_n + row)) * HD + 64u * (uint32_t)grp;
+                    // (packed: rows past the sequence belong to the next one and are not written)
+                    const bool row_ok = q0_n + row < Lq_s;
+                    const size_t off = ((size_t)bh_n * (size_t)p.Lq + (size_t)(yq_n + row)) * HD + 64u * (uint32_t)grp;
 #pragma unroll 1
                     for (int h = 0; h < 2; ++h) {
                         const int pc = 2 * grp + h;

@@ -133,6 +133,19 @@ AJVP_API int attn_jvp_fwd_causal(const void *q, const void *k, const void *v,
                         float scale, void *stream);
 
 /*
+ * attn_jvp_fwd_f32out_causal -- attn_jvp_fwd_f32out with the causal mask of
+ * attn_jvp_fwd_causal (rows that see no key: O = tO = 0, lse = -infinity);
+ * arguments and rules as attn_jvp_fwd_f32out.  The pages describe neither
+ * masks nor this variant; it is the masked definition with the tangent
+ * carried as attn_jvp_fwd_f32out carries it.
+ */
+AJVP_API int attn_jvp_fwd_f32out_causal(const void *q, const void *k, const void *v,
+                        const void *tq, const void *tk, const void *tv,
+                        float *o, float *to, float *lse,
+                        int64_t B, int64_t H, int64_t Lq, int64_t Lk, int64_t d,
+                        float scale, void *stream);
+
+/*
  * attn_jvp_fwd_varlen -- packed variable-length sequences (for example text
  * conditions of different lengths in one batch), optionally causal.
  *
@@ -159,6 +172,20 @@ AJVP_API int attn_jvp_fwd_causal(const void *q, const void *k, const void *v,
 AJVP_API int attn_jvp_fwd_varlen(const void *q, const void *k, const void *v,
                         const void *tq, const void *tk, const void *tv,
                         void *o, void *to, float *lse,
+                        const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                        int64_t n_seq, int64_t H, int64_t total_q, int64_t total_k,
+                        int64_t max_seqlen_q, int64_t d, float scale, int causal,
+                        void *stream);
+
+/*
+ * attn_jvp_fwd_f32out_varlen -- attn_jvp_fwd_varlen with fp32 outputs
+ * o, to (float [H][total_q][d]), as attn_jvp_fwd_f32out computes them;
+ * other arguments and rules as attn_jvp_fwd_varlen (rows past a sequence's
+ * end are never written, empty rows give zeros and lse = -infinity).
+ */
+AJVP_API int attn_jvp_fwd_f32out_varlen(const void *q, const void *k, const void *v,
+                        const void *tq, const void *tk, const void *tv,
+                        float *o, float *to, float *lse,
                         const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
                         int64_t n_seq, int64_t H, int64_t total_q, int64_t total_k,
                         int64_t max_seqlen_q, int64_t d, float scale, int causal,

@@ -97,3 +97,59 @@ def test_zero_tangent_exact_zero():
         inp[n].zero_()
     _, to, _ = run_f32out(inp, w.scale)
     assert torch.count_nonzero(to).item() == 0
+
+
+def _masked_err(got, ref, seen):
+    o, to, lse = (x.float().cpu().numpy() for x in got)
+    ro, rto, rlse = ref
+    err = {"o": max_rel(o[seen], ro[seen]), "to": max_rel(to[seen], rto[seen]),
+           "lse": max_rel(lse[seen], rlse[seen])}
+    empty = ~seen
+    if empty.any():
+        assert np.all(o[empty] == 0) and np.all(to[empty] == 0) and np.all(np.isneginf(lse[empty]))
+    return err
+
+
+@pytest.mark.parametrize("B,H,Lq,Lk", [(1, 2, 200, 200), (1, 2, 129, 300), (1, 1, 333, 130)])
+def test_causal_against_masked_oracle(B, H, Lq, Lk):
+    # the causal mask of attn_jvp_fwd_causal; rows that see no key: zeros, lse = -inf
+    w = custom(B, H, Lq, Lk, 128)
+    inp = gpu_inputs(w, seed=2 * Lq + Lk)
+    names = ("q", "k", "v", "tq", "tk", "tv")
+    got = ajvp.attn_jvp_fwd_f32out_causal(*(inp[n] for n in names), w.scale)
+    bf = ajvp.attn_jvp_fwd_causal(*(inp[n] for n in names), w.scale)
+    torch.cuda.synchronize()
+    assert got[0].dtype == torch.float32
+    ref = oracle.attn_jvp_causal(*(inp[n] for n in names), w.scale)
+    i = np.arange(Lq)
+    seen = np.broadcast_to((i + (Lk - Lq) >= 0)[None, None], (B, H, Lq))
+    err = _masked_err(got, ref, seen)
+    err_bf = _masked_err(bf, ref, seen)
+    print(w.name, err, err_bf)
+    check(err, w.name, Lk)
+    assert err["to"] * 10 <= err_bf["to"], (err, err_bf)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_varlen_against_masked_oracle(causal):
+    H, lq, lk = 2, [300, 1, 129, 0, 64], [200, 513, 7, 40, 0]
+    g = torch.Generator(device="cuda").manual_seed(77)
+    names = ("q", "k", "v", "tq", "tk", "tv")
+    x = {n: torch.randn((H, sum(lq) if n in ("q", "tq") else sum(lk), 128), generator=g,
+                        device="cuda").to(torch.bfloat16) for n in names}
+    cq = torch.tensor(np.concatenate([[0], np.cumsum(lq)]), dtype=torch.int32, device="cuda")
+    ck = torch.tensor(np.concatenate([[0], np.cumsum(lk)]), dtype=torch.int32, device="cuda")
+    s = 128 ** -0.5
+    got = ajvp.attn_jvp_fwd_f32out_varlen(*(x[n] for n in names), cq, ck, max(lq), s, causal=causal)
+    torch.cuda.synchronize()
+    assert got[0].dtype == torch.float32
+    ref = oracle.attn_jvp_packed(*(x[n] for n in names), s, cq.cpu().numpy(), ck.cpu().numpy(), causal)
+    seen = np.zeros(sum(lq), dtype=bool)
+    r0 = 0
+    for a, b in zip(lq, lk):
+        i = np.arange(a)
+        seen[r0:r0 + a] = ((i + (b - a) >= 0) if causal else np.full(a, True)) & (b > 0)
+        r0 += a
+    err = _masked_err(got, ref, np.broadcast_to(seen[None], (H, sum(lq))))
+    print(causal, err)
+    check(err, f"varlen causal={causal}", max(lk))
