@@ -40,18 +40,20 @@
 //   tensor-memory columns per tile; Pd = P .* (u - mu); the elementwise
 //   results E1, E2 are bf16, the A operands of G2.)  V_Q and V_K hold one
 //   set of X, Y, Z, W next to their accumulators: the elementwise warps read
-//   Z and W first and release them, so that the next tile's [Z|W] products
-//   run while they read X, Y and compute; each group writes its E1, E2 over its
-//   own 32 columns of X (16 packed columns each), so the next
-//   tile's [X|Y] products are issued after this tile's G2 (tensor-core
-//   operations run in issue order).  V_V double-buffers its two score tiles
-//   and writes E1, E2 over them, as the forward kernel does.
+//   Z and W as soon as the [Z|W] products complete, release them (the next
+//   tile's [Z|W] products may then run) and form their statistics terms
+//   while the [X|Y] products still run; each group writes its E1 over its own
+//   32 columns of X and E2 over its own 32 columns of Y (16 packed columns
+//   each), so the next tile's [X|Y] products are issued after this tile's G2
+//   (tensor-core operations run in issue order).  V_V double-buffers its two
+//   score tiles and writes E1, E2 over them, as the forward kernel does.
 //
-// Warp roles (384 threads): warp 0 TMA producer, warp 1 MMA issuer, warp 2
-// tensor-memory allocation, warps 4-11 elementwise in two groups of four
-// warps (group g takes columns 32g .. 32g+31 of each tile; one thread per
-// row and group), which also run the epilogue (acc * scale -> bf16 -> TMA
-// store).
+// Warp roles (384 threads): warps 0 and 3 TMA producers (the long and the
+// short ring), warp 1 MMA issuer, warp 2 tensor-memory allocation, warps
+// 4-11 elementwise in two groups of four warps (group g takes columns
+// 32g .. 32g+31 of each tile; one thread per row and group), which also run
+// the epilogue (acc * scale -> bf16 -> tensor store; packed sequences:
+// guarded row stores).
 #pragma once
 
 #include "ptx_sm100.cuh"
