@@ -49,3 +49,63 @@ def test_forward_and_backward_in_a_graph(Lq, Lk):
         for a, b in zip(got, ref):
             assert torch.equal(a, b)
     assert ajvp.check_device_status() == ajvp.AJVP_OK
+
+
+@pytest.mark.parametrize("mode", ["causal", "varlen"])
+def test_masked_forward_and_backward_in_a_graph(mode):
+    # the causal pair on dense tensors, the packed pair on three sequences (one
+    # without keys), captured after one eager call and replayed on changed inputs
+    if mode == "causal":
+        w = custom(1, 2, 300, 260, 128)
+        inp = gpu_inputs(w, seed=5)
+        cot = make_cotangents(w, seed=6, device="cuda")
+        shp_q, shp_s = inp["q"].shape, (1, 2, 300)
+    else:
+        lq, lk = [150, 90, 40], [130, 0, 220]
+        gen = torch.Generator(device="cuda").manual_seed(5)
+        inp = {n: torch.randn((2, sum(lq) if n in ("q", "tq") else sum(lk), 128), generator=gen,
+                              device="cuda").to(torch.bfloat16) for n in NAMES}
+        cot = {n: torch.randn((2, sum(lq), 128), generator=gen, device="cuda").to(torch.bfloat16)
+               for n in ("dout", "dtout")}
+        cq = torch.tensor([0, 150, 240, 280], dtype=torch.int32, device="cuda")
+        ck = torch.tensor([0, 130, 130, 350], dtype=torch.int32, device="cuda")
+        shp_q, shp_s = inp["q"].shape, (2, sum(lq))
+    o, to = torch.empty(shp_q, dtype=torch.bfloat16, device="cuda"), torch.empty(shp_q, dtype=torch.bfloat16,
+                                                                                   device="cuda")
+    lse, mu = torch.empty(shp_s, device="cuda"), torch.empty(shp_s, device="cuda")
+    grads = {n: torch.empty_like(inp["q"] if n in ("dq", "dtq") else inp["k"]) for n in ajvp.GRAD_NAMES}
+    ws = torch.empty(ajvp.bwd_workspace_bytes(1, shp_s[-2] if mode == "varlen" else 2, shp_s[-1]),
+                     dtype=torch.uint8, device="cuda")
+    s = 128 ** -0.5
+
+    def step(stream=None):
+        if mode == "causal":
+            ajvp.attn_jvp_fwd_causal_stats(*(inp[n] for n in NAMES), s, o=o, to=to, lse=lse, mu=mu, stream=stream)
+            ajvp.attn_jvp_bwd_causal(*(inp[n] for n in NAMES), o, to, lse, mu, cot["dout"], cot["dtout"], s,
+                                     grads=grads, workspace=ws, stream=stream)
+        else:
+            ajvp.attn_jvp_fwd_varlen_stats(*(inp[n] for n in NAMES), cq, ck, 150, s, o=o, to=to, lse=lse, mu=mu,
+                                           stream=stream)
+            ajvp.attn_jvp_bwd_varlen(*(inp[n] for n in NAMES), o, to, lse, mu, cot["dout"], cot["dtout"], cq, ck,
+                                     150, 220, s, grads=grads, workspace=ws, stream=stream)
+
+    step()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    st = torch.cuda.Stream()
+    with torch.cuda.stream(st):
+        with torch.cuda.graph(g, stream=st):
+            step(stream=st)
+    for seed in (7, 8):
+        gen2 = torch.Generator(device="cuda").manual_seed(seed)
+        for n in NAMES:
+            inp[n].copy_(torch.randn(inp[n].shape, generator=gen2, device="cuda").to(torch.bfloat16))
+        g.replay()
+        torch.cuda.synchronize()
+        got = [t.clone() for t in (o, to, lse, mu)] + [grads[n].clone() for n in ajvp.GRAD_NAMES]
+        step()
+        torch.cuda.synchronize()
+        ref = [o, to, lse, mu] + [grads[n] for n in ajvp.GRAD_NAMES]
+        for a, b in zip(got, ref):
+            assert torch.equal(a, b)
+    assert ajvp.check_device_status() == ajvp.AJVP_OK
