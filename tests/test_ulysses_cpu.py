@@ -224,3 +224,44 @@ def test_ulysses_causal_matches_unsharded(world, shape):
         res = dict(out)
     for r in range(world):
         assert all(res[r].values()), (r, res[r])
+
+
+def _dropout_worker(rank, world, port, out):
+    # rank 1 leaves before the exchange; rank 0's all-to-all must end with an error
+    # (the peer's connection closes, or the short process-group timeout expires),
+    # not wait for good
+    import datetime
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=5))
+    if rank == 1:
+        out[rank] = "left"
+        os._exit(0)  # no collective, no clean shutdown: the rank is simply gone
+    try:
+        from attention_forward_mode_b200.ulysses import ulysses_attn_jvp
+        t = _inputs(1, 2, 8, 8, 4, seed=1)
+        shard = {n: x[:, :, :4].contiguous() for n, x in t.items()}
+        ulysses_attn_jvp(shard["q"], shard["k"], shard["v"], shard["tq"], shard["tk"], shard["tv"], scale=0.5,
+                         local_fn=_oracle_fn)
+        out[rank] = "completed"
+    except Exception as e:  # the expected outcome
+        out[rank] = f"raised {type(e).__name__}"
+
+
+@pytest.mark.timeout(120)
+def test_ulysses_peer_loss_raises_instead_of_hanging():
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as m:
+        out = m.dict()
+        procs = [ctx.Process(target=_dropout_worker, args=(r, 2, port, out)) for r in range(2)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(90)
+        alive = [p.is_alive() for p in procs]
+        for p in procs:
+            if p.is_alive():
+                p.kill()
+        res = dict(out)
+    assert not any(alive), (alive, res)
+    assert res.get(1) == "left" and str(res.get(0, "")).startswith("raised"), res
