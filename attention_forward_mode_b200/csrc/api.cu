@@ -509,9 +509,11 @@ uint64_t attn_jvp_bwd_workspace_bytes(int64_t B, int64_t H, int64_t Lq) {
 
 namespace {
 // Kernels first..last of the backward (0 row statistics, 1 dQ and dtQ, 2 dK
-// and dtK, 3 dV and dtV) after the full argument check.
-int bwd_steps(int first, int last, int mask, const BwdPack &pk, const void *q, const void *k, const void *v, const void *tq, const void *tk,
-              const void *tv, const void *o, const void *to, const float *lse, const float *mu, const void *dout,
+// and dtK, 3 dV and dtV) after the full argument check; mask: causal and/or
+// packed (pk: the sequences of a packed call).
+int bwd_steps(int first, int last, int mask, const BwdPack &pk, const void *q, const void *k, const void *v,
+              const void *tq, const void *tk, const void *tv, const void *o, const void *to, const float *lse,
+              const float *mu, const void *dout,
               const void *dtout, void *dq, void *dk, void *dv, void *dtq, void *dtk, void *dtv, int64_t B, int64_t H,
               int64_t Lq, int64_t Lk, int64_t d, float scale, void *workspace, uint64_t workspace_bytes,
               void *stream) {
