@@ -31,7 +31,7 @@ AJVP_ERR_DEVICE_LAYOUT = -9
 EXPORTED = ("attn_jvp_fwd", "attn_jvp_fwd_causal", "attn_jvp_fwd_varlen", "attn_jvp_fwd_f32out", "attn_jvp_fwd_stats", "attn_jvp_fwd_causal_stats", "attn_jvp_bwd", "attn_jvp_bwd_step",
             "attn_jvp_bwd_causal", "attn_jvp_fwd_varlen_stats", "attn_jvp_bwd_varlen",
             "attn_jvp_fwd_f32out_causal", "attn_jvp_fwd_f32out_varlen",
-            "attn_jvp_bwd_workspace_bytes", "attn_jvp_fwd_f32", "attn_jvp_fwd_host",
+            "attn_jvp_bwd_workspace_bytes", "attn_jvp_bwd_workspace_bytes_split", "attn_jvp_fwd_f32", "attn_jvp_fwd_host",
             "attn_jvp_fwd_host_noalloc", "attn_jvp_host_workspace_bytes", "attn_jvp_bwd_host",
             "attn_jvp_bwd_host_workspace_bytes", "attn_jvp_strerror",
             "attn_jvp_last_cuda_error",
@@ -90,6 +90,8 @@ def load_library(path: str = LIB_PATH):
         lib.attn_jvp_bwd_step.restype = ctypes.c_int
         lib.attn_jvp_bwd_workspace_bytes.argtypes = [i64] * 3
         lib.attn_jvp_bwd_workspace_bytes.restype = ctypes.c_uint64
+        lib.attn_jvp_bwd_workspace_bytes_split.argtypes = [i64] * 4
+        lib.attn_jvp_bwd_workspace_bytes_split.restype = ctypes.c_uint64
         lib.attn_jvp_bwd_host.argtypes = [vp] * 18 + [i64] * 5 + [f32, vp, ctypes.c_uint64, vp]
         lib.attn_jvp_bwd_host.restype = ctypes.c_int
         lib.attn_jvp_bwd_host_workspace_bytes.argtypes = [i64] * 4
@@ -379,9 +381,14 @@ def _fwd_stats(entry, q, k, v, tq, tk, tv, scale, o, to, lse, mu, stream):
     return o, to, lse, mu
 
 
-def bwd_workspace_bytes(B: int, H: int, Lq: int) -> int:
-    """Device workspace ``attn_jvp_bwd`` needs (row statistics)."""
-    return int(load_library().attn_jvp_bwd_workspace_bytes(int(B), int(H), int(Lq)))
+def bwd_workspace_bytes(B: int, H: int, Lq: int, Lk: int | None = None) -> int:
+    """Device workspace ``attn_jvp_bwd`` needs (row statistics); with ``Lk``,
+    the size that also lets the key-side kernels split short key sequences
+    (``attn_jvp_bwd_workspace_bytes_split``, for the current device)."""
+    lib = load_library()
+    if Lk is None:
+        return int(lib.attn_jvp_bwd_workspace_bytes(int(B), int(H), int(Lq)))
+    return int(lib.attn_jvp_bwd_workspace_bytes_split(int(B), int(H), int(Lq), int(Lk)))
 
 
 GRAD_NAMES = ("dq", "dk", "dv", "dtq", "dtk", "dtv")
@@ -426,7 +433,9 @@ def _bwd(entry, q, k, v, tq, tk, tv, o, to, lse, mu, dout, dtout, scale, grads, 
     if scale is None:
         scale = d ** -0.5
     if workspace is None:
-        workspace = torch.empty(max(1, bwd_workspace_bytes(B, H, Lq)), dtype=torch.uint8, device=q.device)
+        with torch.cuda.device(q.device):  # the split size reads this device's SM count
+            nbytes = bwd_workspace_bytes(B, H, Lq, None if entry == "attn_jvp_bwd_causal" else Lk)
+            workspace = torch.empty(max(1, nbytes), dtype=torch.uint8, device=q.device)
     if not workspace.is_cuda or workspace.dtype != torch.uint8 or not workspace.is_contiguous():
         raise ValueError("workspace must be a contiguous CUDA uint8 tensor")
     lib = load_library()

@@ -74,6 +74,9 @@ cudaError_t set_bwd_smem() {
     if (e == cudaSuccess) e = set_bwd_smem_one<VAR, 1>();
     if (e == cudaSuccess) e = set_bwd_smem_one<VAR, 2>();
     if (e == cudaSuccess) e = set_bwd_smem_one<VAR, 3>();
+    if constexpr (VAR != ajvp::bwd::V_Q) {  // the key-side variants' split form
+        if (e == cudaSuccess) e = set_bwd_smem_one<VAR, ajvp::bwd::MASK_SPLIT>();
+    }
     return e;
 }
 
@@ -268,6 +271,26 @@ struct BwdPack {
     int64_t n_seq = 0, max_q = 0, max_k = 0;
 };
 
+// Parts of the streamed range for the unmasked key-side kernels: when their
+// 128-key tiles alone cannot fill the GPU (short key sequences, as in
+// cross-attention to a few hundred text tokens), each part goes to a CTA of
+// its own, so that about eight waves of CTAs run, with at least four 64-query
+// tiles per part and at most 16 parts.
+int64_t bwd_key_split(int64_t BH, int64_t Lq, int64_t Lk, int sm_count) {
+    const int64_t ctas = (Lk + ajvp::bwd::BM - 1) / ajvp::bwd::BM * BH;
+    const int64_t tiles = (Lq + ajvp::bwd::BN - 1) / ajvp::bwd::BN;
+    if (ctas <= 0 || ctas >= 4 * (int64_t)sm_count) return 1;
+    int64_t s = std::min<int64_t>(16, (8 * (int64_t)sm_count + ctas - 1) / ctas);
+    while (s > 1 && (tiles + s - 1) / s < 4) --s;
+    return std::max<int64_t>(s, 1);
+}
+
+// fp32 partial sums of the split key-side kernels: [parts][B*H][Lk][2][128]
+uint64_t bwd_partial_bytes(int64_t BH, int64_t Lk, int64_t parts) {
+    if (parts <= 1) return 0;
+    return ((uint64_t)parts * (uint64_t)(BH * Lk) * 2u * ajvp::bwd::HD * 4u + 255u) / 256u * 256u;
+}
+
 // One backward variant: resident tensors r (row side, Lrow rows), streamed
 // tensors l (the long ring) and sh (the short stage), Lcol rows; outputs
 // out[] (Lrow rows) scaled by sc[]; MASK: causal and/or packed (cu_row /
@@ -277,11 +300,11 @@ int launch_bwd_var(std::initializer_list<const void *> r, std::initializer_list<
                    std::initializer_list<const void *> sh, std::initializer_list<void *> out,
                    std::initializer_list<float> sc, const void *stats, int64_t BH, int64_t Lrow, int64_t Lcol,
                    int64_t Lq, int64_t d, float scale, cudaStream_t stream, const int *cu_row, const int *cu_col,
-                   int64_t n_seq, int64_t max_row) {
+                   int64_t n_seq, int64_t max_row, int64_t n_split = 1, float *partial = nullptr) {
     using namespace ajvp::bwd;
     constexpr bool kPacked = (MASK & MASK_PACKED) != 0;
     const int64_t n_rtiles = ((kPacked ? max_row : Lrow) + BM - 1) / BM;
-    const int64_t n_cta = n_rtiles * BH * (kPacked ? n_seq : 1);
+    const int64_t n_cta = n_rtiles * BH * (kPacked ? n_seq : 1) * n_split;
     if (n_cta >= (int64_t(1) << 31)) return AJVP_ERR_TOO_LARGE;
     if (n_cta == 0) return AJVP_OK;
     int rc;
@@ -307,6 +330,8 @@ int launch_bwd_var(std::initializer_list<const void *> r, std::initializer_list<
     p.n_seq = (int)n_seq;
     p.cu_row = cu_row;
     p.cu_col = cu_col;
+    p.n_split = (int)n_split;
+    p.partial = partial;
     p.stats = static_cast<const float4 *>(stats);
     p.Lrow = (int)Lrow;
     p.Lcol = (int)Lcol;
@@ -338,6 +363,29 @@ int launch_bwd_mask(int mask, std::initializer_list<const void *> r, std::initia
         default: return launch_bwd_var<VAR, 3>(r, l, sh, out, sc, stats, BH, Lrow, Lcol, Lq, d, scale, stream,
                                                cu_row, cu_col, n_seq, max_row);
     }
+}
+
+// An unmasked key-side variant with its streamed range cut into n_split parts:
+// the kernel writes fp32 partial sums, the reduction adds them up (in part
+// order) into the two bf16 outputs.
+template <int VAR>
+int launch_bwd_split(std::initializer_list<const void *> r, std::initializer_list<const void *> l,
+                     std::initializer_list<const void *> sh, void *out0, void *out1, float s0, float s1,
+                     const void *stats, int64_t BH, int64_t Lrow, int64_t Lcol, int64_t Lq, int64_t d, float scale,
+                     cudaStream_t stream, int64_t n_split, float *partial) {
+    int rc = launch_bwd_var<VAR, ajvp::bwd::MASK_SPLIT>(r, l, sh, {out0, out1}, {s0, s1}, stats, BH, Lrow, Lcol, Lq,
+                                                        d, scale, stream, nullptr, nullptr, 0, 0, n_split, partial);
+    if (rc != AJVP_OK) return rc;
+    const long long rows = (long long)(BH * Lrow);
+    const long long n4 = rows * 2 * (ajvp::bwd::HD / 4);
+    const unsigned grid = (unsigned)std::min<long long>((n4 + 255) / 256, 148LL * 16);
+    ajvp::bwd::bwd_split_reduce_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const float4 *>(partial),
+                                                                  (int)n_split, rows,
+                                                                  static_cast<__nv_bfloat16 *>(out0),
+                                                                  static_cast<__nv_bfloat16 *>(out1), s0, s1);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail_cuda(e);
+    return AJVP_OK;
 }
 
 // ---------------------------------------------------------- host pipeline
@@ -505,6 +553,14 @@ uint64_t attn_jvp_bwd_workspace_bytes(int64_t B, int64_t H, int64_t Lq) {
     return bwd_stats_bytes(B * H, Lq);
 }
 
+uint64_t attn_jvp_bwd_workspace_bytes_split(int64_t B, int64_t H, int64_t Lq, int64_t Lk) {
+    if (B < 0 || H < 0 || Lq < 0 || Lk < 0) return 0;
+    const uint64_t base = bwd_stats_bytes(B * H, Lq);
+    int dev = 0;
+    if (device_setup(&dev) != AJVP_OK) return base;  // no usable device: the minimum
+    return base + bwd_partial_bytes(B * H, Lk, bwd_key_split(B * H, Lq, Lk, g_dev[dev].sm_count));
+}
+
 }  // extern "C"
 
 namespace {
@@ -554,6 +610,11 @@ int bwd_steps(int first, int last, int mask, const BwdPack &pk, const void *q, c
     int dev = 0;
     if ((rc = device_setup(&dev)) != AJVP_OK) return rc;
     if ((rc = get_encoder()) != AJVP_OK) return rc;
+    // unmasked key side: cut the query range into parts when the key tiles alone
+    // cannot fill the GPU and the workspace holds the partial sums
+    int64_t n_split = mask == 0 ? bwd_key_split(BH, Lq, Lk, g_dev[dev].sm_count) : 1;
+    if (n_split > 1 && workspace_bytes < bwd_stats_bytes(BH, Lq) + bwd_partial_bytes(BH, Lk, n_split)) n_split = 1;
+    float *partial = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + bwd_stats_bytes(BH, Lq));
 
     using namespace ajvp::bwd;
     if (first <= 0 && last >= 0) {
@@ -573,15 +634,24 @@ int bwd_steps(int first, int last, int mask, const BwdPack &pk, const void *q, c
                                               workspace, BH, Lq, Lk, Lq, d, scale, st, pk.cu_q, pk.cu_k, pk.n_seq,
                                               pk.max_q)) != AJVP_OK)
         return rc;
-    // rows = keys, streamed queries: dk, dtk; dv, dtv
-    if (want(2) && (rc = launch_bwd_mask<V_K>(mask, {k, tk, v, tv}, {q, tq}, {dtout, dout}, {dk, dtk}, {s1, s1},
-                                              workspace, BH, Lk, Lq, Lq, d, scale, st, pk.cu_k, pk.cu_q, pk.n_seq,
-                                              pk.max_k)) != AJVP_OK)
-        return rc;
-    if (want(3) && (rc = launch_bwd_mask<V_V>(mask, {k, tk}, {dout, dtout}, {q, tq}, {dv, dtv}, {1.0f, 1.0f},
-                                              workspace, BH, Lk, Lq, Lq, d, scale, st, pk.cu_k, pk.cu_q, pk.n_seq,
-                                              pk.max_k)) != AJVP_OK)
-        return rc;
+    // rows = keys, streamed queries: dk, dtk; dv, dtv (the split parts share one
+    // partial-sum buffer: each reduction finishes before the next kernel, on the stream)
+    if (want(2)) {
+        rc = n_split > 1 ? launch_bwd_split<V_K>({k, tk, v, tv}, {q, tq}, {dtout, dout}, dk, dtk, s1, s1, workspace,
+                                                 BH, Lk, Lq, Lq, d, scale, st, n_split, partial)
+                         : launch_bwd_mask<V_K>(mask, {k, tk, v, tv}, {q, tq}, {dtout, dout}, {dk, dtk}, {s1, s1},
+                                                workspace, BH, Lk, Lq, Lq, d, scale, st, pk.cu_k, pk.cu_q, pk.n_seq,
+                                                pk.max_k);
+        if (rc != AJVP_OK) return rc;
+    }
+    if (want(3)) {
+        rc = n_split > 1 ? launch_bwd_split<V_V>({k, tk}, {dout, dtout}, {q, tq}, dv, dtv, 1.0f, 1.0f, workspace, BH,
+                                                 Lk, Lq, Lq, d, scale, st, n_split, partial)
+                         : launch_bwd_mask<V_V>(mask, {k, tk}, {dout, dtout}, {q, tq}, {dv, dtv}, {1.0f, 1.0f},
+                                                workspace, BH, Lk, Lq, Lq, d, scale, st, pk.cu_k, pk.cu_q, pk.n_seq,
+                                                pk.max_k);
+        if (rc != AJVP_OK) return rc;
+    }
     return AJVP_OK;
 }
 }  // namespace

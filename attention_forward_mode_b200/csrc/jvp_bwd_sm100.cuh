@@ -98,7 +98,11 @@ constexpr uint32_t NB_EPI = 1;
 // j <= i + (Lk - Lq) of its sequence, bottom-right aligned; 2 packed -- the
 // tensors are [H][total][128] and sequence b owns row-side rows
 // cu_row[b] .. cu_row[b+1]-1 and streamed rows cu_col[b] .. cu_col[b+1]-1.
-constexpr int MASK_CAUSAL = 1, MASK_PACKED = 2;
+// 4 split (unmasked key-side variants only) -- the streamed range is cut into
+// n_split consecutive parts, one per CTA, each writing its fp32 partial sums
+// to partial[split][B*H][Lrow][2][128] (unscaled); bwd_split_reduce_kernel adds
+// them up in split order, so the result stays deterministic.
+constexpr int MASK_CAUSAL = 1, MASK_PACKED = 2, MASK_SPLIT = 4;
 
 struct Params {
     CUtensorMap tm_r[4], tm_l[2], tm_s[2], tm_out[2];
@@ -110,6 +114,8 @@ struct Params {
     int n_seq;            // packed: sequences per head
     const int *cu_row, *cu_col;  // packed: starts of each sequence's row-side / streamed rows
     __nv_bfloat16 *out[2];       // packed: the outputs as plain pointers (guarded row stores)
+    int n_split;                 // split: parts of the streamed range
+    float *partial;              // split: [n_split][B*H][Lrow][2][128] fp32 partial sums
     float scale;          // s
     float scale_log2;     // s * log2(e)
     float out_scale[2];   // factor applied to each accumulator at the end (s or 1)
@@ -152,6 +158,33 @@ __global__ void __launch_bounds__(256) bwd_rowstats_kernel(const __nv_bfloat16 *
             const float m = mu[r];
             stats[r] = make_float4(lse[r] * 1.4426950408889634f, m, a, b - a * m);
         }
+    }
+}
+
+// Sum of the split parts' fp32 partial sums, in part order, times the
+// accumulator's output scale, rounded to bf16: out[a][row][:] for the
+// rows x 2 accumulators of one key-side variant.  One thread per 4 columns.
+__global__ void __launch_bounds__(256) bwd_split_reduce_kernel(const float4 *__restrict__ partial, int n_split,
+                                                               long long rows, __nv_bfloat16 *__restrict__ out0,
+                                                               __nv_bfloat16 *__restrict__ out1, float s0, float s1) {
+    const long long n4 = rows * 2 * (HD / 4);  // float4s of one part
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
+         i += (long long)gridDim.x * blockDim.x) {
+        float4 acc = partial[i];
+        for (int s = 1; s < n_split; ++s) {
+            const float4 v = partial[(size_t)s * (size_t)n4 + (size_t)i];
+            acc.x += v.x;
+            acc.y += v.y;
+            acc.z += v.z;
+            acc.w += v.w;
+        }
+        const long long row = i / (2 * (HD / 4));
+        const int a = (int)((i / (HD / 4)) & 1), c4 = (int)(i % (HD / 4));
+        const float sc = a ? s1 : s0;
+        uint2 w;
+        w.x = pack_bf16x2(acc.x * sc, acc.y * sc);
+        w.y = pack_bf16x2(acc.z * sc, acc.w * sc);
+        *reinterpret_cast<uint2 *>((a ? out1 : out0) + (size_t)row * HD + 4u * c4) = w;
     }
 }
 
@@ -202,6 +235,8 @@ template <int VAR, int MASK = 0>
 __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_constant__ Params p) {
     using C = Var<VAR>;
     constexpr bool kCausal = (MASK & MASK_CAUSAL) != 0, kPacked = (MASK & MASK_PACKED) != 0;
+    constexpr bool kSplitK = (MASK & MASK_SPLIT) != 0;
+    static_assert(!kSplitK || (MASK == MASK_SPLIT && VAR != V_Q), "the split is for the unmasked key side");
     extern __shared__ __align__(1024) uint8_t bwd_smem[];
     const uint32_t base = smem_u32(bwd_smem);
     if (base & 1023u) {  // the tile layout needs 1024-byte alignment and leaves no slack
@@ -226,17 +261,29 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
         Lrow_s = max(min(max(p.cu_row[b + 1], 0), p.Lrow), yr0) - yr0;
         yc0 = min(max(p.cu_col[b], 0), p.Lcol);
         Lcol_s = max(min(max(p.cu_col[b + 1], 0), p.Lcol), yc0) - yc0;
+    } else if (kSplitK) {
+        // split-major: the n_rtiles * BH tiles of part 0, then of part 1, ...
+        const int cta = (int)(blockIdx.x % (unsigned)(p.n_rtiles * p.BH));
+        rt = cta % p.n_rtiles;
+        bh = cta / p.n_rtiles;
     } else {
         // causal dQ / dtQ: the late (heavy) query tiles of each head first
         rt = (kCausal && VAR == V_Q) ? p.n_rtiles - 1 - (int)(blockIdx.x % p.n_rtiles)
                                      : (int)(blockIdx.x % p.n_rtiles);
         bh = blockIdx.x / p.n_rtiles;
     }
+    // split: this CTA's part of the streamed range
+    const int sp = kSplitK ? (int)(blockIdx.x / (unsigned)(p.n_rtiles * p.BH)) : 0;
     const int r0 = rt * BM;  // local first row
     if (kPacked && r0 >= Lrow_s) return;  // past the end of this sequence (uniform for the CTA)
     const int yr = yr0 + r0;              // tensor row of the tile's first row
     // streamed tiles jt0 .. jt0 + nt - 1 (local index j = 0 .. nt - 1)
     int jt0 = 0, nt = (Lcol_s + BN - 1) / BN;
+    if (kSplitK) {
+        const int chunk = (nt + p.n_split - 1) / p.n_split;
+        jt0 = sp * chunk;
+        nt = max(0, min(chunk, nt - jt0));
+    }
     // koff = Lk - Lq of the sequence: the causal diagonal's offset
     const int koff = VAR == V_Q ? Lcol_s - Lrow_s : Lrow_s - Lcol_s;
     if (kCausal) {
@@ -652,40 +699,55 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
                 for (int h = 0; h < 2; ++h) {
                     const int pc = 2 * grp + h;
                     uint32_t ra[32];
-                    if (MASK != 0 && nt == 0) {  // no row of the tile sees anything: zeros
+                    if (MASK != 0 && nt == 0) {  // no row of the tile sees anything (or an empty part): zeros
 #pragma unroll
                         for (int i = 0; i < 32; ++i) ra[i] = 0u;
                     } else {
                         tmem_ld32(tbase + lane_off + 128u * a + 32u * pc, ra);
                         tmem_wait_ld();
                     }
-                    uint32_t wa[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        wa[i] = pack_bf16x2(__uint_as_float(ra[2 * i]) * os, __uint_as_float(ra[2 * i + 1]) * os);
-                    if (kPacked) {
-                        // rows past the sequence's end belong to the next one: not written
+                    if constexpr (kSplitK) {
+                        // this part's fp32 partial sums, unscaled (the reduction scales them)
                         if (r0 + row < Lrow_s) {
-                            uint4 *dst = reinterpret_cast<uint4 *>(
-                                p.out[a] + ((size_t)bh * (size_t)p.Lrow + (size_t)(yr + row)) * HD + 64u * grp + 32u * h);
+                            float4 *dst = reinterpret_cast<float4 *>(
+                                p.partial + ((((size_t)sp * (size_t)p.BH + (size_t)bh) * (size_t)p.Lrow +
+                                              (size_t)(yr + row)) * 2u + (size_t)a) * HD + 64u * grp + 32u * h);
 #pragma unroll
-                            for (int u = 0; u < 4; ++u)
-                                dst[u] = make_uint4(wa[4 * u], wa[4 * u + 1], wa[4 * u + 2], wa[4 * u + 3]);
+                            for (int u = 0; u < 8; ++u)
+                                dst[u] = make_float4(__uint_as_float(ra[4 * u]), __uint_as_float(ra[4 * u + 1]),
+                                                     __uint_as_float(ra[4 * u + 2]), __uint_as_float(ra[4 * u + 3]));
                         }
-                        continue;
-                    }
-                    const uint32_t dst = base + SM_R + (uint32_t)a * R_TILE + (uint32_t)grp * CHUNK_R + (uint32_t)row * 128u;
+                    } else {
+                        uint32_t wa[16];
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const uint32_t phys = (((uint32_t)h * 4u + u) ^ (uint32_t)(row & 7)) * 16u;
-                        st_shared_v4(dst + phys, wa[4 * u], wa[4 * u + 1], wa[4 * u + 2], wa[4 * u + 3]);
-                    }
+                        for (int i = 0; i < 16; ++i)
+                            wa[i] = pack_bf16x2(__uint_as_float(ra[2 * i]) * os, __uint_as_float(ra[2 * i + 1]) * os);
+                        if (kPacked) {
+                            // rows past the sequence's end belong to the next one: not written
+                            if (r0 + row < Lrow_s) {
+                                uint4 *dst = reinterpret_cast<uint4 *>(
+                                    p.out[a] + ((size_t)bh * (size_t)p.Lrow + (size_t)(yr + row)) * HD + 64u * grp +
+                                    32u * h);
+#pragma unroll
+                                for (int u = 0; u < 4; ++u)
+                                    dst[u] = make_uint4(wa[4 * u], wa[4 * u + 1], wa[4 * u + 2], wa[4 * u + 3]);
+                            }
+                            continue;
+                        }
+                        const uint32_t dst =
+                            base + SM_R + (uint32_t)a * R_TILE + (uint32_t)grp * CHUNK_R + (uint32_t)row * 128u;
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const uint32_t phys = (((uint32_t)h * 4u + u) ^ (uint32_t)(row & 7)) * 16u;
+                            st_shared_v4(dst + phys, wa[4 * u], wa[4 * u + 1], wa[4 * u + 2], wa[4 * u + 3]);
+                        }
+                    }  // bf16 outputs
                 }
             }
         }
         fence_proxy_async_smem();
         named_bar_sync(NB_EPI, EW_THREADS);  // staging complete
-        if (!kPacked && warp == 4 && lane == 0 && !any_failed && *abort_flag == 0) {
+        if (!kPacked && !kSplitK && warp == 4 && lane == 0 && !any_failed && *abort_flag == 0) {
             for (int a = 0; a < 2; ++a) {
                 tma_store_3d(&p.tm_out[a], base + SM_R + a * R_TILE, 0, yr, bh);
                 tma_store_3d(&p.tm_out[a], base + SM_R + a * R_TILE + CHUNK_R, 64, yr, bh);

@@ -621,7 +621,7 @@ def run_ours_bwd(args, w):
         o, to, lse, mu = fwd(*(inp[n] for n in names), w.scale, stream=stream)
     grads = {n: torch.empty_like(inp["q"] if n in ("dq", "dtq") else inp["k"]) for n in ajvp.GRAD_NAMES}
     gpk = {n: g.reshape(-1, g.shape[-2], g.shape[-1]) for n, g in grads.items()}
-    ws = torch.empty(ajvp.bwd_workspace_bytes(w.B, w.H, w.Lq), dtype=torch.uint8, device=dev)
+    ws = torch.empty(ajvp.bwd_workspace_bytes(w.B, w.H, w.Lq, w.Lk), dtype=torch.uint8, device=dev)
     in_bytes = sum(t.numel() * t.element_size() for t in list(inp.values()) + list(cot.values()) + [o, to])
     flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev) if in_bytes <= L2_BYTES else None
 

@@ -346,6 +346,21 @@ AJVP_API int attn_jvp_bwd_varlen(const void *q, const void *k, const void *v,
 AJVP_API uint64_t attn_jvp_bwd_workspace_bytes(int64_t B, int64_t H, int64_t Lq);
 
 /*
+ * attn_jvp_bwd_workspace_bytes_split -- the workspace with which
+ * attn_jvp_bwd (and attn_jvp_bwd_step) may split the query range of its two
+ * key-side kernels (dk, dtk and dv, dtv) over several CTAs per 128-key tile:
+ * when the key tiles alone cannot fill the current device (short key
+ * sequences, such as cross-attention to a few hundred text tokens), each
+ * part writes fp32 partial sums to the workspace and a reduction adds them
+ * up in part order (the result stays deterministic, though not bit-identical
+ * to the unsplit kernels).  At least attn_jvp_bwd_workspace_bytes; equal to
+ * it when no split applies.  Reads the current device's SM count (the
+ * minimum is returned when no usable device is current).  A call whose
+ * workspace is smaller than this runs the unsplit kernels.
+ */
+AJVP_API uint64_t attn_jvp_bwd_workspace_bytes_split(int64_t B, int64_t H, int64_t Lq, int64_t Lk);
+
+/*
  * attn_jvp_bwd_host -- attn_jvp_bwd on HOST buffers: every tensor argument
  * (the twelve inputs, lse and mu included, and the six gradients) is host
  * memory in the layouts of attn_jvp_bwd; pinned memory gives overlapped
@@ -357,7 +372,8 @@ AJVP_API uint64_t attn_jvp_bwd_workspace_bytes(int64_t B, int64_t H, int64_t Lq)
  * on one internal stream, its four backward kernels run on one of two
  * others, and its gradients are copied back on a fourth, so copies overlap
  * the kernels of neighbouring chunks.  Results are identical to attn_jvp_bwd
- * on the same data.  Stream-ordered with respect to `stream` (the call
+ * on the same data with a workspace of attn_jvp_bwd_workspace_bytes (the
+ * chunks' key-side kernels never split).  Stream-ordered with respect to `stream` (the call
  * returns once everything is enqueued; the host buffers must stay valid and
  * unchanged until `stream` reaches that point).  Lq == 0 writes zeros to dk,
  * dv, dtk, dtv on the host after synchronising `stream`.  Errors as

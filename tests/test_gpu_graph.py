@@ -13,16 +13,17 @@ pytestmark = pytest.mark.gpu
 NAMES = ("q", "k", "v", "tq", "tk", "tv")
 
 
-@pytest.mark.parametrize("Lq,Lk", [(300, 260),     # one CTA per query tile
-                                   (19000, 300)])  # 298 query tiles: the persistent forward
-def test_forward_and_backward_in_a_graph(Lq, Lk):
+@pytest.mark.parametrize("Lq,Lk,split", [(300, 260, False),     # one CTA per query tile
+                                         (19000, 300, False),   # 298 query tiles: the persistent forward
+                                         (3000, 300, True)])    # the key side split over the queries
+def test_forward_and_backward_in_a_graph(Lq, Lk, split):
     w = custom(1, 2, Lq, Lk, 128)
     inp = gpu_inputs(w, seed=1)
     cot = make_cotangents(w, seed=2, device="cuda")
     o, to, lse, mu = (torch.empty_like(inp["q"]), torch.empty_like(inp["q"]),
                       torch.empty((1, 2, Lq), device="cuda"), torch.empty((1, 2, Lq), device="cuda"))
     grads = {n: torch.empty_like(inp["q"] if n in ("dq", "dtq") else inp["k"]) for n in ajvp.GRAD_NAMES}
-    ws = torch.empty(ajvp.bwd_workspace_bytes(1, 2, Lq), dtype=torch.uint8, device="cuda")
+    ws = torch.empty(ajvp.bwd_workspace_bytes(1, 2, Lq, Lk if split else None), dtype=torch.uint8, device="cuda")
 
     def step(stream=None):
         ajvp.attn_jvp_fwd_stats(*(inp[n] for n in NAMES), w.scale, o=o, to=to, lse=lse, mu=mu, stream=stream)

@@ -86,7 +86,11 @@ def _bwd_case(w, seed):
     inp = gpu_inputs(w, seed=seed)
     cot = make_cotangents(w, seed=seed + 1, device="cuda")
     o, to, lse, mu = ajvp.attn_jvp_fwd_stats(*(inp[n] for n in NAMES), w.scale)
-    ref = ajvp.attn_jvp_bwd(*(inp[n] for n in NAMES), o, to, lse, mu, cot["dout"], cot["dtout"], w.scale)
+    # the staged path's workspace holds each chunk's row statistics only, so its key
+    # side never splits: compare with a device call whose workspace is as small
+    ws = torch.empty(ajvp.bwd_workspace_bytes(w.B, w.H, w.Lq), dtype=torch.uint8, device="cuda")
+    ref = ajvp.attn_jvp_bwd(*(inp[n] for n in NAMES), o, to, lse, mu, cot["dout"], cot["dtout"], w.scale,
+                            workspace=ws)
     torch.cuda.synchronize()
     dev = {**inp, "o": o, "to": to, "lse": lse, "mu": mu, **cot}
     return dev, {n: g.cpu() for n, g in ref.items()}
