@@ -271,18 +271,33 @@ struct BwdPack {
     int64_t n_seq = 0, max_q = 0, max_k = 0;
 };
 
-// Parts of the streamed range for the unmasked key-side kernels: when their
-// 128-key tiles alone cannot fill the GPU (short key sequences, as in
-// cross-attention to a few hundred text tokens), each part goes to a CTA of
-// its own, so that about eight waves of CTAs run, with at least four 64-query
-// tiles per part and at most 16 parts.
+// Parts of the streamed range for the unmasked key-side kernels.  When their
+// 128-key tiles alone give fewer than four CTAs per SM (short key sequences,
+// as in cross-attention to a few hundred text tokens), the 64-query tiles are
+// cut into s parts (1 <= s <= 16), one CTA each, with s minimising a wave
+// model of the run time: ceil(ctas * s / SMs) waves, each as long as one
+// part's query tiles plus a fixed cost of about eight tiles per CTA (resident
+// loads, pipeline fill and drain, epilogue), times 1 + s / 100 for the
+// partial sums' traffic and their reduction.  On B200, over key sides of 96
+// to 640 CTAs and s = 1 .. 16, the model's choice was the fastest measured or
+// within 1 % of it.  For a given part length the smallest s wins, so no part
+// is ever empty (the kernels still handle one).
 int64_t bwd_key_split(int64_t BH, int64_t Lq, int64_t Lk, int sm_count) {
     const int64_t ctas = (Lk + ajvp::bwd::BM - 1) / ajvp::bwd::BM * BH;
     const int64_t tiles = (Lq + ajvp::bwd::BN - 1) / ajvp::bwd::BN;
-    if (ctas <= 0 || ctas >= 4 * (int64_t)sm_count) return 1;
-    int64_t s = std::min<int64_t>(16, (8 * (int64_t)sm_count + ctas - 1) / ctas);
-    while (s > 1 && (tiles + s - 1) / s < 4) --s;
-    return std::max<int64_t>(s, 1);
+    if (ctas <= 0 || tiles <= 1 || sm_count <= 0 || ctas >= 4 * (int64_t)sm_count) return 1;
+    int64_t best = 1;
+    double best_t = 0.0;
+    for (int64_t s = 1; s <= 16 && s <= tiles; ++s) {
+        const int64_t chunk = (tiles + s - 1) / s;
+        const int64_t waves = (ctas * s + sm_count - 1) / sm_count;
+        const double t = (double)waves * (double)(chunk + 8) * (1.0 + 0.01 * (double)s);
+        if (s == 1 || t < best_t) {
+            best = s;
+            best_t = t;
+        }
+    }
+    return best;
 }
 
 // fp32 partial sums of the split key-side kernels: [parts][B*H][Lk][2][128]

@@ -133,7 +133,8 @@ def test_steps_equal_all_in_one():
     inp = gpu_inputs(w, seed=12)
     cot = make_cotangents(w, seed=13, device="cuda")
     full, (o, to, lse, mu) = run(inp, cot, w.scale)
-    ws = torch.empty(ajvp.bwd_workspace_bytes(w.B, w.H, w.Lq), dtype=torch.uint8, device="cuda")
+    # the whole call's default workspace (the split size): the steps take the same split
+    ws = torch.empty(ajvp.bwd_workspace_bytes(w.B, w.H, w.Lq, w.Lk), dtype=torch.uint8, device="cuda")
     grads = None
     for step in (0, 3, 1, 2):  # steps 1-3 only need step 0 before them
         grads = ajvp.attn_jvp_bwd(*(inp[n] for n in NAMES), o, to, lse, mu, cot["dout"], cot["dtout"], w.scale,

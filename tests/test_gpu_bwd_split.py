@@ -32,9 +32,9 @@ def _bwd(w, inp, cot, split, step=None, grads=None):
     return g
 
 
-@pytest.mark.parametrize("B,H,Lq,Lk", [(1, 2, 3000, 300),   # 15 parts of 4 query tiles, the last three empty
-                                       (2, 1, 1000, 77),    # one ragged key tile per head
-                                       (1, 3, 700, 513)])   # a one-key last tile
+@pytest.mark.parametrize("B,H,Lq,Lk", [(1, 2, 3000, 300),   # 16 parts of 3 query tiles, the last one of 2
+                                       (2, 1, 1000, 77),    # one ragged key tile per head, 16 one-tile parts
+                                       (1, 3, 700, 513)])   # a one-key last tile, the last part one ragged tile
 def test_split_against_oracle(B, H, Lq, Lk):
     assert ajvp.bwd_workspace_bytes(B, H, Lq, Lk) > ajvp.bwd_workspace_bytes(B, H, Lq), "no split at this shape"
     w = custom(B, H, Lq, Lk, 128)
@@ -46,6 +46,28 @@ def test_split_against_oracle(B, H, Lq, Lk):
     print(w.name, err)
     for n, e in err.items():
         assert e <= TOL, f"{w.name}: {n} max-rel error {e:.3e} > {TOL} ({err})"
+
+
+def test_split_many_key_tiles_sampled():
+    # 24 heads x 4 key tiles = 96 key-side CTAs: 3 parts of 22 query tiles (the last
+    # part 21, one of them ragged); sampled rows and keys on three heads
+    w = custom(1, 24, 4100, 512, 128)
+    assert ajvp.bwd_workspace_bytes(w.B, w.H, w.Lq, w.Lk) > ajvp.bwd_workspace_bytes(w.B, w.H, w.Lq)
+    inp = gpu_inputs(w, seed=16)
+    cot = make_cotangents(w, seed=17, device="cuda")
+    got = _bwd(w, inp, cot, split=True)
+    rows, keys = sample_rows(w.Lq, 10), sample_rows(w.Lk, 12, seed=2)
+    err = {n: 0.0 for n in GRADS}
+    for h in (0, 11, 23):
+        fl = {n: t[0, h].cpu() for n, t in {**inp, **cot}.items()}
+        ref = oracle.attn_jvp_bwd(*(fl[n][None] for n in NAMES), fl["dout"][None], fl["dtout"][None], w.scale,
+                                  qrows=rows, krows=keys)
+        for n in GRADS:
+            sel = rows if n in ("dq", "dtq") else keys
+            err[n] = max(err[n], max_rel(got[n][0, h][sel].float().cpu().numpy(), ref[n][0]))
+    print(w.name, err)
+    for n, e in err.items():
+        assert e <= TOL, f"{n}: {e:.3e}"
 
 
 def test_split_deterministic_and_close_to_unsplit():

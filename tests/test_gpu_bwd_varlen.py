@@ -75,14 +75,16 @@ def test_varlen(lq, lk, causal):
 @pytest.mark.parametrize("causal", [False, True])
 def test_one_sequence_equals_dense(causal):
     # one packed sequence: the dense kernels' arithmetic, bit for bit (the packed
-    # epilogue stores rows directly instead of through the tensor-store unit)
+    # epilogue stores rows directly instead of through the tensor-store unit; the
+    # dense call gets the statistics-only workspace, so its key side does not split)
     w = custom(1, 3, 333, 517, 128)
     inp = gpu_inputs(w, seed=41)
     cot = make_cotangents(w, seed=42, device="cuda")
     fwd = ajvp.attn_jvp_fwd_causal_stats if causal else ajvp.attn_jvp_fwd_stats
     bwd = ajvp.attn_jvp_bwd_causal if causal else ajvp.attn_jvp_bwd
     o, to, lse, mu = fwd(*(inp[n] for n in NAMES), w.scale)
-    dense = bwd(*(inp[n] for n in NAMES), o, to, lse, mu, cot["dout"], cot["dtout"], w.scale)
+    ws = torch.empty(ajvp.bwd_workspace_bytes(w.B, w.H, w.Lq), dtype=torch.uint8, device="cuda")
+    dense = bwd(*(inp[n] for n in NAMES), o, to, lse, mu, cot["dout"], cot["dtout"], w.scale, workspace=ws)
     x = {n: t[0] for n, t in {**inp, **cot}.items()}
     cq = torch.tensor([0, w.Lq], dtype=torch.int32, device="cuda")
     ck = torch.tensor([0, w.Lk], dtype=torch.int32, device="cuda")
