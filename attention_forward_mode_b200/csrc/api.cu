@@ -300,7 +300,9 @@ int64_t bwd_key_split(int64_t BH, int64_t Lq, int64_t Lk, int sm_count) {
     return best;
 }
 
-// fp32 partial sums of the split key-side kernels: [parts][B*H][Lk][2][128]
+// fp32 partial sums of one split key-side kernel: [parts][B*H][Lk][2][128]
+// (the dK/dtK and dV/dtV kernels each get a region of this size, after the
+// row statistics, so that the two steps stay independent of each other)
 uint64_t bwd_partial_bytes(int64_t BH, int64_t Lk, int64_t parts) {
     if (parts <= 1) return 0;
     return ((uint64_t)parts * (uint64_t)(BH * Lk) * 2u * ajvp::bwd::HD * 4u + 255u) / 256u * 256u;
@@ -573,7 +575,7 @@ uint64_t attn_jvp_bwd_workspace_bytes_split(int64_t B, int64_t H, int64_t Lq, in
     const uint64_t base = bwd_stats_bytes(B * H, Lq);
     int dev = 0;
     if (device_setup(&dev) != AJVP_OK) return base;  // no usable device: the minimum
-    return base + bwd_partial_bytes(B * H, Lk, bwd_key_split(B * H, Lq, Lk, g_dev[dev].sm_count));
+    return base + 2u * bwd_partial_bytes(B * H, Lk, bwd_key_split(B * H, Lq, Lk, g_dev[dev].sm_count));
 }
 
 }  // extern "C"
@@ -628,8 +630,11 @@ int bwd_steps(int first, int last, int mask, const BwdPack &pk, const void *q, c
     // unmasked key side: cut the query range into parts when the key tiles alone
     // cannot fill the GPU and the workspace holds the partial sums
     int64_t n_split = mask == 0 ? bwd_key_split(BH, Lq, Lk, g_dev[dev].sm_count) : 1;
-    if (n_split > 1 && workspace_bytes < bwd_stats_bytes(BH, Lq) + bwd_partial_bytes(BH, Lk, n_split)) n_split = 1;
-    float *partial = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + bwd_stats_bytes(BH, Lq));
+    const uint64_t part_bytes = bwd_partial_bytes(BH, Lk, n_split);
+    if (n_split > 1 && workspace_bytes < bwd_stats_bytes(BH, Lq) + 2u * part_bytes) n_split = 1;
+    uint8_t *const part_base = static_cast<uint8_t *>(workspace) + bwd_stats_bytes(BH, Lq);
+    float *const partial_k = reinterpret_cast<float *>(part_base);
+    float *const partial_v = reinterpret_cast<float *>(part_base + part_bytes);
 
     using namespace ajvp::bwd;
     if (first <= 0 && last >= 0) {
@@ -649,11 +654,11 @@ int bwd_steps(int first, int last, int mask, const BwdPack &pk, const void *q, c
                                               workspace, BH, Lq, Lk, Lq, d, scale, st, pk.cu_q, pk.cu_k, pk.n_seq,
                                               pk.max_q)) != AJVP_OK)
         return rc;
-    // rows = keys, streamed queries: dk, dtk; dv, dtv (the split parts share one
-    // partial-sum buffer: each reduction finishes before the next kernel, on the stream)
+    // rows = keys, streamed queries: dk, dtk; dv, dtv (split: each kernel with its
+    // own partial-sum region, reduced on the stream before the step returns)
     if (want(2)) {
         rc = n_split > 1 ? launch_bwd_split<V_K>({k, tk, v, tv}, {q, tq}, {dtout, dout}, dk, dtk, s1, s1, workspace,
-                                                 BH, Lk, Lq, Lq, d, scale, st, n_split, partial)
+                                                 BH, Lk, Lq, Lq, d, scale, st, n_split, partial_k)
                          : launch_bwd_mask<V_K>(mask, {k, tk, v, tv}, {q, tq}, {dtout, dout}, {dk, dtk}, {s1, s1},
                                                 workspace, BH, Lk, Lq, Lq, d, scale, st, pk.cu_k, pk.cu_q, pk.n_seq,
                                                 pk.max_k);
@@ -661,7 +666,7 @@ int bwd_steps(int first, int last, int mask, const BwdPack &pk, const void *q, c
     }
     if (want(3)) {
         rc = n_split > 1 ? launch_bwd_split<V_V>({k, tk}, {dout, dtout}, {q, tq}, dv, dtv, 1.0f, 1.0f, workspace, BH,
-                                                 Lk, Lq, Lq, d, scale, st, n_split, partial)
+                                                 Lk, Lq, Lq, d, scale, st, n_split, partial_v)
                          : launch_bwd_mask<V_V>(mask, {k, tk}, {dout, dtout}, {q, tq}, {dv, dtv}, {1.0f, 1.0f},
                                                 workspace, BH, Lk, Lq, Lq, d, scale, st, pk.cu_k, pk.cu_q, pk.n_seq,
                                                 pk.max_k);

@@ -225,7 +225,10 @@ AJVP_API int attn_jvp_fwd_stats(const void *q, const void *k, const void *v,
  *
  * Four kernels on `stream`: per-row statistics into the workspace, then
  * three gradient kernels (tcgen05: dq and dtq; dk and dtk; dv and dtv), each
- * owning its outputs (no atomics: results are deterministic).  Gradients are
+ * owning its outputs (no atomics: results are deterministic).  With a
+ * workspace of attn_jvp_bwd_workspace_bytes_split bytes the dk/dtk and
+ * dv/dtv kernels may split short key sequences over several CTAs, each
+ * followed by an ordered reduction kernel (six kernels in all).  Gradients are
  * accumulated in fp32 and rounded to bf16 (round-to-nearest-even).
  * Supported: d == 128, every pointer non-NULL and 16-byte aligned, sizes as
  * attn_jvp_fwd.  B*H == 0 is a no-op; Lq == 0 writes zeros to dk, dv, dtk,
@@ -351,9 +354,10 @@ AJVP_API uint64_t attn_jvp_bwd_workspace_bytes(int64_t B, int64_t H, int64_t Lq)
  * key-side kernels (dk, dtk and dv, dtv) over several CTAs per 128-key tile:
  * when the key tiles alone cannot fill the current device (short key
  * sequences, such as cross-attention to a few hundred text tokens), each
- * part writes fp32 partial sums to the workspace and a reduction adds them
- * up in part order (the result stays deterministic, though not bit-identical
- * to the unsplit kernels).  At least attn_jvp_bwd_workspace_bytes; equal to
+ * part writes fp32 partial sums to the workspace (one region for dk/dtk,
+ * one for dv/dtv, so that attn_jvp_bwd_step's steps 2 and 3 stay
+ * independent) and a reduction adds them up in part order (the result stays
+ * deterministic, though not bit-identical to the unsplit kernels).  At least attn_jvp_bwd_workspace_bytes; equal to
  * it when no split applies.  Reads the current device's SM count (the
  * minimum is returned when no usable device is current).  A call whose
  * workspace is smaller than this runs the unsplit kernels.

@@ -107,6 +107,31 @@ def test_split_steps_one_at_a_time():
         assert torch.equal(grads[n], whole[n]), n
 
 
+def test_split_key_steps_on_two_streams():
+    # steps 2 (dk, dtk) and 3 (dv, dtv) keep their partial sums in separate regions
+    # of the workspace, so they may run at the same time on two streams
+    w = custom(1, 2, 3000, 300, 128)
+    inp = gpu_inputs(w, seed=18)
+    cot = make_cotangents(w, seed=19, device="cuda")
+    whole = _bwd(w, inp, cot, split=True)
+    o, to, lse, mu = ajvp.attn_jvp_fwd_stats(*(inp[n] for n in NAMES), w.scale)
+    ws = torch.empty(ajvp.bwd_workspace_bytes(w.B, w.H, w.Lq, w.Lk), dtype=torch.uint8, device="cuda")
+    grads = {n: torch.empty_like(inp["q"] if n in ("dq", "dtq") else inp["k"]) for n in GRADS}
+    args = [inp[n] for n in NAMES] + [o, to, lse, mu, cot["dout"], cot["dtout"], w.scale]
+    for _ in range(3):
+        ajvp.attn_jvp_bwd(*args, workspace=ws, grads=grads, step=0)
+        s2, s3 = torch.cuda.Stream(), torch.cuda.Stream()
+        s2.wait_stream(torch.cuda.current_stream())
+        s3.wait_stream(torch.cuda.current_stream())
+        ajvp.attn_jvp_bwd(*args, workspace=ws, grads=grads, step=2, stream=s2)
+        ajvp.attn_jvp_bwd(*args, workspace=ws, grads=grads, step=3, stream=s3)
+        ajvp.attn_jvp_bwd(*args, workspace=ws, grads=grads, step=1)
+        torch.cuda.synchronize()
+        for n in GRADS:
+            assert torch.equal(grads[n], whole[n]), n
+    assert ajvp.check_device_status() == ajvp.AJVP_OK
+
+
 def test_zero_cotangents_give_zero_gradients():
     w = custom(1, 2, 3000, 300, 128)
     inp = gpu_inputs(w, seed=15)
