@@ -70,6 +70,19 @@ def test_split_many_key_tiles_sampled():
         assert e <= TOL, f"{n}: {e:.3e}"
 
 
+@pytest.mark.parametrize("H,Lk,parts", [(24, 512, 3), (40, 512, 6), (40, 1024, 4), (40, 2048, 1)])
+def test_part_count_on_measured_shapes(H, Lk, parts):
+    # the part counts the wave model picks for the key sides of 96, 160, 320 and 640
+    # CTAs (32760 queries; 16384 for the first) on a 148-SM B200, each the fastest or
+    # within 1 % of it in a sweep of 1..16 parts; read back from the workspace size
+    # (statistics, then two regions of parts x heads x keys x 1 KB)
+    if torch.cuda.get_device_properties(0).multi_processor_count != 148:
+        pytest.skip("part counts measured on 148 SMs")
+    Lq = 16384 if H == 24 else 32760
+    extra = ajvp.bwd_workspace_bytes(1, H, Lq, Lk) - ajvp.bwd_workspace_bytes(1, H, Lq)
+    assert extra == (2 * parts * H * Lk * 1024 if parts > 1 else 0)
+
+
 def test_split_deterministic_and_close_to_unsplit():
     w = custom(1, 2, 3000, 300, 128)
     inp = gpu_inputs(w, seed=11)
