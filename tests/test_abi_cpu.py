@@ -90,6 +90,17 @@ def test_host_workspace_bytes(lib):
     assert f(1, 1, 128, 1) == 3 * 9 * 256  # every array padded to its own 256-byte boundary
 
 
+def test_bwd_workspace_bytes(lib):
+    f, fs = lib.attn_jvp_bwd_workspace_bytes, lib.attn_jvp_bwd_workspace_bytes_split
+    # per (batch, head) row 16 bytes of statistics, 64 rows of padding, rounded to 256
+    assert f(1, 2, 100) == 4352  # (200 + 64) x 16 = 4224, rounded up
+    assert f(2, 3, 4096) == (6 * 4096 + 64) * 16
+    assert f(-1, 2, 100) == 0 and fs(1, 2, 100, -1) == 0
+    # no usable device here: the split size is the minimum (the kernels then do not split)
+    for shape in ((1, 40, 32760, 512), (1, 2, 3000, 300), (1, 12, 32760, 32760)):
+        assert fs(*shape) == f(*shape[:3]), shape
+
+
 def test_host_entry_rejections(lib):
     # host-side checks, before any CUDA call
     assert _call_host(lib, Lk=0) == B.AJVP_ERR_INVALID_ARG
