@@ -31,7 +31,7 @@ AJVP_ERR_DEVICE_LAYOUT = -9
 EXPORTED = ("attn_jvp_fwd", "attn_jvp_fwd_causal", "attn_jvp_fwd_varlen", "attn_jvp_fwd_f32out", "attn_jvp_fwd_stats", "attn_jvp_fwd_causal_stats", "attn_jvp_bwd", "attn_jvp_bwd_step",
             "attn_jvp_bwd_causal", "attn_jvp_fwd_varlen_stats", "attn_jvp_bwd_varlen",
             "attn_jvp_fwd_f32out_causal", "attn_jvp_fwd_f32out_varlen",
-            "attn_jvp_bwd_workspace_bytes", "attn_jvp_bwd_workspace_bytes_split", "attn_jvp_fwd_f32", "attn_jvp_fwd_host",
+            "attn_jvp_bwd_workspace_bytes", "attn_jvp_bwd_workspace_bytes_split", "attn_jvp_bwd_key_split_parts", "attn_jvp_fwd_f32", "attn_jvp_fwd_host",
             "attn_jvp_fwd_host_noalloc", "attn_jvp_host_workspace_bytes", "attn_jvp_bwd_host",
             "attn_jvp_bwd_host_workspace_bytes", "attn_jvp_strerror",
             "attn_jvp_last_cuda_error",
@@ -92,6 +92,8 @@ def load_library(path: str = LIB_PATH):
         lib.attn_jvp_bwd_workspace_bytes.restype = ctypes.c_uint64
         lib.attn_jvp_bwd_workspace_bytes_split.argtypes = [i64] * 4
         lib.attn_jvp_bwd_workspace_bytes_split.restype = ctypes.c_uint64
+        lib.attn_jvp_bwd_key_split_parts.argtypes = [i64] * 5
+        lib.attn_jvp_bwd_key_split_parts.restype = i64
         lib.attn_jvp_bwd_host.argtypes = [vp] * 18 + [i64] * 5 + [f32, vp, ctypes.c_uint64, vp]
         lib.attn_jvp_bwd_host.restype = ctypes.c_int
         lib.attn_jvp_bwd_host_workspace_bytes.argtypes = [i64] * 4
@@ -447,6 +449,18 @@ def _bwd(entry, q, k, v, tq, tk, tv, o, to, lse, mu, dout, dtout, scale, grads, 
     else:
         _check(lib.attn_jvp_bwd_step(int(step), *args), "attn_jvp_bwd_step")
     return grads
+
+
+def bwd_key_split_parts(B: int, H: int, Lq: int, Lk: int, sm_count: int | None = None) -> int:
+    """Parts into which ``attn_jvp_bwd`` (with the split workspace) cuts the
+    key-side kernels' query range; ``sm_count`` defaults to the current CUDA
+    device's.  Host arithmetic only."""
+    if sm_count is None:
+        sm_count = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    n = int(load_library().attn_jvp_bwd_key_split_parts(int(B), int(H), int(Lq), int(Lk), int(sm_count)))
+    if n < 1:
+        raise ValueError("invalid sizes or SM count")
+    return n
 
 
 def bwd_host_workspace_bytes(Lq: int, Lk: int, d: int, heads_per_chunk: int = 1) -> int:

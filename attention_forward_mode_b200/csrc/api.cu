@@ -570,6 +570,12 @@ uint64_t attn_jvp_bwd_workspace_bytes(int64_t B, int64_t H, int64_t Lq) {
     return bwd_stats_bytes(B * H, Lq);
 }
 
+int64_t attn_jvp_bwd_key_split_parts(int64_t B, int64_t H, int64_t Lq, int64_t Lk, int64_t sm_count) {
+    if (B < 0 || H < 0 || Lq < 0 || Lk < 0 || sm_count < 1 || sm_count > (int64_t(1) << 20)) return 0;
+    if (B > 0 && H > (int64_t(1) << 40) / B) return 0;
+    return bwd_key_split(B * H, Lq, Lk, (int)sm_count);
+}
+
 uint64_t attn_jvp_bwd_workspace_bytes_split(int64_t B, int64_t H, int64_t Lq, int64_t Lk) {
     if (B < 0 || H < 0 || Lq < 0 || Lk < 0) return 0;
     const uint64_t base = bwd_stats_bytes(B * H, Lq);

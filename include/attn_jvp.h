@@ -365,6 +365,20 @@ AJVP_API uint64_t attn_jvp_bwd_workspace_bytes(int64_t B, int64_t H, int64_t Lq)
 AJVP_API uint64_t attn_jvp_bwd_workspace_bytes_split(int64_t B, int64_t H, int64_t Lq, int64_t Lk);
 
 /*
+ * attn_jvp_bwd_key_split_parts -- the number of parts (1 = no split) into
+ * which attn_jvp_bwd, given the split workspace, cuts the query range of
+ * its key-side kernels on a device with `sm_count` SMs.  Pure host
+ * arithmetic (no CUDA call).  Splits only when the 128-key tiles give
+ * fewer than four CTAs per SM; the count (at most 16, at most the number
+ * of 64-query tiles) minimises a wave model of the run time:
+ * ceil(key CTAs x parts / SMs) waves, each as long as one part's query
+ * tiles plus about eight tiles of fixed cost per CTA, times 1 + parts / 100;
+ * ties go to fewer parts, so no part is empty.  Returns 0 for negative
+ * sizes or an sm_count outside 1 .. 2^20.
+ */
+AJVP_API int64_t attn_jvp_bwd_key_split_parts(int64_t B, int64_t H, int64_t Lq, int64_t Lk, int64_t sm_count);
+
+/*
  * attn_jvp_bwd_host -- attn_jvp_bwd on HOST buffers: every tensor argument
  * (the twelve inputs, lse and mu included, and the six gradients) is host
  * memory in the layouts of attn_jvp_bwd; pinned memory gives overlapped

@@ -101,6 +101,32 @@ def test_bwd_workspace_bytes(lib):
         assert fs(*shape) == f(*shape[:3]), shape
 
 
+def test_bwd_key_split_parts(lib):
+    f = lib.attn_jvp_bwd_key_split_parts
+    # the counts a sweep of 1..16 parts measured fastest (or within 1 %) on a 148-SM B200:
+    # key sides of 96, 160, 320 and 640 CTAs
+    assert f(1, 24, 16384, 512, 148) == 3
+    assert f(1, 40, 32760, 512, 148) == 6
+    assert f(1, 40, 32760, 1024, 148) == 4
+    assert f(1, 40, 32760, 2048, 148) == 1
+    # invalid arguments
+    assert f(-1, 1, 64, 64, 148) == 0 and f(1, 1, 64, 64, 0) == 0 and f(1, 1, 64, -1, 148) == 0
+    # properties over a grid of shapes: 1 <= parts <= min(16, query tiles); no split when the
+    # key tiles give four CTAs per SM or there is one query tile; no part is empty
+    for sm in (148, 132, 8):
+        for bh in (1, 3, 24, 40, 200):
+            for Lq in (1, 64, 65, 1000, 4100, 32760):
+                for Lk in (1, 77, 512, 1024, 4096):
+                    s = f(1, bh, Lq, Lk, sm)
+                    tiles, ctas = -(-Lq // 64), -(-Lk // 128) * bh
+                    assert 1 <= s <= max(1, min(16, tiles)), (sm, bh, Lq, Lk, s)
+                    if ctas >= 4 * sm or tiles <= 1:
+                        assert s == 1, (sm, bh, Lq, Lk, s)
+                    chunk = -(-tiles // s)
+                    assert (s - 1) * chunk < tiles, (sm, bh, Lq, Lk, s)
+    assert B.bwd_key_split_parts(1, 40, 32760, 512, sm_count=148) == 6
+
+
 def test_host_entry_rejections(lib):
     # host-side checks, before any CUDA call
     assert _call_host(lib, Lk=0) == B.AJVP_ERR_INVALID_ARG
