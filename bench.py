@@ -53,6 +53,7 @@ BWD_MASKED_METRIC = ("attention+JVP masked backward TFLOP/s (30·d per visible q
 BWD_KERNEL_SOURCES = ["attention_forward_mode_b200/csrc/jvp_bwd_sm100.cuh",
                       "attention_forward_mode_b200/csrc/ptx_sm100.cuh"]
 BWD_TRAFFIC_FILE = "profiles/attn_jvp_bwd_kernel.video_selfattn_b1h12_l32760.md"
+BWD_TRAFFIC_WORKLOAD = "video_selfattn_b1h12_l32760_d128"  # the workload and kernel (V_K) it covers
 L2_BYTES = 126 * 1024 * 1024
 # backward kernels (steps of attn_jvp_bwd): name, contraction FLOPs per (Lq*Lk*d) per head
 BWD_STEPS = [("bwd_rowstats_kernel", 0.0), ("attn_jvp_bwd_kernel<V_Q> (dQ, dtQ)", 18.0),
@@ -670,10 +671,14 @@ def run_ours_bwd(args, w):
         return finish_bwd_masked(args, w, rank, world, value, flops, ms_max, clocks, inp, cot,
                                  seq_lens if varlen else None)
 
-    # each of the four kernels alone, K launches each, events on the stream
+    # each of the four kernels alone, K launches each, events on the stream (a split
+    # key-side step is its kernel plus the reduction of its partial sums)
+    parts = ajvp.bwd_key_split_parts(w.B, w.H, w.Lq, w.Lk)
     per_kernel = []
     nk = max(3, args.steps // 2)
     for i, (kname, fl) in enumerate(BWD_STEPS):
+        if parts > 1 and i >= 2:
+            kname = f"{kname}, split into {parts} parts + bwd_split_reduce_kernel"
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         step(i)
         torch.cuda.synchronize(dev)
@@ -724,11 +729,13 @@ def run_ours_bwd(args, w):
                 "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
                 "config": dict(workload_config(w, world), entry="attn_jvp_bwd",
-                               flops_per_step="30·Lq·Lk·d per head (minimal contraction count)"),
+                               flops_per_step="30·Lq·Lk·d per head (minimal contraction count)",
+                               key_side_parts=parts),
                 "pct_of_bf16_peak": 100.0 * value / world / burst,
                 "roofline": {"bound": "tensor", "achieved": achieved, "peak": burst, "unit": "TFLOP/s",
                              "frac": achieved / burst,
-                             "traffic": committed_traffic(BWD_TRAFFIC_FILE, BWD_KERNEL_SOURCES),
+                             "traffic": committed_traffic(BWD_TRAFFIC_FILE, BWD_KERNEL_SOURCES)
+                             if w.name == BWD_TRAFFIC_WORKLOAD and dom["kernel"] == BWD_STEPS[2][0] else None,
                              "peak_source": f"{src} bf16 dense (burst) from MEASURED_PEAKS.json"
                              if src == "measured" else "fallback 1.59 PFLOP/s",
                              "kernel": dom["kernel"], "algorithmic_flops_per_launch": dom["flops"],
@@ -737,7 +744,8 @@ def run_ours_bwd(args, w):
                 "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                         "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps,
                         "path": f"attn_jvp_bwd_host (pipelined, chunks of {nh} head(s))"},
-                "gpu_launches": len(BWD_STEPS) * args.steps, "clocks": clocks.summary()}
+                "gpu_launches": (len(BWD_STEPS) + (2 if parts > 1 else 0)) * args.steps,
+                "clocks": clocks.summary()}
         if world == 1 and not args.no_cpu_baseline:
             v, n, el, threads = oracle_bwd_sample(w, bwd_head0_cpu(inp, cot), args.cpu_seconds)
             line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
