@@ -110,7 +110,7 @@ struct Params {
     int Lrow, Lcol;       // row-side and streamed lengths (packed: the tensors' totals)
     int Lq;               // query rows per (batch, head): the stats row stride
     int n_rtiles;         // 128-row tiles per (batch, head) (packed: of the longest sequence)
-    int BH;               // packed: heads (the tensors' outermost extent)
+    int BH;               // packed: heads (the tensors' outermost extent); split: B*H
     int n_seq;            // packed: sequences per head
     const int *cu_row, *cu_col;  // packed: starts of each sequence's row-side / streamed rows
     __nv_bfloat16 *out[2];       // packed: the outputs as plain pointers (guarded row stores)
