@@ -401,9 +401,12 @@ def attn_jvp_bwd(q, k, v, tq, tk, tv, o, to, lse, mu, dout, dtout, scale=None, g
     """Gradients of <dout, O> + <dtout, tO> with respect to q, k, v, tq, tk,
     tv, through the C ABI's ``attn_jvp_bwd`` (bf16, d = 128).  o, to, lse,
     mu are the outputs of ``attn_jvp_fwd_stats`` on the same inputs.
-    ``grads``: optional dict of preallocated outputs.  Returns a dict
-    dq, dk, dv, dtq, dtk, dtv.  Asynchronous on ``stream``.  ``step`` (0-3)
-    runs one of the four kernels only (``attn_jvp_bwd_step``)."""
+    ``grads``: optional dict of preallocated outputs.  ``workspace``: a CUDA
+    uint8 tensor (allocated per call when omitted, with room for the split
+    key side: ``bwd_workspace_bytes(B, H, Lq, Lk)``; one of
+    ``bwd_workspace_bytes(B, H, Lq)`` bytes runs the unsplit kernels).
+    Returns a dict dq, dk, dv, dtq, dtk, dtv.  Asynchronous on ``stream``.
+    ``step`` (0-3) runs one of the four steps only (``attn_jvp_bwd_step``)."""
     return _bwd("attn_jvp_bwd" if step is None else "attn_jvp_bwd_step", q, k, v, tq, tk, tv, o, to, lse, mu,
                 dout, dtout, scale, grads, workspace, stream, step)
 
