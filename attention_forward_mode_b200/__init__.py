@@ -56,8 +56,12 @@ from ._binding import (  # noqa: F401
 from .autograd import AttnJvpFunction, attn_jvp_autograd  # noqa: E402,F401
 
 __all__ = [
-    "AttnJvpFunction", "attn_jvp_autograd",
-    "attn_jvp", "attn_jvp_bwd", "attn_jvp_bwd_causal", "attn_jvp_fwd_causal_stats", "attn_jvp_bwd_varlen", "attn_jvp_fwd_varlen_stats", "attn_jvp_bwd_host", "bwd_host_workspace_bytes", "default_bwd_heads_per_chunk", "attn_jvp_fwd_causal", "attn_jvp_fwd_varlen", "attn_jvp_fwd_stats", "bwd_workspace_bytes", "bwd_key_split_parts", "attn_jvp_fwd", "attn_jvp_fwd_f32", "attn_jvp_fwd_f32out", "attn_jvp_fwd_f32out_causal", "attn_jvp_fwd_f32out_varlen", "attn_jvp_fwd_host", "attn_jvp_fwd_host_noalloc", "check_device_status",
-    "default_heads_per_chunk", "host_workspace_bytes", "load_library",
-    "selftest_wait_timeout", "set_persistent_key_tiles", "DEFAULT_PERSISTENT_KEY_TILES", "set_wait_bound_ns", "strerror", "version", "AttnJvpError",
+    "AttnJvpFunction", "attn_jvp_autograd", "attn_jvp", "attn_jvp_bwd", "attn_jvp_bwd_causal",
+    "attn_jvp_fwd_causal_stats", "attn_jvp_bwd_varlen", "attn_jvp_fwd_varlen_stats", "attn_jvp_bwd_host",
+    "bwd_host_workspace_bytes", "default_bwd_heads_per_chunk", "attn_jvp_fwd_causal", "attn_jvp_fwd_varlen",
+    "attn_jvp_fwd_stats", "bwd_workspace_bytes", "bwd_key_split_parts", "attn_jvp_fwd", "attn_jvp_fwd_f32",
+    "attn_jvp_fwd_f32out", "attn_jvp_fwd_f32out_causal", "attn_jvp_fwd_f32out_varlen", "attn_jvp_fwd_host",
+    "attn_jvp_fwd_host_noalloc", "check_device_status", "default_heads_per_chunk", "host_workspace_bytes",
+    "load_library", "selftest_wait_timeout", "set_persistent_key_tiles", "DEFAULT_PERSISTENT_KEY_TILES",
+    "set_wait_bound_ns", "strerror", "version", "AttnJvpError",
 ]

@@ -28,15 +28,17 @@ AJVP_ERR_WORKSPACE = -8
 AJVP_ERR_DEVICE_LAYOUT = -9
 
 # every symbol the header declares
-EXPORTED = ("attn_jvp_fwd", "attn_jvp_fwd_causal", "attn_jvp_fwd_varlen", "attn_jvp_fwd_f32out", "attn_jvp_fwd_stats", "attn_jvp_fwd_causal_stats", "attn_jvp_bwd", "attn_jvp_bwd_step",
-            "attn_jvp_bwd_causal", "attn_jvp_fwd_varlen_stats", "attn_jvp_bwd_varlen",
-            "attn_jvp_fwd_f32out_causal", "attn_jvp_fwd_f32out_varlen",
-            "attn_jvp_bwd_workspace_bytes", "attn_jvp_bwd_workspace_bytes_split", "attn_jvp_bwd_key_split_parts", "attn_jvp_fwd_f32", "attn_jvp_fwd_host",
-            "attn_jvp_fwd_host_noalloc", "attn_jvp_host_workspace_bytes", "attn_jvp_bwd_host",
-            "attn_jvp_bwd_host_workspace_bytes", "attn_jvp_strerror",
-            "attn_jvp_last_cuda_error",
-            "attn_jvp_check_device_status", "attn_jvp_set_wait_bound_ns", "attn_jvp_set_persistent_key_tiles",
-            "attn_jvp_selftest_wait_timeout", "attn_jvp_version")
+EXPORTED = (
+    "attn_jvp_fwd", "attn_jvp_fwd_causal", "attn_jvp_fwd_varlen", "attn_jvp_fwd_f32out", "attn_jvp_fwd_stats",
+    "attn_jvp_fwd_causal_stats", "attn_jvp_bwd", "attn_jvp_bwd_step", "attn_jvp_bwd_causal",
+    "attn_jvp_fwd_varlen_stats", "attn_jvp_bwd_varlen", "attn_jvp_fwd_f32out_causal",
+    "attn_jvp_fwd_f32out_varlen", "attn_jvp_bwd_workspace_bytes", "attn_jvp_bwd_workspace_bytes_split",
+    "attn_jvp_bwd_key_split_parts", "attn_jvp_fwd_f32", "attn_jvp_fwd_host", "attn_jvp_fwd_host_noalloc",
+    "attn_jvp_host_workspace_bytes", "attn_jvp_bwd_host", "attn_jvp_bwd_host_workspace_bytes",
+    "attn_jvp_strerror", "attn_jvp_last_cuda_error", "attn_jvp_check_device_status",
+    "attn_jvp_set_wait_bound_ns", "attn_jvp_set_persistent_key_tiles", "attn_jvp_selftest_wait_timeout",
+    "attn_jvp_version",
+)
 
 _lock = threading.Lock()
 _lib = None

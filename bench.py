@@ -583,11 +583,13 @@ def run_reference_bwd(args, w):
             + (" of its longest packed sequence" if args.entry == "bwd_varlen" else ""))
     sample = f"{what}, {rows_total} rows over {args.steps} steps, {el_total:.1f} s of fp64 oracle time"
     masked = args.entry in ("bwd_causal", "bwd_varlen")
-    line = {"impl": "reference", "metric": BWD_MASKED_METRIC if masked else BWD_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+    line = {"impl": "reference", "metric": BWD_MASKED_METRIC if masked else BWD_METRIC, "value": value,
+            "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * el_total / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": dict(workload_config(w0, world), entry={"bwd": "attn_jvp_bwd", "bwd_causal": "attn_jvp_bwd_causal",
-                                                              "bwd_varlen": "attn_jvp_bwd_varlen"}[args.entry]),
+            "config": dict(workload_config(w0, world),
+                           entry={"bwd": "attn_jvp_bwd", "bwd_causal": "attn_jvp_bwd_causal",
+                                  "bwd_varlen": "attn_jvp_bwd_varlen"}[args.entry]),
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -689,7 +691,8 @@ def run_ours_bwd(args, w):
         torch.cuda.synchronize(dev)
         kms = a.elapsed_time(b) / nk
         kfl = fl * w.B * w.H * w.Lq * w.Lk * w.d
-        per_kernel.append({"kernel": kname, "ms": kms, "flops": kfl, "tflops": kfl / (kms / 1e3) / 1e12 if fl else None})
+        per_kernel.append({"kernel": kname, "ms": kms, "flops": kfl,
+                           "tflops": kfl / (kms / 1e3) / 1e12 if fl else None})
     dom = max(per_kernel, key=lambda r: r["ms"])
 
     # end to end: pinned host inputs -> attn_jvp_bwd_host (head chunks staged through a
