@@ -10,13 +10,15 @@ Predict2 image models, Wan2.1 480p video with text conditioning): an image
 token grid of 64x64, video latent grids of 21x30x52 and 21x45x80 tokens, and
 512 text tokens for cross-attention.  No dataset or trained weights are used.
 
-Draw order, fixed so a seed names one input set: from one torch.Generator
-seeded with ``seed`` on the target device, standard-normal fp32 draws for
+Draw order, fixed so a seed names one input set: from one CPU
+torch.Generator seeded with ``seed``, standard-normal fp32 draws for
 Q, K, V, tQ, tK, tV in that order, each [B, H, L, d]; then, for the
 cross-attention workload only, per-key factors uK and uV ~ U(0.5, 2) of shape
 [B, H, Lk] (uniform draw * 1.5 + 0.5).  Each tensor is multiplied by its
 stated standard deviation (and K, V rows by uK, uV), then rounded to the I/O
-dtype (round-to-nearest-even).
+dtype (round-to-nearest-even), all on the host; only the rounded tensor is
+moved to the target device.  So one seed names the same tensors whatever the
+device, and a host can re-draw exactly what a GPU run used.
 """
 from __future__ import annotations
 
@@ -98,45 +100,52 @@ def custom(B, H, Lq, Lk, d, dtype="bf16", scale=None, **kw) -> Workload:
 
 
 def make_inputs(w: Workload | str, seed: int = 0, device="cpu", dtype=None):
-    """Q, K, V, tQ, tK, tV as a dict of contiguous [B, H, L, d] tensors."""
+    """Q, K, V, tQ, tK, tV as a dict of contiguous [B, H, L, d] tensors on
+    `device`, drawn and rounded on the host (the same tensors for every
+    device)."""
     if isinstance(w, str):
         w = WORKLOADS[w]
     out_dtype = dtype if dtype is not None else w.torch_dtype
-    g = torch.Generator(device=device)
+    g = torch.Generator(device="cpu")
     g.manual_seed(seed)
     shapes = {"q": (w.B, w.H, w.Lq, w.d), "k": (w.B, w.H, w.Lk, w.d),
               "v": (w.B, w.H, w.Lk, w.d), "tq": (w.B, w.H, w.Lq, w.d),
               "tk": (w.B, w.H, w.Lk, w.d), "tv": (w.B, w.H, w.Lk, w.d)}
     std = {"q": w.q_std, "k": w.k_std, "v": w.v_std, "tq": w.t_std, "tk": w.t_std, "tv": w.t_std}
-    raw = {}
-    for name in ("q", "k", "v", "tq", "tk", "tv"):
-        raw[name] = torch.randn(shapes[name], generator=g, device=device, dtype=torch.float32)
-    if w.kv_row_scale:
-        uk = torch.rand((w.B, w.H, w.Lk), generator=g, device=device, dtype=torch.float32) * 1.5 + 0.5
-        uv = torch.rand((w.B, w.H, w.Lk), generator=g, device=device, dtype=torch.float32) * 1.5 + 0.5
-        raw["k"].mul_(uk[..., None])
-        raw["v"].mul_(uv[..., None])
-    out = {}
-    for name in ("q", "k", "v", "tq", "tk", "tv"):
-        x = raw.pop(name)
+
+    def finish(name, x):
         if std[name] != 1.0:
             x.mul_(std[name])
-        out[name] = x.to(out_dtype).contiguous()
+        return x.to(out_dtype).contiguous().to(device)
+
+    out, raw = {}, {}
+    for name in ("q", "k", "v", "tq", "tk", "tv"):
+        x = torch.randn(shapes[name], generator=g, dtype=torch.float32)
+        if w.kv_row_scale and name in ("k", "v"):
+            raw[name] = x  # the per-key factors are drawn after all six tensors
+        else:
+            out[name] = finish(name, x)
         del x
-    return out
+    if w.kv_row_scale:
+        uk = torch.rand((w.B, w.H, w.Lk), generator=g, dtype=torch.float32) * 1.5 + 0.5
+        uv = torch.rand((w.B, w.H, w.Lk), generator=g, dtype=torch.float32) * 1.5 + 0.5
+        out["k"] = finish("k", raw.pop("k").mul_(uk[..., None]))
+        out["v"] = finish("v", raw.pop("v").mul_(uv[..., None]))
+    return {n: out[n] for n in ("q", "k", "v", "tq", "tk", "tv")}
 
 
 def make_cotangents(w: Workload | str, seed: int = 1, device="cpu", dtype=None):
     """Cotangents dO, dtO of the outputs (for the backward pass): standard
     normal [B, H, Lq, d] tensors, drawn in that order from their own seeded
-    generator (the pages give no training signal to imitate)."""
+    CPU generator and rounded on the host (the pages give no training signal
+    to imitate)."""
     if isinstance(w, str):
         w = WORKLOADS[w]
     out_dtype = dtype if dtype is not None else w.torch_dtype
-    g = torch.Generator(device=device)
+    g = torch.Generator(device="cpu")
     g.manual_seed(seed)
     shape = (w.B, w.H, w.Lq, w.d)
-    return {n: torch.randn(shape, generator=g, device=device, dtype=torch.float32).to(out_dtype).contiguous()
+    return {n: torch.randn(shape, generator=g, dtype=torch.float32).to(out_dtype).contiguous().to(device)
             for n in ("dout", "dtout")}
 
 

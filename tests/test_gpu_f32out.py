@@ -133,10 +133,10 @@ def test_causal_against_masked_oracle(B, H, Lq, Lk):
 @pytest.mark.parametrize("causal", [False, True])
 def test_varlen_against_masked_oracle(causal):
     H, lq, lk = 2, [300, 1, 129, 0, 64], [200, 513, 7, 40, 0]
-    g = torch.Generator(device="cuda").manual_seed(77)
+    g = torch.Generator().manual_seed(77)
     names = ("q", "k", "v", "tq", "tk", "tv")
-    x = {n: torch.randn((H, sum(lq) if n in ("q", "tq") else sum(lk), 128), generator=g,
-                        device="cuda").to(torch.bfloat16) for n in names}
+    x = {n: torch.randn((H, sum(lq) if n in ("q", "tq") else sum(lk), 128), generator=g).to(torch.bfloat16).cuda()
+         for n in names}
     cq = torch.tensor(np.concatenate([[0], np.cumsum(lq)]), dtype=torch.int32, device="cuda")
     ck = torch.tensor(np.concatenate([[0], np.cumsum(lk)]), dtype=torch.int32, device="cuda")
     s = 128 ** -0.5

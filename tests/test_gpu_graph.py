@@ -63,10 +63,10 @@ def test_masked_forward_and_backward_in_a_graph(mode):
         shp_q, shp_s = inp["q"].shape, (1, 2, 300)
     else:
         lq, lk = [150, 90, 40], [130, 0, 220]
-        gen = torch.Generator(device="cuda").manual_seed(5)
-        inp = {n: torch.randn((2, sum(lq) if n in ("q", "tq") else sum(lk), 128), generator=gen,
-                              device="cuda").to(torch.bfloat16) for n in NAMES}
-        cot = {n: torch.randn((2, sum(lq), 128), generator=gen, device="cuda").to(torch.bfloat16)
+        gen = torch.Generator().manual_seed(5)
+        inp = {n: torch.randn((2, sum(lq) if n in ("q", "tq") else sum(lk), 128),
+                              generator=gen).to(torch.bfloat16).cuda() for n in NAMES}
+        cot = {n: torch.randn((2, sum(lq), 128), generator=gen).to(torch.bfloat16).cuda()
                for n in ("dout", "dtout")}
         cq = torch.tensor([0, 150, 240, 280], dtype=torch.int32, device="cuda")
         ck = torch.tensor([0, 130, 130, 350], dtype=torch.int32, device="cuda")
@@ -98,9 +98,9 @@ def test_masked_forward_and_backward_in_a_graph(mode):
         with torch.cuda.graph(g, stream=st):
             step(stream=st)
     for seed in (7, 8):
-        gen2 = torch.Generator(device="cuda").manual_seed(seed)
+        gen2 = torch.Generator().manual_seed(seed)
         for n in NAMES:
-            inp[n].copy_(torch.randn(inp[n].shape, generator=gen2, device="cuda").to(torch.bfloat16))
+            inp[n].copy_(torch.randn(inp[n].shape, generator=gen2).to(torch.bfloat16).cuda())
         g.replay()
         torch.cuda.synchronize()
         got = [t.clone() for t in (o, to, lse, mu)] + [grads[n].clone() for n in ajvp.GRAD_NAMES]

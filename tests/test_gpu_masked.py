@@ -61,9 +61,9 @@ def test_causal_image_workload_sampled():
 
 
 def _packed_inputs(H, lq, lk, seed):
-    g = torch.Generator(device="cuda").manual_seed(seed)
+    g = torch.Generator().manual_seed(seed)
     Tq, Tk = sum(lq), sum(lk)
-    x = {n: torch.randn((H, Tq if n in ("q", "tq") else Tk, 128), generator=g, device="cuda").to(torch.bfloat16)
+    x = {n: torch.randn((H, Tq if n in ("q", "tq") else Tk, 128), generator=g).to(torch.bfloat16).cuda()
          for n in NAMES}
     cq = torch.tensor(np.concatenate([[0], np.cumsum(lq)]), dtype=torch.int32, device="cuda")
     ck = torch.tensor(np.concatenate([[0], np.cumsum(lk)]), dtype=torch.int32, device="cuda")
