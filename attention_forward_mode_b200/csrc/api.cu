@@ -458,13 +458,12 @@ BwdStageLayout bwd_stage_layout(int64_t Lq, int64_t Lk, int64_t d, int64_t nh) {
     return s;
 }
 
-// Streams and events of one host-entry call, released on scope exit
-// (the driver defers the release of objects with work still pending).
+// Streams and events of the host-buffer pipeline.
 // Chunk c uses staging buffer c % kBuffers and compute stream 1 + c % 2, so
 // consecutive chunk kernels may overlap (the next one fills the SMs the
 // previous one's last wave leaves idle).
 constexpr int kBuffers = 3;
-struct HostPipe {
+struct PipeObjects {
     cudaStream_t st[4] = {nullptr, nullptr, nullptr, nullptr};  // copy in, compute x2, copy out
     cudaEvent_t ev[1 + 3 * kBuffers] = {};                      // start, then in / comp / out per buffer
     cudaEvent_t &start() { return ev[0]; }
@@ -478,6 +477,17 @@ struct HostPipe {
             e = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming);
         return e;
     }
+    // after a failed enqueue: wait until the chunks already issued are done, so
+    // that no copy or kernel of this call still touches the staging memory
+    // when the error is returned
+    void drain() {
+        for (cudaStream_t s : st)
+            if (s) cudaStreamSynchronize(s);
+    }
+};
+// one call's pipeline, released on scope exit (the driver defers the release
+// of objects with work still pending)
+struct HostPipe : PipeObjects {
     ~HostPipe() {
         for (cudaStream_t s : st)
             if (s) cudaStreamDestroy(s);
@@ -509,6 +519,78 @@ int launch_varlen(const void *q, const void *k, const void *v, const void *tq, c
     return launch_sm100<kSplit, ajvp::sm100::MASK_PACKED>(q, k, v, tq, tk, tv, o, to, lse, 1, H, total_q, total_k, d,
                                                            scale, stream, mu, cu_seqlens_q, cu_seqlens_k, n_seq,
                                                            max_qtiles);
+}
+
+// The forward's host-buffer pipeline on `pipe`'s streams and events: chunks of
+// nh (batch, head) slabs staged through kBuffers buffers of layout L at
+// `workspace`, ordered after the caller's stream and before its continuation.
+// On an error the chunks already issued are waited for before returning.
+int fwd_host_enqueue(PipeObjects &pipe, const void *q, const void *k, const void *v, const void *tq, const void *tk,
+                     const void *tv, void *o, void *to, float *lse, int64_t BH, int64_t Lq, int64_t Lk, int64_t d,
+                     float scale, int64_t nh, const StageLayout &L, uint8_t *workspace, cudaStream_t caller) {
+    auto bail = [&](int status) {
+        pipe.drain();
+        return status;
+    };
+    cudaError_t e = cudaEventRecord(pipe.start(), caller);
+    if (e != cudaSuccess) return fail_cuda(e);
+    for (cudaStream_t s : pipe.st)
+        if ((e = cudaStreamWaitEvent(s, pipe.start(), 0)) != cudaSuccess) return bail(fail_cuda(e));
+
+    const uint64_t qrow = (uint64_t)(Lq * d * 2), krow = (uint64_t)(Lk * d * 2);  // bytes per (b, h) slab
+    const int64_t nchunks = (BH + nh - 1) / nh;
+    const void *src[6] = {q, tq, k, v, tk, tv};
+    const uint64_t dst_off[6] = {L.q, L.tq, L.k, L.v, L.tk, L.tv};
+    for (int64_t c = 0; c < nchunks; ++c) {
+        const int b = (int)(c % kBuffers);
+        const int64_t h0 = c * nh, n = std::min<int64_t>(nh, BH - h0);
+        uint8_t *buf = workspace + (uint64_t)b * L.bytes;
+        // copy in, once the chunk that last used this buffer has been copied out
+        if (c >= kBuffers && (e = cudaStreamWaitEvent(pipe.st[0], pipe.out(b), 0)) != cudaSuccess)
+            return bail(fail_cuda(e));
+        for (int t = 0; t < 6; ++t) {
+            const uint64_t row = t < 2 ? qrow : krow;
+            e = cudaMemcpyAsync(buf + dst_off[t], static_cast<const uint8_t *>(src[t]) + (uint64_t)h0 * row,
+                                (uint64_t)n * row, cudaMemcpyHostToDevice, pipe.st[0]);
+            if (e != cudaSuccess) return bail(fail_cuda(e));
+        }
+        if ((e = cudaEventRecord(pipe.in(b), pipe.st[0])) != cudaSuccess) return bail(fail_cuda(e));
+        // compute
+        const cudaStream_t cs = pipe.st[1 + (c & 1)];
+        if ((e = cudaStreamWaitEvent(cs, pipe.in(b), 0)) != cudaSuccess) return bail(fail_cuda(e));
+        const int rc = launch_sm100<false>(buf + L.q, buf + L.k, buf + L.v, buf + L.tq, buf + L.tk, buf + L.tv,
+                                           buf + L.o, buf + L.to,
+                                           lse ? reinterpret_cast<float *>(buf + L.lse) : nullptr, 1, n, Lq, Lk, d,
+                                           scale, cs);
+        if (rc != AJVP_OK) return bail(rc);
+        if ((e = cudaEventRecord(pipe.comp(b), cs)) != cudaSuccess) return bail(fail_cuda(e));
+        // copy out (in chunk order on one stream)
+        if ((e = cudaStreamWaitEvent(pipe.st[3], pipe.comp(b), 0)) != cudaSuccess) return bail(fail_cuda(e));
+        e = cudaMemcpyAsync(static_cast<uint8_t *>(o) + (uint64_t)h0 * qrow, buf + L.o, (uint64_t)n * qrow,
+                            cudaMemcpyDeviceToHost, pipe.st[3]);
+        if (e == cudaSuccess)
+            e = cudaMemcpyAsync(static_cast<uint8_t *>(to) + (uint64_t)h0 * qrow, buf + L.to, (uint64_t)n * qrow,
+                                cudaMemcpyDeviceToHost, pipe.st[3]);
+        if (e == cudaSuccess && lse)
+            e = cudaMemcpyAsync(lse + h0 * Lq, buf + L.lse, (uint64_t)(n * Lq * 4), cudaMemcpyDeviceToHost,
+                                pipe.st[3]);
+        if (e != cudaSuccess) return bail(fail_cuda(e));
+        if ((e = cudaEventRecord(pipe.out(b), pipe.st[3])) != cudaSuccess) return bail(fail_cuda(e));
+    }
+    // the caller's stream continues once the last chunk (and so every chunk) is copied out
+    if ((e = cudaStreamWaitEvent(caller, pipe.out((int)((nchunks - 1) % kBuffers)), 0)) != cudaSuccess)
+        return bail(fail_cuda(e));
+    return AJVP_OK;
+}
+
+// heads per chunk of the forward's host pipeline: as many as `workspace_bytes`
+// holds in kBuffers buffers, at most a quarter of B*H (0 if one does not fit)
+int64_t fwd_host_heads_per_chunk(int64_t BH, int64_t Lq, int64_t Lk, int64_t d, uint64_t workspace_bytes) {
+    const uint64_t one = stage_layout(Lq, Lk, d, 1).bytes;
+    if (workspace_bytes < kBuffers * one) return 0;
+    int64_t nh = std::min<int64_t>((int64_t)(workspace_bytes / (kBuffers * one)), (BH + 3) / 4);
+    while (nh > 1 && kBuffers * stage_layout(Lq, Lk, d, nh).bytes > workspace_bytes) --nh;
+    return std::max<int64_t>(nh, 1);
 }
 
 }  // namespace
@@ -768,67 +850,17 @@ int attn_jvp_fwd_host(const void *q, const void *k, const void *v, const void *t
     if (rc != AJVP_OK || noop) return rc;
     if (d != ajvp::sm100::HD) return AJVP_ERR_UNSUPPORTED_DIM;
     const int64_t BH = B * H;
-    const uint64_t one = stage_layout(Lq, Lk, d, 1).bytes;
-    if (!workspace || !aligned(workspace, kStageAlign) || workspace_bytes < kBuffers * one) return AJVP_ERR_WORKSPACE;
-    // heads per chunk: as many as the workspace holds, at most a quarter of B*H
-    int64_t nh = std::min<int64_t>((int64_t)(workspace_bytes / (kBuffers * one)), (BH + 3) / 4);
-    while (nh > 1 && kBuffers * stage_layout(Lq, Lk, d, nh).bytes > workspace_bytes) --nh;
-    nh = std::max<int64_t>(nh, 1);
+    const int64_t nh = fwd_host_heads_per_chunk(BH, Lq, Lk, d, workspace_bytes);
+    if (!workspace || !aligned(workspace, kStageAlign) || nh < 1) return AJVP_ERR_WORKSPACE;
     const StageLayout L = stage_layout(Lq, Lk, d, nh);
     int dev = 0;
     if ((rc = device_setup(&dev)) != AJVP_OK) return rc;
 
     HostPipe pipe;
-    cudaError_t e = pipe.create();
+    const cudaError_t e = pipe.create();
     if (e != cudaSuccess) return fail_cuda(e);
-    const cudaStream_t caller = (cudaStream_t)stream;
-    if ((e = cudaEventRecord(pipe.start(), caller)) != cudaSuccess) return fail_cuda(e);
-    for (cudaStream_t s : pipe.st)
-        if ((e = cudaStreamWaitEvent(s, pipe.start(), 0)) != cudaSuccess) return fail_cuda(e);
-
-    const uint64_t qrow = (uint64_t)(Lq * d * 2), krow = (uint64_t)(Lk * d * 2);  // bytes per (b, h) slab
-    const int64_t nchunks = (BH + nh - 1) / nh;
-    const void *src[6] = {q, tq, k, v, tk, tv};
-    const uint64_t dst_off[6] = {L.q, L.tq, L.k, L.v, L.tk, L.tv};
-    for (int64_t c = 0; c < nchunks; ++c) {
-        const int b = (int)(c % kBuffers);
-        const int64_t h0 = c * nh, n = std::min<int64_t>(nh, BH - h0);
-        uint8_t *buf = static_cast<uint8_t *>(workspace) + (uint64_t)b * L.bytes;
-        // copy in, once the chunk that last used this buffer has been copied out
-        if (c >= kBuffers && (e = cudaStreamWaitEvent(pipe.st[0], pipe.out(b), 0)) != cudaSuccess)
-            return fail_cuda(e);
-        for (int t = 0; t < 6; ++t) {
-            const uint64_t row = t < 2 ? qrow : krow;
-            e = cudaMemcpyAsync(buf + dst_off[t], static_cast<const uint8_t *>(src[t]) + (uint64_t)h0 * row,
-                                (uint64_t)n * row, cudaMemcpyHostToDevice, pipe.st[0]);
-            if (e != cudaSuccess) return fail_cuda(e);
-        }
-        if ((e = cudaEventRecord(pipe.in(b), pipe.st[0])) != cudaSuccess) return fail_cuda(e);
-        // compute
-        const cudaStream_t cs = pipe.st[1 + (c & 1)];
-        if ((e = cudaStreamWaitEvent(cs, pipe.in(b), 0)) != cudaSuccess) return fail_cuda(e);
-        rc = launch_sm100<false>(buf + L.q, buf + L.k, buf + L.v, buf + L.tq, buf + L.tk, buf + L.tv, buf + L.o,
-                                 buf + L.to, lse ? reinterpret_cast<float *>(buf + L.lse) : nullptr, 1, n, Lq, Lk,
-                                 d, scale, cs);
-        if (rc != AJVP_OK) return rc;
-        if ((e = cudaEventRecord(pipe.comp(b), cs)) != cudaSuccess) return fail_cuda(e);
-        // copy out (in chunk order on one stream)
-        if ((e = cudaStreamWaitEvent(pipe.st[3], pipe.comp(b), 0)) != cudaSuccess) return fail_cuda(e);
-        e = cudaMemcpyAsync(static_cast<uint8_t *>(o) + (uint64_t)h0 * qrow, buf + L.o, (uint64_t)n * qrow,
-                            cudaMemcpyDeviceToHost, pipe.st[3]);
-        if (e == cudaSuccess)
-            e = cudaMemcpyAsync(static_cast<uint8_t *>(to) + (uint64_t)h0 * qrow, buf + L.to, (uint64_t)n * qrow,
-                                cudaMemcpyDeviceToHost, pipe.st[3]);
-        if (e == cudaSuccess && lse)
-            e = cudaMemcpyAsync(lse + h0 * Lq, buf + L.lse, (uint64_t)(n * Lq * 4), cudaMemcpyDeviceToHost,
-                                pipe.st[3]);
-        if (e != cudaSuccess) return fail_cuda(e);
-        if ((e = cudaEventRecord(pipe.out(b), pipe.st[3])) != cudaSuccess) return fail_cuda(e);
-    }
-    // the caller's stream continues once the last chunk (and so every chunk) is copied out
-    if ((e = cudaStreamWaitEvent(caller, pipe.out((int)((nchunks - 1) % kBuffers)), 0)) != cudaSuccess)
-        return fail_cuda(e);
-    return AJVP_OK;
+    return fwd_host_enqueue(pipe, q, k, v, tq, tk, tv, o, to, lse, BH, Lq, Lk, d, scale, nh, L,
+                            static_cast<uint8_t *>(workspace), (cudaStream_t)stream);
 }
 
 uint64_t attn_jvp_bwd_host_workspace_bytes(int64_t Lq, int64_t Lk, int64_t d, int64_t heads_per_chunk) {
@@ -873,10 +905,15 @@ int attn_jvp_bwd_host(const void *q, const void *k, const void *v, const void *t
     HostPipe pipe;
     cudaError_t e = pipe.create();
     if (e != cudaSuccess) return fail_cuda(e);
+    // after the start event: on an error, wait for the chunks already issued
+    auto bail = [&](int status) {
+        pipe.drain();
+        return status;
+    };
     const cudaStream_t caller = (cudaStream_t)stream;
     if ((e = cudaEventRecord(pipe.start(), caller)) != cudaSuccess) return fail_cuda(e);
     for (cudaStream_t s : pipe.st)
-        if ((e = cudaStreamWaitEvent(s, pipe.start(), 0)) != cudaSuccess) return fail_cuda(e);
+        if ((e = cudaStreamWaitEvent(s, pipe.start(), 0)) != cudaSuccess) return bail(fail_cuda(e));
 
     // bytes per (b, h) slab of each array, in the layout's order
     const uint64_t qrow = (uint64_t)(Lq * d * 2), krow = (uint64_t)(Lk * d * 2), srow = (uint64_t)(Lq * 4);
@@ -891,34 +928,34 @@ int attn_jvp_bwd_host(const void *q, const void *k, const void *v, const void *t
         uint8_t *buf = static_cast<uint8_t *>(workspace) + (uint64_t)b * L.bytes;
         // copy in, once the chunk that last used this buffer has been copied out
         if (c >= kBuffers && (e = cudaStreamWaitEvent(pipe.st[0], pipe.out(b), 0)) != cudaSuccess)
-            return fail_cuda(e);
+            return bail(fail_cuda(e));
         for (int t = 0; t < 12; ++t) {
             e = cudaMemcpyAsync(buf + L.in[t], static_cast<const uint8_t *>(src[t]) + (uint64_t)h0 * in_row[t],
                                 (uint64_t)n * in_row[t], cudaMemcpyHostToDevice, pipe.st[0]);
-            if (e != cudaSuccess) return fail_cuda(e);
+            if (e != cudaSuccess) return bail(fail_cuda(e));
         }
-        if ((e = cudaEventRecord(pipe.in(b), pipe.st[0])) != cudaSuccess) return fail_cuda(e);
+        if ((e = cudaEventRecord(pipe.in(b), pipe.st[0])) != cudaSuccess) return bail(fail_cuda(e));
         // compute: the four backward kernels on the chunk's n (batch, head) slabs
         const cudaStream_t cs = pipe.st[1 + (c & 1)];
-        if ((e = cudaStreamWaitEvent(cs, pipe.in(b), 0)) != cudaSuccess) return fail_cuda(e);
+        if ((e = cudaStreamWaitEvent(cs, pipe.in(b), 0)) != cudaSuccess) return bail(fail_cuda(e));
         rc = bwd_steps(0, 3, 0, BwdPack(), buf + L.in[0], buf + L.in[6], buf + L.in[7], buf + L.in[1], buf + L.in[8],
                        buf + L.in[9], buf + L.in[2], buf + L.in[3], reinterpret_cast<const float *>(buf + L.in[10]),
                        reinterpret_cast<const float *>(buf + L.in[11]), buf + L.in[4], buf + L.in[5],
                        buf + L.out[0], buf + L.out[2], buf + L.out[3], buf + L.out[1], buf + L.out[4],
                        buf + L.out[5], 1, n, Lq, Lk, d, scale, buf + L.stats, L.stats_bytes, cs);
-        if (rc != AJVP_OK) return rc;
-        if ((e = cudaEventRecord(pipe.comp(b), cs)) != cudaSuccess) return fail_cuda(e);
+        if (rc != AJVP_OK) return bail(rc);
+        if ((e = cudaEventRecord(pipe.comp(b), cs)) != cudaSuccess) return bail(fail_cuda(e));
         // copy out (in chunk order on one stream)
-        if ((e = cudaStreamWaitEvent(pipe.st[3], pipe.comp(b), 0)) != cudaSuccess) return fail_cuda(e);
+        if ((e = cudaStreamWaitEvent(pipe.st[3], pipe.comp(b), 0)) != cudaSuccess) return bail(fail_cuda(e));
         for (int t = 0; t < 6; ++t) {
             e = cudaMemcpyAsync(static_cast<uint8_t *>(dst[t]) + (uint64_t)h0 * out_row[t], buf + L.out[t],
                                 (uint64_t)n * out_row[t], cudaMemcpyDeviceToHost, pipe.st[3]);
-            if (e != cudaSuccess) return fail_cuda(e);
+            if (e != cudaSuccess) return bail(fail_cuda(e));
         }
-        if ((e = cudaEventRecord(pipe.out(b), pipe.st[3])) != cudaSuccess) return fail_cuda(e);
+        if ((e = cudaEventRecord(pipe.out(b), pipe.st[3])) != cudaSuccess) return bail(fail_cuda(e));
     }
     if ((e = cudaStreamWaitEvent(caller, pipe.out((int)((nchunks - 1) % kBuffers)), 0)) != cudaSuccess)
-        return fail_cuda(e);
+        return bail(fail_cuda(e));
     return AJVP_OK;
 }
 
@@ -1027,15 +1064,19 @@ extern "C" int attn_jvp_selftest_wait_timeout(uint64_t bound_ns, void *stream) {
 
 // ------------------------------------------- host entry on static scratch
 // attn_jvp_fwd_host_noalloc stages its chunks in this file-scope device
-// array instead of a caller-supplied workspace.  Its device address is looked
-// up once per device (that device current) on the entry point's first call
-// there.  Nothing in it needs to start at zero: every byte a kernel reads is
-// first written by the same call's copies.
+// array instead of a caller-supplied workspace.  On the entry point's first
+// call on a device (that device current) it looks up the array's device
+// address there and creates the pipeline's streams and events, which every
+// later call on the device reuses, so that a call itself creates and frees
+// nothing.  Nothing in the array needs to start at zero: every byte a kernel
+// reads is first written by the same call's copies.
 namespace {
 constexpr uint64_t kNoallocScratchBytes = 64ull << 20;  // 64 MiB per device
 struct NoallocState {
     std::once_flag once;
+    std::mutex enqueue;  // one call at a time enqueues on the shared streams and events
     void *ptr = nullptr;
+    PipeObjects pipe;    // kept until the process exits
     int cuda_error = 0;
 };
 NoallocState g_noalloc[kMaxDevices];
@@ -1051,13 +1092,15 @@ extern "C" int attn_jvp_fwd_host_noalloc(const void *q, const void *k, const voi
     if (rc != AJVP_OK || noop) return rc;
     if (d != ajvp::sm100::HD) return AJVP_ERR_UNSUPPORTED_DIM;
     // one (batch, head) slab, three staging buffers, must fit the scratch
-    if (attn_jvp_host_workspace_bytes(Lq, Lk, d, 1) > kNoallocScratchBytes) return AJVP_ERR_TOO_LARGE;
+    const int64_t nh = fwd_host_heads_per_chunk(B * H, Lq, Lk, d, kNoallocScratchBytes);
+    if (nh < 1) return AJVP_ERR_TOO_LARGE;
     int dev = 0;
     if ((rc = device_setup(&dev)) != AJVP_OK) return rc;
     NoallocState &st = g_noalloc[dev];
     std::call_once(st.once, [&]() {
         void *p = nullptr;
-        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e == cudaSuccess) e = st.pipe.create();
         if (e == cudaSuccess)
             st.ptr = p;
         else
@@ -1067,6 +1110,7 @@ extern "C" int attn_jvp_fwd_host_noalloc(const void *q, const void *k, const voi
         t_last_cuda_error = st.cuda_error;
         return AJVP_ERR_CUDA;
     }
-    return attn_jvp_fwd_host(q, k, v, tq, tk, tv, o, to, lse, B, H, Lq, Lk, d, scale, st.ptr,
-                             kNoallocScratchBytes, stream);
+    std::lock_guard<std::mutex> lock(st.enqueue);
+    return fwd_host_enqueue(st.pipe, q, k, v, tq, tk, tv, o, to, lse, B * H, Lq, Lk, d, scale, nh,
+                            stage_layout(Lq, Lk, d, nh), static_cast<uint8_t *>(st.ptr), (cudaStream_t)stream);
 }

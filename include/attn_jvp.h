@@ -396,7 +396,8 @@ AJVP_API int64_t attn_jvp_bwd_key_split_parts(int64_t B, int64_t H, int64_t Lq, 
  * unchanged until `stream` reaches that point).  Lq == 0 writes zeros to dk,
  * dv, dtk, dtv on the host after synchronising `stream`.  Errors as
  * attn_jvp_bwd; AJVP_ERR_WORKSPACE for a missing, misaligned or too small
- * workspace.
+ * workspace.  On an error after work was enqueued, the call waits for that
+ * work to finish before returning.
  */
 AJVP_API int attn_jvp_bwd_host(const void *q, const void *k, const void *v,
                       const void *tq, const void *tk, const void *tv,
@@ -445,6 +446,8 @@ AJVP_API int attn_jvp_fwd_f32(const float *q, const float *k, const float *v,
  * `stream` afterwards (e.g. a synchronisation) sees the host outputs written.
  * The internal streams and events are created and released per call, so the
  * call must not be made while `stream` is being captured into a CUDA graph.
+ * On an error after work was enqueued, the call waits for that work to
+ * finish before returning, so nothing of it still touches the workspace.
  * Same size, device and error rules as attn_jvp_fwd, plus AJVP_ERR_WORKSPACE.
  */
 AJVP_API int attn_jvp_fwd_host(const void *q, const void *k, const void *v,
@@ -479,14 +482,21 @@ AJVP_API uint64_t attn_jvp_host_workspace_bytes(int64_t Lq, int64_t Lk, int64_t 
  * (for d = 128 about Lq + Lk <= 21800); larger sizes return
  * AJVP_ERR_TOO_LARGE before anything is enqueued.  Chunks hold as many heads
  * as fit, at most a quarter of B*H.
- * Allocates nothing (no cudaMalloc, cudaFree or allocating library call).
- * The first call on a device looks up the array's device address there
- * (cudaGetSymbolAddress, with that device current); make that first call
- * before any stream capture begins.  Nothing in the array needs to start at
- * zero.  The array is shared by every call on the device: calls on one
- * stream are ordered and safe, but calls on different streams (or from
- * different threads) whose executions overlap race on it and give undefined
- * results; serialise them.  Other rules as attn_jvp_fwd_host.
+ * A call allocates nothing: no cudaMalloc, cudaFree or allocating library
+ * call, and no stream or event is created or destroyed.  The first call on a
+ * device does a one-time set-up there, with that device current: it looks up
+ * the array's device address (cudaGetSymbolAddress) and creates the
+ * pipeline's four internal streams and ten events, which every later call on
+ * the device reuses and which are kept until the process exits; make that
+ * first call before any stream capture begins.  If the set-up fails, that
+ * call and every later one on the device return AJVP_ERR_CUDA.  Nothing in
+ * the array needs to start at zero.  The array is shared by every call on
+ * the device: calls on one stream are ordered and safe, but calls on
+ * different streams whose executions overlap race on it and give undefined
+ * results; serialise them.  Calls from several host threads enqueue their
+ * work one at a time.  On an error after work was enqueued, the call waits
+ * for that work to finish before returning.  Other rules as
+ * attn_jvp_fwd_host.
  */
 AJVP_API int attn_jvp_fwd_host_noalloc(const void *q, const void *k, const void *v,
                               const void *tq, const void *tk, const void *tv,

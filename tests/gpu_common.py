@@ -45,10 +45,12 @@ def compare_full(w: Workload, inp: dict, out) -> dict:
     return {"o": max_rel(o, ro), "to": max_rel(to, rto), "lse": max_rel(lse, rlse)}
 
 
-def compare_rows(w: Workload, inp: dict, out, heads, n_rows: int, seed: int = 0) -> dict:
+def compare_rows(w: Workload, inp: dict, out, heads, n_rows: int, seed: int = 0, rows=None) -> dict:
     """Oracle on sampled query rows of sampled heads (rows are independent,
-    so this is the full oracle restricted to them)."""
-    rows = sample_rows(w.Lq, n_rows, seed=seed)
+    so this is the full oracle restricted to them).  ``rows``: an explicit
+    row list instead of the seeded sample."""
+    if rows is None:
+        rows = sample_rows(w.Lq, n_rows, seed=seed)
     fl = {n: flat(t) for n, t in inp.items()}
     got_o, got_to, got_l = [], [], []
     ref_o, ref_to, ref_l = [], [], []

@@ -4,8 +4,16 @@ existing host entry point attn_jvp_fwd_host with a caller workspace: two
 calls in a row on different inputs must each give bit-identical outputs (the
 same kernel on the same slabs; the second call reuses the scratch the first
 one filled).  Kept in a file collected last so that it also runs after every
-other test in the process; it passes alone as well."""
+other test in the process; it passes alone as well.  On the CPU: sizes
+beyond the scratch are rejected before any CUDA call, and the source of the
+entry point and of the pipeline routine it enqueues through creates no
+stream or event and allocates nothing outside its one-time per-device set-up
+(some callers cannot allocate device memory or create CUDA objects per
+call: a plain C caller without a device allocator of its own, or a process
+whose device memory a framework's caching allocator already holds)."""
 import ctypes
+import os
+import re
 
 import pytest
 import torch
@@ -60,3 +68,30 @@ def test_noalloc_rejects_sizes_beyond_the_scratch():
     assert rc == B.AJVP_ERR_TOO_LARGE
     assert lib.attn_jvp_fwd_host_noalloc(p, p, p, p, p, p, p, p, None, 1, 1, 8, 8, 64, 0.1, None) == \
         B.AJVP_ERR_UNSUPPORTED_DIM
+
+
+def _function_body(src, signature_start):
+    """Text of the C function whose definition starts with `signature_start`."""
+    i = src.index(signature_start)
+    j = src.index("{", i)
+    depth = 0
+    for k in range(j, len(src)):
+        depth += {"{": 1, "}": -1}.get(src[k], 0)
+        if depth == 0:
+            return src[j:k + 1]
+    raise AssertionError("unbalanced braces")
+
+
+def test_noalloc_path_creates_nothing_per_call():
+    # the entry point and the pipeline it enqueues through: the only creation is
+    # the one-time set-up inside std::call_once; nothing is freed or destroyed
+    src = open(os.path.join(os.path.dirname(B.__file__), "csrc", "api.cu")).read()
+    entry = _function_body(src, 'extern "C" int attn_jvp_fwd_host_noalloc(')
+    enqueue = _function_body(src, "int fwd_host_enqueue(")
+    once = _function_body(entry, "std::call_once(")
+    creating = re.compile(r"cuda(Malloc\w*|Free\w*|Stream(Create|Destroy)\w*|Event(Create|Destroy)\w*)\s*\("
+                          r"|HostPipe|\.create\(")
+    assert creating.search(enqueue) is None, creating.search(enqueue)
+    outside = entry.replace(once, "")
+    assert creating.search(outside) is None, creating.search(outside)
+    assert "pipe.create()" in once and "cudaGetSymbolAddress" in once
