@@ -112,6 +112,11 @@ constexpr uint32_t OFF_ABORT = OFF_TMEM_SLOT + 4;  // int
 
 constexpr uint32_t TM_O = 0, TM_T = 128, TM_BUF = 256;
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units: P entries stay <= 256
+// kSplit: every SPLIT_FOLD_TILES key tiles the O / T accumulators are added
+// into the fp32 outputs (round-to-nearest fp32 adds on the CUDA cores) and the
+// next tile's products start them afresh in tensor memory, so that no
+// accumulator takes more than SPLIT_FOLD_TILES tiles of tensor-core adds
+constexpr int SPLIT_FOLD_TILES = 32;
 
 // named barriers of the 256 softmax threads
 constexpr uint32_t NB_TILE = 2, NB_EPI = 1;
@@ -166,6 +171,15 @@ constexpr int MASK_CAUSAL = 1, MASK_PACKED = 2;
 // kSplit = true : P and P.*s dS' are each split into bf16 hi + lo parts
 //                 (x = hi + lo to ~16 significant bits), both multiplied into
 //                 O and T, and O, tO are written in fp32; 1.5x the MMA work.
+//                 The tensor cores' fp32 accumulation loses a little on every
+//                 add into a large accumulator, and over tens of thousands of
+//                 keys that loss adds up: so every SPLIT_FOLD_TILES tiles each
+//                 softmax thread adds its row's accumulators into the fp32
+//                 output rows (the running sums live there until the end) and
+//                 the next P.V products overwrite tensor memory instead of
+//                 adding to it.  A rescale of the reference max between folds
+//                 is carried by one factor per row (opend) applied at the next
+//                 fold and in the epilogue.
 template <bool kSplit, int MASK = 0, bool kPersist = false>
 __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_constant__ Params p) {
     static_assert(!kPersist || (!kSplit && MASK == 0), "the persistent form is the unmasked bf16 kernel");
@@ -476,6 +490,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                 mma_commit(BAR(B_VT_EMPTY + s));
                 return true;
             };
+            // key tile t of a unit starts O / T afresh: the unit's first tile and,
+            // with kSplit, each tile whose accumulators were just folded out
+            auto restarts = [](int t) { return t == 0 || (kSplit && t % SPLIT_FOLD_TILES == 0); };
             int n = 0, qt_n = qt, bh_n = bh;
             do {
                 const int G0 = n * nk;
@@ -483,9 +500,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                 if (ok) ok = issue_sd(G0);
                 for (int j = 1; j < nk && ok; ++j) {
                     ok = issue_sd(G0 + j);
-                    if (ok) ok = issue_pv(G0 + j - 1, j == 1, n);
+                    if (ok) ok = issue_pv(G0 + j - 1, restarts(j - 1), n);
                 }
-                if (ok) ok = issue_pv(G0 + nk - 1, nk == 1, n);
+                if (ok) ok = issue_pv(G0 + nk - 1, restarts(nk - 1), n);
                 // O and T are final once everything issued so far completes (a barrier
                 // of its own: a parity wait on a per-tile barrier could be ambiguous here)
                 if (ok) mma_commit(BAR(B_O_FULL));
@@ -539,6 +556,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
             const int G0 = n * nk;  // CTA-wide index of this unit's first key tile
             const int q0_n = qt_n * BR, yq_n = yq0 + q0_n;
             float m_ref = -INFINITY, l = 0.f, g = 0.f;
+            // kSplit: the folded sums in this row's fp32 output columns 64*grp.. of O and
+            // tO, to be multiplied by opend (the rescales since the last fold)
+            float opend = 1.f;
+            // (recomputed where used rather than kept live through the tile loop)
+            auto row_ok = [&]() { return q0_n + row < Lq_s; };  // rows past the sequence are never written
+            auto out_off = [&]() {
+                return ((size_t)bh_n * (size_t)p.Lq + (size_t)(yq_n + row)) * HD + 64u * (uint32_t)grp;
+            };
             // keys this row sees (a prefix of the sequence's keys; may be <= 0 when causal)
             const int kcount = kCausal ? min(Lk_s, q0_n + row + koff + 1) : Lk_s;
 
@@ -597,7 +622,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                     m_ref = m_tile;
                 } else {
                     const bool need = m_tile > m_ref + RESCALE_THRESHOLD;
-                    if (__any_sync(0xffffffffu, need)) {
+                    const bool fold = kSplit && j % SPLIT_FOLD_TILES == 0;  // the same for every thread
+                    if (fold || __any_sync(0xffffffffu, need)) {
                         float alpha = 1.f;
                         if (need) {
                             alpha = ex2_approx(m_ref - m_tile);
@@ -606,10 +632,45 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                         l *= alpha;
                         g *= alpha;
                         // O and T may only be touched once the P.V products of tile j-1
-                        // are complete (the V-side barrier of its stage); group 0
-                        // rescales O, group 1 rescales T
+                        // are complete (the V-side barrier of its stage)
                         failed = !mbar_wait_warp(BAR(B_VT_EMPTY + ((G - 1) & 1)), ((G - 1) >> 1) & 1, abort_flag, bound);
-                        if (!failed) {
+                        if (!failed && fold) {
+                            // sums = (sums * opend + acc) * alpha over this thread's 64 O and
+                            // 64 T columns (the ones its epilogue writes): the first fold
+                            // stores acc * alpha, later ones add acc with fire-and-forget L2
+                            // reductions unless a rescale since the last fold makes them
+                            // read, scale and write the sums.  Tile j's P.V then overwrites
+                            // O / T.
+                            tc_fence_after();
+                            const bool first_fold = j == SPLIT_FOLD_TILES;
+                            const bool plain_add = opend == 1.f && alpha == 1.f;
+#pragma unroll 1
+                            for (int cc = 0; cc < 8; ++cc) {
+                                const uint32_t col = 64u * (uint32_t)grp + 16u * (uint32_t)(cc & 3);
+                                float *dst = (cc < 4 ? p.o_f32 : p.to_f32) + out_off() + 16 * (cc & 3);
+                                uint32_t r[16];
+                                tmem_ld16(tbase + lane_off + (cc < 4 ? TM_O : TM_T) + col, r);
+                                tmem_wait_ld();
+                                if (!row_ok()) continue;
+#pragma unroll
+                                for (int u = 0; u < 4; ++u) {
+                                    float4 v = make_float4(__uint_as_float(r[4 * u]), __uint_as_float(r[4 * u + 1]),
+                                                           __uint_as_float(r[4 * u + 2]), __uint_as_float(r[4 * u + 3]));
+                                    float4 *d4 = reinterpret_cast<float4 *>(dst) + u;
+                                    if (first_fold) {
+                                        *d4 = make_float4(v.x * alpha, v.y * alpha, v.z * alpha, v.w * alpha);
+                                    } else if (plain_add) {
+                                        red_add_f32x4(dst + 4 * u, v.x, v.y, v.z, v.w);
+                                    } else {
+                                        const float4 o = __ldcg(d4);
+                                        *d4 = make_float4(fmaf(o.x, opend, v.x) * alpha, fmaf(o.y, opend, v.y) * alpha,
+                                                          fmaf(o.z, opend, v.z) * alpha, fmaf(o.w, opend, v.w) * alpha);
+                                    }
+                                }
+                            }
+                            opend = 1.f;
+                        } else if (!failed) {
+                            // group 0 rescales O, group 1 rescales T
                             tc_fence_after();
 #pragma unroll 1
                             for (int cc = 0; cc < 4; ++cc) {
@@ -621,6 +682,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                                 for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
                                 tmem_st32(ta, r);
                             }
+                            if (kSplit) opend *= alpha;
                         }
                     }
                 }
@@ -695,26 +757,47 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                 // group grp writes output columns 64*grp .. 64*grp+63
                 if (kSplit) {
                     // fp32 outputs straight from registers, 16 bytes per store
-                    // (packed: rows past the sequence belong to the next one and are not written)
-                    const bool row_ok = q0_n + row < Lq_s;
-                    const size_t off = ((size_t)bh_n * (size_t)p.Lq + (size_t)(yq_n + row)) * HD + 64u * (uint32_t)grp;
+                    // (packed: rows past the sequence belong to the next one and are not written);
+                    // after folds the row's sums so far sit in the same output words
+                    const bool folded = nk > SPLIT_FOLD_TILES;
 #pragma unroll 1
-                    for (int h = 0; h < 2; ++h) {
-                        const int pc = 2 * grp + h;
-                        uint32_t ro[32], rt[32];
-                        tmem_ld32(tbase + lane_off + TM_O + 32u * pc, ro);
-                        tmem_ld32(tbase + lane_off + TM_T + 32u * pc, rt);
-                        tmem_wait_ld();
-                        if (row_ok) {
-                            float4 *po = reinterpret_cast<float4 *>(p.o_f32 + off + 32 * h);
-                            float4 *pt = reinterpret_cast<float4 *>(p.to_f32 + off + 32 * h);
+                    for (int h = 0; h < 4; ++h) {  // 16 output columns at a time
+                        const uint32_t col = 64u * (uint32_t)grp + 16u * (uint32_t)h;
+                        float4 *po = reinterpret_cast<float4 *>(p.o_f32 + out_off() + 16 * h);
+                        float4 *pt = reinterpret_cast<float4 *>(p.to_f32 + out_off() + 16 * h);
+                        float4 so[4], st[4];
+                        if (folded && row_ok()) {
 #pragma unroll
-                            for (int u = 0; u < 8; ++u) {
+                            for (int u = 0; u < 4; ++u) {  // (the folds' L2 reductions included)
+                                so[u] = __ldcg(po + u);
+                                st[u] = __ldcg(pt + u);
+                            }
+                        }
+                        uint32_t ro[16], rt[16];
+                        tmem_ld16(tbase + lane_off + TM_O + col, ro);
+                        tmem_ld16(tbase + lane_off + TM_T + col, rt);
+                        tmem_wait_ld();
+                        if (row_ok()) {
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) {
+                                float ao[4] = {__uint_as_float(ro[4 * u]), __uint_as_float(ro[4 * u + 1]),
+                                               __uint_as_float(ro[4 * u + 2]), __uint_as_float(ro[4 * u + 3])};
+                                float at[4] = {__uint_as_float(rt[4 * u]), __uint_as_float(rt[4 * u + 1]),
+                                               __uint_as_float(rt[4 * u + 2]), __uint_as_float(rt[4 * u + 3])};
+                                if (folded) {
+                                    const float fo[4] = {so[u].x, so[u].y, so[u].z, so[u].w};
+                                    const float ft[4] = {st[u].x, st[u].y, st[u].z, st[u].w};
+#pragma unroll
+                                    for (int e = 0; e < 4; ++e) {
+                                        ao[e] = fmaf(fo[e], opend, ao[e]);
+                                        at[e] = fmaf(ft[e], opend, at[e]);
+                                    }
+                                }
                                 float o4[4], t4[4];
 #pragma unroll
                                 for (int e = 0; e < 4; ++e) {
-                                    o4[e] = __uint_as_float(ro[4 * u + e]) * inv_l;
-                                    t4[e] = fmaf(-mu, o4[e], __uint_as_float(rt[4 * u + e]) * inv_l);
+                                    o4[e] = ao[e] * inv_l;
+                                    t4[e] = fmaf(-mu, o4[e], at[e] * inv_l);
                                 }
                                 po[u] = make_float4(o4[0], o4[1], o4[2], o4[3]);
                                 pt[u] = make_float4(t4[0], t4[1], t4[2], t4[3]);

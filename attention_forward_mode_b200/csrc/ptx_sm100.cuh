@@ -285,6 +285,13 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(uint32_t M, uint32_t N, ui
 }
 
 // ----------------------------------------------------------------- misc
+// four fp32 adds into global memory, performed at the L2 (round to nearest), without
+// waiting for them: x[0..3] += {a, b, c, d}; 16-byte aligned
+__device__ __forceinline__ void red_add_f32x4(float *x, float a, float b, float c, float d) {
+    asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(x), "f"(a), "f"(b), "f"(c), "f"(d)
+                 : "memory");
+}
+
 __device__ __forceinline__ float ex2_approx(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
