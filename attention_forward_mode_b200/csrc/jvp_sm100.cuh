@@ -640,33 +640,49 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                             // stores acc * alpha, later ones add acc with fire-and-forget L2
                             // reductions unless a rescale since the last fold makes them
                             // read, scale and write the sums.  Tile j's P.V then overwrites
-                            // O / T.
+                            // O / T.  Each 16-column block goes through the warp's staging
+                            // slot (row = lane, 16-byte unit u of row r at
+                            // r*64 + ((u ^ ((r >> 1) & 3)) << 4), conflict-free both ways) and
+                            // out as 8 rows x 64 contiguous bytes per instruction, the lanes
+                            // taking the rows' scale factors by shuffle.
                             tc_fence_after();
                             const bool first_fold = j == SPLIT_FOLD_TILES;
-                            const bool plain_add = opend == 1.f && alpha == 1.f;
+                            const uint32_t slot = base + SM_STG + (uint32_t)(warp - 4) * STG_SLOT;
+                            const int rows_here = Lq_s - (q0_n + wl * 32);  // rows of this warp in the sequence
+                            const size_t warp_row0 = (size_t)bh_n * (size_t)p.Lq + (size_t)(yq_n + wl * 32);
 #pragma unroll 1
                             for (int cc = 0; cc < 8; ++cc) {
                                 const uint32_t col = 64u * (uint32_t)grp + 16u * (uint32_t)(cc & 3);
-                                float *dst = (cc < 4 ? p.o_f32 : p.to_f32) + out_off() + 16 * (cc & 3);
                                 uint32_t r[16];
                                 tmem_ld16(tbase + lane_off + (cc < 4 ? TM_O : TM_T) + col, r);
                                 tmem_wait_ld();
-                                if (!row_ok()) continue;
 #pragma unroll
-                                for (int u = 0; u < 4; ++u) {
-                                    float4 v = make_float4(__uint_as_float(r[4 * u]), __uint_as_float(r[4 * u + 1]),
-                                                           __uint_as_float(r[4 * u + 2]), __uint_as_float(r[4 * u + 3]));
-                                    float4 *d4 = reinterpret_cast<float4 *>(dst) + u;
+                                for (int u = 0; u < 4; ++u)
+                                    st_shared_v4(slot + (uint32_t)lane * 64u + (((uint32_t)u ^ (((uint32_t)lane >> 1) & 3u)) << 4),
+                                                 r[4 * u], r[4 * u + 1], r[4 * u + 2], r[4 * u + 3]);
+                                __syncwarp();
+                                float *dst0 = (cc < 4 ? p.o_f32 : p.to_f32) + col;
+#pragma unroll
+                                for (int k = 0; k < 4; ++k) {
+                                    const int rr = 8 * k + (lane >> 2);  // this lane's row of the warp
+                                    const uint32_t u = (uint32_t)lane & 3u;
+                                    const float a_r = __shfl_sync(0xffffffffu, alpha, rr);
+                                    const float o_r = __shfl_sync(0xffffffffu, opend, rr);
+                                    const float4 v = ld_shared_f4(slot + (uint32_t)rr * 64u + ((u ^ (((uint32_t)rr >> 1) & 3u)) << 4));
+                                    if (rr >= rows_here) continue;  // past the sequence: never written
+                                    float *d = dst0 + (warp_row0 + (size_t)rr) * HD + 4u * u;
                                     if (first_fold) {
-                                        *d4 = make_float4(v.x * alpha, v.y * alpha, v.z * alpha, v.w * alpha);
-                                    } else if (plain_add) {
-                                        red_add_f32x4(dst + 4 * u, v.x, v.y, v.z, v.w);
+                                        *reinterpret_cast<float4 *>(d) = make_float4(v.x * a_r, v.y * a_r, v.z * a_r, v.w * a_r);
+                                    } else if (o_r == 1.f && a_r == 1.f) {
+                                        red_add_f32x4(d, v.x, v.y, v.z, v.w);
                                     } else {
-                                        const float4 o = __ldcg(d4);
-                                        *d4 = make_float4(fmaf(o.x, opend, v.x) * alpha, fmaf(o.y, opend, v.y) * alpha,
-                                                          fmaf(o.z, opend, v.z) * alpha, fmaf(o.w, opend, v.w) * alpha);
+                                        const float4 w = __ldcg(reinterpret_cast<const float4 *>(d));
+                                        *reinterpret_cast<float4 *>(d) =
+                                            make_float4(fmaf(w.x, o_r, v.x) * a_r, fmaf(w.y, o_r, v.y) * a_r,
+                                                        fmaf(w.z, o_r, v.z) * a_r, fmaf(w.w, o_r, v.w) * a_r);
                                     }
                                 }
+                                __syncwarp();  // the slot is free again
                             }
                             opend = 1.f;
                         } else if (!failed) {

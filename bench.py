@@ -46,6 +46,9 @@ TRAFFIC_FILE = "profiles/attn_jvp_fwd_kernel.video_selfattn_b1h12_l32760.md"
 FWD_TRAFFIC_FILES = {"video_selfattn_b1h12_l32760_d128": TRAFFIC_FILE,
                      "video_crossattn_b1h40_lq32760_lk512_d128":
                          "profiles/attn_jvp_fwd_kernel_persistent.video_crossattn_b1h40_lq32760_lk512.md"}
+# the same for the fp32-output instantiation (--entry f32out)
+F32OUT_TRAFFIC_FILES = {"video_selfattn_b1h12_l32760_d128":
+                        "profiles/attn_jvp_fwd_kernel_f32out.video_selfattn_b1h12_l32760.md"}
 MASKED_METRIC = "attention+JVP TFLOP/s (12·d per visible query-key pair) and % of B200 BF16 tensor peak"
 BWD_METRIC = "attention+JVP backward TFLOP/s (30·Lq·Lk·d/head) and % of B200 BF16 tensor peak"
 BWD_MASKED_METRIC = ("attention+JVP masked backward TFLOP/s (30·d per visible query-key pair) and % of B200 "
@@ -435,12 +438,15 @@ def run_ours(args, w):
                 "roofline": {"bound": "tensor", "achieved": achieved, "peak": burst, "unit": "TFLOP/s",
                              "frac": achieved / burst,
                              "traffic": committed_traffic(FWD_TRAFFIC_FILES[w.name])
-                             if args.entry == "bf16" and w.name in FWD_TRAFFIC_FILES else None,
+                             if args.entry == "bf16" and w.name in FWD_TRAFFIC_FILES else
+                             committed_traffic(F32OUT_TRAFFIC_FILES[w.name])
+                             if args.entry == "f32out" and w.name in F32OUT_TRAFFIC_FILES else None,
                              "peak_source": f"{src} bf16 dense (burst) from MEASURED_PEAKS.json"
                              if src == "measured" else "fallback 1.59 PFLOP/s",
                              "kernel": "attn_jvp_fwd_kernel" + (" (persistent form)" if persistent else ""),
                              "algorithmic_flops_per_launch": flops,
-                             "algorithmic_bytes_per_launch": w.io_bytes},
+                             "algorithmic_bytes_per_launch": w.io_bytes
+                             + (4 * w.B * w.H * w.Lq * w.d if args.entry == "f32out" else 0)},  # fp32 O, tO
                 "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                         "d2h_bytes_per_step": d2h, "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps,
                         "path": e2e_path},
