@@ -58,7 +58,8 @@ std::atomic<int64_t> g_persist_key_tiles{kDefaultPersistKeyTiles};
 template <bool kSplit, int MASK, bool kPersist = false>
 cudaError_t set_fwd_smem() {
     return cudaFuncSetAttribute(ajvp::sm100::attn_jvp_fwd_kernel<kSplit, MASK, kPersist>,
-                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ajvp::sm100::SMEM_BYTES);
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)(kPersist ? ajvp::sm100::SMEM_BYTES_P : ajvp::sm100::SMEM_BYTES));
 }
 
 template <int VAR, int MASK>
@@ -244,10 +245,11 @@ int launch_sm100(const void *q, const void *k, const void *v, const void *tq, co
 
     const int sm_count = g_dev[dev].sm_count;
     const int64_t nk = (Lk + ajvp::sm100::BC - 1) / ajvp::sm100::BC;
-    if (!kSplit && MASK == 0 && nk <= g_persist_key_tiles.load() && n_cta > sm_count) {
-        // one CTA per SM walks the query tiles
+    if (!kSplit && MASK == 0 && nk >= 3 && nk <= g_persist_key_tiles.load() && n_cta > sm_count) {
+        // one CTA per SM walks the query tiles (its V-side ring keeps the next tile's first
+        // V tile clear of the staged outputs for units of at least three key tiles)
         ajvp::sm100::attn_jvp_fwd_kernel<false, 0, true><<<(unsigned)sm_count, ajvp::sm100::NTHREADS,
-                                                          ajvp::sm100::SMEM_BYTES, (cudaStream_t)stream>>>(p);
+                                                          ajvp::sm100::SMEM_BYTES_P, (cudaStream_t)stream>>>(p);
     } else {
         ajvp::sm100::attn_jvp_fwd_kernel<kSplit, MASK><<<(unsigned)n_cta, ajvp::sm100::NTHREADS,
                                                          ajvp::sm100::SMEM_BYTES, (cudaStream_t)stream>>>(p);

@@ -86,6 +86,16 @@ constexpr uint32_t STG_SLOT = 32 * 64;                 // one softmax warp's 32 
 constexpr uint32_t SM_STG = SM_XCH + 4 * XCH_FLOATS;  // 8 staging slots for the plain-store epilogue
 constexpr uint32_t SMEM_BYTES = SM_STG + 8 * STG_SLOT + 1024;  // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "dynamic shared memory above the sm_100 per-CTA limit");
+// Persistent form: a third V-side stage (the next unit's first V tile never shares a
+// stage with the previous unit's staged outputs); the exchange area holds only the
+// per-tile maxima, which the final l, g exchange reuses; no staging slots, and no
+// alignment slack (the kernel checks that the dynamic shared memory starts on a
+// 1024-byte boundary)
+constexpr int VSTAGES_P = 3;
+constexpr uint32_t SM_BAR_P = SM_VT + VSTAGES_P * VT_STAGE;
+constexpr uint32_t SM_XCH_P = SM_BAR_P + 256;
+constexpr uint32_t SMEM_BYTES_P = SM_XCH_P + 2 * 2 * 128 * 4;
+static_assert(SMEM_BYTES_P <= 232448, "dynamic shared memory above the sm_100 per-CTA limit");
 
 // barrier slots (8 bytes each).  Two MMA commits per key tile:
 //   B_SD_FULL[j % 2]  S_j / dS'_j complete: the softmax may read them, and
@@ -95,16 +105,16 @@ static_assert(SMEM_BYTES <= 232448, "dynamic shared memory above the sm_100 per-
 enum : int {
     B_Q_FULL = 0,
     B_KT_FULL = 1,   // + stage
-    B_VT_FULL = 3,   // + stage
-    B_VT_EMPTY = 5,  // + stage
-    B_SD_FULL = 7,   // + buffer (= K-side stage)
-    B_P_FULL = 9,    // + buffer
-    B_O_FULL = 11,   // every MMA of the unit has completed (one phase per unit)
-    B_MMA_DRAIN = 12,
-    B_OT_FREE = 13,   // persistent: the epilogue has read O / T (one arrival per softmax warp)
-    B_STG_FULL = 14,  // persistent: O, tO staged in the V-side ring (one arrival per softmax warp)
-    B_STG_FREE = 15,  // persistent: + 0 the stores have read O's stage, + 1 tO's as well
-    N_BARS = 17
+    B_VT_FULL = 3,   // + V-side stage (3 in the persistent form)
+    B_VT_EMPTY = 6,  // + V-side stage
+    B_SD_FULL = 9,   // + buffer (= K-side stage)
+    B_P_FULL = 11,   // + buffer
+    B_O_FULL = 13,   // every MMA of the unit has completed (one phase per unit)
+    B_MMA_DRAIN = 14,
+    B_OT_FREE = 15,   // persistent: the epilogue has read O / T (one arrival per softmax warp)
+    B_STG_FULL = 16,  // persistent: O, tO staged in the V-side ring (one arrival per softmax warp)
+    B_STG_FREE = 17,  // persistent: + 0 the stores have read O's stage, + 1 tO's as well
+    N_BARS = 19
 };
 static_assert(STAGES == 2, "the K-side ring reuses the two S/dS' buffer barriers");
 constexpr uint32_t OFF_TMEM_SLOT = 8 * N_BARS;     // u32
@@ -188,6 +198,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t *gbase = smem_raw + (base - raw);
+    // V-side ring depth, barrier area and exchange area of this form
+    constexpr int VST = kPersist ? VSTAGES_P : STAGES;
+    constexpr uint32_t kBar = kPersist ? SM_BAR_P : SM_BAR, kXch = kPersist ? SM_XCH_P : SM_XCH;
+    if (kPersist && base != raw) {  // its layout leaves no alignment slack
+        if (threadIdx.x == 0) atomicOr(&g_status_word, 2);
+        return;
+    }
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -276,9 +293,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
         return;
     }
     const uint64_t bound = p.bound_ns;
-    // persistent: unit n's staged O goes to the V-side stage of unit n + 1's first
-    // key tile (G = (n + 1) * nk), tO to the other stage
-    auto stage_o = [&](int n) -> uint32_t { return SM_VT + (uint32_t)(((n + 1) * nk) % STAGES) * VT_STAGE; };
+    // persistent (nk >= 3): unit n's staged O goes to the V-side stage of unit n + 1's
+    // second key tile (G = (n + 1) * nk + 1), tO to that of its third; unit n's last
+    // two tiles used those stages, and unit n + 1's first tile has the third stage
+    auto stage_o = [&](int n) -> uint32_t { return SM_VT + (uint32_t)(((n + 1) * nk + 1) % VST) * VT_STAGE; };
+    auto stage_t = [&](int n) -> uint32_t { return SM_VT + (uint32_t)(((n + 1) * nk + 2) % VST) * VT_STAGE; };
     // persistent: the n-th unit of this CTA (unit 0 is blockIdx.x, decoded above);
     // false past the last one, else its query tile and outer index
     auto next_unit = [&](int n, int &qt_n, int &bh_n) -> bool {
@@ -289,15 +308,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
         return true;
     };
 
-    const uint32_t bars = base + SM_BAR;
+    const uint32_t bars = base + kBar;
     auto BAR = [&](int i) -> uint32_t { return bars + 8u * (uint32_t)i; };
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + SM_BAR + OFF_TMEM_SLOT);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(gbase + SM_BAR + OFF_ABORT);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + kBar + OFF_TMEM_SLOT);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(gbase + kBar + OFF_ABORT);
 
     if (threadIdx.x == 0) {
         mbar_init(BAR(B_Q_FULL), 1);
-        for (int s = 0; s < STAGES; ++s) {
-            mbar_init(BAR(B_KT_FULL + s), 1);
+        for (int s = 0; s < STAGES; ++s) mbar_init(BAR(B_KT_FULL + s), 1);
+        for (int s = 0; s < VST; ++s) {
             mbar_init(BAR(B_VT_FULL + s), 1);
             mbar_init(BAR(B_VT_EMPTY + s), 1);
         }
@@ -335,8 +354,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
         // ------------------------------------------------------ TMA producer
         if (lane == 0) {
             bool ok = true;
-            int kt_last[STAGES], vt_last[STAGES], q_last = -1;
-            for (int s = 0; s < STAGES; ++s) kt_last[s] = vt_last[s] = -1;
+            int kt_last[STAGES], vt_last[VST], q_last = -1;
+            for (int s = 0; s < STAGES; ++s) kt_last[s] = -1;
+            for (int s = 0; s < VST; ++s) vt_last[s] = -1;
             int n = 0, qt_n = qt, bh_n = bh;
             do {
                 const int G0 = n * nk;  // CTA-wide index of this unit's first key tile
@@ -375,22 +395,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                     }
                     if (t >= 1) {
                         const int i = G0 + t - 1;
-                        const int s = i % STAGES;
-                        if (!mbar_wait(BAR(B_VT_EMPTY + s), ((i / STAGES) & 1) ^ 1, abort_flag, bound)) {
+                        const int s = i % VST;
+                        if (!mbar_wait(BAR(B_VT_EMPTY + s), ((i / VST) & 1) ^ 1, abort_flag, bound)) {
                             ok = false;
                             break;
                         }
-                        // persistent: the V-side ring held the previous unit's staged outputs,
-                        // O in the stage of this unit's first V tile (stored first), tO in
-                        // the other (a unit of one key tile waits for both: this unit's
-                        // epilogue stages into them only after its own P.V completes)
-                        if (kPersist && n > 0 && t <= 2 &&
-                            !mbar_wait(BAR(B_STG_FREE + (t - 1)), (n - 1) & 1, abort_flag, bound)) {
-                            ok = false;
-                            break;
-                        }
-                        if (kPersist && n > 0 && t == 1 && nk == 1 &&
-                            !mbar_wait(BAR(B_STG_FREE + 1), (n - 1) & 1, abort_flag, bound)) {
+                        // persistent: the previous unit's staged O sits in the stage of this
+                        // unit's second V tile (stored first), tO in that of its third; the
+                        // first V tile has a stage of its own and loads as soon as the ring
+                        // frees it, ahead of the previous unit's epilogue
+                        if (kPersist && n > 0 && (t == 2 || t == 3) &&
+                            !mbar_wait(BAR(B_STG_FREE + (t - 2)), (n - 1) & 1, abort_flag, bound)) {
                             ok = false;
                             break;
                         }
@@ -409,10 +424,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
             } while (kPersist && ok && next_unit(++n, qt_n, bh_n));
             // let every copy already issued land before shared memory is released
             if (q_last >= 0) mbar_wait_drain(BAR(B_Q_FULL), q_last & 1, bound);
-            for (int s = 0; s < STAGES; ++s) {
+            for (int s = 0; s < STAGES; ++s)
                 if (kt_last[s] >= 0) mbar_wait_drain(BAR(B_KT_FULL + s), (kt_last[s] / STAGES) & 1, bound);
-                if (vt_last[s] >= 0) mbar_wait_drain(BAR(B_VT_FULL + s), (vt_last[s] / STAGES) & 1, bound);
-            }
+            for (int s = 0; s < VST; ++s)
+                if (vt_last[s] >= 0) mbar_wait_drain(BAR(B_VT_FULL + s), (vt_last[s] / VST) & 1, bound);
         }
         __syncwarp();
     } else if (warp == 1) {
@@ -454,10 +469,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
             };
             // first: the unit's first tile (overwrites O / T); n: the unit
             auto issue_pv = [&](int G, bool first, int n) -> bool {
-                const int s = G % STAGES;
+                const int s = G % VST;  // V-side stage
                 const int b = G & 1;
                 if (!mbar_wait(BAR(B_P_FULL + b), (G >> 1) & 1, abort_flag, bound)) return false;
-                if (!mbar_wait(BAR(B_VT_FULL + s), (G / STAGES) & 1, abort_flag, bound)) return false;
+                if (!mbar_wait(BAR(B_VT_FULL + s), (G / VST) & 1, abort_flag, bound)) return false;
                 // the previous unit's epilogue must have read O / T before they are overwritten
                 if (kPersist && first && n > 0 && !mbar_wait(BAR(B_OT_FREE), (n - 1) & 1, abort_flag, bound))
                     return false;
@@ -522,7 +537,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
             do {
                 if (!mbar_wait(BAR(B_STG_FULL), n & 1, abort_flag, bound) || *abort_flag != 0) break;
                 const int yq_n = yq0 + qt_n * BR;
-                const uint32_t so = stage_o(n), st = SM_VT + VT_STAGE - (so - SM_VT);
+                const uint32_t so = stage_o(n), st = stage_t(n);
                 tma_store_3d(&p.tm_o, base + so, 0, yq_n, bh_n);
                 tma_store_3d(&p.tm_o, base + so + CHUNK_Q, 64, yq_n, bh_n);
                 tma_store_commit();
@@ -549,7 +564,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
         const float2 s2 = make_float2(p.scale, p.scale);
         const bool up = c >= 0.f;  // row max of c*S is c * max(S) (min(S) for c < 0)
         const float sentinel = up ? -INFINITY : INFINITY;
-        float *xch = reinterpret_cast<float *>(gbase + SM_XCH);
+        float *xch = reinterpret_cast<float *>(gbase + kXch);
         bool failed = false;
         int n = 0, qt_n = qt, bh_n = bh;
         do {
@@ -633,7 +648,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                         g *= alpha;
                         // O and T may only be touched once the P.V products of tile j-1
                         // are complete (the V-side barrier of its stage)
-                        failed = !mbar_wait_warp(BAR(B_VT_EMPTY + ((G - 1) & 1)), ((G - 1) >> 1) & 1, abort_flag, bound);
+                        failed = !mbar_wait_warp(BAR(B_VT_EMPTY + (G - 1) % VST), ((G - 1) / VST) & 1, abort_flag, bound);
                         if (!failed && fold) {
                             // sums = (sums * opend + acc) * alpha over this thread's 64 O and
                             // 64 T columns (the ones its epilogue writes): the first fold
@@ -757,7 +772,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
             }
 
             if (!failed) failed = !mbar_wait_warp(BAR(B_O_FULL), n & 1, abort_flag, bound);
-            float *lg = xch + 2 * 2 * 128;  // [l, g][group][row]
+            // [l, g][group][row]; the persistent form reuses the per-tile maxima area, whose
+            // last reads (the unit's last tile) precede every P arrival and so O_FULL
+            float *lg = kPersist ? xch : xch + 2 * 2 * 128;
             if (!failed) {
                 lg[(0 * 2 + grp) * 128 + row] = l;
                 lg[(1 * 2 + grp) * 128 + row] = g;
@@ -767,6 +784,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                 tc_fence_after();
                 const float lt = l + lg[(0 * 2 + (grp ^ 1)) * 128 + row];
                 const float gt = g + lg[(1 * 2 + (grp ^ 1)) * 128 + row];
+                // persistent: every thread has read the other group's l, g before the next
+                // unit's first tile writes its maxima over them
+                if (kPersist) named_bar_sync(NB_EPI, SOFTMAX_THREADS);
                 // a row that saw no key (masks only) has lt = 0: zeros, lse = -inf
                 const float inv_l = (MASK != 0 && !(lt > 0.f)) ? 0.f : 1.f / lt;
                 const float mu = gt * inv_l;
@@ -859,7 +879,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_fwd_kernel(const __grid_
                     const uint32_t chunk_off = (uint32_t)grp * CHUNK_Q + (uint32_t)row * 128u;
                     const uint32_t unit0 = (uint32_t)h * 4u;
                     const uint32_t so = kPersist ? stage_o(n) : SM_Q;
-                    const uint32_t st = kPersist ? SM_VT + VT_STAGE - (so - SM_VT) : SM_TQ;
+                    const uint32_t st = kPersist ? stage_t(n) : SM_TQ;
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
                         const uint32_t phys = (((unit0 + u) ^ (uint32_t)(row & 7)) * 16u);

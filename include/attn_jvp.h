@@ -514,8 +514,8 @@ AJVP_API int attn_jvp_last_cuda_error(void);
  * Synchronise `stream`, then read and clear the device status word of the
  * current device.  Returns AJVP_OK, AJVP_ERR_TIMEOUT (some kernel wait ran
  * past its bound since the last check), AJVP_ERR_DEVICE_LAYOUT (a backward
- * kernel found its dynamic shared memory not 1024-byte aligned and returned
- * without work) or AJVP_ERR_CUDA.
+ * kernel or the persistent forward found its dynamic shared memory not
+ * 1024-byte aligned and returned without work) or AJVP_ERR_CUDA.
  */
 AJVP_API int attn_jvp_check_device_status(void *stream);
 
@@ -528,9 +528,9 @@ AJVP_API int attn_jvp_set_wait_bound_ns(uint64_t ns);
 
 /*
  * Scheduling of the bf16 forward entry points without masks (attn_jvp_fwd,
- * attn_jvp_fwd_stats, the host entries): when the keys span at most
- * `max_key_tiles` tiles of 64 and there are more 128-row query tiles than
- * SMs, one persistent CTA per SM walks the query tiles and overlaps each
+ * attn_jvp_fwd_stats, the host entries): when the keys span at least 3 and
+ * at most `max_key_tiles` tiles of 64 and there are more 128-row query tiles
+ * than SMs, one persistent CTA per SM walks the query tiles and overlaps each
  * tile's epilogue with the next tile's loads and score products (short key
  * sequences, e.g. cross-attention to a few hundred text tokens).  Results are
  * bit-identical either way.  Default 32; 0 turns the persistent form off;

@@ -160,6 +160,50 @@ def test_causal_against_masked_oracle(B, H, Lq, Lk):
     assert err["to"] * 10 <= err_bf["to"], (err, err_bf)
 
 
+def test_causal_long_keys_fold():
+    # long enough that the later query tiles' key ranges pass several folds (every 32
+    # tiles of 64 keys), with a ragged tail on both sides; rows checked: a sample that
+    # includes the first and last tiles
+    B, H, Lq, Lk = 1, 2, 4500, 4600
+    w = custom(B, H, Lq, Lk, 128)
+    inp = gpu_inputs(w, seed=61)
+    names = ("q", "k", "v", "tq", "tk", "tv")
+    got = ajvp.attn_jvp_fwd_f32out_causal(*(inp[n] for n in names), w.scale)
+    torch.cuda.synchronize()
+    rows = sample_rows(Lq, 160, seed=3)
+    fl = {n: t.reshape(-1, t.shape[-2], t.shape[-1]) for n, t in inp.items()}
+    err = {"o": 0.0, "to": 0.0, "lse": 0.0}
+    for h in range(B * H):
+        # each sampled row alone against its visible keys (causal, bottom-right aligned)
+        ref = oracle.attn_jvp_causal(*(fl[n][h][None].cpu() for n in names), w.scale)
+        for i, key in enumerate(("o", "to", "lse")):
+            g = got[i].reshape(-1, Lq, *(() if key == "lse" else (128,)))[h][rows].cpu().numpy()
+            err[key] = max(err[key], max_rel(g, ref[i][0][rows]))
+    print(w.name, "causal, long keys", err)
+    check(err, w.name, Lk)
+
+
+def test_varlen_long_sequences_fold():
+    # packed sequences long enough to fold (2100 and 4200 keys) next to short ones, so
+    # that the folds' row guard keeps a tile's overhang out of the next sequence
+    H, lq, lk = 2, [700, 90, 300], [4200, 130, 2100]
+    g = torch.Generator().manual_seed(78)
+    names = ("q", "k", "v", "tq", "tk", "tv")
+    x = {n: torch.randn((H, sum(lq) if n in ("q", "tq") else sum(lk), 128), generator=g).to(torch.bfloat16).cuda()
+         for n in names}
+    cq = torch.tensor(np.concatenate([[0], np.cumsum(lq)]), dtype=torch.int32, device="cuda")
+    ck = torch.tensor(np.concatenate([[0], np.cumsum(lk)]), dtype=torch.int32, device="cuda")
+    s = 128 ** -0.5
+    for causal in (False, True):
+        got = ajvp.attn_jvp_fwd_f32out_varlen(*(x[n] for n in names), cq, ck, max(lq), s, causal=causal)
+        torch.cuda.synchronize()
+        ref = oracle.attn_jvp_packed(*(x[n] for n in names), s, cq.cpu().numpy(), ck.cpu().numpy(), causal)
+        seen = np.ones(sum(lq), dtype=bool)  # Lq <= Lk in every sequence: every row sees a key
+        err = _masked_err(got, ref, np.broadcast_to(seen[None], (H, sum(lq))))
+        print("varlen long, causal", causal, err)
+        check(err, f"varlen long causal={causal}", max(lk))
+
+
 @pytest.mark.parametrize("causal", [False, True])
 def test_varlen_against_masked_oracle(causal):
     H, lq, lk = 2, [300, 1, 129, 0, 64], [200, 513, 7, 40, 0]
