@@ -56,6 +56,8 @@
 // guarded row stores).
 #pragma once
 
+#include <type_traits>
+
 #include "ptx_sm100.cuh"
 
 namespace ajvp {
@@ -546,8 +548,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
         bool failed = false;
         // one pair of columns (c, c + 1 of this group): x scores, y score tangent,
         // z A, w B -> r1, r2 (see the variant table)
-        auto pair = [&](int c, int lo, int hi, uint32_t st_base, uint32_t xa, uint32_t xb, uint32_t ya, uint32_t yb,
-                        uint32_t za, uint32_t zb, uint32_t wa, uint32_t wb, float2 &r1, float2 &r2) {
+        auto pair = [&](int c, int lo, int hi, bool masked, uint32_t st_base, uint32_t xa, uint32_t xb, uint32_t ya,
+                        uint32_t yb, uint32_t za, uint32_t zb, uint32_t wa, uint32_t wb, float2 &r1, float2 &r2) {
             float4 sa = rs, sb = rs;  // statistics of columns c and c + 1
             if (C::kColStats) {
                 sa = ld_shared_f4(st_base + 16u * c);
@@ -573,8 +575,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
                 r2 = dsb;
             }
             // columns past the end of the tensor, or hidden by the causal mask
-            if (c >= hi || c < lo) r1.x = r2.x = 0.f;
-            if (c + 1 >= hi || c + 1 < lo) r1.y = r2.y = 0.f;
+            if (masked) {
+                if (c >= hi || c < lo) r1.x = r2.x = 0.f;
+                if (c + 1 >= hi || c + 1 < lo) r1.y = r2.y = 0.f;
+            }
         };
 
         for (int j = 0; j < nt; ++j) {
@@ -633,46 +637,73 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
                 }
                 tc_fence_after();
                 // X and Y in two halves of 16 columns; each half's E1, E2 (8 packed columns
-                // each) go over columns of X and Y that half has already read
+                // each) go over columns of X and Y that half has already read.  The
+                // per-column mask only for tiles that reach past the end or cross the
+                // causal diagonal: most tiles see all their columns and take a copy of the
+                // loop without the tests.
+                auto e_halves = [&](auto masked_c) {
+                    constexpr bool kMasked = decltype(masked_c)::value;
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    uint32_t xr[16], yr[16], h1[8], h2[8];
-                    tmem_ld16(tb + col0 + C::X + 16u * hh, xr);
-                    tmem_ld16(tb + col0 + C::Y + 16u * hh, yr);
-                    tmem_wait_ld();
+                    for (int hh = 0; hh < 2; ++hh) {
+                        uint32_t xr[16], yr[16], h1[8], h2[8];
+                        tmem_ld16(tb + col0 + C::X + 16u * hh, xr);
+                        tmem_ld16(tb + col0 + C::Y + 16u * hh, yr);
+                        tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 16; i += 2) {
-                        const int c = 16 * hh + i;
-                        // lse2 of columns c, c + 1 (column statistics: read again from the
-                        // slot, which stays valid until E_DONE)
-                        const float2 ls = C::kColStats ? make_float2(stf[4 * c], stf[4 * c + 4]) : make_float2(rs.x, rs.x);
-                        const float2 x = make_float2(__uint_as_float(xr[i]), __uint_as_float(xr[i + 1]));
-                        const float2 tt = __ffma2_rn(x, c2, make_float2(-ls.x, -ls.y));
-                        const float2 pp = make_float2(ex2_approx(tt.x), ex2_approx(tt.y));
-                        const float2 u = __fmul2_rn(make_float2(__uint_as_float(yr[i]), __uint_as_float(yr[i + 1])), s2);
-                        const float2 zz = make_float2(za[c], za[c + 1]);
-                        const float2 pb = __ffma2_rn(u, zz, make_float2(wz[c], wz[c + 1]));
-                        float2 r1 = __fmul2_rn(pp, pb), r2 = __fmul2_rn(pp, zz);
-                        // columns past the end of the tensor, or hidden by the causal mask
-                        if (c >= hi || c < lo) r1.x = r2.x = 0.f;
-                        if (c + 1 >= hi || c + 1 < lo) r1.y = r2.y = 0.f;
-                        h1[i / 2] = pack_bf16x2(r1.x, r1.y);
-                        h2[i / 2] = pack_bf16x2(r2.x, r2.y);
+                        for (int i = 0; i < 16; i += 2) {
+                            const int c = 16 * hh + i;
+                            // lse2 of columns c, c + 1 (column statistics: read again from the
+                            // slot, which stays valid until E_DONE)
+                            const float2 ls =
+                                C::kColStats ? make_float2(stf[4 * c], stf[4 * c + 4]) : make_float2(rs.x, rs.x);
+                            const float2 x = make_float2(__uint_as_float(xr[i]), __uint_as_float(xr[i + 1]));
+                            const float2 tt = __ffma2_rn(x, c2, make_float2(-ls.x, -ls.y));
+                            const float2 pp = make_float2(ex2_approx(tt.x), ex2_approx(tt.y));
+                            const float2 u =
+                                __fmul2_rn(make_float2(__uint_as_float(yr[i]), __uint_as_float(yr[i + 1])), s2);
+                            const float2 zz = make_float2(za[c], za[c + 1]);
+                            const float2 pb = __ffma2_rn(u, zz, make_float2(wz[c], wz[c + 1]));
+                            float2 r1 = __fmul2_rn(pp, pb), r2 = __fmul2_rn(pp, zz);
+                            if (kMasked) {  // columns past the end of the tensor, or hidden by the causal mask
+                                if (c >= hi || c < lo) r1.x = r2.x = 0.f;
+                                if (c + 1 >= hi || c + 1 < lo) r1.y = r2.y = 0.f;
+                            }
+                            h1[i / 2] = pack_bf16x2(r1.x, r1.y);
+                            h2[i / 2] = pack_bf16x2(r2.x, r2.y);
+                        }
+                        tmem_st8(tb + col0 + C::E1 + 8u * hh, h1);
+                        tmem_st8(tb + col0 + C::E2 + 8u * hh, h2);
                     }
-                    tmem_st8(tb + col0 + C::E1 + 8u * hh, h1);
-                    tmem_st8(tb + col0 + C::E2 + 8u * hh, h2);
-                }
+                };
+                // the choice must be the same for the whole warp: the copies hold
+                // warp-collective tensor-memory loads and stores
+                if (__all_sync(0xffffffffu, lo <= 0 && hi >= 32))
+                    e_halves(std::false_type{});
+                else
+                    e_halves(std::true_type{});
             } else {
                 uint32_t xr[32], yr[32];
                 tmem_ld32(tb + col0 + C::X, xr);
                 tmem_ld32(tb + col0 + C::Y, yr);
                 tmem_wait_ld();
+                // the per-column mask only for tiles that reach past the end or cross the
+                // causal diagonal (most tiles see all their columns); one choice per warp
+                if (__all_sync(0xffffffffu, lo <= 0 && hi >= 32)) {
 #pragma unroll
-                for (int i = 0; i < 32; i += 2) {
-                    float2 r1, r2;
-                    pair(i, lo, hi, st_base, xr[i], xr[i + 1], yr[i], yr[i + 1], 0u, 0u, 0u, 0u, r1, r2);
-                    e1[i / 2] = pack_bf16x2(r1.x, r1.y);
-                    e2[i / 2] = pack_bf16x2(r2.x, r2.y);
+                    for (int i = 0; i < 32; i += 2) {
+                        float2 r1, r2;
+                        pair(i, lo, hi, false, st_base, xr[i], xr[i + 1], yr[i], yr[i + 1], 0u, 0u, 0u, 0u, r1, r2);
+                        e1[i / 2] = pack_bf16x2(r1.x, r1.y);
+                        e2[i / 2] = pack_bf16x2(r2.x, r2.y);
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; i += 2) {
+                        float2 r1, r2;
+                        pair(i, lo, hi, true, st_base, xr[i], xr[i + 1], yr[i], yr[i + 1], 0u, 0u, 0u, 0u, r1, r2);
+                        e1[i / 2] = pack_bf16x2(r1.x, r1.y);
+                        e2[i / 2] = pack_bf16x2(r2.x, r2.y);
+                    }
                 }
             }
             // over this group's own columns of X and Y (the previous tile's G2, which read
