@@ -559,9 +559,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
             const float2 t = __ffma2_rn(x, c2, make_float2(-sa.x, -sb.x));
             const float2 pp = make_float2(ex2_approx(t.x), ex2_approx(t.y));
             if (VAR == V_V) {
-                const float2 u = __fmul2_rn(make_float2(__uint_as_float(ya), __uint_as_float(yb)), s2);
-                r1 = pp;                                                          // P
-                r2 = __fmul2_rn(pp, __fadd2_rn(u, make_float2(-sa.y, -sb.y)));  // P (u - mu)
+                // u - mu = s Y - mu in one packed FMA
+                const float2 umu = __ffma2_rn(make_float2(__uint_as_float(ya), __uint_as_float(yb)), s2,
+                                              make_float2(-sa.y, -sb.y));
+                r1 = pp;                     // P
+                r2 = __fmul2_rn(pp, umu);    // P (u - mu)
             } else {  // dS_bar = P (A - a), S_bar = P (B + A (u - mu) - a u - D)
                 const float2 z = make_float2(__uint_as_float(za), __uint_as_float(zb));
                 const float2 na = make_float2(-sa.z, -sb.z);
@@ -624,11 +626,18 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
                     tmem_wait_ld();
                     warp_arrive_after_tc(BAR(B_X_FREE));
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const float4 st = C::kColStats ? ld_shared_f4(st_base + 16u * i) : rs;
-                        const float z = __uint_as_float(zr[i]);
-                        za[i] = z - st.z;
-                        wz[i] = fmaf(-z, st.y, __uint_as_float(wr[i]) - st.w);
+                    for (int i = 0; i < 32; i += 2) {  // two columns per packed instruction
+                        const float4 sa = C::kColStats ? ld_shared_f4(st_base + 16u * i) : rs;
+                        const float4 sb = C::kColStats ? ld_shared_f4(st_base + 16u * (i + 1)) : rs;
+                        const float2 z = make_float2(__uint_as_float(zr[i]), __uint_as_float(zr[i + 1]));
+                        const float2 w = make_float2(__uint_as_float(wr[i]), __uint_as_float(wr[i + 1]));
+                        const float2 d = __fadd2_rn(z, make_float2(-sa.z, -sb.z));
+                        const float2 e = __ffma2_rn(make_float2(-z.x, -z.y), make_float2(sa.y, sb.y),
+                                                    __fadd2_rn(w, make_float2(-sa.w, -sb.w)));
+                        za[i] = d.x;
+                        za[i + 1] = d.y;
+                        wz[i] = e.x;
+                        wz[i + 1] = e.y;
                     }
                 }
                 if (!mbar_wait_warp(BAR(B_G1_DONE), j & 1, abort_flag, bound)) {
