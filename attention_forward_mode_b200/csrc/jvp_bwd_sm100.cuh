@@ -190,6 +190,34 @@ __global__ void __launch_bounds__(256) bwd_split_reduce_kernel(const float4 *__r
     }
 }
 
+// Bounded warp-wide wait of the elementwise warps: all 32 lanes poll the
+// barrier together and leave when every lane has seen the phase complete
+// (no lane spins alone while the others wait at a reconvergence point, so
+// the warp resumes as soon as the phase flips).  The phase cannot move on
+// again before this warp releases its stage, so a lane that has seen it keeps
+// seeing it and the vote ends.  Lane 0 checks the abort flag and the time
+// bound every 32 polls; on failure it raises the flag and the status bit and
+// the whole warp returns false.
+__device__ __forceinline__ bool ew_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag, uint64_t bound_ns) {
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t n = 1;; ++n) {
+        if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+        if ((n & 31u) == 0) {
+            int bad = 0;
+            if ((threadIdx.x & 31) == 0) {
+                if (*abort_flag) {
+                    bad = 1;
+                } else if (global_timer_ns() - t0 > bound_ns) {
+                    *abort_flag = 1;
+                    atomicOr(&g_status_word, 1);
+                    bad = 1;
+                }
+            }
+            if (__shfl_sync(0xffffffffu, bad, 0)) return false;
+        }
+    }
+}
+
 // Compile-time shape of one variant.
 template <int VAR>
 struct Var {
@@ -587,12 +615,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
             const int b = j % C::kNB, s = j % C::kLS;
             // V_Q, V_K: Z and W first (complete well before X and Y)
             const int g1bar = C::kSingle ? (int)B_ZW_DONE : (int)B_G1_DONE + b;
-            if (!failed) failed = !mbar_wait_warp(BAR(g1bar), (j / C::kNB) & 1, abort_flag, bound);
+            if (!failed) failed = !ew_wait(BAR(g1bar), (j / C::kNB) & 1, abort_flag, bound);
             // the statistics came with the long-ring stage (bulk copy): observe its barrier too
             if (C::kStatsRing && !failed)
-                failed = !mbar_wait_warp(BAR(B_ST_FULL + (j & 1)), (j >> 1) & 1, abort_flag, bound);
+                failed = !ew_wait(BAR(B_ST_FULL + (j & 1)), (j >> 1) & 1, abort_flag, bound);
             else if (C::kColStats && !failed)
-                failed = !mbar_wait_warp(BAR(B_L_FULL + s), (j / C::kLS) & 1, abort_flag, bound);
+                failed = !ew_wait(BAR(B_L_FULL + s), (j / C::kLS) & 1, abort_flag, bound);
             if (failed) continue;
             tc_fence_after();
             // this group's columns lo .. hi - 1 are inside the tensor and visible
@@ -640,7 +668,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
                         wz[i + 1] = e.y;
                     }
                 }
-                if (!mbar_wait_warp(BAR(B_G1_DONE), j & 1, abort_flag, bound)) {
+                if (!ew_wait(BAR(B_G1_DONE), j & 1, abort_flag, bound)) {
                     failed = true;
                     continue;
                 }
@@ -725,7 +753,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
             warp_arrive_after_tc(BAR(B_E_DONE + b));
         }
 
-        if (!failed) failed = !mbar_wait_warp(BAR(B_ACC_FULL), 0, abort_flag, bound);
+        if (!failed) failed = !ew_wait(BAR(B_ACC_FULL), 0, abort_flag, bound);
         const bool any_failed = named_bar_or(NB_EPI, EW_THREADS, failed);
         if (!any_failed) {
             tc_fence_after();
