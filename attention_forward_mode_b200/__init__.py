@@ -18,6 +18,7 @@ from ._binding import (  # noqa: F401
     AJVP_ERR_UNSUPPORTED_DIM,
     AJVP_ERR_WORKSPACE,
     AJVP_OK,
+    DEFAULT_BWD_PAIRS,
     DEFAULT_PERSISTENT_KEY_TILES,
     GRAD_NAMES,
     AttnJvpError,
@@ -47,6 +48,7 @@ from ._binding import (  # noqa: F401
     host_workspace_bytes,
     load_library,
     selftest_wait_timeout,
+    set_bwd_pairs,
     set_persistent_key_tiles,
     set_wait_bound_ns,
     strerror,
@@ -62,6 +64,7 @@ __all__ = [
     "attn_jvp_fwd_stats", "bwd_workspace_bytes", "bwd_key_split_parts", "attn_jvp_fwd", "attn_jvp_fwd_f32",
     "attn_jvp_fwd_f32out", "attn_jvp_fwd_f32out_causal", "attn_jvp_fwd_f32out_varlen", "attn_jvp_fwd_host",
     "attn_jvp_fwd_host_noalloc", "check_device_status", "default_heads_per_chunk", "host_workspace_bytes",
-    "load_library", "selftest_wait_timeout", "set_persistent_key_tiles", "DEFAULT_PERSISTENT_KEY_TILES",
+    "load_library", "selftest_wait_timeout", "set_bwd_pairs", "set_persistent_key_tiles", "DEFAULT_BWD_PAIRS",
+    "DEFAULT_PERSISTENT_KEY_TILES",
     "set_wait_bound_ns", "strerror", "version", "AttnJvpError",
 ]

@@ -36,7 +36,8 @@ EXPORTED = (
     "attn_jvp_bwd_key_split_parts", "attn_jvp_fwd_f32", "attn_jvp_fwd_host", "attn_jvp_fwd_host_noalloc",
     "attn_jvp_host_workspace_bytes", "attn_jvp_bwd_host", "attn_jvp_bwd_host_workspace_bytes",
     "attn_jvp_strerror", "attn_jvp_last_cuda_error", "attn_jvp_check_device_status",
-    "attn_jvp_set_wait_bound_ns", "attn_jvp_set_persistent_key_tiles", "attn_jvp_selftest_wait_timeout",
+    "attn_jvp_set_wait_bound_ns", "attn_jvp_set_persistent_key_tiles", "attn_jvp_set_bwd_pairs",
+    "attn_jvp_selftest_wait_timeout",
     "attn_jvp_version",
 )
 
@@ -116,6 +117,8 @@ def load_library(path: str = LIB_PATH):
         lib.attn_jvp_set_wait_bound_ns.restype = ctypes.c_int
         lib.attn_jvp_set_persistent_key_tiles.argtypes = [ctypes.c_int64]
         lib.attn_jvp_set_persistent_key_tiles.restype = ctypes.c_int
+        lib.attn_jvp_set_bwd_pairs.argtypes = [ctypes.c_int]
+        lib.attn_jvp_set_bwd_pairs.restype = ctypes.c_int
         lib.attn_jvp_selftest_wait_timeout.argtypes = [ctypes.c_uint64, vp]
         lib.attn_jvp_selftest_wait_timeout.restype = ctypes.c_int
         lib.attn_jvp_version.argtypes = []
@@ -643,6 +646,16 @@ def set_persistent_key_tiles(max_key_tiles: int) -> None:
     persistent form of the unmasked bf16 forward (0: never).  Process-wide."""
     _check(load_library().attn_jvp_set_persistent_key_tiles(int(max_key_tiles)),
            "attn_jvp_set_persistent_key_tiles")
+
+
+DEFAULT_BWD_PAIRS = False
+
+
+def set_bwd_pairs(on: bool) -> None:
+    """The backward's unmasked dQ/dtQ and dK/dtK kernels as CTA pairs sharing
+    each tensor-core product, or one CTA per row tile (the default,
+    ``DEFAULT_BWD_PAIRS``).  Process-wide."""
+    _check(load_library().attn_jvp_set_bwd_pairs(1 if on else 0), "attn_jvp_set_bwd_pairs")
 
 
 def selftest_wait_timeout(bound_ns: int, stream=None) -> None:

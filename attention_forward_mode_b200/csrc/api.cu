@@ -55,6 +55,12 @@ int fail_cuda(cudaError_t e) {
 constexpr int64_t kDefaultPersistKeyTiles = 32;
 std::atomic<int64_t> g_persist_key_tiles{kDefaultPersistKeyTiles};
 
+// The unmasked, unsplit dQ and dK kernels run as CTA pairs (cta_group::2)
+// when this is set.  Off by default: on B200 the pairs measured as fast as
+// single CTAs for dQ and 3-4 % slower for dK (the odd CTA's arrivals on the
+// even CTA's barriers add latency to the per-tile chain the kernels wait on).
+std::atomic<int> g_bwd_pairs{0};
+
 template <bool kSplit, int MASK, bool kPersist = false>
 cudaError_t set_fwd_smem() {
     return cudaFuncSetAttribute(ajvp::sm100::attn_jvp_fwd_kernel<kSplit, MASK, kPersist>,
@@ -68,10 +74,17 @@ cudaError_t set_bwd_smem_one() {
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ajvp::bwd::Var<VAR>::SMEM_BYTES);
 }
 
-// every mask instantiation (none, causal, packed, both) of one variant
+// every mask instantiation (none, causal, packed, both) of one variant, and
+// the pair form of the dQ / dK variants
 template <int VAR>
 cudaError_t set_bwd_smem() {
     cudaError_t e = set_bwd_smem_one<VAR, 0>();
+    if constexpr (VAR != ajvp::bwd::V_V) {
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(ajvp::bwd::attn_jvp_bwd_kernel_pair<VAR>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)ajvp::bwd::Var<VAR, true>::SMEM_BYTES);
+    }
     if (e == cudaSuccess) e = set_bwd_smem_one<VAR, 1>();
     if (e == cudaSuccess) e = set_bwd_smem_one<VAR, 2>();
     if (e == cudaSuccess) e = set_bwd_smem_one<VAR, 3>();
@@ -322,7 +335,10 @@ int launch_bwd_var(std::initializer_list<const void *> r, std::initializer_list<
                    int64_t n_seq, int64_t max_row, int64_t n_split = 1, float *partial = nullptr) {
     using namespace ajvp::bwd;
     constexpr bool kPacked = (MASK & MASK_PACKED) != 0;
-    const int64_t n_rtiles = ((kPacked ? max_row : Lrow) + BM - 1) / BM;
+    // CTA pairs: the unmasked dQ / dK kernels, an even number of row tiles per head
+    const bool pair = MASK == 0 && VAR != V_V && g_bwd_pairs.load() != 0;
+    int64_t n_rtiles = ((kPacked ? max_row : Lrow) + BM - 1) / BM;
+    if (pair) n_rtiles = (n_rtiles + 1) / 2 * 2;
     const int64_t n_cta = n_rtiles * BH * (kPacked ? n_seq : 1) * n_split;
     if (n_cta >= (int64_t(1) << 31)) return AJVP_ERR_TOO_LARGE;
     if (n_cta == 0) return AJVP_OK;
@@ -341,6 +357,10 @@ int launch_bwd_var(std::initializer_list<const void *> r, std::initializer_list<
     i = 0;
     for (void *x : out)
         if ((rc = encode_3d(&p.tm_out[i++], x, d, Lrow, BH, 128)) != AJVP_OK) return rc;
+    if (pair) {  // the first streamed tensor of each ring in boxes of 32 rows
+        if ((rc = encode_3d(&p.tm_l32, *l.begin(), d, Lcol, BH, 32)) != AJVP_OK) return rc;
+        if ((rc = encode_3d(&p.tm_s32, *sh.begin(), d, Lcol, BH, 32)) != AJVP_OK) return rc;
+    }
     i = 0;
     for (void *x : out) p.out[i++] = static_cast<__nv_bfloat16 *>(x);
     i = 0;
@@ -359,7 +379,14 @@ int launch_bwd_var(std::initializer_list<const void *> r, std::initializer_list<
     p.scale = scale;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.bound_ns = g_bound_ns.load();
-    attn_jvp_bwd_kernel<VAR, MASK><<<(unsigned)n_cta, NTHREADS, Var<VAR>::SMEM_BYTES, stream>>>(p);
+    if constexpr (MASK == 0 && VAR != V_V) {
+        if (pair)
+            attn_jvp_bwd_kernel_pair<VAR><<<(unsigned)n_cta, NTHREADS, Var<VAR, true>::SMEM_BYTES, stream>>>(p);
+        else
+            attn_jvp_bwd_kernel<VAR, MASK><<<(unsigned)n_cta, NTHREADS, Var<VAR>::SMEM_BYTES, stream>>>(p);
+    } else {
+        attn_jvp_bwd_kernel<VAR, MASK><<<(unsigned)n_cta, NTHREADS, Var<VAR>::SMEM_BYTES, stream>>>(p);
+    }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail_cuda(e);
     return AJVP_OK;
@@ -1027,6 +1054,11 @@ int attn_jvp_set_wait_bound_ns(uint64_t ns) {
 int attn_jvp_set_persistent_key_tiles(int64_t max_key_tiles) {
     if (max_key_tiles < 0) return AJVP_ERR_INVALID_ARG;
     g_persist_key_tiles.store(max_key_tiles);
+    return AJVP_OK;
+}
+
+int attn_jvp_set_bwd_pairs(int on) {
+    g_bwd_pairs.store(on != 0 ? 1 : 0);
     return AJVP_OK;
 }
 

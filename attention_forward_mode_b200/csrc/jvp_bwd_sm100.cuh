@@ -108,6 +108,7 @@ constexpr int MASK_CAUSAL = 1, MASK_PACKED = 2, MASK_SPLIT = 4;
 
 struct Params {
     CUtensorMap tm_r[4], tm_l[2], tm_s[2], tm_out[2];
+    CUtensorMap tm_l32, tm_s32;  // pairs: L0 and S0 in boxes of 32 rows (the B2 halves)
     const float4 *stats;  // [B*H][Lq] {lse*log2(e), mu, a, D}, plus BN rows of padding
     int Lrow, Lcol;       // row-side and streamed lengths (packed: the tensors' totals)
     int Lq;               // query rows per (batch, head): the stats row stride
@@ -218,9 +219,103 @@ __device__ __forceinline__ bool ew_wait(uint32_t bar, uint32_t parity, volatile 
     }
 }
 
-// Compile-time shape of one variant.
-template <int VAR>
+// ------------------------------------------------ CTA pairs (cta_group::2)
+// A pair of CTAs on two SMs of one cluster shares each product: the even CTA
+// issues M = 256 MMAs whose A rows 0..127 come from its own shared (or tensor)
+// memory and rows 128..255 from its peer's, and whose B operand is split by
+// N halves, the first half in the even CTA's shared memory and the second in
+// the odd CTA's, at the same offsets; each CTA's tensor memory receives the
+// accumulator rows of its own A rows, all N columns.
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// shared::cluster address of the same shared-memory offset in CTA `rank`
+__device__ __forceinline__ uint32_t cluster_addr(uint32_t addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+// one arrival (release at cluster scope) on a barrier of another CTA of the cluster
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_bar) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// bounded wait (acquire at cluster scope) for a barrier that other CTAs arrive on
+__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                                  uint64_t bound_ns) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t n = 1;; ++n) {
+        if (mbar_try_wait_cluster(bar, parity)) return true;
+        if ((n & 31u) == 0) {
+            if (*abort_flag) return false;
+            if (global_timer_ns() - t0 > bound_ns) {
+                *abort_flag = 1;
+                atomicOr(&g_status_word, 1);
+                return false;
+            }
+        }
+    }
+}
+// every thread of both CTAs (aligned: whole warps)
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void mma_ss_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void mma_ts_pair(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// one arrival on the barrier at this offset in both CTAs of the pair once the
+// pair's tensor-core operations issued so far have completed
+__device__ __forceinline__ void mma_commit_pair(uint32_t bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            bar),
+        "h"((unsigned short)3)
+        : "memory");
+}
+
+// Compile-time shape of one variant.  kPair: the dQ / dK variants as CTA
+// pairs (the unmasked kernels only).
+template <int VAR, bool kPair = false>
 struct Var {
+    static_assert(!kPair || VAR != V_V, "pairs are built for the dQ and dK variants");
     static constexpr bool kSingle = VAR != V_V;     // one set of X..W (E1, E2 written over X)
     static constexpr bool kColStats = VAR != V_Q;   // statistics per streamed query
     static constexpr int kNR = kSingle ? 4 : 2;     // resident tiles R0..R(kNR-1)
@@ -234,9 +329,16 @@ struct Var {
     // two-slot ring of their own freed by the elementwise warps (V_K)
     static constexpr bool kStatsRing = VAR == V_K;
     // a stage holds two [64 rows][128] tiles x, y as [x c0 | y c0 | x c1 | y c1]
-    // (c = 64-column chunk), so that [x; y] is one N = 128 operand
+    // (c = 64-column chunk), so that [x; y] is one N = 128 operand.
+    // Pairs: each CTA holds its halves of the B operands (x: L0 / S0, y: L1 / S1):
+    //   B1 [c0 | c1]  the N = 128 product's half: y in the even CTA, x in the odd one
+    //   B2 [c0 | c1]  rows 32r .. 32r + 31 of x (CTA r): the N = 64 product's half
+    //   B3            x's columns 64r .. 64r + 63 (long stage only): the N = 128 G2
+    //                 product's half (B1, read MN-major, is the N = 256 one's)
     static constexpr uint32_t L_CH = 2u * CHUNK_C, S_CH = 2u * CHUNK_C;
-    static constexpr uint32_t L_BYTES = 2 * L_CH, S_BYTES = 2 * S_CH;
+    static constexpr uint32_t P_B2 = 2u * CHUNK_C, P_B3 = 3u * CHUNK_C, B2_CH = CHUNK_C / 2;
+    static constexpr uint32_t L_BYTES = kPair ? 4u * CHUNK_C : 2 * L_CH;
+    static constexpr uint32_t S_BYTES = kPair ? 3u * CHUNK_C : 2 * S_CH;
     static constexpr uint32_t SM_L = SM_R + kNR * R_TILE;
     static constexpr uint32_t SM_S = SM_L + kLS * L_BYTES;
     static constexpr uint32_t SM_ST = SM_S + kSS * S_BYTES;  // column statistics
@@ -248,7 +350,11 @@ struct Var {
     // tensor memory: two accumulators, then the score buffer(s)
     static constexpr uint32_t BUF0 = 256u;
     static constexpr uint32_t BUF_COLS = kSingle ? 256u : 128u;
-    static constexpr uint32_t X = 0, Y = 64, Z = 128, W = 192;  // inside a buffer (Z, W: V_Q, V_K)
+    // inside a buffer (Z, W: V_Q, V_K).  The N = 128 products write [X|Y] and
+    // [Z|W]; pairs write [Y|X] and [W|Z] (their first N half is y's), so the
+    // N = 64 products, whose halves are rows of x, accumulate into Y and W
+    static constexpr uint32_t X = kPair ? 64 : 0, Y = kPair ? 0 : 64, Z = kPair ? 192 : 128, W = kPair ? 128 : 192;
+    static constexpr uint32_t G1B_D = 0, G1A_D = 128;  // the N = 128 products' first column
     // E1, E2 (16 packed columns per group) over each group's own columns of X and Y
     static constexpr uint32_t E1 = X, E2 = Y;
     static_assert(BUF0 + kNB * BUF_COLS == 512u, "tensor-memory layout");
@@ -261,19 +367,33 @@ struct Var {
 // start at the sequence's first streamed row and columns past its end are
 // hidden; rows past the sequence's end (the tile may overhang into the next
 // sequence) are computed but not stored.
-template <int VAR, int MASK = 0>
-__global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_constant__ Params p) {
-    using C = Var<VAR>;
+//
+// Pairs (kPair, unmasked V_Q / V_K): a cluster of two CTAs takes row tiles
+// 2m and 2m + 1 of a head.  The even CTA's MMA warp issues every product of
+// the pair (cta_group::2, M = 256) and commits to the barriers of both CTAs;
+// each CTA loads its own resident rows and its halves of the streamed
+// operands; the odd CTA's warp 1 relays the completion of its loads to the
+// even CTA's barriers (one remote arrival each), and its elementwise warps
+// arrive on the even CTA's X_FREE and E_DONE (which count both CTAs' warps).
+// Both CTAs meet at a cluster barrier after setting up and before releasing
+// tensor memory, so neither leaves while the other may still reach it.
+template <int VAR, int MASK, bool kPair>
+__device__ __forceinline__ void bwd_body(const Params &p) {
+    using C = Var<VAR, kPair>;
     constexpr bool kCausal = (MASK & MASK_CAUSAL) != 0, kPacked = (MASK & MASK_PACKED) != 0;
     constexpr bool kSplitK = (MASK & MASK_SPLIT) != 0;
     static_assert(!kSplitK || (MASK == MASK_SPLIT && VAR != V_Q), "the split is for the unmasked key side");
+    static_assert(!kPair || MASK == 0, "pairs are built for the unmasked kernels");
     extern __shared__ __align__(1024) uint8_t bwd_smem[];
     const uint32_t base = smem_u32(bwd_smem);
     if (base & 1023u) {  // the tile layout needs 1024-byte alignment and leaves no slack
+        // (the same in both CTAs of a pair: both leave here)
         if (threadIdx.x == 0) atomicOr(&g_status_word, 2);
         return;
     }
     uint8_t *gbase = bwd_smem;
+    const uint32_t crank = kPair ? cluster_rank() : 0u;  // 0: the CTA that issues the pair's products
+    const bool issuer = crank == 0;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -307,6 +427,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
     const int r0 = rt * BM;  // local first row
     if (kPacked && r0 >= Lrow_s) return;  // past the end of this sequence (uniform for the CTA)
     const int yr = yr0 + r0;              // tensor row of the tile's first row
+    // pairs: the odd CTA of a head's last pair may lie past the end (an odd tile
+    // count); it loads rows 0.. instead, takes its part in the products and stores nothing
+    const bool rows_live = r0 < Lrow_s;
+    const int yr_load = (kPair && !rows_live) ? 0 : yr;
     // streamed tiles jt0 .. jt0 + nt - 1 (local index j = 0 .. nt - 1)
     int jt0 = 0, nt = (Lcol_s + BN - 1) / BN;
     if (kSplitK) {
@@ -333,19 +457,22 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + C::SM_BAR + OFF_TMEM_SLOT);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(gbase + C::SM_BAR + OFF_ABORT);
 
+    // the even CTA of a pair counts its own loads and the odd CTA's relayed ones,
+    // and both CTAs' elementwise warps
+    const uint32_t n_load = (kPair && issuer) ? 2u : 1u, n_ew = (kPair && issuer) ? 2u : 1u;
     if (threadIdx.x == 0) {
-        mbar_init(BAR(B_R_FULL), 1);
+        mbar_init(BAR(B_R_FULL), n_load);
         for (int s = 0; s < 4; ++s) {
-            mbar_init(BAR(B_L_FULL + s), 1);
-            mbar_init(BAR(B_S_FULL + s), 1);
+            mbar_init(BAR(B_L_FULL + s), n_load);
+            mbar_init(BAR(B_S_FULL + s), n_load);
             mbar_init(BAR(B_S_EMPTY + s), 1);
             mbar_init(BAR(B_G2_DONE + s), 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(BAR(B_G1_DONE + b), 1);
-            mbar_init(BAR(B_E_DONE + b), EW_THREADS / 32);  // one arrival per elementwise warp
+            mbar_init(BAR(B_E_DONE + b), n_ew * (EW_THREADS / 32));  // one arrival per elementwise warp
         }
-        mbar_init(BAR(B_X_FREE), EW_THREADS / 32);
+        mbar_init(BAR(B_X_FREE), n_ew * (EW_THREADS / 32));
         mbar_init(BAR(B_ZW_DONE), 1);
         mbar_init(BAR(B_ST_FULL), 1);
         mbar_init(BAR(B_ST_FULL + 1), 1);
@@ -360,15 +487,27 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
             tma_prefetch_desc(&p.tm_l[lane]);
             tma_prefetch_desc(&p.tm_s[lane]);
         }
+        if (kPair && lane == 2) tma_prefetch_desc(&p.tm_l32);
+        if (kPair && lane == 3) tma_prefetch_desc(&p.tm_s32);
     }
     if (warp == 2) {
-        tmem_alloc(smem_u32(tmem_slot), 512);
-        tmem_relinquish();
+        if constexpr (kPair) {  // the same columns in both CTAs (warp 2 of each)
+            tmem_alloc_pair(smem_u32(tmem_slot), 512);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(smem_u32(tmem_slot), 512);
+            tmem_relinquish();
+        }
     }
     tc_fence_before();
-    __syncthreads();
+    if constexpr (kPair)
+        cluster_sync_all();  // both CTAs' barriers initialised before any remote arrival
+    else
+        __syncthreads();
     tc_fence_after();
     const uint32_t tbase = *tmem_slot;
+    // the even CTA's copy of one of this CTA's barriers (pairs)
+    auto LEAD = [&](int i) -> uint32_t { return cluster_addr(BAR(i), 0u); };
 
     if (warp == 0 || warp == 3) {
         // ------------------------------------------------------ TMA producers
@@ -383,8 +522,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
             if (lp) {
                 mbar_arrive_expect_tx(BAR(B_R_FULL), C::kNR * R_TILE);
                 for (int i = 0; i < C::kNR; ++i) {
-                    tma_load_3d(base + SM_R + i * R_TILE, &p.tm_r[i], BAR(B_R_FULL), 0, yr, bh);
-                    tma_load_3d(base + SM_R + i * R_TILE + CHUNK_R, &p.tm_r[i], BAR(B_R_FULL), 64, yr, bh);
+                    tma_load_3d(base + SM_R + i * R_TILE, &p.tm_r[i], BAR(B_R_FULL), 0, yr_load, bh);
+                    tma_load_3d(base + SM_R + i * R_TILE + CHUNK_R, &p.tm_r[i], BAR(B_R_FULL), 64, yr_load, bh);
                 }
             }
             // a stage [x c0 | y c0 | x c1 | y c1] of two streamed tensors, rows y..y+63
@@ -406,7 +545,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
                     const uint32_t fb = BAR(B_L_FULL + s);
                     constexpr bool kWithStats = C::kColStats && !C::kStatsRing;
                     mbar_arrive_expect_tx(fb, 4 * CHUNK_C + (kWithStats ? STATS_TILE : 0));
-                    if (VAR == V_V) {
+                    if constexpr (kPair) {
+                        // B1: y (even CTA) or x (odd CTA); B2: rows 32r.. of x; B3: x's columns 64r..
+                        const uint32_t st = base + C::long_off(s);
+                        const CUtensorMap *b1 = issuer ? &p.tm_l[1] : &p.tm_l[0];
+                        tma_load_3d(st, b1, fb, 0, y, bh);
+                        tma_load_3d(st + CHUNK_C, b1, fb, 64, y, bh);
+                        tma_load_3d(st + C::P_B2, &p.tm_l32, fb, 0, y + 32 * (int)crank, bh);
+                        tma_load_3d(st + C::P_B2 + C::B2_CH, &p.tm_l32, fb, 64, y + 32 * (int)crank, bh);
+                        tma_load_3d(st + C::P_B3, &p.tm_l[0], fb, 64 * (int)crank, y, bh);
+                    } else if (VAR == V_V) {
                         // only G2 reads it, as one N = 256 operand [x | y]: [x c0 | x c1 | y c0 | y c1]
                         const uint32_t st = base + C::long_off(s);
                         tma_load_3d(st, &p.tm_l[0], fb, 0, y, bh);
@@ -427,8 +575,18 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
                         break;
                     }
                     const uint32_t fb = BAR(B_S_FULL + ss);
-                    mbar_arrive_expect_tx(fb, 4 * CHUNK_C);
-                    load_pair(base + C::SM_S + ss * C::S_BYTES, &p.tm_s[0], &p.tm_s[1], fb, y);
+                    const uint32_t st = base + C::SM_S + ss * C::S_BYTES;
+                    if constexpr (kPair) {  // B1: y (even CTA) or x (odd CTA); B2: rows 32r.. of x
+                        mbar_arrive_expect_tx(fb, 3 * CHUNK_C);
+                        const CUtensorMap *b1 = issuer ? &p.tm_s[1] : &p.tm_s[0];
+                        tma_load_3d(st, b1, fb, 0, y, bh);
+                        tma_load_3d(st + CHUNK_C, b1, fb, 64, y, bh);
+                        tma_load_3d(st + C::P_B2, &p.tm_s32, fb, 0, y + 32 * (int)crank, bh);
+                        tma_load_3d(st + C::P_B2 + C::B2_CH, &p.tm_s32, fb, 64, y + 32 * (int)crank, bh);
+                    } else {
+                        mbar_arrive_expect_tx(fb, 4 * CHUNK_C);
+                        load_pair(st, &p.tm_s[0], &p.tm_s[1], fb, y);
+                    }
                     s_last[ss] = t;
                     if (C::kStatsRing) {
                         // statistics slot t % 2: free once the elementwise warps finished tile t - 2
@@ -454,13 +612,36 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
                 if (C::kStatsRing && u >= 0) mbar_wait_drain(BAR(B_ST_FULL + (u & 1)), (u >> 1) & 1, bound);
         }
         __syncwarp();
+    } else if (warp == 1 && kPair && !issuer) {
+        // ------------------------------------- odd CTA of a pair: load relay
+        // the even CTA issues the pair's products once this CTA's halves have
+        // landed too: one remote arrival per completed load, in the order the
+        // products consume them (short stage of tile t, then long stage of tile t)
+        if (lane == 0) {
+            auto relay = [&](int bar, uint32_t parity) -> bool {
+                if (!mbar_wait(BAR(bar), parity, abort_flag, bound)) return false;
+                mbar_arrive_remote(LEAD(bar));
+                return true;
+            };
+            bool ok = relay(B_R_FULL, 0);
+            for (int t = 0; t < nt && ok; ++t)
+                ok = relay(B_S_FULL + t % C::kSS, (t / C::kSS) & 1) && relay(B_L_FULL + t % C::kLS, (t / C::kLS) & 1);
+        }
+        __syncwarp();
     } else if (warp == 1) {
         // -------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            constexpr uint32_t ID_W = idesc_bf16_f32(128, 128, 0);  // R [Cx; Cy]^T
-            constexpr uint32_t ID_N = idesc_bf16_f32(128, 64, 0);   // R Cx^T
-            constexpr uint32_t ID_G2 = idesc_bf16_f32(128, 128, 1);  // E C (C read MN-major)
-            constexpr uint32_t ID_G2W = idesc_bf16_f32(128, 256, 1);  // V_V: E1 [L0 | L1]
+            constexpr uint32_t M = kPair ? 256 : 128;
+            constexpr uint32_t ID_W = idesc_bf16_f32(M, 128, 0);  // R [Cx; Cy]^T
+            constexpr uint32_t ID_N = idesc_bf16_f32(M, 64, 0);   // R Cx^T
+            constexpr uint32_t ID_G2 = idesc_bf16_f32(M, 128, 1);  // E C (C read MN-major)
+            constexpr uint32_t ID_G2W = idesc_bf16_f32(M, 256, 1);  // V_V: E1 [L0 | L1]; pairs: E2 [L1 | L0]
+            auto commit = [&](int bar) {
+                if constexpr (kPair)
+                    mma_commit_pair(BAR(bar));
+                else
+                    mma_commit(BAR(bar));
+            };
             // descriptors of the resident tiles, as scalars (an array captured by the
             // lambdas below would live in local memory and delay every MMA issue)
             const uint64_t dr0 = smem_desc_sw128(base + SM_R, 16, 1024);
@@ -472,11 +653,21 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
                 for (int kk = 0; kk < HD / 16; ++kk) {
                     const uint32_t offr = (kk >> 2) * CHUNK_R + (kk & 3) * 32;
                     const uint32_t offc = (kk >> 2) * ch + (kk & 3) * 32;
-                    mma_ss(d, desc_add(a, offr), desc_add(b, offc), id, (acc || kk > 0) ? 1u : 0u);
+                    if constexpr (kPair)
+                        mma_ss_pair(d, desc_add(a, offr), desc_add(b, offc), id, (acc || kk > 0) ? 1u : 0u);
+                    else
+                        mma_ss(d, desc_add(a, offr), desc_add(b, offc), id, (acc || kk > 0) ? 1u : 0u);
                 }
             };
+            // (pairs: the odd CTA arrives on these barriers too; acquire at cluster scope)
+            auto wait_bar = [&](int bar, uint32_t parity) -> bool {
+                if constexpr (kPair)
+                    return mbar_wait_cluster(BAR(bar), parity, abort_flag, bound);
+                else
+                    return mbar_wait(BAR(bar), parity, abort_flag, bound);
+            };
             auto wait_full = [&](int bar, int j, int stages) -> bool {
-                if (!mbar_wait(BAR(bar + j % stages), (j / stages) & 1, abort_flag, bound)) return false;
+                if (!wait_bar(bar + j % stages, (j / stages) & 1)) return false;
                 tc_fence_after();
                 return true;
             };
@@ -488,16 +679,20 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
                 const uint32_t tb = tbase + C::BUF0 + (uint32_t)b * C::BUF_COLS;
                 const uint64_t ds = smem_desc_sw128(base + C::SM_S + ss * C::S_BYTES, 16, 1024);
                 if (!wait_full(B_S_FULL, j, C::kSS)) return false;
-                if (C::kSingle) {
+                if (kPair) {  // [W|Z] = R2 [S1 | S0]^T by halves, W += R3 S0^T by row halves
+                    g1(tb + C::G1A_D, dr2, ds, CHUNK_C, ID_W, false);
+                    g1(tb + C::W, dr3, desc_add(ds, C::P_B2), C::B2_CH, ID_N, true);
+                    commit(B_ZW_DONE);
+                } else if (C::kSingle) {
                     g1(tb + C::Z, dr2, ds, SC, ID_W, false);
                     g1(tb + C::W, dr3, ds, SC, ID_N, true);
-                    mma_commit(BAR(B_ZW_DONE));
+                    commit(B_ZW_DONE);
                 } else {
                     g1(tb + C::X, dr0, ds, SC, ID_W, false);
                     g1(tb + C::Y, dr1, ds, SC, ID_N, true);
-                    mma_commit(BAR(B_G1_DONE + b));
+                    commit(B_G1_DONE + b);
                 }
-                mma_commit(BAR(B_S_EMPTY + ss));
+                commit(B_S_EMPTY + ss);
                 return true;
             };
             // G1, second part (V_Q, V_K): [X|Y] = R0 [L0; L1]^T, Y += R1 L0^T, over the X
@@ -507,9 +702,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
                 const uint32_t tb = tbase + C::BUF0;
                 const uint64_t dl = smem_desc_sw128(base + C::long_off(j % C::kLS), 16, 1024);
                 if (!wait_full(B_L_FULL, j, C::kLS)) return false;
-                g1(tb + C::X, dr0, dl, LC, ID_W, false);
-                g1(tb + C::Y, dr1, dl, LC, ID_N, true);
-                mma_commit(BAR(B_G1_DONE));
+                if (kPair) {  // [Y|X] = R0 [L1 | L0]^T by halves, Y += R1 L0^T by row halves
+                    g1(tb + C::G1B_D, dr0, dl, CHUNK_C, ID_W, false);
+                    g1(tb + C::Y, dr1, desc_add(dl, C::P_B2), C::B2_CH, ID_N, true);
+                } else {
+                    g1(tb + C::X, dr0, dl, LC, ID_W, false);
+                    g1(tb + C::Y, dr1, dl, LC, ID_N, true);
+                }
+                commit(B_G1_DONE);
                 return true;
             };
             auto issue_g2 = [&](int j) -> bool {
@@ -525,10 +725,21 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
                     for (int kk = 0; kk < BN / 16; ++kk) {
                         // streamed items 16kk..16kk+15: group kk / 2's columns, 8 packed per K-step
                         const uint32_t a_col = (kk >> 1) * 32u + (kk & 1) * 8u;
-                        mma_ts(tbase + acc, e + a_col, desc_add(bm, kk * 2048), id, (!first || j > 0 || kk > 0) ? 1u : 0u);
+                        const uint32_t en = (!first || j > 0 || kk > 0) ? 1u : 0u;
+                        if constexpr (kPair)
+                            mma_ts_pair(tbase + acc, e + a_col, desc_add(bm, kk * 2048), id, en);
+                        else
+                            mma_ts(tbase + acc, e + a_col, desc_add(bm, kk * 2048), id, en);
                     }
                 };
-                if (VAR == V_V) {
+                if (kPair) {
+                    // B1 read MN-major (two 64-column chunks CHUNK_C apart, 8 rows 1024 B apart):
+                    // [acc0 | acc1] += E2 [L1 | L0] (the first product of the tile: it starts
+                    // both accumulators), then acc0 += E1 L0 with B3 (x's columns by halves)
+                    const uint64_t mw = smem_desc_sw128(base + C::long_off(s), CHUNK_C, 1024);
+                    g2(0, e2, mw, ID_G2W, true);
+                    g2(0, e1, desc_add(mw, C::P_B3), ID_G2, false);
+                } else if (VAR == V_V) {
                     // MN-major [L0 | L1]: 64-column chunks CHUNK_C apart (LBO), 8 rows 1024 B apart
                     const uint64_t mw = smem_desc_sw128(base + C::long_off(s), CHUNK_C, 1024);
                     g2(0, e1, mw, ID_G2W, true);                         // [dV | dtV] += E1 [L0 | L1]
@@ -541,10 +752,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
                     g2(0, e2, m1, ID_G2, false);   //       + E2 L1
                     g2(128, e2, m0, ID_G2, true);  // dtQ / dtK += E2 L0
                 }
-                mma_commit(BAR(B_G2_DONE + s));
+                commit(B_G2_DONE + s);
                 return true;
             };
-            bool ok = mbar_wait(BAR(B_R_FULL), 0, abort_flag, bound);
+            bool ok = wait_bar(B_R_FULL, 0);
             // one call site per issue routine.  V_Q, V_K: [X|Y] of tile j, [Z|W] of tile
             // j + 1 once the elementwise warps have read tile j's Z and W (they do so as
             // soon as tile j's [Z|W] completes, long before its [X|Y]), then G2 of tile j.
@@ -552,13 +763,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
             for (int j = -1; j < nt && ok; ++j) {
                 if (C::kSingle && j >= 0 && !(ok = issue_g1b(j))) break;
                 if (j + 1 < nt) {
-                    if (C::kSingle && j >= 0 && !(ok = mbar_wait(BAR(B_X_FREE), j & 1, abort_flag, bound))) break;
+                    if (C::kSingle && j >= 0 && !(ok = wait_bar(B_X_FREE, j & 1))) break;
                     if (!(ok = issue_g1a(j + 1))) break;
                 }
                 if (j >= 0 && !(ok = issue_g2(j))) break;
             }
-            if (ok) mma_commit(BAR(B_ACC_FULL));
-            mma_commit(BAR(B_MMA_DRAIN));
+            if (ok) commit(B_ACC_FULL);
+            commit(B_MMA_DRAIN);
             mbar_wait_drain(BAR(B_MMA_DRAIN), 0, bound);
         }
         __syncwarp();
@@ -574,6 +785,25 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
         float4 rs = make_float4(0.f, 0.f, 0.f, 0.f);  // row statistics {lse2, mu, a, D} (query rows)
         if (!C::kColStats && r0 + row < Lrow_s) rs = p.stats[(size_t)bh * p.Lq + (size_t)(yr + row)];
         bool failed = false;
+        // one arrival per warp for the MMA warp (pairs: on the even CTA's barrier; the
+        // odd CTA's warps also arrive on their own E_DONE, which frees the column
+        // statistics slot for this CTA's producer)
+        auto arrive_mma = [&](int bar, bool local_too) {
+            if constexpr (kPair) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    if (issuer) {
+                        mbar_arrive(BAR(bar));
+                    } else {
+                        mbar_arrive_remote(LEAD(bar));
+                        if (local_too) mbar_arrive(BAR(bar));
+                    }
+                }
+            } else {
+                warp_arrive_after_tc(BAR(bar));
+            }
+        };
         // one pair of columns (c, c + 1 of this group): x scores, y score tangent,
         // z A, w B -> r1, r2 (see the variant table)
         auto pair = [&](int c, int lo, int hi, bool masked, uint32_t st_base, uint32_t xa, uint32_t xb, uint32_t ya,
@@ -652,7 +882,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
                     tmem_ld32(tb + col0 + C::Z, zr);
                     tmem_ld32(tb + col0 + C::W, wr);
                     tmem_wait_ld();
-                    warp_arrive_after_tc(BAR(B_X_FREE));
+                    arrive_mma(B_X_FREE, false);
 #pragma unroll
                     for (int i = 0; i < 32; i += 2) {  // two columns per packed instruction
                         const float4 sa = C::kColStats ? ld_shared_f4(st_base + 16u * i) : rs;
@@ -750,7 +980,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
                 tmem_st16(tb + col0 + C::E2, e2);
             }
             tmem_wait_st();
-            warp_arrive_after_tc(BAR(B_E_DONE + b));
+            arrive_mma(B_E_DONE + b, true);
         }
 
         if (!failed) failed = !ew_wait(BAR(B_ACC_FULL), 0, abort_flag, bound);
@@ -815,7 +1045,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
         }
         fence_proxy_async_smem();
         named_bar_sync(NB_EPI, EW_THREADS);  // staging complete
-        if (!kPacked && !kSplitK && warp == 4 && lane == 0 && !any_failed && *abort_flag == 0) {
+        if (!kPacked && !kSplitK && warp == 4 && lane == 0 && !any_failed && *abort_flag == 0 && rows_live) {
             for (int a = 0; a < 2; ++a) {
                 tma_store_3d(&p.tm_out[a], base + SM_R + a * R_TILE, 0, yr, bh);
                 tma_store_3d(&p.tm_out[a], base + SM_R + a * R_TILE + CHUNK_R, 64, yr, bh);
@@ -827,11 +1057,29 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_
     }
 
     tc_fence_before();
-    __syncthreads();
+    if constexpr (kPair)
+        cluster_sync_all();  // the peer's loads, relays, arrivals and products are all over
+    else
+        __syncthreads();
     if (warp == 2) {
         tc_fence_after();
-        tmem_dealloc(tbase, 512);
+        if constexpr (kPair)
+            tmem_dealloc_pair(tbase, 512);
+        else
+            tmem_dealloc(tbase, 512);
     }
+}
+
+template <int VAR, int MASK = 0>
+__global__ void __launch_bounds__(NTHREADS, 1) attn_jvp_bwd_kernel(const __grid_constant__ Params p) {
+    bwd_body<VAR, MASK, false>(p);
+}
+
+// The dQ / dK variants as CTA pairs (grid: an even number of row tiles per head).
+template <int VAR>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
+    attn_jvp_bwd_kernel_pair(const __grid_constant__ Params p) {
+    bwd_body<VAR, 0, true>(p);
 }
 
 }  // namespace bwd

@@ -540,6 +540,22 @@ AJVP_API int attn_jvp_set_wait_bound_ns(uint64_t ns);
 AJVP_API int attn_jvp_set_persistent_key_tiles(int64_t max_key_tiles);
 
 /*
+ * Scheduling of the backward's unmasked dQ/dtQ and dK/dtK kernels (steps 1
+ * and 2 of attn_jvp_bwd, attn_jvp_bwd_step and attn_jvp_bwd_host, without a
+ * split key side): with `on` != 0 two CTAs on two SMs of a cluster share
+ * each tensor-core product (cta_group::2, 256 rows per product), each
+ * holding its own 128 rows and half of each streamed operand; with 0 (the
+ * default) every CTA works alone.  The pairs read half the shared-memory B
+ * operand per product, which on B200 bought no time (dQ as fast, dK 3-4 %
+ * slower: the kernels wait on their per-tile chain, to which the pairs add
+ * cross-CTA arrivals).  The two forms add the same products in a different
+ * order within a tile, so results agree to rounding, not bit for bit.
+ * Applies to launches made after the call, process-wide.  Returns AJVP_OK.
+ * A scheduling choice with no counterpart in the method.
+ */
+AJVP_API int attn_jvp_set_bwd_pairs(int on);
+
+/*
  * Failure-detection self test: enqueue a one-warp kernel that waits, through
  * the same bounded-wait routine the attention kernel uses, on a barrier that
  * nothing ever completes, with a bound of `bound_ns`.  The kernel gives up,

@@ -181,3 +181,10 @@ def test_persistent_key_tiles_setting(lib):
     assert lib.attn_jvp_set_persistent_key_tiles(-1) == B.AJVP_ERR_INVALID_ARG
     assert lib.attn_jvp_set_persistent_key_tiles(0) == B.AJVP_OK
     assert lib.attn_jvp_set_persistent_key_tiles(B.DEFAULT_PERSISTENT_KEY_TILES) == B.AJVP_OK
+
+
+def test_bwd_pairs_setting(lib):
+    """The backward's pair switch takes any int (0 off, else on) and needs no GPU."""
+    assert lib.attn_jvp_set_bwd_pairs(0) == B.AJVP_OK
+    assert lib.attn_jvp_set_bwd_pairs(7) == B.AJVP_OK
+    assert lib.attn_jvp_set_bwd_pairs(1) == B.AJVP_OK

@@ -70,14 +70,20 @@ def test_causal_stats_forward():
 
 def test_single_query_row_equals_unmasked():
     # one query row sees every key (bottom-right alignment): the causal kernels do
-    # the unmasked arithmetic, bit for bit
+    # the unmasked arithmetic, bit for bit (the unmasked call with its dQ / dK
+    # kernels one CTA per row tile, as the causal ones run: the CTA-pair form adds
+    # each tile's products in another order)
     w = custom(1, 3, 1, 517, 128)
     inp = gpu_inputs(w, seed=22)
     cot = make_cotangents(w, seed=23, device="cuda")
     got, _ = run(inp, cot, w.scale)
     o, to, lse, mu = ajvp.attn_jvp_fwd_stats(*(inp[n] for n in NAMES), w.scale)
-    ref = ajvp.attn_jvp_bwd(*(inp[n] for n in NAMES), o, to, lse, mu, cot["dout"], cot["dtout"], w.scale)
-    torch.cuda.synchronize()
+    ajvp.set_bwd_pairs(False)
+    try:
+        ref = ajvp.attn_jvp_bwd(*(inp[n] for n in NAMES), o, to, lse, mu, cot["dout"], cot["dtout"], w.scale)
+        torch.cuda.synchronize()
+    finally:
+        ajvp.set_bwd_pairs(ajvp.DEFAULT_BWD_PAIRS)
     for n in GRADS:
         assert torch.equal(got[n], ref[n]), n
 

@@ -133,7 +133,9 @@ def test_varlen(lq, lk, causal):
 def test_one_sequence_equals_dense(causal):
     # one packed sequence: the dense kernels' arithmetic, bit for bit (the packed
     # epilogue stores rows directly instead of through the tensor-store unit; the
-    # dense call gets the statistics-only workspace, so its key side does not split)
+    # dense call gets the statistics-only workspace, so its key side does not split,
+    # and runs its dQ / dK kernels one CTA per row tile, as the packed ones do: the
+    # CTA-pair form adds each tile's products in another order)
     w = custom(1, 3, 333, 517, 128)
     inp = gpu_inputs(w, seed=41)
     cot = make_cotangents(w, seed=42, device="cuda")
@@ -141,7 +143,12 @@ def test_one_sequence_equals_dense(causal):
     bwd = ajvp.attn_jvp_bwd_causal if causal else ajvp.attn_jvp_bwd
     o, to, lse, mu = fwd(*(inp[n] for n in NAMES), w.scale)
     ws = torch.empty(ajvp.bwd_workspace_bytes(w.B, w.H, w.Lq), dtype=torch.uint8, device="cuda")
-    dense = bwd(*(inp[n] for n in NAMES), o, to, lse, mu, cot["dout"], cot["dtout"], w.scale, workspace=ws)
+    ajvp.set_bwd_pairs(False)
+    try:
+        dense = bwd(*(inp[n] for n in NAMES), o, to, lse, mu, cot["dout"], cot["dtout"], w.scale, workspace=ws)
+        torch.cuda.synchronize()
+    finally:
+        ajvp.set_bwd_pairs(ajvp.DEFAULT_BWD_PAIRS)
     x = {n: t[0] for n, t in {**inp, **cot}.items()}
     cq = torch.tensor([0, w.Lq], dtype=torch.int32, device="cuda")
     ck = torch.tensor([0, w.Lk], dtype=torch.int32, device="cuda")
