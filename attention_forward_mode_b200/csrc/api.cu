@@ -220,6 +220,7 @@ int launch_sm100(const void *q, const void *k, const void *v, const void *tq, co
     int dev = 0;
     rc = device_setup(&dev);
     if (rc != AJVP_OK) return rc;
+
     rc = get_encoder();
     if (rc != AJVP_OK) return rc;
 

@@ -269,6 +269,23 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
         }
     }
 }
+// the odd CTA of a pair announces its part of a load on the even CTA's barrier
+// (one arrival plus the bytes its copies will complete there)
+__device__ __forceinline__ void mbar_arrive_expect_tx_remote(uint32_t cluster_bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(cluster_bar),
+                 "r"(bytes)
+                 : "memory");
+}
+// 3-D tiled load global -> this CTA's shared memory whose completion is counted
+// (bytes) on a barrier of either CTA of the pair (cta_group::2; no multicast)
+__device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const void *tmap, uint32_t cluster_bar, int x, int y,
+                                                 int z) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, "
+        "%5}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(cluster_bar), "r"(x), "r"(y), "r"(z)
+        : "memory");
+}
 // every thread of both CTAs (aligned: whole warps)
 __device__ __forceinline__ void cluster_sync_all() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
@@ -372,9 +389,10 @@ struct Var {
 // 2m and 2m + 1 of a head.  The even CTA's MMA warp issues every product of
 // the pair (cta_group::2, M = 256) and commits to the barriers of both CTAs;
 // each CTA loads its own resident rows and its halves of the streamed
-// operands; the odd CTA's warp 1 relays the completion of its loads to the
-// even CTA's barriers (one remote arrival each), and its elementwise warps
-// arrive on the even CTA's X_FREE and E_DONE (which count both CTAs' warps).
+// operands, and the copies of both complete on the even CTA's barriers
+// (cta_group::2 loads, each CTA announcing its bytes there); the odd CTA's
+// elementwise warps arrive on the even CTA's X_FREE and E_DONE (which count
+// both CTAs' warps).
 // Both CTAs meet at a cluster barrier after setting up and before releasing
 // tensor memory, so neither leaves while the other may still reach it.
 template <int VAR, int MASK, bool kPair>
@@ -457,7 +475,7 @@ __device__ __forceinline__ void bwd_body(const Params &p) {
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + C::SM_BAR + OFF_TMEM_SLOT);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(gbase + C::SM_BAR + OFF_ABORT);
 
-    // the even CTA of a pair counts its own loads and the odd CTA's relayed ones,
+    // the even CTA of a pair counts its own loads and the odd CTA's,
     // and both CTAs' elementwise warps
     const uint32_t n_load = (kPair && issuer) ? 2u : 1u, n_ew = (kPair && issuer) ? 2u : 1u;
     if (threadIdx.x == 0) {
@@ -515,15 +533,30 @@ __device__ __forceinline__ void bwd_body(const Params &p) {
         // two rings are released at different points, so neither waits on the other)
         const bool lp = warp == 0;
         if (lane == 0) {
+            // pairs: both CTAs' copies of the resident tiles and the rings complete on the
+            // even CTA's barriers (cta_group::2 loads), each CTA announcing its own bytes
+            // there; the odd CTA's own barriers of these kinds stay unused
+            auto expect = [&](int bar, uint32_t bytes) {
+                if (kPair && !issuer)
+                    mbar_arrive_expect_tx_remote(LEAD(bar), bytes);
+                else
+                    mbar_arrive_expect_tx(BAR(bar), bytes);
+            };
+            auto load = [&](uint32_t dst, const CUtensorMap *m, int bar, int x, int y) {
+                if constexpr (kPair)
+                    tma_load_3d_pair(dst, m, LEAD(bar), x, y, bh);
+                else
+                    tma_load_3d(dst, m, BAR(bar), x, y, bh);
+            };
             bool ok = true;
             int l_last[C::kLS], s_last[C::kSS], st_last = -1;
             for (int s = 0; s < C::kLS; ++s) l_last[s] = -1;
             for (int s = 0; s < C::kSS; ++s) s_last[s] = -1;
             if (lp) {
-                mbar_arrive_expect_tx(BAR(B_R_FULL), C::kNR * R_TILE);
+                expect(B_R_FULL, C::kNR * R_TILE);
                 for (int i = 0; i < C::kNR; ++i) {
-                    tma_load_3d(base + SM_R + i * R_TILE, &p.tm_r[i], BAR(B_R_FULL), 0, yr_load, bh);
-                    tma_load_3d(base + SM_R + i * R_TILE + CHUNK_R, &p.tm_r[i], BAR(B_R_FULL), 64, yr_load, bh);
+                    load(base + SM_R + i * R_TILE, &p.tm_r[i], B_R_FULL, 0, yr_load);
+                    load(base + SM_R + i * R_TILE + CHUNK_R, &p.tm_r[i], B_R_FULL, 64, yr_load);
                 }
             }
             // a stage [x c0 | y c0 | x c1 | y c1] of two streamed tensors, rows y..y+63
@@ -544,16 +577,18 @@ __device__ __forceinline__ void bwd_body(const Params &p) {
                     }
                     const uint32_t fb = BAR(B_L_FULL + s);
                     constexpr bool kWithStats = C::kColStats && !C::kStatsRing;
-                    mbar_arrive_expect_tx(fb, 4 * CHUNK_C + (kWithStats ? STATS_TILE : 0));
+                    if (!kPair) mbar_arrive_expect_tx(fb, 4 * CHUNK_C + (kWithStats ? STATS_TILE : 0));
                     if constexpr (kPair) {
                         // B1: y (even CTA) or x (odd CTA); B2: rows 32r.. of x; B3: x's columns 64r..
                         const uint32_t st = base + C::long_off(s);
                         const CUtensorMap *b1 = issuer ? &p.tm_l[1] : &p.tm_l[0];
-                        tma_load_3d(st, b1, fb, 0, y, bh);
-                        tma_load_3d(st + CHUNK_C, b1, fb, 64, y, bh);
-                        tma_load_3d(st + C::P_B2, &p.tm_l32, fb, 0, y + 32 * (int)crank, bh);
-                        tma_load_3d(st + C::P_B2 + C::B2_CH, &p.tm_l32, fb, 64, y + 32 * (int)crank, bh);
-                        tma_load_3d(st + C::P_B3, &p.tm_l[0], fb, 64 * (int)crank, y, bh);
+                        const int fi = B_L_FULL + s;
+                        expect(fi, 4 * CHUNK_C);
+                        load(st, b1, fi, 0, y);
+                        load(st + CHUNK_C, b1, fi, 64, y);
+                        load(st + C::P_B2, &p.tm_l32, fi, 0, y + 32 * (int)crank);
+                        load(st + C::P_B2 + C::B2_CH, &p.tm_l32, fi, 64, y + 32 * (int)crank);
+                        load(st + C::P_B3, &p.tm_l[0], fi, 64 * (int)crank, y);
                     } else if (VAR == V_V) {
                         // only G2 reads it, as one N = 256 operand [x | y]: [x c0 | x c1 | y c0 | y c1]
                         const uint32_t st = base + C::long_off(s);
@@ -577,12 +612,13 @@ __device__ __forceinline__ void bwd_body(const Params &p) {
                     const uint32_t fb = BAR(B_S_FULL + ss);
                     const uint32_t st = base + C::SM_S + ss * C::S_BYTES;
                     if constexpr (kPair) {  // B1: y (even CTA) or x (odd CTA); B2: rows 32r.. of x
-                        mbar_arrive_expect_tx(fb, 3 * CHUNK_C);
+                        const int fi = B_S_FULL + ss;
+                        expect(fi, 3 * CHUNK_C);
                         const CUtensorMap *b1 = issuer ? &p.tm_s[1] : &p.tm_s[0];
-                        tma_load_3d(st, b1, fb, 0, y, bh);
-                        tma_load_3d(st + CHUNK_C, b1, fb, 64, y, bh);
-                        tma_load_3d(st + C::P_B2, &p.tm_s32, fb, 0, y + 32 * (int)crank, bh);
-                        tma_load_3d(st + C::P_B2 + C::B2_CH, &p.tm_s32, fb, 64, y + 32 * (int)crank, bh);
+                        load(st, b1, fi, 0, y);
+                        load(st + CHUNK_C, b1, fi, 64, y);
+                        load(st + C::P_B2, &p.tm_s32, fi, 0, y + 32 * (int)crank);
+                        load(st + C::P_B2 + C::B2_CH, &p.tm_s32, fi, 64, y + 32 * (int)crank);
                     } else {
                         mbar_arrive_expect_tx(fb, 4 * CHUNK_C);
                         load_pair(st, &p.tm_s[0], &p.tm_s[1], fb, y);
@@ -602,8 +638,14 @@ __device__ __forceinline__ void bwd_body(const Params &p) {
                     }
                 }
             }
-            // every copy already issued lands before shared memory is released
-            if (lp) mbar_wait_drain(BAR(B_R_FULL), 0, bound);
+            // every copy already issued lands before shared memory is released (pairs: the
+            // even CTA drains both CTAs' copies, and the cluster barrier at the end keeps the
+            // odd CTA's shared memory until then; the statistics copies stay local)
+            if (kPair && !issuer) {
+                for (int s = 0; s < C::kLS; ++s) l_last[s] = -1;
+                for (int s = 0; s < C::kSS; ++s) s_last[s] = -1;
+            }
+            if (lp && (!kPair || issuer)) mbar_wait_drain(BAR(B_R_FULL), 0, bound);
             for (int s = 0; s < C::kLS; ++s)
                 if (l_last[s] >= 0) mbar_wait_drain(BAR(B_L_FULL + s), (l_last[s] / C::kLS) & 1, bound);
             for (int s = 0; s < C::kSS; ++s)
@@ -612,25 +654,10 @@ __device__ __forceinline__ void bwd_body(const Params &p) {
                 if (C::kStatsRing && u >= 0) mbar_wait_drain(BAR(B_ST_FULL + (u & 1)), (u >> 1) & 1, bound);
         }
         __syncwarp();
-    } else if (warp == 1 && kPair && !issuer) {
-        // ------------------------------------- odd CTA of a pair: load relay
-        // the even CTA issues the pair's products once this CTA's halves have
-        // landed too: one remote arrival per completed load, in the order the
-        // products consume them (short stage of tile t, then long stage of tile t)
-        if (lane == 0) {
-            auto relay = [&](int bar, uint32_t parity) -> bool {
-                if (!mbar_wait(BAR(bar), parity, abort_flag, bound)) return false;
-                mbar_arrive_remote(LEAD(bar));
-                return true;
-            };
-            bool ok = relay(B_R_FULL, 0);
-            for (int t = 0; t < nt && ok; ++t)
-                ok = relay(B_S_FULL + t % C::kSS, (t / C::kSS) & 1) && relay(B_L_FULL + t % C::kLS, (t / C::kLS) & 1);
-        }
-        __syncwarp();
     } else if (warp == 1) {
         // -------------------------------------------------------- MMA issuer
-        if (lane == 0) {
+        // (pairs: the even CTA's; the odd CTA's warp 1 has nothing to do)
+        if (lane == 0 && (!kPair || issuer)) {
             constexpr uint32_t M = kPair ? 256 : 128;
             constexpr uint32_t ID_W = idesc_bf16_f32(M, 128, 0);  // R [Cx; Cy]^T
             constexpr uint32_t ID_N = idesc_bf16_f32(M, 64, 0);   // R Cx^T
@@ -1058,7 +1085,7 @@ __device__ __forceinline__ void bwd_body(const Params &p) {
 
     tc_fence_before();
     if constexpr (kPair)
-        cluster_sync_all();  // the peer's loads, relays, arrivals and products are all over
+        cluster_sync_all();  // the peer's loads, arrivals and products are all over
     else
         __syncthreads();
     if (warp == 2) {

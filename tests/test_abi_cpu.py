@@ -188,3 +188,4 @@ def test_bwd_pairs_setting(lib):
     assert lib.attn_jvp_set_bwd_pairs(0) == B.AJVP_OK
     assert lib.attn_jvp_set_bwd_pairs(7) == B.AJVP_OK
     assert lib.attn_jvp_set_bwd_pairs(1) == B.AJVP_OK
+
