@@ -56,9 +56,8 @@ constexpr int64_t kDefaultPersistKeyTiles = 32;
 std::atomic<int64_t> g_persist_key_tiles{kDefaultPersistKeyTiles};
 
 // The unmasked, unsplit dQ and dK kernels run as CTA pairs (cta_group::2)
-// when this is set.  Off by default: on B200 the pairs measured as fast as
-// single CTAs for dQ and 3-4 % slower for dK (the odd CTA's arrivals on the
-// even CTA's barriers add latency to the per-tile chain the kernels wait on).
+// when this is set.  Off by default: on B200 the pairs measured 4-5 % slower
+// than single CTAs for both kernels.
 std::atomic<int> g_bwd_pairs{0};
 
 template <bool kSplit, int MASK, bool kPersist = false>

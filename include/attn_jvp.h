@@ -546,10 +546,11 @@ AJVP_API int attn_jvp_set_persistent_key_tiles(int64_t max_key_tiles);
  * each tensor-core product (cta_group::2, 256 rows per product), each
  * holding its own 128 rows and half of each streamed operand; with 0 (the
  * default) every CTA works alone.  The pairs read half the shared-memory B
- * operand per product, which on B200 bought no time (dQ as fast, dK 3-4 %
- * slower: the kernels wait on their per-tile chain, to which the pairs add
- * cross-CTA arrivals).  The two forms add the same products in a different
- * order within a tile, so results agree to rounding, not bit for bit.
+ * operand per product, which on B200 bought no time (both kernels 4-5 %
+ * slower: the tensor pipe is not bound by the operand reads there, and the
+ * pairs tie each tile to two SMs).  The two forms add the same products in
+ * a different order within a tile, so results agree to rounding, not bit
+ * for bit.
  * Applies to launches made after the call, process-wide.  Returns AJVP_OK.
  * A scheduling choice with no counterpart in the method.
  */
