@@ -277,7 +277,7 @@ __device__ __forceinline__ void mbar_arrive_expect_tx_remote(uint32_t cluster_ba
                  : "memory");
 }
 // 3-D tiled load global -> this CTA's shared memory whose completion is counted
-// (bytes) on a barrier of either CTA of the pair (cta_group::2; no multicast)
+// (bytes) on a barrier of either CTA of the pair (cta_group::2; this CTA is the only destination)
 __device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const void *tmap, uint32_t cluster_bar, int x, int y,
                                                  int z) {
     asm volatile(
