@@ -78,7 +78,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     }
 }
 
-// Warp-wide bounded wait: lane 0 polls, the verdict is broadcast.  Must be
+// Warp-wide bounded wait: lane 0 polls, the outcome is broadcast.  Must be
 // called by all 32 lanes.  After it returns true the caller's tcgen05 loads
 // are ordered by tcgen05.fence::after_thread_sync as usual.
 __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, volatile int *abort_flag,
