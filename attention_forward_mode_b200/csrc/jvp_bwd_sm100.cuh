@@ -603,9 +603,11 @@ __device__ __forceinline__ void bwd_body(const Params &p) {
                         bulk_load(base + C::SM_ST + s * STATS_TILE, p.stats + (size_t)bh * p.Lq + y, STATS_TILE, fb);
                     l_last[s] = t;
                 } else {  // short ring, stage t % kSS: free once G1 of tile t - kSS is complete
+                    // (V_Q, V_K: one stage, freed by the [Z|W] products' own completion barrier)
                     const int ss = t % C::kSS;
+                    const int free_bar = C::kSingle ? (int)B_ZW_DONE : (int)B_S_EMPTY + ss;
                     if (t >= C::kSS &&
-                        !mbar_wait(BAR(B_S_EMPTY + ss), ((t - C::kSS) / C::kSS) & 1, abort_flag, bound)) {
+                        !mbar_wait(BAR(free_bar), ((t - C::kSS) / C::kSS) & 1, abort_flag, bound)) {
                         ok = false;
                         break;
                     }
@@ -706,6 +708,7 @@ __device__ __forceinline__ void bwd_body(const Params &p) {
                 const uint32_t tb = tbase + C::BUF0 + (uint32_t)b * C::BUF_COLS;
                 const uint64_t ds = smem_desc_sw128(base + C::SM_S + ss * C::S_BYTES, 16, 1024);
                 if (!wait_full(B_S_FULL, j, C::kSS)) return false;
+                // V_Q, V_K: ZW_DONE also frees the (single) short stage
                 if (kPair) {  // [W|Z] = R2 [S1 | S0]^T by halves, W += R3 S0^T by row halves
                     g1(tb + C::G1A_D, dr2, ds, CHUNK_C, ID_W, false);
                     g1(tb + C::W, dr3, desc_add(ds, C::P_B2), C::B2_CH, ID_N, true);
@@ -718,8 +721,8 @@ __device__ __forceinline__ void bwd_body(const Params &p) {
                     g1(tb + C::X, dr0, ds, SC, ID_W, false);
                     g1(tb + C::Y, dr1, ds, SC, ID_N, true);
                     commit(B_G1_DONE + b);
+                    commit(B_S_EMPTY + ss);
                 }
-                commit(B_S_EMPTY + ss);
                 return true;
             };
             // G1, second part (V_Q, V_K): [X|Y] = R0 [L0; L1]^T, Y += R1 L0^T, over the X
